@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark of the expert-parallel MoE-layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one forward of the whole layer (route -> preprocess -> dispatch ->
+grouped expert FFN -> combine) over one batch of T synthetic tokens, inputs
+resident in HBM.  L2 is flushed (a 256 MiB write) before every timed step, and
+each step is timed with CUDA events on the launching stream; the max over ranks
+is taken.  With N > 1 (torchrun) every rank runs an independent replica on its
+own batch (replicas only: the layer needs no collective on one node here), so
+scaling is weak and value = tokens of all ranks / max time.
+
+`--impl reference` times the CPU oracle (float64 numpy, the definition the CUDA
+path is checked against) on host cores over a bounded token sample per step.
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_workloads as W  # noqa: E402
+
+DEFAULT_WORKLOAD = "small_e8_d2048"
+METRIC = "MoE-layer fwd tokens/s on 1 B200; grouped-FFN % BF16 peak; permute/combine GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=W.WORKLOAD_ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-sample", type=int, default=0,
+                    help="tokens per CPU-oracle sample (0 = choose for ~10-30 s)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, ws):
+    if ws == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
+               0x2: "applications_clocks_setting"}
+
+    def __init__(self, index, period=0.002):
+        self.samples, self.reasons, self.period = [], 0, period
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"],
+                    "samples": 0}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def stage_bytes(wl):
+    sx = 4 if wl.x_dtype == "f32" else 2
+    T, D, R = wl.T, wl.D, wl.R
+    dispatch = T * D * sx + R * D * 2 + R * 4
+    combine = R * D * 2 + 2 * T * D * sx + (T * D * 2 if wl.n_shared else 0) + R * 8
+    return dispatch, combine
+
+
+def cpu_oracle_time(wl, inp_host, n_tok, seed=0):
+    """Time the oracle's layer forward on a token sample (weights already float64 on the host)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    toks = np.sort(rng.choice(wl.T, size=n_tok, replace=False))
+    x = inp_host["x"][toks]
+    t0 = time.perf_counter()
+    oracle.moe_layer(x, inp_host["w_router"], inp_host["bias"], inp_host["w_up"], inp_host["w_down"],
+                     inp_host["ws_up"], inp_host["ws_down"], E=wl.E, ep_size=wl.ep_size,
+                     top_k=wl.top_k, act=wl.act, renormalize=wl.renormalize,
+                     x_is_f32=(wl.x_dtype == "f32"))
+    return time.perf_counter() - t0
+
+
+def host_inputs_f64(wl, inp):
+    f = lambda t: None if t is None else t.detach().cpu().to(torch.float64).numpy()
+    return dict(x=f(inp["x"]), w_router=inp["w_router"].cpu().numpy(),
+                bias=None if inp["bias"] is None else inp["bias"].cpu().numpy(),
+                w_up=f(inp["w_gate_up"] if wl.act == "swiglu" else inp["w1"]), w_down=f(inp["w_down"]),
+                ws_up=f(inp["ws_gate_up"]), ws_down=f(inp["ws_down"]))
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def pick_sample(wl, budget_s=12.0):
+    """Tokens per oracle sample so one sample costs about budget_s on the host."""
+    per_tok_flop = 2 * wl.D * wl.F * (3 if wl.act == "swiglu" else 2) * wl.top_k \
+        + 6 * wl.D * wl.F_shared * wl.n_shared + 2 * wl.D * wl.E
+    est_flops = 30e9            # a conservative float64 BLAS rate for an 8-core host
+    return int(max(16, min(wl.T, budget_s * est_flops / per_tok_flop)))
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = W.get(args.workload)
+    inp = W.make_inputs(wl, device="cpu")
+    host = host_inputs_f64(wl, inp)
+    del inp
+    n_tok = args.cpu_sample or pick_sample(wl, budget_s=min(10.0, max(0.5, 120.0 / max(1, args.steps))))
+    for i in range(args.warmup):
+        cpu_oracle_time(wl, host, min(n_tok, 16), seed=i)
+    times = [cpu_oracle_time(wl, host, n_tok, seed=100 + i) for i in range(args.steps)]
+    total = sum(times)
+    value = n_tok * args.steps / total
+    cores = cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "D": wl.D, "E": wl.E, "ep_size": wl.ep_size,
+                   "top_k": wl.top_k, "F": wl.F, "n_shared": wl.n_shared, "F_shared": wl.F_shared,
+                   "tokens_per_step": n_tok},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n_tok} random tokens of the {wl.name} batch per step "
+                                   f"(tokens are independent: dropless routing)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    ws, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    import expert_dispatch_fp32_b200 as M
+
+    wl = W.get(args.workload)
+    peaks, peak_src = load_peaks()
+    inp = W.make_inputs(wl, device="cuda")
+    if rank > 0:
+        inp["x"] = W.make_x(wl, device="cuda", seed=wl.seed + 1000 * rank)
+    cpu_host = None
+    want_cpu = (rank == 0 and ws == 1 and not args.no_cpu_baseline)
+    if want_cpu:
+        cpu_host = host_inputs_f64(wl, inp)
+    up = inp["w_gate_up"] if wl.act == "swiglu" else inp["w1"]
+    layer = M.MoELayer(D=wl.D, E=wl.E, ep_size=wl.ep_size, top_k=wl.top_k, F=wl.F,
+                       w_router=inp["w_router"], w_gate_up=up, w_down=inp["w_down"],
+                       expert_bias=inp["bias"], ws_gate_up=inp["ws_gate_up"], ws_down=inp["ws_down"],
+                       act=wl.act, renormalize=wl.renormalize, x_dtype=wl.x_dtype)
+    torch.cuda.synchronize()
+    for key in ("w_gate_up", "w1", "w_down", "ws_gate_up", "ws_down"):
+        inp.pop(key, None)
+    torch.cuda.empty_cache()
+    x = inp["x"]
+    T = wl.T
+    b = layer.allocate(T)
+    cfg = layer.config(T)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    x_bf = x if wl.x_dtype == "bf16" else None
+
+    def step(ev):
+        ev[0].record(stream)
+        M.moe_route(cfg, x, layer.w_router, layer.expert_bias, None, b["topk_idx"], b["topk_w"],
+                    b["workspace"], stream)
+        ev[1].record(stream)
+        M.moe_preprocess(cfg, b["topk_idx"], b["counts"], b["expert_offsets"], b["rank_splits"],
+                         b["rank_offsets"], b["pos"], b["src"], b["workspace"], b["status"], stream)
+        ev[2].record(stream)
+        M.moe_dispatch_permute(cfg, x, b["src"], b["x_perm"], stream)
+        ev[3].record(stream)
+        M.moe_expert_ffn(cfg, b["x_perm"], x_bf, b["expert_offsets"], layer.packed, b["act"],
+                         b["y_perm"], b["shared_out"], b["workspace"], b["status"], stream)
+        ev[4].record(stream)
+        M.moe_combine_unpermute(cfg, b["y_perm"], b["pos"], b["topk_w"], x, b["shared_out"],
+                                b["out"], stream)
+        ev[5].record(stream)
+
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    # the stage-by-stage step is moe_forward: check once that both give the same bits
+    step(mk())
+    ref_out = b["out"].clone()
+    layer.forward(x, stream)
+    torch.cuda.synchronize()
+    assert torch.equal(ref_out, b["out"]), "stage-by-stage step differs from moe_forward"
+    layer.check_status()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(mk())
+    torch.cuda.synchronize()
+    barrier(ws)
+    evs = [mk() for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize()
+    barrier(ws)
+    layer.check_status()
+    stage_ms = np.zeros(5)
+    for ev in evs:
+        stage_ms += [ev[j].elapsed_time(ev[j + 1]) for j in range(5)]
+    total_ms = float(stage_ms.sum())
+    total_ms_max = max_over_ranks(total_ms, ws)
+    value = T * ws * args.steps / (total_ms_max / 1e3)
+
+    # end to end: pinned host x -> device, forward, device -> pinned host out
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty(b["out"].shape, dtype=b["out"].dtype).pin_memory()
+    x_dev = torch.empty_like(x)
+    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    for _ in range(args.warmup):
+        x_dev.copy_(x_host, non_blocking=True)
+        layer.forward(x_dev, stream)
+        out_host.copy_(b["out"], non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(ws)
+    for i in range(args.steps):
+        flush.zero_()
+        e_ev[i][0].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        layer.forward(x_dev, stream)
+        out_host.copy_(b["out"], non_blocking=True)
+        e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    layer.check_status()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(z) for a, z in e_ev), ws)
+    e2e_value = T * ws * args.steps / (e2e_ms / 1e3)
+    sx = 4 if wl.x_dtype == "f32" else 2
+
+    # roofline of the dominant kernel: the grouped expert FFN (tcgen05 GEMMs)
+    ffn_ms = stage_ms[3] / args.steps
+    ffn_tflops = wl.ffn_flop() / (ffn_ms / 1e3) / 1e12
+    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "ffn_traffic.json")
+    if os.path.exists(tpath):
+        try:
+            import hashlib
+            with open(tpath) as f:
+                tj = json.load(f)
+            src = open(os.path.join(ROOT, "expert_dispatch_fp32_b200", "csrc", "grouped_gemm.cu"), "rb").read()
+            ent = tj.get(wl.name)
+            if ent and ent.get("kernel_sha256") == hashlib.sha256(src).hexdigest():
+                traffic = ent["dram_bytes_per_step"]
+        except Exception:
+            traffic = None
+    disp_b, comb_b = stage_bytes(wl)
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    disp_gbs = disp_b / (stage_ms[2] / args.steps / 1e3) / 1e9
+    comb_gbs = comb_b / (stage_ms[4] / args.steps / 1e3) / 1e9
+    launches_per_step = 2 + 3 + 1 + (4 if wl.n_shared else 2) + 1
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "D": wl.D, "E": wl.E, "ep_size": wl.ep_size,
+                   "top_k": wl.top_k, "F": wl.F, "act": wl.act, "n_shared": wl.n_shared,
+                   "F_shared": wl.F_shared, "router": "fp32", "parallelism": f"replicas{ws}",
+                   "l2": "flushed (256 MiB write) before every timed step"},
+        "roofline": {"bound": "tensor", "achieved": ffn_tflops, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": ffn_tflops / peak_tf, "traffic": traffic,
+                     "kernel": "grouped_gemm_kernel (moe_expert_ffn: routed gate_up+down"
+                               + (", shared gate_up+down" if wl.n_shared else "") + ")",
+                     "peak_source": f"{peak_src} bf16 burst"},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * wl.D * sx,
+                "d2h_bytes_per_step": T * wl.D * sx},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "stages_us": {n: 1e3 * float(v) / args.steps for n, v in
+                      zip(("route", "preprocess", "dispatch", "expert_ffn", "combine"), stage_ms)},
+        "ffn_tflops": ffn_tflops,
+        "dispatch_gbs": disp_gbs, "dispatch_frac_hbm": disp_gbs / hbm,
+        "combine_gbs": comb_gbs, "combine_frac_hbm": comb_gbs / hbm,
+    }
+    if want_cpu:
+        n_tok = args.cpu_sample or pick_sample(wl)
+        cpu_oracle_time(wl, cpu_host, min(16, n_tok))          # warm BLAS
+        t = cpu_oracle_time(wl, cpu_host, n_tok, seed=1)
+        line["cpu_baseline"] = {"value": n_tok / t, "unit": "tokens/s", "cores": cpu_threads(),
+                                "kind": "oracle",
+                                "sample": f"{n_tok} random tokens of the {wl.name} batch "
+                                          f"({t:.1f} s of float64 numpy on the host)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

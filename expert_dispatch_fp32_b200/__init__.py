@@ -1,0 +1,16 @@
+"""Expert-parallel MoE-layer forward on one NVIDIA B200 (sm_100a).
+
+The compute path is libmoe.so (hand-written CUDA behind a C ABI, include/moe.h);
+this package holds its ctypes binding and a small layer object that allocates
+buffers with PyTorch.  Stages, after "Expert Parallel (EP)", Communication
+Pattern: moe_route -> moe_preprocess -> moe_dispatch_permute -> moe_expert_ffn
+-> moe_combine_unpermute (or moe_forward for all five).
+"""
+from ._binding import (  # noqa: F401
+    LIB_PATH, MOE_ACT_GELU, MOE_ACT_SWIGLU, MOE_DT_BF16, MOE_DT_F32, MOE_ERR_CUDA,
+    MOE_ERR_INDEX_OOB, MOE_ERR_INVALID_ARG, MOE_ERR_TIMEOUT, MOE_ERR_UNSUPPORTED, MOE_OK,
+    MoeConfig, MoeError, lib, moe_abi_version, moe_combine_unpermute, moe_dispatch_permute,
+    moe_expert_ffn, moe_forward, moe_packed_weights_size, moe_prepare_weights, moe_preprocess,
+    moe_route, moe_status_string, moe_validate_config, moe_workspace_size,
+)
+from .layer import MoELayer, make_config  # noqa: F401

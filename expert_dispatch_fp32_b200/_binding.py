@@ -1,0 +1,154 @@
+"""ctypes binding of libmoe.so: argument marshalling only.
+
+Every function here has the name and argument order of the C entry point it
+wraps (see include/moe.h); tensors are passed as raw device pointers, ``None``
+as NULL, and the stream defaults to torch's current stream.  No arithmetic of
+the layer happens in Python: a missing or unloadable library raises at import
+of the first call, and there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_INDEX_OOB, MOE_ERR_TIMEOUT = range(6)
+MOE_DT_F32, MOE_DT_BF16 = 0, 1
+MOE_ACT_GELU, MOE_ACT_SWIGLU = 0, 1
+
+
+class MoeConfig(ctypes.Structure):
+    """Mirror of ``moe_config`` (include/moe.h)."""
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "T", "D", "E", "ep_size", "top_k", "F", "act", "renormalize", "x_dtype",
+        "router_dtype", "n_shared", "F_shared")]
+
+    def __repr__(self):
+        return "MoeConfig(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class MoeError(RuntimeError):
+    def __init__(self, name, status):
+        super().__init__(f"{name} failed: {moe_status_string(status)} ({status})")
+        self.status = status
+
+
+_lib = None
+_vp, _i32p, _f32p, _cfgp = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(MoeConfig)
+_SIGS = {
+    "moe_validate_config": (ctypes.c_int, [_cfgp]),
+    "moe_workspace_size": (ctypes.c_size_t, [_cfgp]),
+    "moe_packed_weights_size": (ctypes.c_size_t, [_cfgp]),
+    "moe_prepare_weights": (ctypes.c_int, [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_route": (ctypes.c_int, [_cfgp, _vp, _f32p, _f32p, _f32p, _i32p, _f32p, _vp, _vp]),
+    "moe_preprocess": (ctypes.c_int, [_cfgp, _i32p, _i32p, _i32p, _i32p, _i32p, _i32p, _i32p, _vp,
+                                      _i32p, _vp]),
+    "moe_dispatch_permute": (ctypes.c_int, [_cfgp, _vp, _i32p, _vp, _vp]),
+    "moe_expert_ffn": (ctypes.c_int, [_cfgp, _vp, _vp, _i32p, _vp, _vp, _vp, _vp, _vp, _i32p, _vp]),
+    "moe_combine_unpermute": (ctypes.c_int, [_cfgp, _vp, _i32p, _f32p, _vp, _vp, _vp, _vp]),
+    "moe_forward": (ctypes.c_int, [_cfgp, _vp, _f32p, _f32p, _vp, _f32p, _i32p, _f32p, _i32p, _i32p,
+                                   _i32p, _i32p, _i32p, _i32p, _vp, _vp, _vp, _vp, _vp, _vp, _i32p,
+                                   _vp]),
+    "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "moe_abi_version": (ctypes.c_int32, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so (built in-tree by ``expert_dispatch_fp32_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libmoe.so not built: {LIB_PATH} is missing "
+                              "(run `python -m expert_dispatch_fp32_b200.build`)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _s(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _call(name, *args):
+    st = getattr(lib(), name)(*args)
+    if st != MOE_OK:
+        raise MoeError(name, st)
+
+
+def moe_status_string(status: int) -> str:
+    return lib().moe_status_string(status).decode()
+
+
+def moe_abi_version() -> int:
+    return lib().moe_abi_version()
+
+
+def moe_validate_config(cfg: MoeConfig) -> int:
+    return lib().moe_validate_config(ctypes.byref(cfg))
+
+
+def moe_workspace_size(cfg: MoeConfig) -> int:
+    return lib().moe_workspace_size(ctypes.byref(cfg))
+
+
+def moe_packed_weights_size(cfg: MoeConfig) -> int:
+    return lib().moe_packed_weights_size(ctypes.byref(cfg))
+
+
+def moe_prepare_weights(cfg, w_gate_up, w_down, ws_gate_up, ws_down, packed, stream=None):
+    _call("moe_prepare_weights", ctypes.byref(cfg), _p(w_gate_up), _p(w_down), _p(ws_gate_up),
+          _p(ws_down), _p(packed), _s(stream))
+
+
+def moe_route(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w, workspace, stream=None):
+    _call("moe_route", ctypes.byref(cfg), _p(x), _p(w_router), _p(expert_bias), _p(logits_out),
+          _p(topk_idx), _p(topk_w), _p(workspace), _s(stream))
+
+
+def moe_preprocess(cfg, topk_idx, counts, expert_offsets, rank_splits, rank_offsets, pos, src,
+                   workspace, status, stream=None):
+    _call("moe_preprocess", ctypes.byref(cfg), _p(topk_idx), _p(counts), _p(expert_offsets),
+          _p(rank_splits), _p(rank_offsets), _p(pos), _p(src), _p(workspace), _p(status), _s(stream))
+
+
+def moe_dispatch_permute(cfg, x, src, x_perm, stream=None):
+    _call("moe_dispatch_permute", ctypes.byref(cfg), _p(x), _p(src), _p(x_perm), _s(stream))
+
+
+def moe_expert_ffn(cfg, x_perm, x, expert_offsets, packed, act, y_perm, shared_out, workspace,
+                   status, stream=None):
+    _call("moe_expert_ffn", ctypes.byref(cfg), _p(x_perm), _p(x), _p(expert_offsets), _p(packed),
+          _p(act), _p(y_perm), _p(shared_out), _p(workspace), _p(status), _s(stream))
+
+
+def moe_combine_unpermute(cfg, y_perm, pos, topk_w, x, shared_out, out, stream=None):
+    _call("moe_combine_unpermute", ctypes.byref(cfg), _p(y_perm), _p(pos), _p(topk_w), _p(x),
+          _p(shared_out), _p(out), _s(stream))
+
+
+def moe_forward(cfg, x, w_router, expert_bias, packed, logits_out, topk_idx, topk_w, counts,
+                expert_offsets, rank_splits, rank_offsets, pos, src, x_perm, act, y_perm, shared_out,
+                out, workspace, status, stream=None):
+    _call("moe_forward", ctypes.byref(cfg), _p(x), _p(w_router), _p(expert_bias), _p(packed),
+          _p(logits_out), _p(topk_idx), _p(topk_w), _p(counts), _p(expert_offsets), _p(rank_splits),
+          _p(rank_offsets), _p(pos), _p(src), _p(x_perm), _p(act), _p(y_perm), _p(shared_out),
+          _p(out), _p(workspace), _p(status), _s(stream))

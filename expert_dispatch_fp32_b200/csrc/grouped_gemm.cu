@@ -1,0 +1,498 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// "Expert Parallel (EP)", Communication Pattern step 3 (each rank runs its local
+// experts on the tokens it received); "Worked Example: Tracing a Token Through
+// Expert Parallelism", Step 3 (two-layer FFN per expert).  Here every expert of
+// every virtual rank runs in one persistent launch over the rank-major buffer.
+//
+// out[row, :] = epilogue( A[row, :] . B[g]^T ) for the rows of group g
+//   A  bf16 [rows, K] row-major (K-major), rows of group g contiguous at
+//      [group_offsets[g], group_offsets[g+1]);
+//   B  bf16 [G, N, K] (K-major), one [N, K] matrix per group.
+//
+// Tiles are 128 x BN (BN = 256/128/64) output blocks; the tile list is
+// expert-major, then N block, then M tile fastest, so the CTAs that run at the
+// same time share each weight tile through L2 and stream every weight from HBM
+// about once.  The per-expert M-tile prefix (mt_start) comes from the preprocess
+// stage on the device: the host never learns the counts, so grid = #SMs and each
+// CTA walks tiles blockIdx.x, blockIdx.x + gridDim.x, ...  Empty experts own no
+// tiles, so their weights are never read.
+//
+// One CTA per SM, 6 warps:
+//   warp 0      TMA producer: A tile [128 x 64] and B tile [BN x 64] per K step
+//               into a STAGES-deep shared-memory ring (128-byte swizzle).
+//   warp 1      allocates 2*BN TMEM columns; one lane issues tcgen05.mma
+//               (M=128, N=BN, K=16, bf16 in, fp32 accumulate) into one of two
+//               TMEM accumulators and commits to mbarriers.
+//   warps 2-5   epilogue: tcgen05.ld the accumulator (warp w owns TMEM lanes
+//               32*(w%4)..+31 = tile rows), apply the activation, round to bf16
+//               and store the rows that belong to the group (rows past the group
+//               end belong to the next expert and are dropped).
+// The two accumulators let the epilogue of tile i overlap the MMAs of tile i+1.
+//
+// Every mbarrier wait is bounded (about 2 s by %globaltimer): on expiry the
+// kernel writes MOE_ERR_TIMEOUT to the status word, raises a CTA-wide abort flag
+// so the other roles stop waiting, frees its TMEM and returns.
+#include <stdio.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr int kGemmThreads = 192;
+
+struct GemmArgs {
+  CUtensorMap tmap_a;
+  CUtensorMap tmap_b;
+  const int32_t* group_offsets;
+  const int32_t* mt_start;
+  int32_t G, N, K, dense_rows;
+  bf16* out;
+  int32_t ldo;
+  int32_t* status;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for phase `parity` of `bar`; false if the wait gave up.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       int32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        atomicCAS(status, 0, (int32_t)MOE_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row core groups 1024 bytes apart (SBO), sm_100 descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both K-major.
+__host__ __device__ constexpr uint32_t make_idesc(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void decode_tile(int tile, const int* mt, int G, int nb, int& g,
+                                            int& m, int& n) {
+  int lo = 0, hi = G;                      // mt[lo]*nb <= tile < mt[hi]*nb
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (mt[mid] * nb <= tile) lo = mid; else hi = mid;
+  }
+  g = lo;
+  const int mtiles = mt[g + 1] - mt[g];
+  const int local = tile - mt[g] * nb;
+  n = local / mtiles;
+  m = local - n * mtiles;
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+__device__ __forceinline__ float gelu_f(float h) {
+  return 0.5f * h * (1.0f + erff(h * 0.70710678118654752f));
+}
+
+__device__ __forceinline__ void store_row32(bf16* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 t;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&t);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
+    d[q] = t;
+  }
+}
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kStages = BN == 256 ? 4 : BN == 128 ? 6 : 8;
+  static constexpr int kABytes = kTileM * kTileK * 2;
+  static constexpr int kBBytes = BN * kTileK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr uint32_t kIdesc = make_idesc(kTileM, BN);
+  static size_t smem_bytes(int G) {
+    return 1024 + (size_t)kStages * kStageBytes + 256 + 2 * (size_t)(G + 1) * sizeof(int);
+  }
+};
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs p) {
+  using C = GemmCfg<BN>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* a_smem = smem;
+  uint8_t* b_smem = smem + S * C::kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  // bars: full[S], empty[S], tmem_full[2], tmem_empty[2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* mt = reinterpret_cast<int*>(smem + S * C::kStageBytes + 256);
+  const bool dense = p.group_offsets == nullptr;
+  const int G = dense ? 1 : p.G;
+  int* off = mt + (G + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
+  const uint32_t tfull0 = smem_u32(bars + 2 * S), tempty0 = smem_u32(bars + 2 * S + 2);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(full0 + 8 * i, 1);
+      mbar_init(empty0 + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull0 + 8 * i, 1);
+      mbar_init(tempty0 + 8 * i, 4);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_tmap(&p.tmap_a);
+    prefetch_tmap(&p.tmap_b);
+  }
+  if (dense) {
+    if (threadIdx.x == 0) {
+      mt[0] = 0; mt[1] = (p.dense_rows + kTileM - 1) / kTileM;
+      off[0] = 0; off[1] = p.dense_rows;
+    }
+  } else {
+    for (int i = threadIdx.x; i <= G; i += blockDim.x) {
+      mt[i] = p.mt_start[i];
+      off[i] = p.group_offsets[i];
+    }
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(C::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int nb = p.N / BN;
+  const int total = mt[G] * nb;
+  const int ksteps = p.K / kTileK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        int g, m, n;
+        decode_tile(tile, mt, G, nb, g, m, n);
+        const int row0 = off[g] + m * kTileM;
+        bool ok = true;
+        for (int kb = 0; kb < ksteps; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, C::kStageBytes);
+          tma_load_2d(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * kTileK, row0);
+          tma_load_3d(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * kTileK, n * BN, g);
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        bool ok = true;
+        for (int kb = 0; kb < ksteps; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = sw128_desc(smem_u32(a_smem + stage * C::kABytes));
+          const uint64_t bd = sw128_desc(smem_u32(b_smem + stage * C::kBBytes));
+#pragma unroll
+          for (int kk = 0; kk < kTileK / 16; ++kk)   // +32 bytes per K=16 slice
+            tc_mma(d_tmem, ad + 2 * kk, bd + 2 * kk, C::kIdesc, (kb | kk) != 0);
+          tc_commit(empty0 + 8 * stage);
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(tfull0 + 8 * acc);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int g, m, n;
+      decode_tile(tile, mt, G, nb, g, m, n);
+      const int row0 = off[g] + m * kTileM;
+      const int rows_valid = min(kTileM, off[g + 1] - row0);
+      const bool ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) break;     // keep the warp converged for tcgen05.ld
+      tc_fence_after();
+      const int r = q * 32 + lane;
+      const bool valid = r < rows_valid;
+      bf16* orow = p.out + (size_t)(row0 + (valid ? r : 0)) * p.ldo;
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      if (EPI == EPI_SWIGLU) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t gr[32], ur[32];
+          tmem_ld32(tb + c, gr);
+          tmem_ld32(tb + BN / 2 + c, ur);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
+          if (valid) store_row32(orow + n * (BN / 2) + c, v);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t hr[32];
+          tmem_ld32(tb + c, hr);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float h = __uint_as_float(hr[i]);
+            v[i] = (EPI == EPI_GELU) ? gelu_f(h) : h;
+          }
+          if (valid) store_row32(orow + n * BN + c, v);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(C::kTmemCols)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(ptr);
+  }();
+  return fn;
+}
+
+bool make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kTileK, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_3d(CUtensorMap* m, const void* base, uint64_t K, uint64_t N, uint64_t G, uint32_t box_n) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {K, N, G};
+  cuuint64_t strides[2] = {K * 2, N * K * 2};
+  cuuint32_t box[3] = {(cuuint32_t)kTileK, box_n, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int EPI>
+cudaError_t launch_tc(const GemmArgs& a, int grid, cudaStream_t s) {
+  using C = GemmCfg<BN>;
+  const size_t smem = C::smem_bytes(a.group_offsets ? a.G : 1);
+  auto kern = grouped_gemm_kernel<BN, EPI>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  kern<<<grid, kGemmThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  static int cache[64] = {0};
+  if (dev < 64 && cache[dev]) return cache[dev];
+  int n = 148;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (dev < 64) cache[dev] = n;
+  return n;
+}
+
+cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  const int BN = p.tile_n;
+  if (!make_map_2d(&a.tmap_a, p.A, (uint64_t)p.K, (uint64_t)p.a_rows, kTileM)) return cudaErrorInvalidValue;
+  if (!make_map_3d(&a.tmap_b, p.B, (uint64_t)p.K, (uint64_t)p.N, (uint64_t)p.G, (uint32_t)BN))
+    return cudaErrorInvalidValue;
+  a.group_offsets = p.group_offsets;
+  a.mt_start = p.mt_start;
+  a.G = p.G;
+  a.N = p.N;
+  a.K = p.K;
+  a.dense_rows = p.dense_rows;
+  a.out = p.out;
+  a.ldo = p.ldo;
+  a.status = p.status;
+  const int64_t tiles = p.max_tiles > 0 ? p.max_tiles : 1;
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  if (BN == 256) {
+    if (p.epi == EPI_SWIGLU) return launch_tc<256, EPI_SWIGLU>(a, grid, s);
+    if (p.epi == EPI_GELU) return launch_tc<256, EPI_GELU>(a, grid, s);
+    return launch_tc<256, EPI_STORE>(a, grid, s);
+  }
+  if (BN == 128) {
+    if (p.epi == EPI_GELU) return launch_tc<128, EPI_GELU>(a, grid, s);
+    if (p.epi == EPI_STORE) return launch_tc<128, EPI_STORE>(a, grid, s);
+    return cudaErrorInvalidValue;
+  }
+  if (BN == 64) {
+    if (p.epi == EPI_GELU) return launch_tc<64, EPI_GELU>(a, grid, s);
+    if (p.epi == EPI_STORE) return launch_tc<64, EPI_STORE>(a, grid, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

@@ -1,0 +1,305 @@
+// C ABI of libmoe.so: argument validation, buffer layouts and the stage calls.
+// Each call checks its arguments on the host, then only enqueues kernels on the
+// caller's stream.  Nothing here allocates device memory.
+#include <string.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+WsLayout ws_layout(const moe_config& c) {
+  WsLayout L;
+  const size_t T = (size_t)c.T, E = (size_t)c.E;
+  const size_t R = T * (size_t)c.top_k;
+  L.nblk = (int)((R + kPreChunk - 1) / kPreChunk);
+  size_t o = 0;
+  L.logits = o;       o = align256(o + T * E * sizeof(float));
+  L.block_counts = o; o = align256(o + (size_t)L.nblk * E * sizeof(int32_t));
+  L.mt_start = o;     o = align256(o + (E + 1) * sizeof(int32_t));
+  L.act_shared = o;   o = align256(o + T * (size_t)c.n_shared * c.F_shared * sizeof(bf16));
+  L.total = o;
+  return L;
+}
+
+PackLayout pack_layout(const moe_config& c) {
+  PackLayout L;
+  const size_t E = c.E, D = c.D, F = c.F;
+  const size_t nup = c.act == MOE_ACT_SWIGLU ? 2 * F : F;
+  const size_t Fc = (size_t)c.n_shared * c.F_shared;
+  size_t o = 0;
+  L.w_up = o;    o = align256(o + E * nup * D * sizeof(bf16));
+  L.w_down = o;  o = align256(o + E * D * F * sizeof(bf16));
+  L.ws_up = o;   o = align256(o + 2 * Fc * D * sizeof(bf16));
+  L.ws_down = o; o = align256(o + D * Fc * sizeof(bf16));
+  L.total = o;
+  return L;
+}
+
+int up_tile_n(const moe_config& c) {
+  if (c.act == MOE_ACT_SWIGLU) return 256;
+  return c.F % 256 == 0 ? 256 : c.F % 128 == 0 ? 128 : 64;
+}
+int down_tile_n(const moe_config& c) { return c.D % 256 == 0 ? 256 : c.D % 128 == 0 ? 128 : 64; }
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_CHECK_PTR(p) \
+  do {                                                 \
+    if ((p) == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_validate_config(const moe_config* cfg) {
+  if (cfg == nullptr) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = *cfg;
+  if (c.T < 0 || c.D <= 0 || c.E <= 0 || c.ep_size <= 0 || c.top_k <= 0 || c.F <= 0)
+    return MOE_ERR_INVALID_ARG;
+  if (c.E % c.ep_size != 0) return MOE_ERR_INVALID_ARG;        // num_experts % ep_size
+  if (c.top_k > c.E) return MOE_ERR_INVALID_ARG;
+  if (c.act != MOE_ACT_GELU && c.act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
+  if (c.renormalize != 0 && c.renormalize != 1) return MOE_ERR_INVALID_ARG;
+  if (c.x_dtype != MOE_DT_F32 && c.x_dtype != MOE_DT_BF16) return MOE_ERR_INVALID_ARG;
+  if (c.router_dtype != MOE_DT_F32) return MOE_ERR_UNSUPPORTED;   // the fp32 router only
+  if (c.n_shared < 0 || (c.n_shared > 0 && c.F_shared <= 0)) return MOE_ERR_INVALID_ARG;
+  if (c.E > kMaxExperts || c.top_k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
+  if (c.D % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  if (c.act == MOE_ACT_SWIGLU ? (c.F % 128 != 0) : (c.F % 64 != 0)) return MOE_ERR_UNSUPPORTED;
+  if (c.n_shared > 0 && (c.F_shared % 128 != 0 || c.x_dtype != MOE_DT_BF16)) return MOE_ERR_UNSUPPORTED;
+  const int64_t R = (int64_t)c.T * c.top_k;
+  if (R * (c.D / 8) >= (int64_t)1 << 31 || (int64_t)c.T * c.E >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+size_t moe_workspace_size(const moe_config* cfg) {
+  if (moe_validate_config(cfg) != MOE_OK) return 0;
+  return ws_layout(*cfg).total;
+}
+
+size_t moe_packed_weights_size(const moe_config* cfg) {
+  if (moe_validate_config(cfg) != MOE_OK) return 0;
+  return pack_layout(*cfg).total;
+}
+
+moe_status moe_prepare_weights(const moe_config* cfg, const void* w_gate_up, const void* w_down,
+                               const void* ws_gate_up, const void* ws_down, void* packed,
+                               void* stream) {
+  moe_status st = moe_validate_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  MOE_CHECK_PTR(w_gate_up);
+  MOE_CHECK_PTR(w_down);
+  MOE_CHECK_PTR(packed);
+  if (c.n_shared > 0) {
+    MOE_CHECK_PTR(ws_gate_up);
+    MOE_CHECK_PTR(ws_down);
+  }
+  return cuda_status(launch_pack(c, (const bf16*)w_gate_up, (const bf16*)w_down,
+                                 (const bf16*)ws_gate_up, (const bf16*)ws_down, (uint8_t*)packed,
+                                 as_stream(stream)));
+}
+
+moe_status moe_route(const moe_config* cfg, const void* x, const float* w_router,
+                     const float* expert_bias, float* logits_out, int32_t* topk_idx,
+                     float* topk_w, void* workspace, void* stream) {
+  moe_status st = moe_validate_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (c.T == 0) return MOE_OK;
+  MOE_CHECK_PTR(x);
+  MOE_CHECK_PTR(w_router);
+  MOE_CHECK_PTR(topk_idx);
+  MOE_CHECK_PTR(topk_w);
+  MOE_CHECK_PTR(workspace);
+  float* logits = logits_out;
+  if (logits == nullptr) logits = (float*)((uint8_t*)workspace + ws_layout(c).logits);
+  else if (!aligned16(logits)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_route(c, x, w_router, expert_bias, logits, topk_idx, topk_w,
+                                  as_stream(stream)));
+}
+
+moe_status moe_preprocess(const moe_config* cfg, const int32_t* topk_idx, int32_t* counts,
+                          int32_t* expert_offsets, int32_t* rank_splits, int32_t* rank_offsets,
+                          int32_t* pos, int32_t* src, void* workspace, int32_t* status,
+                          void* stream) {
+  moe_status st = moe_validate_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  MOE_CHECK_PTR(counts);
+  MOE_CHECK_PTR(expert_offsets);
+  MOE_CHECK_PTR(rank_splits);
+  MOE_CHECK_PTR(rank_offsets);
+  MOE_CHECK_PTR(workspace);
+  MOE_CHECK_PTR(status);
+  if (c.T > 0) {
+    MOE_CHECK_PTR(topk_idx);
+    MOE_CHECK_PTR(pos);
+    MOE_CHECK_PTR(src);
+  }
+  const WsLayout L = ws_layout(c);
+  uint8_t* ws = (uint8_t*)workspace;
+  return cuda_status(launch_preprocess(c, topk_idx, counts, expert_offsets, rank_splits,
+                                       rank_offsets, pos, src, (int32_t*)(ws + L.block_counts),
+                                       L.nblk, (int32_t*)(ws + L.mt_start), status,
+                                       as_stream(stream)));
+}
+
+moe_status moe_dispatch_permute(const moe_config* cfg, const void* x, const int32_t* src,
+                                void* x_perm, void* stream) {
+  moe_status st = moe_validate_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (c.T == 0) return MOE_OK;
+  MOE_CHECK_PTR(x);
+  MOE_CHECK_PTR(src);
+  MOE_CHECK_PTR(x_perm);
+  return cuda_status(launch_dispatch(c, x, src, (bf16*)x_perm, as_stream(stream)));
+}
+
+moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void* x,
+                          const int32_t* expert_offsets, const void* packed, void* act,
+                          void* y_perm, void* shared_out, void* workspace, int32_t* status,
+                          void* stream) {
+  moe_status st = moe_validate_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (c.T == 0) return MOE_OK;
+  MOE_CHECK_PTR(x_perm);
+  MOE_CHECK_PTR(expert_offsets);
+  MOE_CHECK_PTR(packed);
+  MOE_CHECK_PTR(act);
+  MOE_CHECK_PTR(y_perm);
+  MOE_CHECK_PTR(workspace);
+  MOE_CHECK_PTR(status);
+  if (c.n_shared > 0) {
+    MOE_CHECK_PTR(x);
+    MOE_CHECK_PTR(shared_out);
+  }
+  cudaStream_t s = as_stream(stream);
+  const WsLayout W = ws_layout(c);
+  const PackLayout P = pack_layout(c);
+  const uint8_t* pk = (const uint8_t*)packed;
+  uint8_t* ws = (uint8_t*)workspace;
+  const int64_t R = (int64_t)c.T * c.top_k;
+  const int nup = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
+
+  // Routed experts, gate_up (+ activation) then down, over the rank-major rows.
+  GemmProblem up;
+  memset(&up, 0, sizeof(up));
+  up.A = (const bf16*)x_perm; up.a_rows = R;
+  up.B = (const bf16*)(pk + P.w_up); up.G = c.E;
+  up.N = nup; up.K = c.D;
+  up.group_offsets = expert_offsets;
+  up.mt_start = (const int32_t*)(ws + W.mt_start);
+  up.tile_n = up_tile_n(c);
+  up.max_tiles = (R / kTileM + c.E) * (int64_t)(nup / up.tile_n);
+  up.out = (bf16*)act; up.ldo = c.F;
+  up.epi = c.act == MOE_ACT_SWIGLU ? EPI_SWIGLU : EPI_GELU;
+  up.status = status;
+  cudaError_t err = launch_grouped_gemm(up, s);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+
+  GemmProblem dn = up;
+  dn.A = (const bf16*)act; dn.a_rows = R;
+  dn.B = (const bf16*)(pk + P.w_down);
+  dn.N = c.D; dn.K = c.F;
+  dn.tile_n = down_tile_n(c);
+  dn.max_tiles = (R / kTileM + c.E) * (int64_t)(c.D / dn.tile_n);
+  dn.out = (bf16*)y_perm; dn.ldo = c.D;
+  dn.epi = EPI_STORE;
+  err = launch_grouped_gemm(dn, s);
+  if (err != cudaSuccess || c.n_shared == 0) return cuda_status(err);
+
+  // Shared experts: one dense SwiGLU expert of intermediate S*Fs over all tokens.
+  const int Fc = c.n_shared * c.F_shared;
+  bf16* act_s = (bf16*)(ws + W.act_shared);
+  GemmProblem su;
+  memset(&su, 0, sizeof(su));
+  su.A = (const bf16*)x; su.a_rows = c.T;
+  su.B = (const bf16*)(pk + P.ws_up); su.G = 1;
+  su.N = 2 * Fc; su.K = c.D;
+  su.group_offsets = nullptr; su.mt_start = nullptr; su.dense_rows = c.T;
+  su.tile_n = 256;
+  su.max_tiles = ((int64_t)(c.T + kTileM - 1) / kTileM) * (2 * Fc / 256);
+  su.out = act_s; su.ldo = Fc;
+  su.epi = EPI_SWIGLU;
+  su.status = status;
+  err = launch_grouped_gemm(su, s);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+
+  GemmProblem sd = su;
+  sd.A = act_s; sd.a_rows = c.T;
+  sd.B = (const bf16*)(pk + P.ws_down);
+  sd.N = c.D; sd.K = Fc;
+  sd.tile_n = down_tile_n(c);
+  sd.max_tiles = ((int64_t)(c.T + kTileM - 1) / kTileM) * (c.D / sd.tile_n);
+  sd.out = (bf16*)shared_out; sd.ldo = c.D;
+  sd.epi = EPI_STORE;
+  return cuda_status(launch_grouped_gemm(sd, s));
+}
+
+moe_status moe_combine_unpermute(const moe_config* cfg, const void* y_perm, const int32_t* pos,
+                                 const float* topk_w, const void* x, const void* shared_out,
+                                 void* out, void* stream) {
+  moe_status st = moe_validate_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (c.T == 0) return MOE_OK;
+  MOE_CHECK_PTR(y_perm);
+  MOE_CHECK_PTR(pos);
+  MOE_CHECK_PTR(topk_w);
+  MOE_CHECK_PTR(x);
+  MOE_CHECK_PTR(out);
+  if (out == x) return MOE_ERR_INVALID_ARG;
+  if (c.n_shared > 0) MOE_CHECK_PTR(shared_out);
+  return cuda_status(launch_combine(c, (const bf16*)y_perm, pos, topk_w, x,
+                                    c.n_shared > 0 ? (const bf16*)shared_out : nullptr, out,
+                                    as_stream(stream)));
+}
+
+moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_router,
+                       const float* expert_bias, const void* packed, float* logits_out,
+                       int32_t* topk_idx, float* topk_w, int32_t* counts,
+                       int32_t* expert_offsets, int32_t* rank_splits, int32_t* rank_offsets,
+                       int32_t* pos, int32_t* src, void* x_perm, void* act, void* y_perm,
+                       void* shared_out, void* out, void* workspace, int32_t* status,
+                       void* stream) {
+  moe_status st = moe_route(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w,
+                            workspace, stream);
+  if (st != MOE_OK) return st;
+  st = moe_preprocess(cfg, topk_idx, counts, expert_offsets, rank_splits, rank_offsets, pos, src,
+                      workspace, status, stream);
+  if (st != MOE_OK) return st;
+  st = moe_dispatch_permute(cfg, x, src, x_perm, stream);
+  if (st != MOE_OK) return st;
+  st = moe_expert_ffn(cfg, x_perm, x, expert_offsets, packed, act, y_perm, shared_out, workspace,
+                      status, stream);
+  if (st != MOE_OK) return st;
+  return moe_combine_unpermute(cfg, y_perm, pos, topk_w, x, shared_out, out, stream);
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_INDEX_OOB: return "expert index out of range";
+    case MOE_ERR_TIMEOUT: return "bounded wait expired in a kernel";
+  }
+  return "unknown status";
+}
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+}  // extern "C"

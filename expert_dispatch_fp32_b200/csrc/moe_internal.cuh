@@ -1,0 +1,91 @@
+// Internal declarations shared by the libmoe.so translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+typedef __nv_bfloat16 bf16;
+
+// ---------------------------------------------------------------------------
+// Sizes fixed by the kernels
+// ---------------------------------------------------------------------------
+constexpr int kMaxExperts = 1024;   // preprocess keeps one counter per expert in smem
+constexpr int kMaxTopK = 32;        // top-k kernel keeps selection j in lane j
+constexpr int kPreChunk = 1024;     // flat (token, slot) pairs per preprocess block
+constexpr int kPreThreads = 256;
+constexpr int kTileM = 128;         // GEMM tile rows (one tcgen05 M=128 accumulator)
+constexpr int kTileK = 64;          // GEMM K step: 64 bf16 = one 128-byte swizzle row
+
+// ---------------------------------------------------------------------------
+// Workspace and packed-weight layouts (byte offsets, each 256-aligned)
+// ---------------------------------------------------------------------------
+struct WsLayout {
+  size_t logits;        // fp32 [T, E]
+  size_t block_counts;  // int32 [nblk, E]
+  size_t mt_start;      // int32 [E + 1]: prefix of ceil(count/128) per expert
+  size_t act_shared;    // bf16 [T, S*Fs]
+  size_t total;
+  int nblk;
+};
+WsLayout ws_layout(const moe_config& c);
+
+struct PackLayout {
+  size_t w_up;          // bf16 [E, Nup, D]   (Nup = 2F SwiGLU interleaved, or F)
+  size_t w_down;        // bf16 [E, D, F]
+  size_t ws_up;         // bf16 [1, 2*S*Fs, D] interleaved
+  size_t ws_down;       // bf16 [1, D, S*Fs]
+  size_t total;
+};
+PackLayout pack_layout(const moe_config& c);
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// GEMM tile widths chosen from the shapes
+int up_tile_n(const moe_config& c);
+int down_tile_n(const moe_config& c);
+
+// ---------------------------------------------------------------------------
+// Launchers (each returns cudaGetLastError() of its launches)
+// ---------------------------------------------------------------------------
+cudaError_t launch_route(const moe_config& c, const void* x, const float* w_router,
+                         const float* bias, float* logits, int32_t* topk_idx, float* topk_w,
+                         cudaStream_t s);
+cudaError_t launch_preprocess(const moe_config& c, const int32_t* topk_idx, int32_t* counts,
+                              int32_t* expert_offsets, int32_t* rank_splits,
+                              int32_t* rank_offsets, int32_t* pos, int32_t* src,
+                              int32_t* block_counts, int nblk, int32_t* mt_start,
+                              int32_t* status, cudaStream_t s);
+cudaError_t launch_dispatch(const moe_config& c, const void* x, const int32_t* src,
+                            bf16* x_perm, cudaStream_t s);
+cudaError_t launch_combine(const moe_config& c, const bf16* y_perm, const int32_t* pos,
+                           const float* topk_w, const void* x, const bf16* shared_out, void* out,
+                           cudaStream_t s);
+cudaError_t launch_pack(const moe_config& c, const bf16* w_up, const bf16* w_down,
+                        const bf16* ws_up, const bf16* ws_down, uint8_t* packed, cudaStream_t s);
+
+// Grouped GEMM on the tensor cores.  out[row, :] = epilogue(A[row, :] @ B[g]^T)
+// for rows of group g; B is K-major [G, N, K].
+enum Epilogue { EPI_STORE = 0, EPI_GELU = 1, EPI_SWIGLU = 2 };
+struct GemmProblem {
+  const bf16* A; int64_t a_rows;          // A [a_rows, K]
+  const bf16* B; int G;                   // B [G, N, K]
+  int N, K;
+  const int32_t* group_offsets;           // [G+1] device, or nullptr: one dense group
+  const int32_t* mt_start;                // [G+1] device, or nullptr
+  int dense_rows;                         // rows of the dense group
+  int64_t max_tiles;                      // host upper bound on tiles (grid size)
+  bf16* out; int ldo;                     // output row stride in elements
+  int epi; int tile_n;
+  int32_t* status;
+};
+cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s);
+
+int sm_count();
+
+}  // namespace moe

@@ -1,0 +1,196 @@
+// Router: fp32 logits over all experts, then softmax + top-k per token.
+//
+// "Worked Example: Tracing a Token Through Expert Parallelism", Step 1: the gate
+// scores all E experts for the token, softmax-normalises, keeps the top-k.
+// "Expert Parallel (EP)", Configuration: router_dtype 'fp32'.
+//
+// Logits kernel: a token-tiled SIMT fp32 GEMM (x[T,D] . W_r[E,D]^T).  W_r does not
+// fit in shared memory for large E*D, so tiles of BM tokens x BN experts stream
+// 32-wide K slices of both operands through shared memory.  Each thread sums a
+// 32-term K slice in fp32 and folds the slice into an fp64 running total, so the
+// stored fp32 logit is the dot product rounded once, to within fp32 round-off of
+// a 32-term partial (~1e-8 relative), far inside the 1e-5 near-tie margin.
+//
+// Top-k kernel: one warp per token; selection j is an exact warp argmax on
+// (logit, -index), so ties go to the lower expert index; lane j keeps pick j.
+#include <math.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kRouteBM = 128;
+constexpr int kRouteBK = 32;
+constexpr int kRouteThreads = 256;
+
+__device__ __forceinline__ void load4(const float* p, float (&v)[4]) {
+  float4 t = __ldg(reinterpret_cast<const float4*>(p));
+  v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+}
+__device__ __forceinline__ void load4(const bf16* p, float (&v)[4]) {
+  uint2 t = __ldg(reinterpret_cast<const uint2*>(p));
+  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&t.x);
+  __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&t.y);
+  float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+  v[0] = fa.x; v[1] = fa.y; v[2] = fb.x; v[3] = fb.y;
+}
+
+template <int BN, typename XT>
+__global__ void __launch_bounds__(kRouteThreads)
+route_logits_kernel(const XT* __restrict__ x, const float* __restrict__ w,
+                    const float* __restrict__ bias, float* __restrict__ logits, int T, int D,
+                    int E) {
+  constexpr int BM = kRouteBM, BK = kRouteBK;
+  constexpr int NTN = BN / 4;                 // thread columns, 4 experts each
+  constexpr int NTM = kRouteThreads / NTN;    // thread rows
+  constexpr int TM = BM / NTM;                // tokens per thread
+  static_assert(TM >= 1 && BM % NTM == 0, "tile");
+  __shared__ __align__(16) float xs[BK][BM + 4];
+  __shared__ __align__(16) float ws[BK][BN + 4];
+
+  const int tid = threadIdx.x;
+  const int tx = tid % NTN, ty = tid / NTN;
+  const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
+
+  double tot[TM][4];
+#pragma unroll
+  for (int i = 0; i < TM; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tot[i][j] = 0.0;
+
+  for (int k0 = 0; k0 < D; k0 += BK) {
+    for (int i = tid; i < BM * (BK / 4); i += kRouteThreads) {
+      const int r = i / (BK / 4), c4 = (i % (BK / 4)) * 4;
+      const int t = m0 + r;
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      if (t < T) load4(x + (size_t)t * D + k0 + c4, v);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) xs[c4 + q][r] = v[q];
+    }
+    for (int i = tid; i < BN * (BK / 4); i += kRouteThreads) {
+      const int r = i / (BK / 4), c4 = (i % (BK / 4)) * 4;
+      const int e = n0 + r;
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      if (e < E) load4(w + (size_t)e * D + k0 + c4, v);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) ws[c4 + q][r] = v[q];
+    }
+    __syncthreads();
+    float acc[TM][4];
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 8
+    for (int kk = 0; kk < BK; ++kk) {
+      float a[TM];
+#pragma unroll
+      for (int i = 0; i < TM; ++i) a[i] = xs[kk][ty * TM + i];
+      const float4 b = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
+#pragma unroll
+      for (int i = 0; i < TM; ++i) {
+        acc[i][0] = fmaf(a[i], b.x, acc[i][0]);
+        acc[i][1] = fmaf(a[i], b.y, acc[i][1]);
+        acc[i][2] = fmaf(a[i], b.z, acc[i][2]);
+        acc[i][3] = fmaf(a[i], b.w, acc[i][3]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tot[i][j] += (double)acc[i][j];
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < TM; ++i) {
+    const int t = m0 + ty * TM + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = n0 + tx * 4 + j;
+      if (e >= E) continue;
+      float l = (float)tot[i][j];
+      if (bias != nullptr) l = l + bias[e];
+      logits[(size_t)t * E + e] = l;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256)
+route_topk_kernel(const float* __restrict__ logits, int32_t* __restrict__ topk_idx,
+                  float* __restrict__ topk_w, int T, int E, int k, int renorm) {
+  const int lane = threadIdx.x & 31;
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;
+  const float* row = logits + (size_t)t * E;
+  uint32_t taken = 0;                 // bit c: element c*32+lane already chosen
+  int my_idx = 0;
+  float my_val = 0.f, top = 0.f;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int c = 0; c * 32 + lane < E; ++c) {
+      if ((taken >> c) & 1u) continue;
+      const int e = c * 32 + lane;
+      const float v = row[e];
+      if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == j) { my_idx = bi; my_val = bv; }
+    if (j == 0) top = bv;
+  }
+  const float num = (lane < k) ? expf(my_val - top) : 0.f;
+  float den;
+  if (renorm) {
+    den = num;
+  } else {
+    den = 0.f;
+    for (int e = lane; e < E; e += 32) den += expf(row[e] - top);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  if (lane < k) {
+    topk_idx[(size_t)t * k + lane] = my_idx;
+    topk_w[(size_t)t * k + lane] = num / den;
+  }
+}
+
+template <typename XT>
+cudaError_t launch_logits(const moe_config& c, const XT* x, const float* w, const float* bias,
+                          float* logits, cudaStream_t s) {
+  const int bn = c.E >= 64 ? 64 : c.E > 16 ? 32 : c.E > 8 ? 16 : 8;
+  dim3 grid((c.T + kRouteBM - 1) / kRouteBM, (c.E + bn - 1) / bn);
+  switch (bn) {
+    case 64: route_logits_kernel<64, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E); break;
+    case 32: route_logits_kernel<32, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E); break;
+    case 16: route_logits_kernel<16, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E); break;
+    default: route_logits_kernel<8, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E); break;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_route(const moe_config& c, const void* x, const float* w_router,
+                         const float* bias, float* logits, int32_t* topk_idx, float* topk_w,
+                         cudaStream_t s) {
+  cudaError_t err = (c.x_dtype == MOE_DT_F32)
+      ? launch_logits(c, static_cast<const float*>(x), w_router, bias, logits, s)
+      : launch_logits(c, static_cast<const bf16*>(x), w_router, bias, logits, s);
+  if (err != cudaSuccess) return err;
+  const int warps_per_block = 8;
+  const int blocks = (c.T + warps_per_block - 1) / warps_per_block;
+  route_topk_kernel<<<blocks, warps_per_block * 32, 0, s>>>(logits, topk_idx, topk_w, c.T, c.E,
+                                                             c.top_k, c.renormalize);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

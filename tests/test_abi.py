@@ -1,0 +1,117 @@
+"""C-ABI library checks that need no GPU: it loads, exports every symbol
+include/moe.h declares, and rejects bad arguments on the host before touching
+CUDA.  No call here enqueues device work."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def B():
+    from expert_dispatch_fp32_b200 import build
+    build.build()
+    import expert_dispatch_fp32_b200._binding as binding
+    binding.lib()
+    return binding
+
+
+def declared_symbols():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_declares_the_stage_calls():
+    names = declared_symbols()
+    for stage in ("moe_route", "moe_preprocess", "moe_dispatch_permute", "moe_expert_ffn",
+                  "moe_combine_unpermute", "moe_forward"):
+        assert stage in names
+
+
+def test_library_exports_every_declared_symbol(B):
+    L = ctypes.CDLL(B.LIB_PATH)
+    missing = [n for n in declared_symbols() if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_binding_names_match_header(B):
+    import expert_dispatch_fp32_b200 as pkg
+    for n in declared_symbols():
+        assert callable(getattr(pkg, n, None)), n
+
+
+def good_cfg(B, **kw):
+    c = dict(T=64, D=64, E=16, ep_size=4, top_k=2, F=128, act=B.MOE_ACT_GELU, renormalize=1,
+             x_dtype=B.MOE_DT_F32, router_dtype=B.MOE_DT_F32, n_shared=0, F_shared=0)
+    c.update(kw)
+    return B.MoeConfig(**c)
+
+
+def test_version_and_strings(B):
+    assert B.moe_abi_version() == 1
+    assert B.moe_status_string(B.MOE_OK) == "ok"
+    assert "range" in B.moe_status_string(B.MOE_ERR_INDEX_OOB)
+    assert B.moe_status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("kw,expect", [
+    ({}, 0),
+    ({"E": 10, "ep_size": 4}, 1),          # num_experts must be divisible by ep_size
+    ({"top_k": 17}, 1),                     # k > E
+    ({"top_k": 0}, 1),
+    ({"T": -1}, 1),
+    ({"router_dtype": 1}, 2),               # only the fp32 router
+    ({"D": 96}, 2),                         # rows of 64-element K steps
+    ({"act": 1, "F": 192}, 2),              # SwiGLU tiles need F % 128
+    ({"act": 7}, 1),
+    ({"renormalize": 2}, 1),
+    ({"n_shared": 1, "F_shared": 0}, 1),
+    ({"n_shared": 1, "F_shared": 128}, 2),  # shared experts read bf16 x
+    ({"n_shared": 1, "F_shared": 128, "x_dtype": 1}, 0),
+    ({"E": 2048, "ep_size": 8}, 2),
+    ({"top_k": 33, "E": 64}, 2),
+    ({"T": 0}, 0),
+])
+def test_validate_config(B, kw, expect):
+    assert B.moe_validate_config(good_cfg(B, **kw)) == expect
+
+
+def test_sizes_host_only(B):
+    c = good_cfg(B)
+    ws = B.moe_workspace_size(c)
+    pk = B.moe_packed_weights_size(c)
+    assert ws > 0 and ws % 256 == 0
+    # packed = W1 [16,128,64] + W2 [16,64,128], bf16
+    assert pk == 2 * (16 * 128 * 64) * 2
+    assert B.moe_workspace_size(good_cfg(B, E=10)) == 0
+
+
+def test_null_and_misaligned_pointers_rejected_on_host(B):
+    c = good_cfg(B)
+    lib = B.lib()
+    by = ctypes.byref(c)
+    fake = 1 << 20                    # never dereferenced: validation fails first
+    assert lib.moe_route(by, None, fake, None, None, fake, fake, fake, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_route(by, fake + 4, fake, None, None, fake, fake, fake, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_preprocess(by, fake, fake, fake, fake, fake, fake, fake, fake, None, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_dispatch_permute(by, fake, None, fake, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_ffn(by, fake, None, fake, None, fake, fake, None, fake, fake, None) == B.MOE_ERR_INVALID_ARG
+    # out may not alias the residual
+    assert lib.moe_combine_unpermute(by, fake, fake, fake, fake, None, fake, None) == B.MOE_ERR_INVALID_ARG
+    bad = good_cfg(B, E=10)
+    assert lib.moe_forward(ctypes.byref(bad), *([fake] * 20), None) == B.MOE_ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_no_op(B):
+    c = good_cfg(B, T=0)
+    lib = B.lib()
+    assert lib.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, None) == 0
+    assert lib.moe_dispatch_permute(ctypes.byref(c), None, None, None, None) == 0
+    assert lib.moe_combine_unpermute(ctypes.byref(c), None, None, None, None, None, None, None) == 0

@@ -1,0 +1,162 @@
+"""GPU edge cases: ragged batches, skewed and empty experts, k = E, ties, the
+worked example's closed form, device error reporting and determinism."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import expert_dispatch_fp32_b200 as M
+import moe_workloads as W
+import oracle
+from conftest import read_golden
+from parity_helpers import (assert_layer_close, compare_routing, f64, make_layer, oracle_layer,
+                            oracle_route)
+
+pytestmark = pytest.mark.gpu
+
+BASE = W.Workload(name="edge", T=256, D=128, E=8, ep_size=2, top_k=2, F=256, act="swiglu")
+
+
+def run_and_compare(wl, inp=None, full=True):
+    inp = inp or W.make_inputs(wl, device="cuda")
+    layer = make_layer(wl, inp)
+    out = layer.forward(inp["x"])
+    torch.cuda.synchronize()
+    layer.check_status()
+    ref = oracle_route(wl, inp)
+    b = layer.buf
+    compare_routing(b["topk_idx"].cpu().numpy(), b["topk_w"].cpu().numpy(), ref)
+    pre = oracle.preprocess(ref["idx"], wl.E, wl.ep_size)
+    if np.array_equal(b["topk_idx"].cpu().numpy(), ref["idx"]):
+        for key in ("counts", "expert_offsets", "rank_splits", "rank_offsets", "pos", "src"):
+            assert np.array_equal(b[key].cpu().numpy(), pre[key]), key
+    res = oracle_layer(wl, inp)
+    assert_layer_close(f64(out), res["out"], f64(inp["x"]))
+    return layer, inp, res
+
+
+@pytest.mark.parametrize("T", [1, 3, 127, 128, 129, 1000])
+def test_ragged_batches(T):
+    run_and_compare(BASE.with_(T=T, seed=T))
+
+
+@pytest.mark.parametrize("D,F,act", [(64, 128, "swiglu"), (128, 128, "gelu"), (192, 64, "gelu"),
+                                     (320, 384, "swiglu")])
+def test_tile_widths(D, F, act):
+    # D % 256 != 0 and F % 256 != 0 take the 128- and 64-wide tiles; K = 64 is one K step
+    run_and_compare(BASE.with_(T=300, D=D, F=F, act=act, x_dtype="f32" if act == "gelu" else "bf16"))
+
+
+def test_k_equals_e_and_no_renormalisation():
+    run_and_compare(BASE.with_(T=200, E=8, top_k=8, ep_size=4))
+    run_and_compare(BASE.with_(T=200, renormalize=False))
+
+
+def test_shared_experts_small():
+    run_and_compare(BASE.with_(T=333, E=16, ep_size=4, top_k=3, n_shared=2, F_shared=128))
+
+
+def test_all_tokens_to_one_expert_and_empty_experts():
+    wl = BASE.with_(T=700, E=16, ep_size=4, top_k=2, zipf_bias=False)
+    inp = W.make_inputs(wl, device="cuda")
+    bias = torch.full((16,), -50.0, device="cuda")
+    bias[5] = 50.0       # expert 5 is every token's first choice
+    bias[9] = 40.0       # expert 9 every token's second
+    inp["bias"] = bias
+    layer, _, res = run_and_compare(wl, inp)
+    counts = layer.buf["counts"].cpu().numpy()
+    assert counts[5] == 700 and counts[9] == 700 and counts.sum() == 1400
+    assert list(layer.buf["rank_splits"].cpu().numpy()) == [0, 700, 700, 0]
+
+
+def test_zipf_skew_small():
+    run_and_compare(W.get("zipf_skew_e64").with_(T=2000, D=256, F=256, F_shared=128))
+
+
+def test_ties_go_to_the_lower_index():
+    wl = BASE.with_(T=512, E=8, top_k=2)
+    inp = W.make_inputs(wl, device="cuda")
+    wr = inp["w_router"]
+    wr[6] = wr[1]           # experts 1 and 6 always tie exactly on the device
+    layer = make_layer(wl, inp)
+    layer.forward(inp["x"])
+    torch.cuda.synchronize()
+    idx = layer.buf["topk_idx"].cpu().numpy()
+    logits = layer.buf["logits"].cpu().numpy()
+    assert np.array_equal(logits[:, 1], logits[:, 6])
+    for row in idx:
+        r = row.tolist()
+        if 6 in r:
+            assert 1 in r and r.index(1) < r.index(6)
+
+
+def test_worked_example_on_gpu():
+    g = read_golden("worked_example.txt")
+    E, k, ep = g["num_experts"][0], g["top_k"][0], g["num_devices"][0]
+    D, F = 64, 128
+    e_a, e_b = g["chosen_experts"]
+    wa, wb = g["routing_weights"]
+    x = torch.zeros((1, D), dtype=torch.float32)
+    x[0, 0] = 1.0
+    w_r = torch.zeros((E, D), dtype=torch.float32)
+    w_r[:, 0] = -10.0
+    w_r[e_a, 0] = math.log(wa / wb)
+    w_r[e_b, 0] = 0.0
+    w1 = torch.zeros((E, D, F))
+    w2 = torch.zeros((E, F, D))
+    for e in range(E):
+        w1[e, 0, e], w1[e, 0, 64 + e] = 1.0, -1.0
+        w2[e, e, 1] = w2[e, 64 + e, 2] = (e + 1) / 16.0
+    layer = M.MoELayer(D=D, E=E, ep_size=ep, top_k=k, F=F, w_router=w_r.cuda(),
+                       w_gate_up=w1.to(torch.bfloat16).cuda(), w_down=w2.to(torch.bfloat16).cuda(),
+                       act="gelu", x_dtype="f32")
+    out = layer.forward(x.cuda())
+    torch.cuda.synchronize()
+    b = layer.buf
+    assert b["topk_idx"].cpu().tolist() == [g["chosen_experts"]]
+    assert np.allclose(b["topk_w"].cpu().numpy()[0], g["routing_weights"], atol=1e-6)
+    ro = b["rank_offsets"].cpu().numpy()
+    for j, dev in enumerate(g["device_of_chosen"]):
+        assert ro[dev] <= int(b["pos"][j]) < ro[dev + 1]
+    phi1 = 0.5 * (1 + math.erf(1 / math.sqrt(2)))
+    sa, sb = (e_a + 1) / 16, (e_b + 1) / 16
+    expect = np.zeros(D)
+    expect[0] = 1.0
+    expect[1] = wa * sa * phi1 + wb * sb * phi1
+    expect[2] = -(wa * sa * (1 - phi1) + wb * sb * (1 - phi1))
+    assert np.allclose(out.cpu().numpy()[0], expect, rtol=1e-2, atol=2e-3)
+
+
+def test_out_of_range_index_sets_status():
+    wl = BASE.with_(T=64)
+    cfg = M.make_config(wl.T, wl.D, wl.E, wl.ep_size, wl.top_k, wl.F)
+    idx = torch.zeros((wl.T, wl.top_k), dtype=torch.int32, device="cuda")
+    idx[:, 1] = 1
+    idx[10, 1] = 8                       # outside [0, E)
+    i32 = lambda n: torch.zeros(n, dtype=torch.int32, device="cuda")
+    ws = torch.zeros(M.moe_workspace_size(cfg), dtype=torch.uint8, device="cuda")
+    status = i32(1)
+    M.moe_preprocess(cfg, idx, i32(wl.E), i32(wl.E + 1), i32(wl.ep_size), i32(wl.ep_size + 1),
+                     i32(wl.R), i32(wl.R), ws, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == M.MOE_ERR_INDEX_OOB
+
+
+def test_empty_batch_forward():
+    wl = BASE.with_(T=0)
+    inp = W.make_inputs(BASE, device="cuda")
+    layer = make_layer(BASE, inp)
+    layer.forward(inp["x"][:0])
+    torch.cuda.synchronize()
+    assert int(layer.buf["counts"].sum().item()) == 0
+
+
+def test_deterministic():
+    wl = BASE.with_(T=1000, E=16, ep_size=4, top_k=4)
+    inp = W.make_inputs(wl, device="cuda")
+    layer = make_layer(wl, inp)
+    a = layer.forward(inp["x"]).clone()
+    b = layer.forward(inp["x"]).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)

@@ -1,0 +1,183 @@
+"""GPU parity: every stage of the CUDA path against the CPU oracle, on the five
+seeded workloads at full size.
+
+Stage tests feed the oracle's own intermediate results into one C-ABI call and
+compare that call's output, so no oracle input ever comes from the CUDA path.
+The end-to-end test runs moe_forward (the launch configuration bench.py times)
+and compares routing in full and layer outputs on sampled tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import expert_dispatch_fp32_b200 as M
+import moe_workloads as W
+import oracle
+from parity_helpers import (GAP, assert_layer_close, compare_routing, cuda_inputs, f64, make_layer,
+                            oracle_layer, oracle_route, sample_tokens, up_weights)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", params=W.WORKLOAD_ORDER)
+def ctx(request):
+    wl = W.get(request.param)
+    inp = cuda_inputs(wl)
+    layer = make_layer(wl, inp, keep_logits=True)
+    ref = oracle_route(wl, inp)
+    pre = oracle.preprocess(ref["idx"], wl.E, wl.ep_size)
+    yield dict(wl=wl, inp=inp, layer=layer, ref=ref, pre=pre)
+    del inp, layer
+    torch.cuda.empty_cache()
+
+
+def _preprocess_on_gpu(ctx, idx_np):
+    wl, layer = ctx["wl"], ctx["layer"]
+    b = layer.allocate(wl.T)
+    b["status"].zero_()
+    idx = torch.from_numpy(np.ascontiguousarray(idx_np, dtype=np.int32)).cuda()
+    M.moe_preprocess(layer.config(wl.T), idx, b["counts"], b["expert_offsets"], b["rank_splits"],
+                     b["rank_offsets"], b["pos"], b["src"], b["workspace"], b["status"])
+    torch.cuda.synchronize()
+    return b
+
+
+def test_route_stage(ctx):
+    wl, inp, layer, ref = ctx["wl"], ctx["inp"], ctx["layer"], ctx["ref"]
+    b = layer.allocate(wl.T)
+    M.moe_route(layer.config(wl.T), inp["x"], inp["w_router"], inp["bias"], b["logits"],
+                b["topk_idx"], b["topk_w"], b["workspace"])
+    torch.cuda.synchronize()
+    lg = b["logits"].cpu().numpy()
+    # fp32 logits: the dot product rounded once, to within a few fp32 ulps
+    assert np.allclose(lg, ref["logits"], rtol=2e-6, atol=2e-6)
+    n_exempt, n_differ = compare_routing(b["topk_idx"].cpu().numpy(), b["topk_w"].cpu().numpy(), ref)
+    print(f"\n{wl.name}: near-tie tokens (gap < {GAP}): {n_exempt}, routed differently: {n_differ}")
+
+
+def test_preprocess_stage(ctx):
+    wl, pre = ctx["wl"], ctx["pre"]
+    b = _preprocess_on_gpu(ctx, ctx["ref"]["idx"])
+    assert int(b["status"].item()) == 0
+    for key in ("counts", "expert_offsets", "rank_splits", "rank_offsets", "pos", "src"):
+        assert np.array_equal(b[key].cpu().numpy(), pre[key]), key
+    # split sizes sum to T*k; rank r starts where its first expert starts
+    assert pre["rank_splits"].sum() == wl.R
+
+
+def test_dispatch_stage(ctx):
+    wl, inp, layer, pre = ctx["wl"], ctx["inp"], ctx["layer"], ctx["pre"]
+    b = layer.allocate(wl.T)
+    src = torch.from_numpy(pre["src"]).cuda()
+    M.moe_dispatch_permute(layer.config(wl.T), inp["x"], src, b["x_perm"])
+    torch.cuda.synchronize()
+    # sampled rows against the oracle, bit-exact
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([rng.choice(wl.R, size=min(2048, wl.R), replace=False),
+                                     pre["expert_offsets"][:-1][pre["counts"] > 0], [wl.R - 1]]))
+    x_h = f64(inp["x"][torch.from_numpy(pre["src"][rows] // wl.top_k).cuda()])
+    if wl.x_dtype == "f32":
+        x_h = oracle.bf16_round(x_h)
+    got = f64(b["x_perm"][torch.from_numpy(rows).cuda()])
+    assert np.array_equal(got, x_h)
+    # every row: the gather of x by the oracle's src (torch indexing as the reference)
+    full = inp["x"].to(torch.bfloat16)[src.long() // wl.top_k]
+    assert torch.equal(b["x_perm"], full)
+
+
+def _sample_rows(pre, E, rng, max_experts=8):
+    counts, off = pre["counts"], pre["expert_offsets"]
+    nz = np.nonzero(counts)[0]
+    if nz.size > max_experts:
+        pick = {int(nz[np.argmax(counts[nz])]), int(nz[np.argmin(counts[nz])]), int(nz[0]), int(nz[-1])}
+        pick.update(rng.choice(nz, size=max_experts - len(pick), replace=False).tolist())
+        nz = np.array(sorted(pick))
+    out = {}
+    for e in nz:
+        lo, hi = int(off[e]), int(off[e + 1])
+        cand = {lo, hi - 1, min(lo + 127, hi - 1), min(lo + 128, hi - 1)}
+        cand.update(rng.integers(lo, hi, size=min(4, hi - lo)).tolist())
+        out[int(e)] = np.array(sorted(cand))
+    return out
+
+
+def test_expert_ffn_stage(ctx):
+    wl, inp, layer, pre = ctx["wl"], ctx["inp"], ctx["layer"], ctx["pre"]
+    b = _preprocess_on_gpu(ctx, ctx["ref"]["idx"])
+    src = torch.from_numpy(pre["src"]).cuda()
+    # the oracle's permuted input (a gather by the oracle's src, done by torch on the device)
+    x_perm = inp["x"].to(torch.bfloat16)[src.long() // wl.top_k].contiguous()
+    x_bf = inp["x"] if wl.x_dtype == "bf16" else None
+    M.moe_expert_ffn(layer.config(wl.T), x_perm, x_bf, b["expert_offsets"], layer.packed, b["act"],
+                     b["y_perm"], b["shared_out"], b["workspace"], b["status"])
+    torch.cuda.synchronize()
+    assert int(b["status"].item()) == 0
+    rng = np.random.default_rng(1)
+    wup = up_weights(wl, inp)
+    got, ref, res = [], [], []
+    for e, rows in _sample_rows(pre, wl.E, rng).items():
+        xr = f64(x_perm[torch.from_numpy(rows).cuda()])
+        y = oracle.expert_ffn(xr, f64(wup[e]), f64(inp["w_down"][e]), wl.act)
+        got.append(f64(b["y_perm"][torch.from_numpy(rows).cuda()]))
+        ref.append(y)
+        res.append(np.zeros_like(y))
+    assert_layer_close(np.concatenate(got), np.concatenate(ref), np.concatenate(res), "y_perm")
+    if wl.n_shared:
+        toks = sample_tokens(wl.T, 24)
+        xs = f64(inp["x"][torch.from_numpy(toks).cuda()])
+        s_ref = oracle.shared_experts(xs, f64(inp["ws_gate_up"]), f64(inp["ws_down"]))
+        s_got = f64(b["shared_out"][torch.from_numpy(toks).cuda()])
+        assert_layer_close(s_got, s_ref, np.zeros_like(s_ref), "shared_out")
+
+
+def test_combine_stage(ctx):
+    wl, inp, layer, pre, ref = ctx["wl"], ctx["inp"], ctx["layer"], ctx["pre"], ctx["ref"]
+    b = layer.allocate(wl.T)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7)
+    y_perm = torch.randn((wl.R, wl.D), generator=g, device="cuda").to(torch.bfloat16)
+    shared = (torch.randn((wl.T, wl.D), generator=g, device="cuda").to(torch.bfloat16)
+              if wl.n_shared else None)
+    w32 = ref["w"].astype(np.float32)
+    pos = torch.from_numpy(pre["pos"]).cuda()
+    M.moe_combine_unpermute(layer.config(wl.T), y_perm, pos, torch.from_numpy(w32).cuda(), inp["x"],
+                            shared, b["out"])
+    torch.cuda.synchronize()
+    toks = sample_tokens(wl.T, 256, seed=3)
+    tk = torch.from_numpy(toks).cuda()
+    y_tok = f64(y_perm[pos.long().view(wl.T, wl.top_k)[tk]])
+    s = None if shared is None else f64(shared[tk])
+    expect = oracle.combine(y_tok, w32[toks].astype(np.float64), f64(inp["x"][tk]), s)
+    got = f64(b["out"][tk])
+    if wl.x_dtype == "bf16":       # one rounding of the fp32 sum to bf16
+        assert np.all(np.abs(got - expect) <= 2.0 ** -8 * np.abs(expect) + 1e-5)
+    else:
+        assert np.allclose(got, expect, rtol=1e-5, atol=1e-5)
+
+
+def test_forward_end_to_end(ctx):
+    wl, inp, layer, ref, pre = ctx["wl"], ctx["inp"], ctx["layer"], ctx["ref"], ctx["pre"]
+    out = layer.forward(inp["x"])
+    torch.cuda.synchronize()
+    layer.check_status()
+    b = layer.buf
+    n_exempt, n_differ = compare_routing(b["topk_idx"].cpu().numpy(), b["topk_w"].cpu().numpy(), ref)
+    gpu_idx = b["topk_idx"].cpu().numpy()
+    if n_differ == 0:
+        for key in ("counts", "expert_offsets", "rank_splits", "rank_offsets", "pos", "src"):
+            assert np.array_equal(b[key].cpu().numpy(), pre[key]), key
+    else:   # a near-tie token chose differently: check the bookkeeping is valid for its choice
+        counts = b["counts"].cpu().numpy()
+        assert np.array_equal(counts, np.bincount(gpu_idx.ravel(), minlength=wl.E))
+        pos, src = b["pos"].cpu().numpy(), b["src"].cpu().numpy()
+        assert np.array_equal(src[pos], np.arange(wl.R))
+    # outputs: all tokens for the small workload, a sample otherwise
+    toks = (np.arange(wl.T) if wl.T * wl.D <= 1 << 16
+            else sample_tokens(wl.T, 12 if wl.E <= 64 else 4, seed=5))
+    diff_tok = set(np.nonzero(~np.all(gpu_idx == ref["idx"], axis=1))[0].tolist())
+    toks = np.array([t for t in toks if t not in diff_tok])
+    res = oracle_layer(wl, inp, toks)
+    got = f64(out[torch.from_numpy(toks).cuda()])
+    e = assert_layer_close(got, res["out"], f64(inp["x"][torch.from_numpy(toks).cuda()]))
+    print(f"\n{wl.name}: tokens checked {toks.size}, rel-L2 {e[0]:.2e}, max-abs {e[1]:.2e}, "
+          f"MoE-part rel-L2 {e[2]:.2e}; near-tie {n_exempt}, differ {n_differ}")
