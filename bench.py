@@ -49,7 +49,7 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=W.WORKLOAD_ORDER)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-sample", type=int, default=0,
-                    help="tokens per CPU-oracle sample (0 = choose for ~10-30 s)")
+                    help="tokens per CPU-oracle sample (0 = sized for ~12 s of host time)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -63,13 +63,14 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def dist_setup():
+def dist_setup(backend="nccl"):
+    """Join the process group torchrun describes in the environment (N > 1)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if ws > 1:
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
     return ws, rank, local
 
 
@@ -79,13 +80,19 @@ def barrier(ws):
         dist.barrier()
 
 
-def max_over_ranks(v, ws):
+def max_over_ranks(v, ws, device="cuda"):
+    """Max of a per-rank scalar over all ranks (the slowest rank sets the time)."""
     if ws == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_value(tokens_per_rank, ws, steps, total_ms_max):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * ws * steps / (total_ms_max / 1e3)
 
 
 class ClockSampler:
@@ -180,12 +187,13 @@ def cpu_threads():
     return os.cpu_count()
 
 
-def pick_sample(wl, budget_s=12.0):
-    """Tokens per oracle sample so one sample costs about budget_s on the host."""
-    per_tok_flop = 2 * wl.D * wl.F * (3 if wl.act == "swiglu" else 2) * wl.top_k \
-        + 6 * wl.D * wl.F_shared * wl.n_shared + 2 * wl.D * wl.E
-    est_flops = 30e9            # a conservative float64 BLAS rate for an 8-core host
-    return int(max(16, min(wl.T, budget_s * est_flops / per_tok_flop)))
+def pick_sample(wl, host, budget_s):
+    """Tokens per oracle sample so one sample costs about budget_s on the host:
+    time a 64-token probe and scale (tokens are independent, cost is linear)."""
+    probe = min(64, wl.T)
+    cpu_oracle_time(wl, host, probe, seed=99)            # warm the BLAS threads
+    t = cpu_oracle_time(wl, host, probe, seed=98)
+    return int(max(probe, min(wl.T, budget_s * probe / max(t, 1e-6))))
 
 
 # ---------------------------------------------------------------------------
@@ -200,7 +208,7 @@ def run_reference(args):
     inp = W.make_inputs(wl, device="cpu")
     host = host_inputs_f64(wl, inp)
     del inp
-    n_tok = args.cpu_sample or pick_sample(wl, budget_s=min(10.0, max(0.5, 120.0 / max(1, args.steps))))
+    n_tok = args.cpu_sample or pick_sample(wl, host, min(10.0, max(0.5, 120.0 / max(1, args.steps))))
     for i in range(args.warmup):
         cpu_oracle_time(wl, host, min(n_tok, 16), seed=i)
     times = [cpu_oracle_time(wl, host, n_tok, seed=100 + i) for i in range(args.steps)]
@@ -304,7 +312,7 @@ def run_ours(args):
         stage_ms += [ev[j].elapsed_time(ev[j + 1]) for j in range(5)]
     total_ms = float(stage_ms.sum())
     total_ms_max = max_over_ranks(total_ms, ws)
-    value = T * ws * args.steps / (total_ms_max / 1e3)
+    value = replica_value(T, ws, args.steps, total_ms_max)
 
     # end to end: pinned host x -> device, forward, device -> pinned host out
     x_host = x.cpu().pin_memory()
@@ -329,7 +337,7 @@ def run_ours(args):
     barrier(ws)
     layer.check_status()
     e2e_ms = max_over_ranks(sum(a.elapsed_time(z) for a, z in e_ev), ws)
-    e2e_value = T * ws * args.steps / (e2e_ms / 1e3)
+    e2e_value = replica_value(T, ws, args.steps, e2e_ms)
     sx = 4 if wl.x_dtype == "f32" else 2
 
     # roofline of the dominant kernel: the grouped expert FFN (tcgen05 GEMMs)
@@ -379,8 +387,7 @@ def run_ours(args):
         "combine_gbs": comb_gbs, "combine_frac_hbm": comb_gbs / hbm,
     }
     if want_cpu:
-        n_tok = args.cpu_sample or pick_sample(wl)
-        cpu_oracle_time(wl, cpu_host, min(16, n_tok))          # warm BLAS
+        n_tok = args.cpu_sample or pick_sample(wl, cpu_host, 12.0)
         t = cpu_oracle_time(wl, cpu_host, n_tok, seed=1)
         line["cpu_baseline"] = {"value": n_tok / t, "unit": "tokens/s", "cores": cpu_threads(),
                                 "kind": "oracle",

@@ -124,8 +124,8 @@ moe_status moe_route(const moe_config* cfg, const void* x, const float* w_router
   float* logits = logits_out;
   if (logits == nullptr) logits = (float*)((uint8_t*)workspace + ws_layout(c).logits);
   else if (!aligned16(logits)) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_route(c, x, w_router, expert_bias, logits, topk_idx, topk_w,
-                                  as_stream(stream)));
+  return cuda_status(launch_route(c, x, w_router, expert_bias, logits, logits_out != nullptr,
+                                  topk_idx, topk_w, as_stream(stream)));
 }
 
 moe_status moe_preprocess(const moe_config* cfg, const int32_t* topk_idx, int32_t* counts,

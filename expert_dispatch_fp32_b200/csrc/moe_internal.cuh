@@ -53,9 +53,11 @@ int down_tile_n(const moe_config& c);
 // ---------------------------------------------------------------------------
 // Launchers (each returns cudaGetLastError() of its launches)
 // ---------------------------------------------------------------------------
+// logits: where the tiled path stores fp32 logits (caller's buffer or workspace);
+// keep_logits: the caller asked for them (the fused few-expert path then writes them).
 cudaError_t launch_route(const moe_config& c, const void* x, const float* w_router,
-                         const float* bias, float* logits, int32_t* topk_idx, float* topk_w,
-                         cudaStream_t s);
+                         const float* bias, float* logits, bool keep_logits, int32_t* topk_idx,
+                         float* topk_w, cudaStream_t s);
 cudaError_t launch_preprocess(const moe_config& c, const int32_t* topk_idx, int32_t* counts,
                               int32_t* expert_offsets, int32_t* rank_splits,
                               int32_t* rank_offsets, int32_t* pos, int32_t* src,

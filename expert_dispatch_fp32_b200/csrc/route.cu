@@ -13,6 +13,13 @@
 //
 // Top-k kernel: one warp per token; selection j is an exact warp argmax on
 // (logit, -index), so ties go to the lower expert index; lane j keeps pick j.
+//
+// Few experts (E <= 32 and W_r small enough for shared memory): one fused kernel.
+// W_r is staged in shared memory once per block; each warp streams TW tokens of x
+// with coalesced 16-byte loads (lane l holds columns 8l..8l+7 of every 256), sums
+// each 8-column slice in fp32 and folds it into an fp64 per-lane accumulator, then
+// an fp64 butterfly leaves every lane with all E dot products; lane e keeps logit
+// e and the warp runs the same exact argmax top-k without a logits round trip.
 #include <math.h>
 
 #include "moe_internal.cuh"
@@ -37,12 +44,12 @@ __device__ __forceinline__ void load4(const bf16* p, float (&v)[4]) {
   v[0] = fa.x; v[1] = fa.y; v[2] = fb.x; v[3] = fb.y;
 }
 
-template <int BN, typename XT>
+template <int BN, int BM, typename XT>
 __global__ void __launch_bounds__(kRouteThreads)
 route_logits_kernel(const XT* __restrict__ x, const float* __restrict__ w,
                     const float* __restrict__ bias, float* __restrict__ logits, int T, int D,
                     int E) {
-  constexpr int BM = kRouteBM, BK = kRouteBK;
+  constexpr int BK = kRouteBK;
   constexpr int NTN = BN / 4;                 // thread columns, 4 experts each
   constexpr int NTM = kRouteThreads / NTN;    // thread rows
   constexpr int TM = BM / NTM;                // tokens per thread
@@ -163,34 +170,186 @@ route_topk_kernel(const float* __restrict__ logits, int32_t* __restrict__ topk_i
   }
 }
 
+// Warp argmax top-k over one logit per lane (lanes >= E hold none).
+__device__ __forceinline__ void warp_topk_write(float l, int E, int k, int renorm, size_t t,
+                                                int32_t* __restrict__ topk_idx,
+                                                float* __restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  bool avail = lane < E;
+  int my_idx = 0;
+  float my_val = 0.f, top = 0.f;
+  for (int j = 0; j < k; ++j) {
+    float bv = avail ? l : -INFINITY;
+    int bi = avail ? lane : 0x7fffffff;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    if (lane == bi) avail = false;
+    if (lane == j) { my_idx = bi; my_val = bv; }
+    if (j == 0) top = bv;
+  }
+  const float num = (lane < k) ? expf(my_val - top) : 0.f;
+  float den = renorm ? num : (lane < E ? expf(l - top) : 0.f);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  if (lane < k) {
+    topk_idx[t * k + lane] = my_idx;
+    topk_w[t * k + lane] = num / den;
+  }
+}
+
+constexpr int kSmallThreads = 512;
+
+template <int EP, int TW, typename XT>
+__global__ void __launch_bounds__(kSmallThreads, 1)
+route_small_kernel(const XT* __restrict__ x, const float* __restrict__ w,
+                   const float* __restrict__ bias, float* __restrict__ logits_out,
+                   int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, int T, int D, int E,
+                   int k, int renorm) {
+  extern __shared__ float4 w_s4[];
+  const float* w_s = reinterpret_cast<const float*>(w_s4);
+  const int n4 = E * D / 4;
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) w_s4[i] = __ldg(reinterpret_cast<const float4*>(w) + i);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  const int gwarp = blockIdx.x * wpb + (threadIdx.x >> 5);
+  const int nwarps = gridDim.x * wpb;
+  for (int t0 = gwarp * TW; t0 < T; t0 += nwarps * TW) {
+    double acc[TW][EP];
+#pragma unroll
+    for (int i = 0; i < TW; ++i)
+#pragma unroll
+      for (int e = 0; e < EP; ++e) acc[i][e] = 0.0;
+    for (int d0 = lane * 8; d0 < D; d0 += 256) {
+      float xv[TW][8];
+#pragma unroll
+      for (int i = 0; i < TW; ++i) {
+        if (t0 + i < T) {
+          float a[4], b[4];
+          load4(x + (size_t)(t0 + i) * D + d0, a);
+          load4(x + (size_t)(t0 + i) * D + d0 + 4, b);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) { xv[i][q] = a[q]; xv[i][4 + q] = b[q]; }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) xv[i][q] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < EP; ++e) {
+        if (e < E) {
+          const float4 w0 = *reinterpret_cast<const float4*>(w_s + (size_t)e * D + d0);
+          const float4 w1 = *reinterpret_cast<const float4*>(w_s + (size_t)e * D + d0 + 4);
+#pragma unroll
+          for (int i = 0; i < TW; ++i) {
+            float p = xv[i][0] * w0.x;
+            p = fmaf(xv[i][1], w0.y, p);
+            p = fmaf(xv[i][2], w0.z, p);
+            p = fmaf(xv[i][3], w0.w, p);
+            p = fmaf(xv[i][4], w1.x, p);
+            p = fmaf(xv[i][5], w1.y, p);
+            p = fmaf(xv[i][6], w1.z, p);
+            p = fmaf(xv[i][7], w1.w, p);
+            acc[i][e] += (double)p;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < TW; ++i)
+#pragma unroll
+      for (int e = 0; e < EP; ++e)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[i][e] += __shfl_xor_sync(0xffffffffu, acc[i][e], o);
+#pragma unroll
+    for (int i = 0; i < TW; ++i) {
+      const int t = t0 + i;
+      if (t >= T) break;
+      float l = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < EP; ++e)
+        if (lane == e) l = (float)acc[i][e];
+      if (lane < E && bias != nullptr) l = l + bias[lane];
+      if (logits_out != nullptr && lane < E) logits_out[(size_t)t * E + lane] = l;
+      warp_topk_write(l, E, k, renorm, (size_t)t, topk_idx, topk_w);
+    }
+  }
+}
+
+template <int EP, int TW, typename XT>
+cudaError_t launch_small(const moe_config& c, const XT* x, const float* w, const float* bias,
+                         float* logits_out, int32_t* topk_idx, float* topk_w, cudaStream_t s) {
+  const size_t smem = (size_t)c.E * c.D * sizeof(float);
+  auto kern = route_small_kernel<EP, TW, XT>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  const int per_sm = (int)((227u << 10) / (smem + 1024));
+  const int warps = kSmallThreads / 32;
+  const int need = (c.T + warps * TW - 1) / (warps * TW);
+  const int cap = sm_count() * (per_sm > 0 ? per_sm : 1);
+  kern<<<need < cap ? need : cap, kSmallThreads, smem, s>>>(x, w, bias, logits_out, topk_idx, topk_w,
+                                                            c.T, c.D, c.E, c.top_k, c.renormalize);
+  return cudaGetLastError();
+}
+
+constexpr size_t kSmallRouterSmem = 200u << 10;
+
 template <typename XT>
 cudaError_t launch_logits(const moe_config& c, const XT* x, const float* w, const float* bias,
                           float* logits, cudaStream_t s) {
   const int bn = c.E >= 64 ? 64 : c.E > 16 ? 32 : c.E > 8 ? 16 : 8;
-  dim3 grid((c.T + kRouteBM - 1) / kRouteBM, (c.E + bn - 1) / bn);
+  const int m_blocks128 = (c.T + 127) / 128, n_blocks = (c.E + bn - 1) / bn;
+  // 64-token tiles when 128-token tiles leave SMs idle (needs >= 2 tokens per thread row)
+  const bool small_m = bn >= 32 && (int64_t)m_blocks128 * n_blocks < 2 * sm_count();
+  const int bm = small_m ? 64 : 128;
+  dim3 grid((c.T + bm - 1) / bm, n_blocks);
+#define MOE_ROUTE_TILE(BN_)                                                                        \
+  if (small_m) route_logits_kernel<BN_, 64, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E); \
+  else route_logits_kernel<BN_, 128, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E);
   switch (bn) {
-    case 64: route_logits_kernel<64, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E); break;
-    case 32: route_logits_kernel<32, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E); break;
-    case 16: route_logits_kernel<16, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E); break;
-    default: route_logits_kernel<8, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E); break;
+    case 64: MOE_ROUTE_TILE(64) break;
+    case 32: MOE_ROUTE_TILE(32) break;
+    case 16: route_logits_kernel<16, 128, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E); break;
+    default: route_logits_kernel<8, 128, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E); break;
   }
+#undef MOE_ROUTE_TILE
   return cudaGetLastError();
 }
 
-}  // namespace
-
-cudaError_t launch_route(const moe_config& c, const void* x, const float* w_router,
-                         const float* bias, float* logits, int32_t* topk_idx, float* topk_w,
-                         cudaStream_t s) {
-  cudaError_t err = (c.x_dtype == MOE_DT_F32)
-      ? launch_logits(c, static_cast<const float*>(x), w_router, bias, logits, s)
-      : launch_logits(c, static_cast<const bf16*>(x), w_router, bias, logits, s);
+template <typename XT>
+cudaError_t launch_route_t(const moe_config& c, const XT* x, const float* w_router,
+                           const float* bias, float* logits, bool keep_logits, int32_t* topk_idx,
+                           float* topk_w, cudaStream_t s) {
+  const size_t wbytes = (size_t)c.E * c.D * sizeof(float);
+  if (c.E <= 32 && wbytes <= kSmallRouterSmem) {
+    float* lo = keep_logits ? logits : nullptr;
+    if (c.E <= 8) return launch_small<8, 2, XT>(c, x, w_router, bias, lo, topk_idx, topk_w, s);
+    if (c.E <= 16) return launch_small<16, 1, XT>(c, x, w_router, bias, lo, topk_idx, topk_w, s);
+    return launch_small<32, 1, XT>(c, x, w_router, bias, lo, topk_idx, topk_w, s);
+  }
+  cudaError_t err = launch_logits(c, x, w_router, bias, logits, s);
   if (err != cudaSuccess) return err;
   const int warps_per_block = 8;
   const int blocks = (c.T + warps_per_block - 1) / warps_per_block;
   route_topk_kernel<<<blocks, warps_per_block * 32, 0, s>>>(logits, topk_idx, topk_w, c.T, c.E,
                                                              c.top_k, c.renormalize);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_route(const moe_config& c, const void* x, const float* w_router,
+                         const float* bias, float* logits, bool keep_logits, int32_t* topk_idx,
+                         float* topk_w, cudaStream_t s) {
+  if (c.x_dtype == MOE_DT_F32)
+    return launch_route_t(c, static_cast<const float*>(x), w_router, bias, logits, keep_logits,
+                          topk_idx, topk_w, s);
+  return launch_route_t(c, static_cast<const bf16*>(x), w_router, bias, logits, keep_logits,
+                        topk_idx, topk_w, s);
 }
 
 }  // namespace moe
