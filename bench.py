@@ -275,7 +275,7 @@ def run_ours(args):
         M.moe_preprocess(cfg, b["topk_idx"], b["counts"], b["expert_offsets"], b["rank_splits"],
                          b["rank_offsets"], b["pos"], b["src"], b["workspace"], b["status"], stream)
         ev[2].record(stream)
-        M.moe_dispatch_permute(cfg, x, b["src"], b["x_perm"], stream)
+        M.moe_dispatch_permute(cfg, x, b["pos"], b["x_perm"], stream)
         ev[3].record(stream)
         M.moe_expert_ffn(cfg, b["x_perm"], x_bf, b["expert_offsets"], layer.packed, b["act"],
                          b["y_perm"], b["shared_out"], b["workspace"], b["status"], stream)

@@ -130,8 +130,8 @@ def moe_preprocess(cfg, topk_idx, counts, expert_offsets, rank_splits, rank_offs
           _p(rank_splits), _p(rank_offsets), _p(pos), _p(src), _p(workspace), _p(status), _s(stream))
 
 
-def moe_dispatch_permute(cfg, x, src, x_perm, stream=None):
-    _call("moe_dispatch_permute", ctypes.byref(cfg), _p(x), _p(src), _p(x_perm), _s(stream))
+def moe_dispatch_permute(cfg, x, pos, x_perm, stream=None):
+    _call("moe_dispatch_permute", ctypes.byref(cfg), _p(x), _p(pos), _p(x_perm), _s(stream))
 
 
 def moe_expert_ffn(cfg, x_perm, x, expert_offsets, packed, act, y_perm, shared_out, workspace,

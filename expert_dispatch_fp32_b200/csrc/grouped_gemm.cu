@@ -10,7 +10,10 @@
 //      [group_offsets[g], group_offsets[g+1]);
 //   B  bf16 [G, N, K] (K-major), one [N, K] matrix per group.
 //
-// Tiles are 128 x BN (BN = 256/128/64) output blocks; the tile list is
+// Two kernels share this file.  grouped_gemm_pair_kernel (the default for 256-wide
+// N tiles) runs 256 x 256 output tiles on a cluster of two CTAs with
+// tcgen05.mma.cta_group::2; grouped_gemm_kernel runs 128 x BN tiles (BN = 256/128/64)
+// on one CTA and serves the narrower N tiles.  In both, the tile list is
 // expert-major, then N block, then M tile fastest, so the CTAs that run at the
 // same time share each weight tile through L2 and stream every weight from HBM
 // about once.  The per-expert M-tile prefix (mt_start) comes from the preprocess
@@ -18,7 +21,7 @@
 // CTA walks tiles blockIdx.x, blockIdx.x + gridDim.x, ...  Empty experts own no
 // tiles, so their weights are never read.
 //
-// One CTA per SM, 6 warps:
+// One-CTA kernel: one CTA per SM, 6 warps:
 //   warp 0      TMA producer: A tile [128 x 64] and B tile [BN x 64] per K step
 //               into a STAGES-deep shared-memory ring (128-byte swizzle).
 //   warp 1      allocates 2*BN TMEM columns; one lane issues tcgen05.mma
@@ -160,6 +163,62 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---- CTA-pair (cluster of 2) forms ----
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Shared address of the same object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_cta(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+// Loads into this CTA's shared memory whose bytes complete on `leader_bar`, the
+// shared::cluster address (from mapa) of the barrier in the pair's leader CTA.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t leader_bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t leader_bar, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the barrier at this shared offset in both CTAs of the pair when
+// all tcgen05 operations issued so far by this thread have completed.
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
 }
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
@@ -383,10 +442,222 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     }
   }
 
+  __syncwarp();                 // reconverge lane 0 of warps 0/1 with its warp
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(C::kTmemCols)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// CTA-pair kernel: 256 x 256 output tiles on a cluster of 2 CTAs
+// ---------------------------------------------------------------------------
+// tcgen05.mma.cta_group::2 with M = 256, N = 256: CTA r of the pair holds A rows
+// [row0 + 128 r, +128) and B rows [n0 + 128 r, +128) of every K step in its own
+// shared memory, and its TMEM holds accumulator rows 128 r .. 128 r + 127 (all 256
+// columns).  Per CTA and K step that is 16 KB of A + 16 KB of B for 128 x 256 x 64
+// MACs, two thirds of the operand traffic of the one-CTA 128 x 256 tile.
+//   warp 0 (both CTAs)   TMA producer: waits its own `empty` slot, loads its halves;
+//                        the bytes complete on the leader's `full` barrier, whose
+//                        expected byte count the leader posts for both CTAs.
+//   warp 1 (leader)      issues the pair MMAs and commits to `empty` / `tmem_full`
+//                        in both CTAs; warp 1 of both CTAs allocates the TMEM.
+//   warps 2-5 (both)     epilogue of the CTA's 128 rows, then one arrive per warp
+//                        on the leader's `tmem_empty` (8 arrivals per phase).
+// Every wait is bounded as in the one-CTA kernel.
+struct PairCfg {
+  static constexpr int BN = 256;
+  static constexpr int kStages = 6;
+  static constexpr int kABytes = kTileM * kTileK * 2;            // this CTA's A half
+  static constexpr int kBBytes = (BN / 2) * kTileK * 2;          // this CTA's B half
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr uint32_t kIdesc = make_idesc(2 * kTileM, BN);
+  static size_t smem_bytes(int G) {
+    return 1024 + (size_t)kStages * kStageBytes + 256 + 2 * (size_t)(G + 1) * sizeof(int);
+  }
+};
+
+template <int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(const __grid_constant__ GemmArgs p) {
+  using C = PairCfg;
+  constexpr int S = C::kStages, BN = C::BN, TM2 = 2 * kTileM;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* a_smem = smem;
+  uint8_t* b_smem = smem + S * C::kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* mt = reinterpret_cast<int*>(smem + S * C::kStageBytes + 256);
+  const bool dense = p.group_offsets == nullptr;
+  const int G = dense ? 1 : p.G;
+  int* off = mt + (G + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
+  const uint32_t tfull0 = smem_u32(bars + 2 * S), tempty0 = smem_u32(bars + 2 * S + 2);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(full0 + 8 * i, 1);
+      mbar_init(empty0 + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(tfull0 + 8 * i, 1);
+      mbar_init(tempty0 + 8 * i, 8);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_tmap(&p.tmap_a);
+    prefetch_tmap(&p.tmap_b);
+  }
+  if (dense) {
+    if (threadIdx.x == 0) {
+      mt[0] = 0; mt[1] = (p.dense_rows + TM2 - 1) / TM2;
+      off[0] = 0; off[1] = p.dense_rows;
+    }
+  } else {
+    for (int i = threadIdx.x; i <= G; i += blockDim.x) {
+      mt[i] = p.mt_start[i];
+      off[i] = p.group_offsets[i];
+    }
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(C::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync();               // barriers of both CTAs initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int nb = p.N / BN;
+  const int total = mt[G] * nb;
+  const int ksteps = p.K / kTileK;
+  const int cluster_id = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      const uint32_t full0_leader = map_to_cta(full0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = cluster_id; tile < total; tile += nclusters) {
+        int g, m, n;
+        decode_tile(tile, mt, G, nb, g, m, n);
+        const int arow = off[g] + m * TM2 + (int)rank * kTileM;
+        const int brow = n * BN + (int)rank * (BN / 2);
+        bool ok = true;
+        for (int kb = 0; kb < ksteps; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * C::kStageBytes);
+          const uint32_t fb = full0_leader + 8 * stage;
+          tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * kTileK, arow);
+          tma_load_3d_pair(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * kTileK, brow, g);
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (leader CTA) ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int tile = cluster_id; tile < total; tile += nclusters) {
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        bool ok = true;
+        for (int kb = 0; kb < ksteps; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = sw128_desc(smem_u32(a_smem + stage * C::kABytes));
+          const uint64_t bd = sw128_desc(smem_u32(b_smem + stage * C::kBBytes));
+#pragma unroll
+          for (int kk = 0; kk < kTileK / 16; ++kk)
+            tc_mma_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, C::kIdesc, (kb | kk) != 0);
+          tc_commit_pair_both(empty0 + 8 * stage);
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair_both(tfull0 + 8 * acc);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
+    const int q = warp & 3;
+    const uint32_t tempty_leader = map_to_cta(tempty0, 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cluster_id; tile < total; tile += nclusters) {
+      int g, m, n;
+      decode_tile(tile, mt, G, nb, g, m, n);
+      const int row0 = off[g] + m * TM2 + (int)rank * kTileM;
+      const int rows_valid = min(kTileM, off[g + 1] - row0);
+      const bool ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int r = q * 32 + lane;
+      const bool valid = r < rows_valid;
+      bf16* orow = p.out + (size_t)(row0 + (valid ? r : 0)) * p.ldo;
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      if (EPI == EPI_SWIGLU) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t gr[32], ur[32];
+          tmem_ld32(tb + c, gr);
+          tmem_ld32(tb + BN / 2 + c, ur);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
+          if (valid) store_row32(orow + n * (BN / 2) + c, v);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t hr[32];
+          tmem_ld32(tb + c, hr);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float h = __uint_as_float(hr[i]);
+            v[i] = (EPI == EPI_GELU) ? gelu_f(h) : h;
+          }
+          if (valid) store_row32(orow + n * BN + c, v);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader + 8 * acc);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  // Neither CTA leaves (or frees TMEM) while the pair's MMAs may still touch it.
+  __syncwarp();                 // reconverge lane 0 of warps 0/1 with its warp
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(C::kTmemCols)
                  : "memory");
   }
@@ -436,6 +707,30 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t K, uint64_t N, uint6
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int EPI>
+cudaError_t launch_tc_pair(const GemmArgs& a, int clusters, cudaStream_t s) {
+  const size_t smem = PairCfg::smem_bytes(a.group_offsets ? a.G : 1);
+  auto kern = grouped_gemm_pair_kernel<EPI>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, kern, a);
+  if (err != cudaSuccess) return err;
+  return cudaGetLastError();
+}
+
 template <int BN, int EPI>
 cudaError_t launch_tc(const GemmArgs& a, int grid, cudaStream_t s) {
   using C = GemmCfg<BN>;
@@ -465,7 +760,9 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
   memset(&a, 0, sizeof(a));
   const int BN = p.tile_n;
   if (!make_map_2d(&a.tmap_a, p.A, (uint64_t)p.K, (uint64_t)p.a_rows, kTileM)) return cudaErrorInvalidValue;
-  if (!make_map_3d(&a.tmap_b, p.B, (uint64_t)p.K, (uint64_t)p.N, (uint64_t)p.G, (uint32_t)BN))
+  // each CTA of a pair loads its 128-row half of the 256-row B tile
+  const uint32_t b_box = p.pair ? (uint32_t)(BN / 2) : (uint32_t)BN;
+  if (!make_map_3d(&a.tmap_b, p.B, (uint64_t)p.K, (uint64_t)p.N, (uint64_t)p.G, b_box))
     return cudaErrorInvalidValue;
   a.group_offsets = p.group_offsets;
   a.mt_start = p.mt_start;
@@ -477,6 +774,14 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
   a.ldo = p.ldo;
   a.status = p.status;
   const int64_t tiles = p.max_tiles > 0 ? p.max_tiles : 1;
+  if (p.pair) {                 // 256 x 256 tiles on CTA pairs
+    if (BN != 256) return cudaErrorInvalidValue;
+    const int64_t pairs = sm_count() / 2;
+    const int clusters = (int)(tiles < pairs ? tiles : pairs);
+    if (p.epi == EPI_SWIGLU) return launch_tc_pair<EPI_SWIGLU>(a, clusters, s);
+    if (p.epi == EPI_GELU) return launch_tc_pair<EPI_GELU>(a, clusters, s);
+    return launch_tc_pair<EPI_STORE>(a, clusters, s);
+  }
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   if (BN == 256) {
     if (p.epi == EPI_SWIGLU) return launch_tc<256, EPI_SWIGLU>(a, grid, s);

@@ -1,6 +1,7 @@
 // C ABI of libmoe.so: argument validation, buffer layouts and the stage calls.
 // Each call checks its arguments on the host, then only enqueues kernels on the
 // caller's stream.  Nothing here allocates device memory.
+#include <stdlib.h>
 #include <string.h>
 
 #include "moe_internal.cuh"
@@ -15,7 +16,7 @@ WsLayout ws_layout(const moe_config& c) {
   size_t o = 0;
   L.logits = o;       o = align256(o + T * E * sizeof(float));
   L.block_counts = o; o = align256(o + (size_t)L.nblk * E * sizeof(int32_t));
-  L.mt_start = o;     o = align256(o + (E + 1) * sizeof(int32_t));
+  L.mt_start = o;     o = align256(o + 2 * (E + 1) * sizeof(int32_t));
   L.act_shared = o;   o = align256(o + T * (size_t)c.n_shared * c.F_shared * sizeof(bf16));
   L.total = o;
   return L;
@@ -154,16 +155,16 @@ moe_status moe_preprocess(const moe_config* cfg, const int32_t* topk_idx, int32_
                                        as_stream(stream)));
 }
 
-moe_status moe_dispatch_permute(const moe_config* cfg, const void* x, const int32_t* src,
+moe_status moe_dispatch_permute(const moe_config* cfg, const void* x, const int32_t* pos,
                                 void* x_perm, void* stream) {
   moe_status st = moe_validate_config(cfg);
   if (st != MOE_OK) return st;
   const moe_config& c = *cfg;
   if (c.T == 0) return MOE_OK;
   MOE_CHECK_PTR(x);
-  MOE_CHECK_PTR(src);
+  MOE_CHECK_PTR(pos);
   MOE_CHECK_PTR(x_perm);
-  return cuda_status(launch_dispatch(c, x, src, (bf16*)x_perm, as_stream(stream)));
+  return cuda_status(launch_dispatch(c, x, pos, (bf16*)x_perm, as_stream(stream)));
 }
 
 moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void* x,
@@ -187,9 +188,15 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   }
   cudaStream_t s = as_stream(stream);
   const WsLayout W = ws_layout(c);
+  // 256-wide tiles run on CTA pairs (256 x 256 per pair) unless MOE_GEMM_CTA_PAIR=0
+  // selects the one-CTA 128 x 256 kernel (kept for comparison and for narrow N).
+  const char* pair_env = getenv("MOE_GEMM_CTA_PAIR");
+  const bool use_pair = !(pair_env && pair_env[0] == '0');
   const PackLayout P = pack_layout(c);
   const uint8_t* pk = (const uint8_t*)packed;
   uint8_t* ws = (uint8_t*)workspace;
+  const int32_t* mt128 = (const int32_t*)(ws + W.mt_start);
+  const int32_t* mt256 = mt128 + (c.E + 1);
   const int64_t R = (int64_t)c.T * c.top_k;
   const int nup = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
 
@@ -200,9 +207,10 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   up.B = (const bf16*)(pk + P.w_up); up.G = c.E;
   up.N = nup; up.K = c.D;
   up.group_offsets = expert_offsets;
-  up.mt_start = (const int32_t*)(ws + W.mt_start);
   up.tile_n = up_tile_n(c);
-  up.max_tiles = (R / kTileM + c.E) * (int64_t)(nup / up.tile_n);
+  up.pair = use_pair && up.tile_n == 256;
+  up.mt_start = up.pair ? mt256 : mt128;
+  up.max_tiles = (R / (up.pair ? 2 * kTileM : kTileM) + c.E) * (int64_t)(nup / up.tile_n);
   up.out = (bf16*)act; up.ldo = c.F;
   up.epi = c.act == MOE_ACT_SWIGLU ? EPI_SWIGLU : EPI_GELU;
   up.status = status;
@@ -214,7 +222,9 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   dn.B = (const bf16*)(pk + P.w_down);
   dn.N = c.D; dn.K = c.F;
   dn.tile_n = down_tile_n(c);
-  dn.max_tiles = (R / kTileM + c.E) * (int64_t)(c.D / dn.tile_n);
+  dn.pair = use_pair && dn.tile_n == 256;
+  dn.mt_start = dn.pair ? mt256 : mt128;
+  dn.max_tiles = (R / (dn.pair ? 2 * kTileM : kTileM) + c.E) * (int64_t)(c.D / dn.tile_n);
   dn.out = (bf16*)y_perm; dn.ldo = c.D;
   dn.epi = EPI_STORE;
   err = launch_grouped_gemm(dn, s);
@@ -230,7 +240,9 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   su.N = 2 * Fc; su.K = c.D;
   su.group_offsets = nullptr; su.mt_start = nullptr; su.dense_rows = c.T;
   su.tile_n = 256;
-  su.max_tiles = ((int64_t)(c.T + kTileM - 1) / kTileM) * (2 * Fc / 256);
+  su.pair = use_pair;
+  const int tm_s = su.pair ? 2 * kTileM : kTileM;
+  su.max_tiles = ((int64_t)(c.T + tm_s - 1) / tm_s) * (2 * Fc / 256);
   su.out = act_s; su.ldo = Fc;
   su.epi = EPI_SWIGLU;
   su.status = status;
@@ -242,7 +254,9 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   sd.B = (const bf16*)(pk + P.ws_down);
   sd.N = c.D; sd.K = Fc;
   sd.tile_n = down_tile_n(c);
-  sd.max_tiles = ((int64_t)(c.T + kTileM - 1) / kTileM) * (c.D / sd.tile_n);
+  sd.pair = use_pair && sd.tile_n == 256;
+  const int tm_sd = sd.pair ? 2 * kTileM : kTileM;
+  sd.max_tiles = ((int64_t)(c.T + tm_sd - 1) / tm_sd) * (c.D / sd.tile_n);
   sd.out = (bf16*)shared_out; sd.ldo = c.D;
   sd.epi = EPI_STORE;
   return cuda_status(launch_grouped_gemm(sd, s));
@@ -280,7 +294,7 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_rout
   st = moe_preprocess(cfg, topk_idx, counts, expert_offsets, rank_splits, rank_offsets, pos, src,
                       workspace, status, stream);
   if (st != MOE_OK) return st;
-  st = moe_dispatch_permute(cfg, x, src, x_perm, stream);
+  st = moe_dispatch_permute(cfg, x, pos, x_perm, stream);
   if (st != MOE_OK) return st;
   st = moe_expert_ffn(cfg, x_perm, x, expert_offsets, packed, act, y_perm, shared_out, workspace,
                       status, stream);

@@ -28,7 +28,7 @@ constexpr int kTileK = 64;          // GEMM K step: 64 bf16 = one 128-byte swizz
 struct WsLayout {
   size_t logits;        // fp32 [T, E]
   size_t block_counts;  // int32 [nblk, E]
-  size_t mt_start;      // int32 [E + 1]: prefix of ceil(count/128) per expert
+  size_t mt_start;      // int32 [2][E + 1]: prefixes of ceil(count/128), ceil(count/256)
   size_t act_shared;    // bf16 [T, S*Fs]
   size_t total;
   int nblk;
@@ -63,7 +63,7 @@ cudaError_t launch_preprocess(const moe_config& c, const int32_t* topk_idx, int3
                               int32_t* rank_offsets, int32_t* pos, int32_t* src,
                               int32_t* block_counts, int nblk, int32_t* mt_start,
                               int32_t* status, cudaStream_t s);
-cudaError_t launch_dispatch(const moe_config& c, const void* x, const int32_t* src,
+cudaError_t launch_dispatch(const moe_config& c, const void* x, const int32_t* pos,
                             bf16* x_perm, cudaStream_t s);
 cudaError_t launch_combine(const moe_config& c, const bf16* y_perm, const int32_t* pos,
                            const float* topk_w, const void* x, const bf16* shared_out, void* out,
@@ -84,6 +84,7 @@ struct GemmProblem {
   int64_t max_tiles;                      // host upper bound on tiles (grid size)
   bf16* out; int ldo;                     // output row stride in elements
   int epi; int tile_n;
+  int pair;                               // 1: 256-row tiles on CTA pairs (mt_start per 256 rows)
   int32_t* status;
 };
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s);

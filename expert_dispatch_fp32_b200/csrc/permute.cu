@@ -6,9 +6,9 @@
 // copy of the token), Step 4 (weighted sum of the expert outputs) and Step 5
 // (residual add).  On one GPU the exchange is the gather itself.
 //
-// Both kernels walk a flat index over 16-byte output vectors (8 bf16 or 8 fp32
-// elements of one row), so consecutive threads touch consecutive bytes of a row;
-// each thread handles kUnroll vectors with all loads issued before any store.
+// Both kernels run one warp per token over 16-byte vectors (8 bf16 or 8 fp32
+// elements), so each warp instruction touches 512 contiguous bytes of one row,
+// with several vectors in flight per lane.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -50,118 +50,130 @@ __device__ __forceinline__ void st8(float* p, const Vec8& o) {
   reinterpret_cast<float4*>(p)[1] = make_float4(o.v[4], o.v[5], o.v[6], o.v[7]);
 }
 
-// x_perm[row, :] = bf16(x[src[row] / k, :])
+// Token pre-all-to-all as a scatter in token order: warp w owns token t, reads
+// x[t, :] once (16-byte vectors, 512 contiguous bytes per warp instruction) and
+// writes the bf16 row to its k destinations x_perm[pos[t*k + j], :].  Every byte
+// of x is read from HBM once and every byte of x_perm written once.
 template <typename XT>
 __global__ void __launch_bounds__(kThreads)
-dispatch_kernel(const XT* __restrict__ x, const int32_t* __restrict__ src, bf16* __restrict__ x_perm,
-                uint32_t total_vec, uint32_t vec_per_row, int D, int k, int T) {
-  const uint32_t stride = gridDim.x * blockDim.x;
-  for (uint32_t v0 = blockIdx.x * blockDim.x + threadIdx.x; v0 < total_vec; v0 += stride * kUnroll) {
-    Vec8 buf[kUnroll];
-    uint32_t row[kUnroll], col[kUnroll];
+dispatch_kernel(const XT* __restrict__ x, const int32_t* __restrict__ pos, bf16* __restrict__ x_perm,
+                int T, int D, int k, uint32_t R) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+    const uint32_t my_pos = lane < k ? (uint32_t)__ldg(pos + (size_t)t * k + lane) : 0u;
+    const XT* xrow = x + (size_t)t * D;
+    for (int c0 = lane * 8; c0 < D; c0 += 256 * kUnroll) {
+      uint4 v[kUnroll];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const uint32_t v = v0 + u * stride;
-      row[u] = v / vec_per_row;
-      col[u] = (v - row[u] * vec_per_row) * 8;
-      if (v < total_vec) {
-        const uint32_t t = (uint32_t)__ldg(src + row[u]) / (uint32_t)k;
-        if (t < (uint32_t)T) ld8(x + (size_t)t * D + col[u], buf[u]);
-        else for (int i = 0; i < 8; ++i) buf[u].v[i] = 0.f;   // a pair the preprocess skipped
+      for (int u = 0; u < kUnroll; ++u) {
+        const int c = c0 + u * 256;
+        if (c < D) {
+          Vec8 f;
+          ld8(xrow + c, f);
+          v[u] = pack_bf16(f);
+        }
       }
-    }
+      for (int j = 0; j < k; ++j) {
+        const uint32_t p = __shfl_sync(0xffffffffu, my_pos, j);
+        if (p >= R) continue;                    // a pair the preprocess skipped
+        bf16* dst = x_perm + (size_t)p * D;
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const uint32_t v = v0 + u * stride;
-      if (v < total_vec) st8(x_perm + (size_t)row[u] * D + col[u], buf[u]);
+        for (int u = 0; u < kUnroll; ++u) {
+          const int c = c0 + u * 256;
+          if (c < D) *reinterpret_cast<uint4*>(dst + c) = v[u];
+        }
+      }
     }
   }
 }
 
-// out[t] = x[t] + shared[t] + sum_j w[t,j] * y_perm[pos[t,j]]   (fp32 accumulate)
-// Row indices are clamped to [0, R): pos is only undefined after the preprocess
+// Token post-all-to-all + unpermute + routing weights + residual, warp per token:
+// out[t] = x[t] + shared[t] + sum_j w[t,j] * y_perm[pos[t*k+j]]   (fp32 accumulate,
+// slots in order j = 0..k-1).  pos and w are read once per token into lanes;
+// each of the k row reads is 512 contiguous bytes per warp instruction.  Row
+// indices are clamped to [0, R): pos is only undefined after the preprocess
 // reported an out-of-range expert, and then the output is unspecified anyway.
 template <typename XT>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(const bf16* __restrict__ y_perm, const int32_t* __restrict__ pos,
                const float* __restrict__ topk_w, const XT* __restrict__ x,
-               const bf16* __restrict__ shared, XT* __restrict__ out, uint32_t total_vec,
-               uint32_t vec_per_row, int D, int k, uint32_t R) {
-  const uint32_t stride = gridDim.x * blockDim.x;
-  for (uint32_t v = blockIdx.x * blockDim.x + threadIdx.x; v < total_vec; v += stride) {
-    const uint32_t t = v / vec_per_row;
-    const uint32_t col = (v - t * vec_per_row) * 8;
-    Vec8 acc;
-    ld8(x + (size_t)t * D + col, acc);
-    if (shared != nullptr) {
-      Vec8 s;
-      ld8(shared + (size_t)t * D + col, s);
+               const bf16* __restrict__ shared, XT* __restrict__ out, int T, int D, int k,
+               uint32_t R) {
+  constexpr int U = 2;
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+    const uint32_t my_pos = lane < k ? min((uint32_t)__ldg(pos + (size_t)t * k + lane), R - 1) : 0u;
+    const float my_w = lane < k ? __ldg(topk_w + (size_t)t * k + lane) : 0.f;
+    for (int c0 = lane * 8; c0 < D; c0 += 256 * U) {
+      Vec8 acc[U];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc.v[i] += s.v[i];
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + u * 256;
+        if (c < D) {
+          ld8(x + (size_t)t * D + c, acc[u]);
+          if (shared != nullptr) {
+            Vec8 s;
+            ld8(shared + (size_t)t * D + c, s);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[u].v[i] += s.v[i];
+          }
+        }
+      }
+      for (int j = 0; j < k; ++j) {
+        const uint32_t p = __shfl_sync(0xffffffffu, my_pos, j);
+        const float w = __shfl_sync(0xffffffffu, my_w, j);
+        const bf16* yrow = y_perm + (size_t)p * D;
+        Vec8 y[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (c0 + u * 256 < D) ld8(yrow + c0 + u * 256, y[u]);
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[u].v[i] = fmaf(w, y[u].v[i], acc[u].v[i]);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (c0 + u * 256 < D) st8(out + (size_t)t * D + c0 + u * 256, acc[u]);
     }
-    const int32_t* pt = pos + (size_t)t * k;
-    const float* wt = topk_w + (size_t)t * k;
-    int j = 0;
-    for (; j + 2 <= k; j += 2) {               // two rows in flight per step
-      const uint32_t p0 = min((uint32_t)__ldg(pt + j), R - 1), p1 = min((uint32_t)__ldg(pt + j + 1), R - 1);
-      const float w0 = __ldg(wt + j), w1 = __ldg(wt + j + 1);
-      Vec8 y0, y1;
-      ld8(y_perm + (size_t)p0 * D + col, y0);
-      ld8(y_perm + (size_t)p1 * D + col, y1);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc.v[i] = fmaf(w0, y0.v[i], acc.v[i]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc.v[i] = fmaf(w1, y1.v[i], acc.v[i]);
-    }
-    if (j < k) {
-      const uint32_t p0 = min((uint32_t)__ldg(pt + j), R - 1);
-      const float w0 = __ldg(wt + j);
-      Vec8 y0;
-      ld8(y_perm + (size_t)p0 * D + col, y0);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc.v[i] = fmaf(w0, y0.v[i], acc.v[i]);
-    }
-    st8(out + (size_t)t * D + col, acc);
   }
 }
 
-int grid_for(uint32_t total_vec) {
-  const int max_blocks = sm_count() * 8;
-  const uint32_t need = (total_vec + kThreads - 1) / kThreads;
-  return (int)(need < (uint32_t)max_blocks ? (need > 0 ? need : 1) : max_blocks);
+int warp_grid(int T) {
+  const int wpb = kThreads / 32;
+  const int need = (T + wpb - 1) / wpb;
+  const int cap = sm_count() * 8;
+  return need < cap ? (need > 0 ? need : 1) : cap;
 }
 
 }  // namespace
 
-cudaError_t launch_dispatch(const moe_config& c, const void* x, const int32_t* src, bf16* x_perm,
+cudaError_t launch_dispatch(const moe_config& c, const void* x, const int32_t* pos, bf16* x_perm,
                             cudaStream_t s) {
-  const uint32_t vpr = c.D / 8;
-  const uint32_t total = (uint32_t)c.T * c.top_k * vpr;
-  const int grid = grid_for((total + kUnroll - 1) / kUnroll);
+  const uint32_t R = (uint32_t)c.T * c.top_k;
   if (c.x_dtype == MOE_DT_F32)
-    dispatch_kernel<float><<<grid, kThreads, 0, s>>>(static_cast<const float*>(x), src, x_perm,
-                                                     total, vpr, c.D, c.top_k, c.T);
+    dispatch_kernel<float><<<warp_grid(c.T), kThreads, 0, s>>>(static_cast<const float*>(x), pos,
+                                                               x_perm, c.T, c.D, c.top_k, R);
   else
-    dispatch_kernel<bf16><<<grid, kThreads, 0, s>>>(static_cast<const bf16*>(x), src, x_perm,
-                                                    total, vpr, c.D, c.top_k, c.T);
+    dispatch_kernel<bf16><<<warp_grid(c.T), kThreads, 0, s>>>(static_cast<const bf16*>(x), pos,
+                                                              x_perm, c.T, c.D, c.top_k, R);
   return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const moe_config& c, const bf16* y_perm, const int32_t* pos,
                            const float* topk_w, const void* x, const bf16* shared_out, void* out,
                            cudaStream_t s) {
-  const uint32_t vpr = c.D / 8;
-  const uint32_t total = (uint32_t)c.T * vpr;
-  const int grid = grid_for(total);
+  const uint32_t R = (uint32_t)c.T * c.top_k;
   if (c.x_dtype == MOE_DT_F32)
-    combine_kernel<float><<<grid, kThreads, 0, s>>>(y_perm, pos, topk_w,
-                                                    static_cast<const float*>(x), shared_out,
-                                                    static_cast<float*>(out), total, vpr, c.D,
-                                                    c.top_k, (uint32_t)c.T * c.top_k);
+    combine_kernel<float><<<warp_grid(c.T), kThreads, 0, s>>>(
+        y_perm, pos, topk_w, static_cast<const float*>(x), shared_out, static_cast<float*>(out),
+        c.T, c.D, c.top_k, R);
   else
-    combine_kernel<bf16><<<grid, kThreads, 0, s>>>(y_perm, pos, topk_w, static_cast<const bf16*>(x),
-                                                   shared_out, static_cast<bf16*>(out), total, vpr,
-                                                   c.D, c.top_k, (uint32_t)c.T * c.top_k);
+    combine_kernel<bf16><<<warp_grid(c.T), kThreads, 0, s>>>(
+        y_perm, pos, topk_w, static_cast<const bf16*>(x), shared_out, static_cast<bf16*>(out), c.T,
+        c.D, c.top_k, R);
   return cudaGetLastError();
 }
 

@@ -97,10 +97,15 @@ pre_scan_kernel(int32_t* __restrict__ block_counts, int nblk, int E, int ep,
   const int off = block_exclusive_scan(e < E ? run : 0, warp_sums, &total);
   if (e < E) expert_offsets[e] = off;
   if (e == 0) expert_offsets[E] = total;
+  // GEMM M-tile prefixes: [0, E] for 128-row tiles, [E+1, 2E+1] for 256-row tiles
   const int tiles = e < E ? (run + kTileM - 1) / kTileM : 0;
   const int toff = block_exclusive_scan(tiles, warp_sums, &total);
   if (e < E) mt_start[e] = toff;
   if (e == 0) mt_start[E] = total;
+  const int tiles2 = e < E ? (run + 2 * kTileM - 1) / (2 * kTileM) : 0;
+  const int toff2 = block_exclusive_scan(tiles2, warp_sums, &total);
+  if (e < E) mt_start[E + 1 + e] = toff2;
+  if (e == 0) mt_start[2 * E + 1] = total;
   __syncthreads();
   const int El = E / ep;
   int split = 0;

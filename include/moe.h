@@ -142,10 +142,13 @@ MOE_API moe_status moe_preprocess(const moe_config* cfg, const int32_t* topk_idx
                           void* stream);
 
 /* Stage 2a, dispatch (token pre-all-to-all).  "Expert Parallel (EP)",
- * Communication Pattern, step 2; "Worked Example ...", Step 2.
- *   x_perm[row, :] = bf16( x[src[row] / k, :] )      (fp32 x rounded to nearest even)
- *   x      device [T, D] x_dtype;  src device int32 [R];  x_perm device bf16 [R, D] */
-MOE_API moe_status moe_dispatch_permute(const moe_config* cfg, const void* x, const int32_t* src,
+ * Communication Pattern, step 2; "Worked Example ...", Step 2 (each chosen expert
+ * receives its own copy of the token).
+ *   x_perm[pos[t*k+j], :] = bf16( x[t, :] )  for every token t and slot j
+ *   (equivalently x_perm[row] = bf16(x[src[row] / k]); fp32 x rounds to nearest even)
+ *   x      device [T, D] x_dtype;  pos device int32 [R] from moe_preprocess;
+ *   x_perm device bf16 [R, D], written.  Rows whose pos is outside [0, R) are skipped. */
+MOE_API moe_status moe_dispatch_permute(const moe_config* cfg, const void* x, const int32_t* pos,
                                 void* x_perm, void* stream);
 
 /* Stage 2b, local experts.  "Expert Parallel (EP)", Communication Pattern, step 3;

@@ -160,3 +160,23 @@ def test_deterministic():
     b = layer.forward(inp["x"]).clone()
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("T", [100, 700])
+def test_cta_pair_and_single_cta_gemm_agree(T, monkeypatch):
+    """The 256x256 CTA-pair tiles and the one-CTA 128x256 tiles both match the
+    oracle (ragged expert ends inside a 256-row tile, shared experts included)."""
+    wl = BASE.with_(T=T, D=512, E=16, ep_size=4, top_k=3, F=384, n_shared=1, F_shared=256, seed=T)
+    inp = W.make_inputs(wl, device="cuda")
+    outs = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("MOE_GEMM_CTA_PAIR", flag)
+        layer = make_layer(wl, inp)
+        outs.append(layer.forward(inp["x"]).clone())
+        torch.cuda.synchronize()
+        layer.check_status()
+    res = oracle_layer(wl, inp)
+    for o in outs:
+        assert_layer_close(f64(o), res["out"], f64(inp["x"]))
+    d = (outs[0].float() - outs[1].float()).abs().max().item()
+    assert d <= 2 ** -6 * outs[1].float().abs().max().item()

@@ -69,7 +69,8 @@ def test_dispatch_stage(ctx):
     wl, inp, layer, pre = ctx["wl"], ctx["inp"], ctx["layer"], ctx["pre"]
     b = layer.allocate(wl.T)
     src = torch.from_numpy(pre["src"]).cuda()
-    M.moe_dispatch_permute(layer.config(wl.T), inp["x"], src, b["x_perm"])
+    pos = torch.from_numpy(pre["pos"]).cuda()
+    M.moe_dispatch_permute(layer.config(wl.T), inp["x"], pos, b["x_perm"])
     torch.cuda.synchronize()
     # sampled rows against the oracle, bit-exact
     rng = np.random.default_rng(0)
