@@ -15,7 +15,8 @@ import torch
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libmoe.so")
 
-MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_INDEX_OOB, MOE_ERR_TIMEOUT = range(6)
+(MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_INDEX_OOB, MOE_ERR_TIMEOUT,
+ MOE_ERR_SCRATCH_LIMIT) = range(7)
 MOE_DT_F32, MOE_DT_BF16 = 0, 1
 MOE_ACT_GELU, MOE_ACT_SWIGLU = 0, 1
 
@@ -52,6 +53,8 @@ _SIGS = {
     "moe_forward": (ctypes.c_int, [_cfgp, _vp, _f32p, _f32p, _vp, _f32p, _i32p, _f32p, _i32p, _i32p,
                                    _i32p, _i32p, _i32p, _i32p, _vp, _vp, _vp, _vp, _vp, _vp, _i32p,
                                    _vp]),
+    "moe_preprocess_noalloc": (ctypes.c_int, [_cfgp, _i32p, _i32p, _i32p, _i32p, _i32p, _i32p, _i32p,
+                                              _i32p, _vp]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_abi_version": (ctypes.c_int32, []),
 }
@@ -128,6 +131,16 @@ def moe_preprocess(cfg, topk_idx, counts, expert_offsets, rank_splits, rank_offs
                    workspace, status, stream=None):
     _call("moe_preprocess", ctypes.byref(cfg), _p(topk_idx), _p(counts), _p(expert_offsets),
           _p(rank_splits), _p(rank_offsets), _p(pos), _p(src), _p(workspace), _p(status), _s(stream))
+
+
+def moe_preprocess_noalloc(cfg, topk_idx, counts, expert_offsets, rank_splits, rank_offsets, pos,
+                           src, status, stream=None):
+    """moe_preprocess without a workspace, for callers that cannot allocate device
+    memory (a plugin whose host framework owns all device memory, or a loop that
+    cannot afford cudaMalloc's implicit synchronisation); scratch is a fixed array
+    inside libmoe.so, so overlapping calls on different streams race."""
+    _call("moe_preprocess_noalloc", ctypes.byref(cfg), _p(topk_idx), _p(counts), _p(expert_offsets),
+          _p(rank_splits), _p(rank_offsets), _p(pos), _p(src), _p(status), _s(stream))
 
 
 def moe_dispatch_permute(cfg, x, pos, x_perm, stream=None):

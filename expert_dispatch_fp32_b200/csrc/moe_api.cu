@@ -310,6 +310,7 @@ const char* moe_status_string(moe_status s) {
     case MOE_ERR_CUDA: return "CUDA error";
     case MOE_ERR_INDEX_OOB: return "expert index out of range";
     case MOE_ERR_TIMEOUT: return "bounded wait expired in a kernel";
+    case MOE_ERR_SCRATCH_LIMIT: return "configuration exceeds the no-alloc preprocess scratch";
   }
   return "unknown status";
 }

@@ -1,0 +1,85 @@
+// moe_preprocess_noalloc: the preprocess stage for callers that cannot allocate
+// device memory.
+//
+// moe_preprocess needs a caller-allocated workspace for its per-block expert
+// histograms.  Some callers cannot provide one: code running inside a host
+// framework that owns every device allocation and hands out only the tensors it
+// already has, or a latency-critical loop where a cudaMalloc (which may
+// synchronise the device) is not acceptable.  This entry point takes no
+// workspace and allocates nothing; its scratch is one file-scope device array of
+// MOE_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library holds until
+// the process exits.  The pages describe no such call: it exists for deployment.
+//
+// The kernels are the ones moe_preprocess launches; only the scratch differs.
+// Every call shares the array and leaves its contents behind.  Each call writes
+// every histogram entry before reading it, so nothing needs clearing; calls that
+// overlap on the GPU (two streams with no ordering between them) race on it.
+#include <mutex>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+// Scratch: block histograms [nblk * E] followed by the two GEMM tile prefixes [2 * (E + 1)].
+constexpr size_t kNoAllocScratchInts = MOE_NOALLOC_SCRATCH_BYTES / sizeof(int32_t);
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchInts];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_setup_mutex;
+int32_t* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address must come from
+// cudaGetSymbolAddress, once per device, with that device current.
+cudaError_t scratch_for_current_device(int32_t** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (err != cudaSuccess) return err;
+    g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" moe_status moe_preprocess_noalloc(const moe_config* cfg, const int32_t* topk_idx,
+                                             int32_t* counts, int32_t* expert_offsets,
+                                             int32_t* rank_splits, int32_t* rank_offsets,
+                                             int32_t* pos, int32_t* src, int32_t* status,
+                                             void* stream) {
+  moe_status st = moe_validate_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  const int32_t* ptrs_small[] = {counts, expert_offsets, rank_splits, rank_offsets, status};
+  for (const int32_t* p : ptrs_small)
+    if (p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u)) return MOE_ERR_INVALID_ARG;
+  if (c.T > 0) {
+    const int32_t* ptrs_big[] = {topk_idx, pos, src};
+    for (const int32_t* p : ptrs_big)
+      if (p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u)) return MOE_ERR_INVALID_ARG;
+  }
+  const size_t R = (size_t)c.T * c.top_k;
+  const size_t nblk = (R + kPreChunk - 1) / kPreChunk;
+  const size_t need = nblk * (size_t)c.E + 2 * ((size_t)c.E + 1);
+  if (need > kNoAllocScratchInts) return MOE_ERR_SCRATCH_LIMIT;
+  int32_t* scratch = nullptr;
+  if (scratch_for_current_device(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+  int32_t* block_counts = scratch;
+  int32_t* mt_start = scratch + nblk * (size_t)c.E;
+  // Every histogram entry is written before it is read, so no clearing is needed.
+  const cudaError_t err = launch_preprocess(c, topk_idx, counts, expert_offsets, rank_splits,
+                                            rank_offsets, pos, src, block_counts, (int)nblk,
+                                            mt_start, status, reinterpret_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}

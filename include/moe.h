@@ -54,7 +54,8 @@ typedef enum {
   MOE_ERR_UNSUPPORTED = 2,  /* valid MoE but outside what the kernels implement   */
   MOE_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed                */
   MOE_ERR_INDEX_OOB = 4,    /* device status: an expert index was outside [0, E)   */
-  MOE_ERR_TIMEOUT = 5       /* device status: a bounded wait in a kernel expired   */
+  MOE_ERR_TIMEOUT = 5,      /* device status: a bounded wait in a kernel expired   */
+  MOE_ERR_SCRATCH_LIMIT = 6 /* moe_preprocess_noalloc: config exceeds its fixed scratch */
 } moe_status;
 
 typedef enum { MOE_DT_F32 = 0, MOE_DT_BF16 = 1 } moe_dtype;
@@ -194,6 +195,37 @@ MOE_API moe_status moe_forward(const moe_config* cfg, const void* x, const float
                        int32_t* pos, int32_t* src, void* x_perm, void* act, void* y_perm,
                        void* shared_out, void* out, void* workspace, int32_t* status,
                        void* stream);
+
+/* Preprocess without a workspace -- for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this entry point; it exists for deployment.
+ * moe_preprocess needs a caller-allocated `workspace` for its per-block expert
+ * histograms.  Some callers have no way to provide one: a plugin inside a host
+ * framework that owns every device allocation and only lends out the tensors it
+ * already has, or a latency-critical loop in which cudaMalloc (which may
+ * synchronise the whole device) is not acceptable.  This call takes no workspace
+ * and allocates nothing: its scratch is one file-scope device array of
+ * MOE_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library holds until
+ * the process exits.
+ *
+ * Outputs, layouts, ordering and the device status word are exactly those of
+ * moe_preprocess (bit-identical results); it does not write the GEMM tile prefix
+ * that moe_expert_ffn reads from a workspace, so it is a drop-in for the
+ * bookkeeping outputs only.
+ *   Limit: ceil(T*k / 1024) * E + 2*(E + 1) int32 values must fit in the scratch;
+ *   larger configurations return MOE_ERR_SCRATCH_LIMIT before anything is enqueued.
+ *   First call on each device: finds the scratch array's device address with
+ *   cudaGetSymbolAddress (once per device, with that device current), so make that
+ *   first call before any stream capture.
+ *   Concurrency: every call shares the one array and leaves its contents behind
+ *   (each call rewrites all it reads); calls that may overlap on the GPU, e.g. on
+ *   two streams without ordering between them, race and must not be issued. */
+#define MOE_NOALLOC_SCRATCH_BYTES (1u << 20)
+MOE_API moe_status moe_preprocess_noalloc(const moe_config* cfg, const int32_t* topk_idx,
+                                          int32_t* counts, int32_t* expert_offsets,
+                                          int32_t* rank_splits, int32_t* rank_offsets,
+                                          int32_t* pos, int32_t* src, int32_t* status,
+                                          void* stream);
 
 /* Static description of a status code. */
 MOE_API const char* moe_status_string(moe_status s);
