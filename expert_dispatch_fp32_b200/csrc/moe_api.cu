@@ -12,10 +12,11 @@ WsLayout ws_layout(const moe_config& c) {
   WsLayout L;
   const size_t T = (size_t)c.T, E = (size_t)c.E;
   const size_t R = T * (size_t)c.top_k;
-  L.nblk = (int)((R + kPreChunk - 1) / kPreChunk);
+  L.nblk = preprocess_blocks((int64_t)R);
   size_t o = 0;
   L.logits = o;       o = align256(o + T * E * sizeof(float));
   L.block_counts = o; o = align256(o + (size_t)L.nblk * E * sizeof(int32_t));
+  L.barrier = o;      o = align256(o + 2 * sizeof(uint32_t));
   L.mt_start = o;     o = align256(o + 2 * (E + 1) * sizeof(int32_t));
   L.act_shared = o;   o = align256(o + T * (size_t)c.n_shared * c.F_shared * sizeof(bf16));
   L.total = o;
@@ -151,8 +152,8 @@ moe_status moe_preprocess(const moe_config* cfg, const int32_t* topk_idx, int32_
   uint8_t* ws = (uint8_t*)workspace;
   return cuda_status(launch_preprocess(c, topk_idx, counts, expert_offsets, rank_splits,
                                        rank_offsets, pos, src, (int32_t*)(ws + L.block_counts),
-                                       L.nblk, (int32_t*)(ws + L.mt_start), status,
-                                       as_stream(stream)));
+                                       L.nblk, (int32_t*)(ws + L.mt_start),
+                                       (unsigned*)(ws + L.barrier), status, as_stream(stream)));
 }
 
 moe_status moe_dispatch_permute(const moe_config* cfg, const void* x, const int32_t* pos,

@@ -17,8 +17,8 @@ typedef __nv_bfloat16 bf16;
 // ---------------------------------------------------------------------------
 constexpr int kMaxExperts = 1024;   // preprocess keeps one counter per expert in smem
 constexpr int kMaxTopK = 32;        // top-k kernel keeps selection j in lane j
-constexpr int kPreChunk = 1024;     // flat (token, slot) pairs per preprocess block
-constexpr int kPreThreads = 256;
+constexpr int kPreThreads = 256;    // preprocess block size
+constexpr int kPreMaxBlocks = 160;  // preprocess grid cap (>= one block per SM on B200)
 constexpr int kTileM = 128;         // GEMM tile rows (one tcgen05 M=128 accumulator)
 constexpr int kTileK = 64;          // GEMM K step: 64 bf16 = one 128-byte swizzle row
 
@@ -27,7 +27,8 @@ constexpr int kTileK = 64;          // GEMM K step: 64 bf16 = one 128-byte swizz
 // ---------------------------------------------------------------------------
 struct WsLayout {
   size_t logits;        // fp32 [T, E]
-  size_t block_counts;  // int32 [nblk, E]
+  size_t block_counts;  // int32 [nblk, E]: preprocess per-block histograms
+  size_t barrier;       // uint32 [2]: preprocess grid barrier (zeroed per call)
   size_t mt_start;      // int32 [2][E + 1]: prefixes of ceil(count/128), ceil(count/256)
   size_t act_shared;    // bf16 [T, S*Fs]
   size_t total;
@@ -58,11 +59,14 @@ int down_tile_n(const moe_config& c);
 cudaError_t launch_route(const moe_config& c, const void* x, const float* w_router,
                          const float* bias, float* logits, bool keep_logits, int32_t* topk_idx,
                          float* topk_w, cudaStream_t s);
+// Preprocess grid size for R pairs (<= kPreMaxBlocks); block_counts needs
+// preprocess_blocks(R) * E entries.
+int preprocess_blocks(int64_t R);
 cudaError_t launch_preprocess(const moe_config& c, const int32_t* topk_idx, int32_t* counts,
                               int32_t* expert_offsets, int32_t* rank_splits,
                               int32_t* rank_offsets, int32_t* pos, int32_t* src,
-                              int32_t* block_counts, int nblk, int32_t* mt_start,
-                              int32_t* status, cudaStream_t s);
+                              int32_t* block_counts, int max_blocks, int32_t* mt_start,
+                              unsigned* barrier, int32_t* status, cudaStream_t s);
 cudaError_t launch_dispatch(const moe_config& c, const void* x, const int32_t* pos,
                             bf16* x_perm, cudaStream_t s);
 cudaError_t launch_combine(const moe_config& c, const bf16* y_perm, const int32_t* pos,

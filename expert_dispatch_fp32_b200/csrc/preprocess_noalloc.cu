@@ -11,9 +11,10 @@
 // the process exits.  The pages describe no such call: it exists for deployment.
 //
 // The kernels are the ones moe_preprocess launches; only the scratch differs.
-// Every call shares the array and leaves its contents behind.  Each call writes
-// every histogram entry before reading it, so nothing needs clearing; calls that
-// overlap on the GPU (two streams with no ordering between them) race on it.
+// Every call shares the array and leaves its contents behind.  Each call zeroes
+// the barrier words on its stream and writes every histogram entry before reading
+// it; calls that overlap on the GPU (two streams with no ordering between them)
+// race on it.
 #include <mutex>
 
 #include "moe_internal.cuh"
@@ -21,7 +22,7 @@
 namespace moe {
 namespace {
 
-// Scratch: block histograms [nblk * E] followed by the two GEMM tile prefixes [2 * (E + 1)].
+// Scratch: grid-barrier words, the two GEMM tile prefixes, then block histograms.
 constexpr size_t kNoAllocScratchInts = MOE_NOALLOC_SCRATCH_BYTES / sizeof(int32_t);
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchInts];
 
@@ -70,16 +71,20 @@ extern "C" moe_status moe_preprocess_noalloc(const moe_config* cfg, const int32_
       if (p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u)) return MOE_ERR_INVALID_ARG;
   }
   const size_t R = (size_t)c.T * c.top_k;
-  const size_t nblk = (R + kPreChunk - 1) / kPreChunk;
-  const size_t need = nblk * (size_t)c.E + 2 * ((size_t)c.E + 1);
+  const size_t nblk = (size_t)preprocess_blocks((int64_t)R);
+  // barrier words [2], tile prefixes [2 * (E + 1)], block histograms [nblk * E]
+  const size_t need = 2 + 2 * ((size_t)c.E + 1) + nblk * (size_t)c.E;
   if (need > kNoAllocScratchInts) return MOE_ERR_SCRATCH_LIMIT;
   int32_t* scratch = nullptr;
   if (scratch_for_current_device(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
-  int32_t* block_counts = scratch;
-  int32_t* mt_start = scratch + nblk * (size_t)c.E;
-  // Every histogram entry is written before it is read, so no clearing is needed.
+  unsigned* barrier = reinterpret_cast<unsigned*>(scratch);
+  int32_t* mt_start = scratch + 2;
+  int32_t* block_counts = mt_start + 2 * ((size_t)c.E + 1);
+  // The barrier words are zeroed on the stream before each launch; every histogram
+  // entry is written before it is read, so nothing else needs clearing.
   const cudaError_t err = launch_preprocess(c, topk_idx, counts, expert_offsets, rank_splits,
                                             rank_offsets, pos, src, block_counts, (int)nblk,
-                                            mt_start, status, reinterpret_cast<cudaStream_t>(stream));
+                                            mt_start, barrier, status,
+                                            reinterpret_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

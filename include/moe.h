@@ -212,15 +212,16 @@ MOE_API moe_status moe_forward(const moe_config* cfg, const void* x, const float
  * moe_preprocess (bit-identical results); it does not write the GEMM tile prefix
  * that moe_expert_ffn reads from a workspace, so it is a drop-in for the
  * bookkeeping outputs only.
- *   Limit: ceil(T*k / 1024) * E + 2*(E + 1) int32 values must fit in the scratch;
- *   larger configurations return MOE_ERR_SCRATCH_LIMIT before anything is enqueued.
+ *   Limit: min(160, ceil(T*k / 256)) * E + 2*(E + 1) + 2 int32 values must fit in
+ *   the scratch; larger configurations return MOE_ERR_SCRATCH_LIMIT before anything
+ *   is enqueued.
  *   First call on each device: finds the scratch array's device address with
  *   cudaGetSymbolAddress (once per device, with that device current), so make that
  *   first call before any stream capture.
  *   Concurrency: every call shares the one array and leaves its contents behind
  *   (each call rewrites all it reads); calls that may overlap on the GPU, e.g. on
  *   two streams without ordering between them, race and must not be issued. */
-#define MOE_NOALLOC_SCRATCH_BYTES (1u << 20)
+#define MOE_NOALLOC_SCRATCH_BYTES (1u << 18)
 MOE_API moe_status moe_preprocess_noalloc(const moe_config* cfg, const int32_t* topk_idx,
                                           int32_t* counts, int32_t* expert_offsets,
                                           int32_t* rank_splits, int32_t* rank_offsets,
