@@ -314,36 +314,70 @@ def run_ours(args):
     total_ms_max = max_over_ranks(total_ms, ws)
     value = replica_value(T, ws, args.steps, total_ms_max)
 
-    # end to end: pinned host x -> device, forward, device -> pinned host out
-    x_host = x.cpu().pin_memory()
-    out_host = torch.empty(b["out"].shape, dtype=b["out"].dtype).pin_memory()
-    x_dev = torch.empty_like(x)
-    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
-    for _ in range(args.warmup):
-        x_dev.copy_(x_host, non_blocking=True)
-        layer.forward(x_dev, stream)
-        out_host.copy_(b["out"], non_blocking=True)
+    # end to end through the C ABI with host buffers: every step uploads its batch from
+    # pinned host memory and reads its output back to pinned host memory.  Uploads run on
+    # a copy stream and downloads on another, double-buffered, so step i+1's upload and
+    # step i-1's download overlap step i's forward; the timed region spans the first
+    # upload to the last download (whole-job throughput).
+    NBUF = 2
+    x_host = [x.cpu().pin_memory() for _ in range(NBUF)]
+    out_host = [torch.empty(b["out"].shape, dtype=b["out"].dtype).pin_memory() for _ in range(NBUF)]
+    x_dev = [torch.empty_like(x) for _ in range(NBUF)]
+    out_dev = [torch.empty_like(b["out"]) for _ in range(NBUF)]
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def e2e_run(nsteps, t0=None, t1=None):
+        up_done = [torch.cuda.Event() for _ in range(nsteps)]
+        fw_done = [torch.cuda.Event() for _ in range(nsteps)]
+        dn_done = [torch.cuda.Event() for _ in range(nsteps)]
+        if t0 is not None:
+            t0.record(h2d)
+        for i in range(nsteps):
+            j = i % NBUF
+            with torch.cuda.stream(h2d):
+                if i >= NBUF:
+                    h2d.wait_event(fw_done[i - NBUF])          # x_dev[j] no longer read
+                x_dev[j].copy_(x_host[j], non_blocking=True)
+                up_done[i].record(h2d)
+            stream.wait_event(up_done[i])
+            if i >= NBUF:
+                stream.wait_event(dn_done[i - NBUF])           # out_dev[j] already read back
+            M.moe_forward(cfg, x_dev[j], layer.w_router, layer.expert_bias, layer.packed, None,
+                          b["topk_idx"], b["topk_w"], b["counts"], b["expert_offsets"],
+                          b["rank_splits"], b["rank_offsets"], b["pos"], b["src"], b["x_perm"],
+                          b["act"], b["y_perm"], b["shared_out"], out_dev[j], b["workspace"],
+                          b["status"], stream)
+            fw_done[i].record(stream)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(fw_done[i])
+                out_host[j].copy_(out_dev[j], non_blocking=True)
+                dn_done[i].record(d2h)
+        if t1 is not None:
+            t1.record(d2h)
+
+    e2e_run(max(args.warmup, NBUF))
     torch.cuda.synchronize()
     barrier(ws)
-    for i in range(args.steps):
-        flush.zero_()
-        e_ev[i][0].record(stream)
-        x_dev.copy_(x_host, non_blocking=True)
-        layer.forward(x_dev, stream)
-        out_host.copy_(b["out"], non_blocking=True)
-        e_ev[i][1].record(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_run(args.steps, e0, e1)
     torch.cuda.synchronize()
     barrier(ws)
     layer.check_status()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(z) for a, z in e_ev), ws)
+    assert torch.equal(out_host[(args.steps - 1) % NBUF].to(b["out"].device), ref_out), \
+        "end-to-end output differs from the device-resident forward"
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws)
     e2e_value = replica_value(T, ws, args.steps, e2e_ms)
     sx = 4 if wl.x_dtype == "f32" else 2
 
     # roofline of the dominant kernel: the grouped expert FFN (tcgen05 GEMMs)
     ffn_ms = stage_ms[3] / args.steps
     ffn_tflops = wl.ffn_flop() / (ffn_ms / 1e3) / 1e12
-    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    # a step of several ms keeps the tensor cores busy long enough to meet the power cap:
+    # compare against the sustained figure there, the burst figure for short steps
+    long_step = total_ms_max / args.steps > 2.0
+    peak_key = "bf16_tflops_sustained" if long_step else "bf16_tflops"
+    peak_tf = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
+    burst_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "ffn_traffic.json")
     if os.path.exists(tpath):
@@ -375,7 +409,8 @@ def run_ours(args):
                      "frac": ffn_tflops / peak_tf, "traffic": traffic,
                      "kernel": "grouped_gemm_kernel (moe_expert_ffn: routed gate_up+down"
                                + (", shared gate_up+down" if wl.n_shared else "") + ")",
-                     "peak_source": f"{peak_src} bf16 burst"},
+                     "peak_source": f"{peak_src} bf16 " + ("sustained (step > 2 ms)" if long_step else "burst"),
+                     "frac_of_burst": ffn_tflops / burst_tf},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * wl.D * sx,
                 "d2h_bytes_per_step": T * wl.D * sx},
         "gpu_launches": launches_per_step * args.steps,

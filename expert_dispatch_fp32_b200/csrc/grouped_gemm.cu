@@ -54,6 +54,7 @@ struct GemmArgs {
   const int32_t* mt_start;
   int32_t G, N, K, dense_rows;
   bf16* out;
+  float* outf;               // EPI_PAIRSUM_F32 output
   int32_t ldo;
   int32_t* status;
 };
@@ -102,7 +103,7 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
       if (*abort_flag) return false;
       if (global_ns() - t0 > kWaitLimitNs) {
         *abort_flag = 1;
-        atomicCAS(status, 0, (int32_t)MOE_ERR_TIMEOUT);
+        if (status != nullptr) atomicCAS(status, 0, (int32_t)MOE_ERR_TIMEOUT);
         return false;
       }
     }
@@ -264,6 +265,12 @@ __device__ __forceinline__ void store_row32(bf16* dst, const float (&v)[32]) {
   }
 }
 
+__device__ __forceinline__ void store_row32_f32(float* dst, const float (&v)[32]) {
+  float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
 template <int BN>
 struct GemmCfg {
   static constexpr int kStages = BN == 256 ? 4 : BN == 128 ? 6 : 8;
@@ -418,6 +425,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
           if (valid) store_row32(orow + n * (BN / 2) + c, v);
+        }
+      } else if (EPI == EPI_PAIRSUM_F32) {
+        // columns [0, BN/2) and [BN/2, BN) of the tile are two parts of one value
+        float* frow = p.outf + (size_t)(row0 + (valid ? r : 0)) * p.ldo;
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t hr[32], lr[32];
+          tmem_ld32(tb + c, hr);
+          tmem_ld32(tb + BN / 2 + c, lr);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(hr[i]) + __uint_as_float(lr[i]);
+          if (valid) store_row32_f32(frow + n * (BN / 2) + c, v);
         }
       } else {
 #pragma unroll 1
@@ -628,6 +649,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
           for (int i = 0; i < 32; ++i) v[i] = silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
           if (valid) store_row32(orow + n * (BN / 2) + c, v);
         }
+      } else if (EPI == EPI_PAIRSUM_F32) {
+        // columns [0, BN/2) and [BN/2, BN) of the tile are two parts of one value
+        float* frow = p.outf + (size_t)(row0 + (valid ? r : 0)) * p.ldo;
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t hr[32], lr[32];
+          tmem_ld32(tb + c, hr);
+          tmem_ld32(tb + BN / 2 + c, lr);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(hr[i]) + __uint_as_float(lr[i]);
+          if (valid) store_row32_f32(frow + n * (BN / 2) + c, v);
+        }
       } else {
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
@@ -771,6 +806,7 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
   a.K = p.K;
   a.dense_rows = p.dense_rows;
   a.out = p.out;
+  a.outf = p.outf;
   a.ldo = p.ldo;
   a.status = p.status;
   const int64_t tiles = p.max_tiles > 0 ? p.max_tiles : 1;
@@ -780,12 +816,14 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
     const int clusters = (int)(tiles < pairs ? tiles : pairs);
     if (p.epi == EPI_SWIGLU) return launch_tc_pair<EPI_SWIGLU>(a, clusters, s);
     if (p.epi == EPI_GELU) return launch_tc_pair<EPI_GELU>(a, clusters, s);
+    if (p.epi == EPI_PAIRSUM_F32) return launch_tc_pair<EPI_PAIRSUM_F32>(a, clusters, s);
     return launch_tc_pair<EPI_STORE>(a, clusters, s);
   }
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   if (BN == 256) {
     if (p.epi == EPI_SWIGLU) return launch_tc<256, EPI_SWIGLU>(a, grid, s);
     if (p.epi == EPI_GELU) return launch_tc<256, EPI_GELU>(a, grid, s);
+    if (p.epi == EPI_PAIRSUM_F32) return launch_tc<256, EPI_PAIRSUM_F32>(a, grid, s);
     return launch_tc<256, EPI_STORE>(a, grid, s);
   }
   if (BN == 128) {

@@ -19,6 +19,10 @@ WsLayout ws_layout(const moe_config& c) {
   L.barrier = o;      o = align256(o + 2 * sizeof(uint32_t));
   L.mt_start = o;     o = align256(o + 2 * (E + 1) * sizeof(int32_t));
   L.act_shared = o;   o = align256(o + T * (size_t)c.n_shared * c.F_shared * sizeof(bf16));
+  const size_t Epad = (E + 127) / 128 * 128;
+  L.r_split = o;      o = align256(o + 2 * Epad * (size_t)c.D * sizeof(bf16));
+  L.r_wmax = o;       o = align256(o + (size_t)c.D * sizeof(float));
+  L.r_approx = o;     o = align256(o + T * Epad * sizeof(float));
   L.total = o;
   return L;
 }
@@ -123,11 +127,20 @@ moe_status moe_route(const moe_config* cfg, const void* x, const float* w_router
   MOE_CHECK_PTR(topk_idx);
   MOE_CHECK_PTR(topk_w);
   MOE_CHECK_PTR(workspace);
+  const WsLayout L = ws_layout(c);
+  uint8_t* ws = (uint8_t*)workspace;
   float* logits = logits_out;
-  if (logits == nullptr) logits = (float*)((uint8_t*)workspace + ws_layout(c).logits);
+  if (logits == nullptr) logits = (float*)(ws + L.logits);
   else if (!aligned16(logits)) return MOE_ERR_INVALID_ARG;
+  const char* pair_env = getenv("MOE_GEMM_CTA_PAIR");
+  RouterScratch rs;
+  rs.bsplit = (bf16*)(ws + L.r_split);
+  rs.wmax = (float*)(ws + L.r_wmax);
+  rs.approx = (float*)(ws + L.r_approx);
+  rs.pair = !(pair_env && pair_env[0] == '0');
+  rs.status = nullptr;
   return cuda_status(launch_route(c, x, w_router, expert_bias, logits, logits_out != nullptr,
-                                  topk_idx, topk_w, as_stream(stream)));
+                                  topk_idx, topk_w, rs, as_stream(stream)));
 }
 
 moe_status moe_preprocess(const moe_config* cfg, const int32_t* topk_idx, int32_t* counts,

@@ -31,6 +31,9 @@ struct WsLayout {
   size_t barrier;       // uint32 [2]: preprocess grid barrier (zeroed per call)
   size_t mt_start;      // int32 [2][E + 1]: prefixes of ceil(count/128), ceil(count/256)
   size_t act_shared;    // bf16 [T, S*Fs]
+  size_t r_split;       // bf16 [2*Epad, D]: tensor-core router weights
+  size_t r_wmax;        // fp32 [D]
+  size_t r_approx;      // fp32 [T, Epad]
   size_t total;
   int nblk;
 };
@@ -54,11 +57,19 @@ int down_tile_n(const moe_config& c);
 // ---------------------------------------------------------------------------
 // Launchers (each returns cudaGetLastError() of its launches)
 // ---------------------------------------------------------------------------
+// Workspace buffers of the tensor-core router (bf16 x).
+struct RouterScratch {
+  bf16* bsplit;     // [2 * Epad, D]: W_r hi / mid rows, 128-expert interleave
+  float* wmax;      // [D]: max_e |W_r[e, d]|
+  float* approx;    // [T, Epad]: tensor-core logits (hi + mid)
+  int pair;         // GEMM on CTA pairs
+  int32_t* status;
+};
 // logits: where the tiled path stores fp32 logits (caller's buffer or workspace);
 // keep_logits: the caller asked for them (the fused few-expert path then writes them).
 cudaError_t launch_route(const moe_config& c, const void* x, const float* w_router,
                          const float* bias, float* logits, bool keep_logits, int32_t* topk_idx,
-                         float* topk_w, cudaStream_t s);
+                         float* topk_w, const RouterScratch& rs, cudaStream_t s);
 // Preprocess grid size for R pairs (<= kPreMaxBlocks); block_counts needs
 // preprocess_blocks(R) * E entries.
 int preprocess_blocks(int64_t R);
@@ -77,7 +88,8 @@ cudaError_t launch_pack(const moe_config& c, const bf16* w_up, const bf16* w_dow
 
 // Grouped GEMM on the tensor cores.  out[row, :] = epilogue(A[row, :] @ B[g]^T)
 // for rows of group g; B is K-major [G, N, K].
-enum Epilogue { EPI_STORE = 0, EPI_GELU = 1, EPI_SWIGLU = 2 };
+// EPI_PAIRSUM_F32: out_f32[row, n*BN/2 + c] = acc[c] + acc[BN/2 + c] (256-wide tiles)
+enum Epilogue { EPI_STORE = 0, EPI_GELU = 1, EPI_SWIGLU = 2, EPI_PAIRSUM_F32 = 3 };
 struct GemmProblem {
   const bf16* A; int64_t a_rows;          // A [a_rows, K]
   const bf16* B; int G;                   // B [G, N, K]
@@ -87,6 +99,7 @@ struct GemmProblem {
   int dense_rows;                         // rows of the dense group
   int64_t max_tiles;                      // host upper bound on tiles (grid size)
   bf16* out; int ldo;                     // output row stride in elements
+  float* outf;                            // fp32 output (EPI_PAIRSUM_F32)
   int epi; int tile_n;
   int pair;                               // 1: 256-row tiles on CTA pairs (mt_start per 256 rows)
   int32_t* status;

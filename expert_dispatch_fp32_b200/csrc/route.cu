@@ -21,6 +21,8 @@
 // an fp64 butterfly leaves every lane with all E dot products; lane e keeps logit
 // e and the warp runs the same exact argmax top-k without a logits round trip.
 #include <math.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "moe_internal.cuh"
 
@@ -340,14 +342,263 @@ cudaError_t launch_route_t(const moe_config& c, const XT* x, const float* w_rout
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core router for bf16 x (filter and refine)
+// ---------------------------------------------------------------------------
+// 1. router_split_kernel: W_r (fp32) = hi + mid + lo with hi = bf16(W_r),
+//    mid = bf16(W_r - hi), |lo| <= 2^-18 |W_r|.  hi and mid rows are packed K-major
+//    for the grouped GEMM, interleaved per 128 experts (a 256-row block holds the
+//    hi rows then the mid rows of the same 128 experts); wmax[d] = max_e |W_r[e,d]|.
+// 2. The grouped GEMM (dense group, EPI_PAIRSUM_F32) gives approx[t,e] = x.hi + x.mid
+//    in fp32 on the tensor cores (x is bf16, so every product is exact; only the
+//    fp32 accumulation and the dropped lo part differ from the exact value).
+// 3. route_refine_kernel, one warp per token: with S_t = sum_d |x_d| wmax_d, every
+//    approximate logit is within eps_t = coef * S_t of the exact one (coef covers
+//    one fp32 rounding per MMA instruction in each of the two chains plus the lo
+//    part, with a factor 2 of margin).  Experts whose approx is below the k-th
+//    largest approx minus 2 eps_t cannot be in the exact top-k; the others
+//    (usually k plus one or two) get an exact logit (fp32 8-term slices folded into
+//    fp64, as in the SIMT paths), and the top-k and weights are taken from those.
+constexpr int kRouterRowBlock = 128;      // experts per 256-row (hi, mid) block
+constexpr int kRefineWarps = 4;
+
+__global__ void __launch_bounds__(128)
+router_split_kernel(const float* __restrict__ w, int E, int Epad, int D, bf16* __restrict__ bsplit,
+                    unsigned* __restrict__ wmax_bits) {
+  const int dq = blockIdx.x * blockDim.x + threadIdx.x;     // 8-column chunk
+  if (dq * 8 >= D) return;
+  const int d = dq * 8;
+  const int e0 = blockIdx.y * 16;
+  float mx[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx[i] = 0.f;
+  for (int e = e0; e < e0 + 16 && e < Epad; ++e) {
+    float v[8];
+    if (e < E) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(w + (size_t)e * D + d));
+      const float4 b = __ldg(reinterpret_cast<const float4*>(w + (size_t)e * D + d + 4));
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    }
+    uint4 hi, mid;
+    __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(&hi);
+    __nv_bfloat16* m = reinterpret_cast<__nv_bfloat16*>(&mid);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      h[i] = __float2bfloat16_rn(v[i]);
+      m[i] = __float2bfloat16_rn(v[i] - __bfloat162float(h[i]));
+      mx[i] = fmaxf(mx[i], fabsf(v[i]));
+    }
+    const size_t row_hi = (size_t)(e / kRouterRowBlock) * (2 * kRouterRowBlock) + (e % kRouterRowBlock);
+    *reinterpret_cast<uint4*>(bsplit + row_hi * D + d) = hi;
+    *reinterpret_cast<uint4*>(bsplit + (row_hi + kRouterRowBlock) * D + d) = mid;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) atomicMax(wmax_bits + d + i, __float_as_uint(mx[i]));   // |w| >= 0
+}
+
+__global__ void __launch_bounds__(32 * kRefineWarps)
+route_refine_kernel(const bf16* __restrict__ x, const float* __restrict__ w,
+                    const float* __restrict__ bias, const float* __restrict__ approx, int ld_approx,
+                    const float* __restrict__ wmax, float coef, int32_t* __restrict__ topk_idx,
+                    float* __restrict__ topk_w, int T, int D, int E, int k) {
+  extern __shared__ int refine_sm[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = blockIdx.x * kRefineWarps + warp;
+  if (t >= T) return;                          // warps are independent: no block barrier below
+  int* cidx = refine_sm + (size_t)warp * 2 * E;
+  float* cval = reinterpret_cast<float*>(cidx + E);
+  const bf16* xr = x + (size_t)t * D;
+  const float* ar = approx + (size_t)t * ld_approx;
+
+  // a. S_t = sum_d |x_d| wmax_d
+  float S = 0.f;
+  for (int d0 = lane * 8; d0 < D; d0 += 256) {
+    const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr + d0));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&xv);
+    const float4 m0 = __ldg(reinterpret_cast<const float4*>(wmax + d0));
+    const float4 m1 = __ldg(reinterpret_cast<const float4*>(wmax + d0 + 4));
+    const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      S = fmaf(fabsf(f.x), mm[2 * i], S);
+      S = fmaf(fabsf(f.y), mm[2 * i + 1], S);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+
+  // b. the k-th largest approximate logit (+ bias) and the candidate set
+  uint32_t taken = 0;
+  float vk = 0.f;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int c = 0; c * 32 + lane < E; ++c) {
+      if ((taken >> c) & 1u) continue;
+      const int e = c * 32 + lane;
+      const float v = ar[e] + (bias != nullptr ? bias[e] : 0.f);
+      if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    vk = bv;
+  }
+  const float eps = coef * S * 1.01f + 1e-6f * (fabsf(vk) + 1.f);
+  const float thr = vk - 2.f * eps;
+  int n = 0;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int c = 0; c * 32 < E; ++c) {
+    const int e = c * 32 + lane;
+    const bool is = e < E && ar[e] + (bias != nullptr ? bias[e] : 0.f) >= thr;
+    const unsigned m = __ballot_sync(0xffffffffu, is);
+    if (is) cidx[n + __popc(m & lt)] = e;
+    n += __popc(m);
+  }
+  __syncwarp();
+
+  // c. exact logits of the candidates, four at a time
+  for (int i0 = 0; i0 < n; i0 += 4) {
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    int ce[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) ce[q] = i0 + q < n ? cidx[i0 + q] : -1;
+    for (int d0 = lane * 8; d0 < D; d0 += 256) {
+      const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xr + d0));
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&xv);
+      float xf[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        xf[2 * i] = f.x; xf[2 * i + 1] = f.y;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (ce[q] < 0) continue;
+        const float* wr = w + (size_t)ce[q] * D + d0;
+        const float4 w0 = __ldg(reinterpret_cast<const float4*>(wr));
+        const float4 w1 = __ldg(reinterpret_cast<const float4*>(wr + 4));
+        float p = xf[0] * w0.x;
+        p = fmaf(xf[1], w0.y, p);
+        p = fmaf(xf[2], w0.z, p);
+        p = fmaf(xf[3], w0.w, p);
+        p = fmaf(xf[4], w1.x, p);
+        p = fmaf(xf[5], w1.y, p);
+        p = fmaf(xf[6], w1.z, p);
+        p = fmaf(xf[7], w1.w, p);
+        acc[q] += (double)p;
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], o);
+    if (lane == 0) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (ce[q] < 0) continue;
+        float l = (float)acc[q];
+        if (bias != nullptr) l = l + bias[ce[q]];
+        cval[i0 + q] = l;
+      }
+    }
+  }
+  __syncwarp();
+
+  // d. exact top-k among the candidates (logit descending, ties to the lower index)
+  taken = 0;
+  int my_idx = 0;
+  float my_val = 0.f, top = 0.f;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff, bs = -1;
+    for (int c = 0; c * 32 + lane < n; ++c) {
+      if ((taken >> c) & 1u) continue;
+      const int s = c * 32 + lane;
+      const float v = cval[s];
+      const int e = cidx[s];
+      if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; bs = s; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      const int os = __shfl_xor_sync(0xffffffffu, bs, o);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; bs = os; }
+    }
+    if ((bs & 31) == lane) taken |= 1u << (bs >> 5);
+    if (lane == j) { my_idx = bi; my_val = bv; }
+    if (j == 0) top = bv;
+  }
+  // e. renormalised weights over the top-k
+  const float num = (lane < k) ? expf(my_val - top) : 0.f;
+  float den = num;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  if (lane < k) {
+    topk_idx[(size_t)t * k + lane] = my_idx;
+    topk_w[(size_t)t * k + lane] = num / den;
+  }
+}
+
+cudaError_t launch_route_tc(const moe_config& c, const bf16* x, const float* w, const float* bias,
+                            const RouterScratch& rs, int32_t* topk_idx, float* topk_w,
+                            cudaStream_t s) {
+  const int Epad = (c.E + kRouterRowBlock - 1) / kRouterRowBlock * kRouterRowBlock;
+  cudaError_t err = cudaMemsetAsync(rs.wmax, 0, (size_t)c.D * sizeof(float), s);
+  if (err != cudaSuccess) return err;
+  dim3 sgrid((c.D / 8 + 127) / 128, (Epad + 15) / 16);
+  router_split_kernel<<<sgrid, 128, 0, s>>>(w, c.E, Epad, c.D, rs.bsplit,
+                                            reinterpret_cast<unsigned*>(rs.wmax));
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  GemmProblem g;
+  memset(&g, 0, sizeof(g));
+  g.A = x; g.a_rows = c.T;
+  g.B = rs.bsplit; g.G = 1;
+  g.N = 2 * Epad; g.K = c.D;
+  g.group_offsets = nullptr; g.mt_start = nullptr; g.dense_rows = c.T;
+  g.tile_n = 256;
+  g.pair = rs.pair;
+  const int tm = g.pair ? 2 * kTileM : kTileM;
+  g.max_tiles = ((int64_t)(c.T + tm - 1) / tm) * (2 * Epad / 256);
+  g.outf = rs.approx; g.ldo = Epad;
+  g.epi = EPI_PAIRSUM_F32;
+  g.status = rs.status;
+  err = launch_grouped_gemm(g, s);
+  if (err != cudaSuccess) return err;
+  // every approximate logit is within coef * S_t of the exact one (see above)
+  const float coef = (float)(4.0 * (c.D / 16 + 2) * 0x1p-23 + 0x1p-17);
+  const size_t smem = (size_t)kRefineWarps * 2 * c.E * sizeof(int);
+  route_refine_kernel<<<(c.T + kRefineWarps - 1) / kRefineWarps, 32 * kRefineWarps, smem, s>>>(
+      x, w, bias, rs.approx, Epad, rs.wmax, coef, topk_idx, topk_w, c.T, c.D, c.E, c.top_k);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_route(const moe_config& c, const void* x, const float* w_router,
                          const float* bias, float* logits, bool keep_logits, int32_t* topk_idx,
-                         float* topk_w, cudaStream_t s) {
+                         float* topk_w, const RouterScratch& rs, cudaStream_t s) {
   if (c.x_dtype == MOE_DT_F32)
     return launch_route_t(c, static_cast<const float*>(x), w_router, bias, logits, keep_logits,
                           topk_idx, topk_w, s);
+  // bf16 x with renormalised weights and no logits to return, too many experts for the
+  // fused shared-memory router: tensor-core filter and exact refine (MOE_ROUTER_TC=0
+  // selects the SIMT paths, which compute every logit exactly)
+  const char* env = getenv("MOE_ROUTER_TC");
+  const bool tc_ok = !(env && env[0] == '0');
+  const bool few = c.E <= 32 && (size_t)c.E * c.D * sizeof(float) <= kSmallRouterSmem;
+  if (tc_ok && !few && c.renormalize && !keep_logits && rs.bsplit != nullptr)
+    return launch_route_tc(c, static_cast<const bf16*>(x), w_router, bias, rs, topk_idx, topk_w, s);
   return launch_route_t(c, static_cast<const bf16*>(x), w_router, bias, logits, keep_logits,
                         topk_idx, topk_w, s);
 }

@@ -29,7 +29,7 @@ def up_weights(wl, inp):
     return inp["w_gate_up"] if wl.act == "swiglu" else inp["w1"]
 
 
-def make_layer(wl, inp, keep_logits=True):
+def make_layer(wl, inp, keep_logits=False):
     return M.MoELayer(D=wl.D, E=wl.E, ep_size=wl.ep_size, top_k=wl.top_k, F=wl.F,
                       w_router=inp["w_router"], w_gate_up=up_weights(wl, inp), w_down=inp["w_down"],
                       expert_bias=inp["bias"], ws_gate_up=inp["ws_gate_up"], ws_down=inp["ws_down"],

@@ -79,7 +79,7 @@ def test_ties_go_to_the_lower_index():
     inp = W.make_inputs(wl, device="cuda")
     wr = inp["w_router"]
     wr[6] = wr[1]           # experts 1 and 6 always tie exactly on the device
-    layer = make_layer(wl, inp)
+    layer = make_layer(wl, inp, keep_logits=True)
     layer.forward(inp["x"])
     torch.cuda.synchronize()
     idx = layer.buf["topk_idx"].cpu().numpy()
@@ -180,3 +180,25 @@ def test_cta_pair_and_single_cta_gemm_agree(T, monkeypatch):
         assert_layer_close(f64(o), res["out"], f64(inp["x"]))
     d = (outs[0].float() - outs[1].float()).abs().max().item()
     assert d <= 2 ** -6 * outs[1].float().abs().max().item()
+
+
+@pytest.mark.parametrize("E,k", [(8, 2), (64, 6), (256, 8)])
+def test_ties_on_the_tensor_core_router(E, k):
+    """Exact ties through the filter-and-refine path: duplicated router rows give
+    identical exact logits, and the lower index must come first."""
+    wl = BASE.with_(T=300, D=256, E=E, ep_size=8 if E % 8 == 0 else 1, top_k=k, F=128)
+    inp = W.make_inputs(wl, device="cuda")
+    wr = inp["w_router"]
+    wr[E - 1] = wr[0]
+    wr[E // 2] = wr[1]
+    layer = make_layer(wl, inp)                # no logits returned: tensor-core router
+    layer.forward(inp["x"])
+    torch.cuda.synchronize()
+    idx = layer.buf["topk_idx"].cpu().numpy()
+    for a_, b_ in ((0, E - 1), (1, E // 2)):
+        for row in idx:
+            r = row.tolist()
+            if b_ in r:
+                assert a_ in r and r.index(a_) < r.index(b_)
+    ref = oracle_route(wl, inp)
+    compare_routing(idx, layer.buf["topk_w"].cpu().numpy(), ref)

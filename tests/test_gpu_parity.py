@@ -45,14 +45,22 @@ def _preprocess_on_gpu(ctx, idx_np):
 def test_route_stage(ctx):
     wl, inp, layer, ref = ctx["wl"], ctx["inp"], ctx["layer"], ctx["ref"]
     b = layer.allocate(wl.T)
-    M.moe_route(layer.config(wl.T), inp["x"], inp["w_router"], inp["bias"], b["logits"],
-                b["topk_idx"], b["topk_w"], b["workspace"])
+    cfg = layer.config(wl.T)
+    # with logits returned: every logit computed exactly on the SIMT path
+    M.moe_route(cfg, inp["x"], inp["w_router"], inp["bias"], b["logits"], b["topk_idx"],
+                b["topk_w"], b["workspace"])
     torch.cuda.synchronize()
     lg = b["logits"].cpu().numpy()
     # fp32 logits: the dot product rounded once, to within a few fp32 ulps
     assert np.allclose(lg, ref["logits"], rtol=2e-6, atol=2e-6)
     n_exempt, n_differ = compare_routing(b["topk_idx"].cpu().numpy(), b["topk_w"].cpu().numpy(), ref)
     print(f"\n{wl.name}: near-tie tokens (gap < {GAP}): {n_exempt}, routed differently: {n_differ}")
+    # without logits (bf16 x): tensor-core filter with exact refinement of the candidates
+    idx2 = torch.empty_like(b["topk_idx"])
+    w2 = torch.empty_like(b["topk_w"])
+    M.moe_route(cfg, inp["x"], inp["w_router"], inp["bias"], None, idx2, w2, b["workspace"])
+    torch.cuda.synchronize()
+    compare_routing(idx2.cpu().numpy(), w2.cpu().numpy(), ref)
 
 
 def test_preprocess_stage(ctx):
@@ -158,6 +166,7 @@ def test_combine_stage(ctx):
 
 def test_forward_end_to_end(ctx):
     wl, inp, layer, ref, pre = ctx["wl"], ctx["inp"], ctx["layer"], ctx["ref"], ctx["pre"]
+    layer.allocate(wl.T)["logits"] = None      # the forward bench.py times: no logits returned
     out = layer.forward(inp["x"])
     torch.cuda.synchronize()
     layer.check_status()
