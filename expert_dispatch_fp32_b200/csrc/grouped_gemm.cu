@@ -33,10 +33,11 @@
 //               end belong to the next expert and are dropped).
 // The two accumulators let the epilogue of tile i overlap the MMAs of tile i+1.
 //
-// Every mbarrier wait is bounded (about 2 s by %globaltimer): on expiry the
+// Every mbarrier wait is bounded (about 2 s of SM clock cycles): on expiry the
 // kernel writes MOE_ERR_TIMEOUT to the status word, raises a CTA-wide abort flag
 // so the other roles stop waiting, frees its TMEM and returns.
 #include <stdio.h>
+#include <stdlib.h>
 
 #include "moe_internal.cuh"
 
@@ -44,8 +45,9 @@ namespace moe {
 
 namespace {
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr long long kWaitLimitCycles = 4000000000ll;   // 2 s at 2 GHz (4 s at 1 GHz)
 constexpr int kGemmThreads = 192;
+constexpr int kCtrlBytes = 512;     // barriers, tile queue, TMEM slot, abort flag
 
 struct GemmArgs {
   CUtensorMap tmap_a;
@@ -57,6 +59,8 @@ struct GemmArgs {
   float* outf;               // EPI_PAIRSUM_F32 output
   int32_t ldo;
   int32_t* status;
+  int32_t* counter;          // tile counter, zero at launch
+  int32_t l2hint;            // 1: TMA loads carry L2 evict_last (A) / evict_first (B) policies
 };
 
 // ---------------------------------------------------------------------------
@@ -86,28 +90,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
+// Same, with cluster-scope acquire (the phase was completed by arrivals that
+// release writes made from the other CTA of the cluster).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
 }
 
-// Wait for phase `parity` of `bar`; false if the wait gave up.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                       int32_t* status) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
+// Wait for phase `parity` of `bar`; false if the wait gave up.  The limit is
+// counted in SM clock cycles (clock64 is a cheap register read; %globaltimer is
+// not, and reading it on every missed first try stretched the pipeline's
+// barrier round trips enough to idle the tensor cores a quarter of the time).
+template <bool kCluster>
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                            int32_t* status) {
+  const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (clock64() - t0 > kWaitLimitCycles) {
         *abort_flag = 1;
         if (status != nullptr) atomicCAS(status, 0, (int32_t)MOE_ERR_TIMEOUT);
         return false;
       }
     }
   }
+}
+template <bool kCluster = false>
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int32_t* status) {
+  if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow<kCluster>(bar, parity, abort_flag, status);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
@@ -185,6 +206,63 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
 }
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, int v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// ---- Dynamic tile scheduler ----
+// One thread (the TMA producer of the CTA, or of the pair's leader) takes tile
+// indices in order from a global counter and posts each into a ring of kTileQ
+// shared-memory slots; every other role of the CTA (and of the peer CTA of a
+// pair, whose slot is written through the cluster window) reads the slot, then
+// arrives on the scheduler's `qempty` barrier so the slot can be reused.  A
+// posted -1 ends every role.  Taking tiles in order as CTAs become free keeps
+// tiles of very different cost (a 256-row tile next to a 128-row remainder)
+// balanced across the SMs, and makes the tiles that share a weight tile (the M
+// tiles of one expert and N block, consecutive in the order) start within a
+// fraction of a tile of each other, so that weight tile is read from HBM once.
+constexpr int kTileQ = 8;
+
+template <bool kPair>
+__device__ __forceinline__ int tq_post(int32_t* counter, int& next, int total, int qi, uint32_t qfull0,
+                                       uint32_t qempty0, volatile int* tq,
+                                       volatile int* abort_flag, int32_t* status) {
+  const int slot = qi % kTileQ;
+  const uint32_t ph = (uint32_t)(qi / kTileQ) & 1u;
+  if (!mbar_wait<true>(qempty0 + 8 * slot, ph ^ 1u, abort_flag, status)) return -2;
+  // `next` was taken one tile ahead, so the atomic's round trip overlaps the
+  // previous tile's loads instead of stalling the pipeline at the tile edge
+  int tile = next;
+  if (tile >= total) tile = -1;
+  else next = atomicAdd(counter, 1);
+  tq[slot] = tile;
+  if (kPair) st_cluster_u32(map_to_cta(smem_u32((const void*)(tq + slot)), 1), tile);
+  mbar_arrive(qfull0 + 8 * slot);
+  if (kPair) mbar_arrive_cluster(map_to_cta(qfull0 + 8 * slot, 1));
+  return tile;
+}
+
+// Consumer side.  kWarp: the whole (converged) warp calls, every lane reads, and
+// lane 0 releases the slot after a __syncwarp; otherwise one thread calls and
+// releases.  The slot is released on the scheduler's barrier at `qempty_sched`
+// (a shared::cluster address).  Returns -2 if the wait gave up.
+template <bool kWarp>
+__device__ __forceinline__ int tq_take(int qi, uint32_t qfull0, uint32_t qempty_sched,
+                                       const volatile int* tq, volatile int* abort_flag,
+                                       int32_t* status) {
+  const int slot = qi % kTileQ;
+  const uint32_t ph = (uint32_t)(qi / kTileQ) & 1u;
+  int tile = -2;
+  if (!kWarp || (threadIdx.x & 31) == 0) {      // one lane polls; the others wait in the shuffle
+    if (mbar_wait<true>(qfull0 + 8 * slot, ph, abort_flag, status)) {
+      tile = tq[slot];
+      mbar_arrive_cluster(qempty_sched + 8 * slot);
+    }
+  }
+  if (kWarp) tile = __shfl_sync(0xffffffffu, tile, 0);
+  return tile;
+}
+
 // Loads into this CTA's shared memory whose bytes complete on `leader_bar`, the
 // shared::cluster address (from mapa) of the barrier in the pair's leader CTA.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
@@ -201,6 +279,52 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap
       "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+// The same loads with an L2 cache policy (createpolicy): A rows are re-read by
+// every N block of their band (evict_last), each weight tile only by the M tiles
+// running beside it (evict_first).
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1, int c2, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair_hint(uint32_t dst, const CUtensorMap* map,
+                                                      uint32_t leader_bar, int c0, int c1, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c0), "r"(c1), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair_hint(uint32_t dst, const CUtensorMap* map,
+                                                      uint32_t leader_bar, int c0, int c1, int c2,
+                                                      uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c0), "r"(c1), "r"(c2), "l"(pol)
       : "memory");
 }
 __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
@@ -234,6 +358,15 @@ __host__ __device__ constexpr uint32_t make_idesc(int M, int N) {
          ((uint32_t)(M >> 4) << 24);
 }
 
+// Tile order: group-major; inside a group, M tiles in bands of kBandM, then N
+// block, then M tile fastest inside the band.  Tiles that run at the same time
+// share each weight tile (B) through L2, and a band's A rows (kBandM tiles of
+// rows x K) stay in L2 while every N block of the band reads them, so a group of
+// many rows (a dense shared expert, or one expert taking most tokens) reads A
+// from HBM about once instead of once per N block.  Groups of at most kBandM
+// tiles (the usual case) are plain N-major, M fastest.
+constexpr int kBandM = 8;
+
 __device__ __forceinline__ void decode_tile(int tile, const int* mt, int G, int nb, int& g,
                                             int& m, int& n) {
   int lo = 0, hi = G;                      // mt[lo]*nb <= tile < mt[hi]*nb
@@ -244,8 +377,12 @@ __device__ __forceinline__ void decode_tile(int tile, const int* mt, int G, int 
   g = lo;
   const int mtiles = mt[g + 1] - mt[g];
   const int local = tile - mt[g] * nb;
-  n = local / mtiles;
-  m = local - n * mtiles;
+  const int band = local / (kBandM * nb);
+  const int in_full = mtiles / kBandM;             // full bands
+  const int bw = band < in_full ? kBandM : mtiles - in_full * kBandM;
+  const int rem = local - band * kBandM * nb;
+  n = rem / bw;
+  m = band * kBandM + (rem - n * bw);
 }
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
@@ -271,6 +408,52 @@ __device__ __forceinline__ void store_row32_f32(float* dst, const float (&v)[32]
   for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 }
 
+// Epilogue of one output row: this thread's `tcols` TMEM columns at `tb` hold
+// accumulator values of row `row` (`valid` false: read, store nothing).
+//   EPI_SWIGLU / EPI_PAIRSUM_F32: every 128 columns are [first 64 | second 64] of
+//     64 outputs (packed gate/up or router hi/mid groups); output column
+//     col0 + 64 * group + c = silu(first) * second, or first + second in fp32.
+//   EPI_STORE / EPI_GELU: output column col0 + c = value (or its GELU).
+// tcgen05.ld is warp-collective, so every lane runs the loads.
+template <int EPI>
+__device__ __forceinline__ void epilogue_row(const GemmArgs& p, uint32_t tb, int tcols, int64_t row,
+                                             int col0, bool valid) {
+  if (EPI == EPI_SWIGLU || EPI == EPI_PAIRSUM_F32) {
+#pragma unroll 1
+    for (int c = 0; c < tcols / 2; c += 32) {
+      const int tc = (c >> 6) * 128 + (c & 63);
+      uint32_t a[32], b[32];
+      tmem_ld32(tb + tc, a);
+      tmem_ld32(tb + tc + 64, b);
+      tmem_ld_wait();
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float x = __uint_as_float(a[i]), y = __uint_as_float(b[i]);
+        v[i] = (EPI == EPI_SWIGLU) ? silu_f(x) * y : x + y;
+      }
+      if (valid) {
+        if (EPI == EPI_SWIGLU) store_row32(p.out + row * p.ldo + col0 + c, v);
+        else store_row32_f32(p.outf + row * p.ldo + col0 + c, v);
+      }
+    }
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < tcols; c += 32) {
+      uint32_t h[32];
+      tmem_ld32(tb + c, h);
+      tmem_ld_wait();
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float x = __uint_as_float(h[i]);
+        v[i] = (EPI == EPI_GELU) ? gelu_f(x) : x;
+      }
+      if (valid) store_row32(p.out + row * p.ldo + col0 + c, v);
+    }
+  }
+}
+
 template <int BN>
 struct GemmCfg {
   static constexpr int kStages = BN == 256 ? 4 : BN == 128 ? 6 : 8;
@@ -280,7 +463,7 @@ struct GemmCfg {
   static constexpr int kTmemCols = 2 * BN;
   static constexpr uint32_t kIdesc = make_idesc(kTileM, BN);
   static size_t smem_bytes(int G) {
-    return 1024 + (size_t)kStages * kStageBytes + 256 + 2 * (size_t)(G + 1) * sizeof(int);
+    return 1024 + (size_t)kStages * kStageBytes + kCtrlBytes + 2 * (size_t)(G + 1) * sizeof(int);
   }
 };
 
@@ -294,10 +477,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   uint8_t* a_smem = smem;
   uint8_t* b_smem = smem + S * C::kABytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
-  // bars: full[S], empty[S], tmem_full[2], tmem_empty[2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+  // bars: full[S], empty[S], tmem_full[2], tmem_empty[2], qfull[Q], qempty[Q]
+  volatile int* tq = reinterpret_cast<volatile int*>(bars + 2 * S + 4 + 2 * kTileQ);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(tq) + kTileQ);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* mt = reinterpret_cast<int*>(smem + S * C::kStageBytes + 256);
+  int* mt = reinterpret_cast<int*>(smem + S * C::kStageBytes + kCtrlBytes);
   const bool dense = p.group_offsets == nullptr;
   const int G = dense ? 1 : p.G;
   int* off = mt + (G + 1);
@@ -305,6 +489,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
   const uint32_t tfull0 = smem_u32(bars + 2 * S), tempty0 = smem_u32(bars + 2 * S + 2);
+  const uint32_t qfull0 = smem_u32(bars + 2 * S + 4), qempty0 = smem_u32(bars + 2 * S + 4 + kTileQ);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -314,6 +499,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     for (int i = 0; i < 2; ++i) {
       mbar_init(tfull0 + 8 * i, 1);
       mbar_init(tempty0 + 8 * i, 4);
+    }
+    for (int i = 0; i < kTileQ; ++i) {
+      mbar_init(qfull0 + 8 * i, 1);
+      mbar_init(qempty0 + 8 * i, 5);         // MMA issuer + 4 epilogue warps
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -347,12 +536,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   const int total = mt[G] * nb;
   const int ksteps = p.K / kTileK;
 
+  const uint32_t qempty_sched = map_to_cta(qempty0, 0);
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer ----------------
+      // ---------------- TMA producer (and tile scheduler) ----------------
       int stage = 0;
       uint32_t phase = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      int next = atomicAdd(p.counter, 1);
+      const uint64_t pol_a = l2_policy_evict_last(), pol_b = l2_policy_evict_first();
+      for (int qi = 0;; ++qi) {
+        const int tile = tq_post<false>(p.counter, next, total, qi, qfull0, qempty0, tq, abort_flag, p.status);
+        if (tile < 0) break;
         int g, m, n;
         decode_tile(tile, mt, G, nb, g, m, n);
         const int row0 = off[g] + m * kTileM;
@@ -361,8 +555,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
           const uint32_t fb = full0 + 8 * stage;
           mbar_arrive_expect_tx(fb, C::kStageBytes);
-          tma_load_2d(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * kTileK, row0);
-          tma_load_3d(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * kTileK, n * BN, g);
+          if (p.l2hint) {
+            tma_load_2d_hint(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * kTileK, row0, pol_a);
+            tma_load_3d_hint(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * kTileK, n * BN, g, pol_b);
+          } else {
+            tma_load_2d(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * kTileK, row0);
+            tma_load_3d(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * kTileK, n * BN, g);
+          }
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -375,7 +574,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      for (int qi = 0;; ++qi) {
+        const int tile = tq_take<false>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
+        if (tile < 0) break;
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -402,59 +603,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
     const int q = warp & 3;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    for (int qi = 0;; ++qi) {
+      const int tile = tq_take<true>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
+      if (__any_sync(0xffffffffu, tile < 0)) break;
       int g, m, n;
       decode_tile(tile, mt, G, nb, g, m, n);
       const int row0 = off[g] + m * kTileM;
       const int rows_valid = min(kTileM, off[g + 1] - row0);
-      const bool ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status);
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;     // keep the warp converged for tcgen05.ld
       tc_fence_after();
       const int r = q * 32 + lane;
       const bool valid = r < rows_valid;
-      bf16* orow = p.out + (size_t)(row0 + (valid ? r : 0)) * p.ldo;
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      if (EPI == EPI_SWIGLU) {
-#pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
-          uint32_t gr[32], ur[32];
-          tmem_ld32(tb + c, gr);
-          tmem_ld32(tb + BN / 2 + c, ur);
-          tmem_ld_wait();
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
-          if (valid) store_row32(orow + n * (BN / 2) + c, v);
-        }
-      } else if (EPI == EPI_PAIRSUM_F32) {
-        // columns [0, BN/2) and [BN/2, BN) of the tile are two parts of one value
-        float* frow = p.outf + (size_t)(row0 + (valid ? r : 0)) * p.ldo;
-#pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
-          uint32_t hr[32], lr[32];
-          tmem_ld32(tb + c, hr);
-          tmem_ld32(tb + BN / 2 + c, lr);
-          tmem_ld_wait();
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(hr[i]) + __uint_as_float(lr[i]);
-          if (valid) store_row32_f32(frow + n * (BN / 2) + c, v);
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t hr[32];
-          tmem_ld32(tb + c, hr);
-          tmem_ld_wait();
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float h = __uint_as_float(hr[i]);
-            v[i] = (EPI == EPI_GELU) ? gelu_f(h) : h;
-          }
-          if (valid) store_row32(orow + n * BN + c, v);
-        }
-      }
+      const bool paired = EPI == EPI_SWIGLU || EPI == EPI_PAIRSUM_F32;
+      epilogue_row<EPI>(p, tb, BN, (int64_t)row0 + r, paired ? n * (BN / 2) : n * BN, valid);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
@@ -481,6 +645,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
 // shared memory, and its TMEM holds accumulator rows 128 r .. 128 r + 127 (all 256
 // columns).  Per CTA and K step that is 16 KB of A + 16 KB of B for 128 x 256 x 64
 // MACs, two thirds of the operand traffic of the one-CTA 128 x 256 tile.
+// The last M tile of a group with at most 128 rows left runs as M = 128 instead
+// (each CTA holds 64 A rows and still its 128 B rows): it costs half a full tile,
+// which matters when groups hold a few hundred rows (e.g. 256 +- 18 rows per
+// expert: a second full 256-row tile for 16 spill-over rows would waste a third
+// of the tensor work).  Its accumulator uses the 2-CTA M = 128 layout: the CTA's
+// row i sits in TMEM lane i for tile columns [0, 128) and in lane 64 + i for
+// columns [128, 256), both at TMEM columns 0..127 — so each 128-column half of
+// the B tile must carry matching gate/up (or hi/mid) columns, as packed.
 //   warp 0 (both CTAs)   TMA producer: waits its own `empty` slot, loads its halves;
 //                        the bytes complete on the leader's `full` barrier, whose
 //                        expected byte count the leader posts for both CTAs.
@@ -497,8 +669,9 @@ struct PairCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;
   static constexpr uint32_t kIdesc = make_idesc(2 * kTileM, BN);
+  static constexpr uint32_t kIdescHalf = make_idesc(kTileM, BN);
   static size_t smem_bytes(int G) {
-    return 1024 + (size_t)kStages * kStageBytes + 256 + 2 * (size_t)(G + 1) * sizeof(int);
+    return 1024 + (size_t)kStages * kStageBytes + kCtrlBytes + 2 * (size_t)(G + 1) * sizeof(int);
   }
 };
 
@@ -512,9 +685,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
   uint8_t* a_smem = smem;
   uint8_t* b_smem = smem + S * C::kABytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+  // bars: full[S], empty[S], tmem_full[2], tmem_empty[2], qfull[Q], qempty[Q]
+  volatile int* tq = reinterpret_cast<volatile int*>(bars + 2 * S + 4 + 2 * kTileQ);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(tq) + kTileQ);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* mt = reinterpret_cast<int*>(smem + S * C::kStageBytes + 256);
+  int* mt = reinterpret_cast<int*>(smem + S * C::kStageBytes + kCtrlBytes);
   const bool dense = p.group_offsets == nullptr;
   const int G = dense ? 1 : p.G;
   int* off = mt + (G + 1);
@@ -524,6 +699,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
   const bool leader = rank == 0;
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
   const uint32_t tfull0 = smem_u32(bars + 2 * S), tempty0 = smem_u32(bars + 2 * S + 2);
+  const uint32_t qfull0 = smem_u32(bars + 2 * S + 4), qempty0 = smem_u32(bars + 2 * S + 4 + kTileQ);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -533,6 +709,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
     for (int i = 0; i < 2; ++i) {
       mbar_init(tfull0 + 8 * i, 1);
       mbar_init(tempty0 + 8 * i, 8);
+    }
+    for (int i = 0; i < kTileQ; ++i) {
+      mbar_init(qfull0 + 8 * i, 1);
+      // leader: MMA issuer + 4 epilogue warps; peer: producer + 4 epilogue warps
+      mbar_init(qempty0 + 8 * i, 10);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -565,26 +746,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
   const int nb = p.N / BN;
   const int total = mt[G] * nb;
   const int ksteps = p.K / kTileK;
-  const int cluster_id = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+  const uint32_t qempty_sched = map_to_cta(qempty0, 0);
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer (both CTAs) ----------------
+      // ---------------- TMA producer (both CTAs; the leader's also schedules) ----------------
       const uint32_t full0_leader = map_to_cta(full0, 0);
       int stage = 0;
       uint32_t phase = 0;
-      for (int tile = cluster_id; tile < total; tile += nclusters) {
+      int next = leader ? atomicAdd(p.counter, 1) : 0;
+      const uint64_t pol_a = l2_policy_evict_last(), pol_b = l2_policy_evict_first();
+      for (int qi = 0;; ++qi) {
+        const int tile = leader
+            ? tq_post<true>(p.counter, next, total, qi, qfull0, qempty0, tq, abort_flag, p.status)
+            : tq_take<false>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
+        if (tile < 0) break;
         int g, m, n;
         decode_tile(tile, mt, G, nb, g, m, n);
-        const int arow = off[g] + m * TM2 + (int)rank * kTileM;
+        const int base = off[g] + m * TM2;
+        const bool half = off[g + 1] - base <= kTileM;     // M = 128: 64 rows per CTA
+        const int arow = base + (int)rank * (half ? kTileM / 2 : kTileM);
         const int brow = n * BN + (int)rank * (BN / 2);
         bool ok = true;
         for (int kb = 0; kb < ksteps; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
           if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * C::kStageBytes);
           const uint32_t fb = full0_leader + 8 * stage;
-          tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * kTileK, arow);
-          tma_load_3d_pair(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * kTileK, brow, g);
+          if (p.l2hint) {
+            tma_load_2d_pair_hint(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * kTileK, arow, pol_a);
+            tma_load_3d_pair_hint(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * kTileK, brow, g, pol_b);
+          } else {
+            tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * kTileK, arow);
+            tma_load_3d_pair(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * kTileK, brow, g);
+          }
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -597,7 +791,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int tile = cluster_id; tile < total; tile += nclusters) {
+      for (int qi = 0;; ++qi) {
+        const int tile = tq_take<false>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
+        if (tile < 0) break;
+        int g, m, n;
+        decode_tile(tile, mt, G, nb, g, m, n);
+        const bool half = off[g + 1] - (off[g] + m * TM2) <= kTileM;
+        const uint32_t idesc = half ? C::kIdescHalf : C::kIdesc;
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -609,7 +809,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
           const uint64_t bd = sw128_desc(smem_u32(b_smem + stage * C::kBBytes));
 #pragma unroll
           for (int kk = 0; kk < kTileK / 16; ++kk)
-            tc_mma_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, C::kIdesc, (kb | kk) != 0);
+            tc_mma_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
           tc_commit_pair_both(empty0 + 8 * stage);
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
@@ -625,58 +825,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
     const uint32_t tempty_leader = map_to_cta(tempty0, 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = cluster_id; tile < total; tile += nclusters) {
+    for (int qi = 0;; ++qi) {
+      const int tile = tq_take<true>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
+      if (__any_sync(0xffffffffu, tile < 0)) break;
       int g, m, n;
       decode_tile(tile, mt, G, nb, g, m, n);
-      const int row0 = off[g] + m * TM2 + (int)rank * kTileM;
-      const int rows_valid = min(kTileM, off[g + 1] - row0);
-      const bool ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status);
+      const int base = off[g] + m * TM2;
+      const bool half = off[g + 1] - base <= kTileM;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const int r = q * 32 + lane;
-      const bool valid = r < rows_valid;
-      bf16* orow = p.out + (size_t)(row0 + (valid ? r : 0)) * p.ldo;
+      const bool paired = EPI == EPI_SWIGLU || EPI == EPI_PAIRSUM_F32;
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      if (EPI == EPI_SWIGLU) {
-#pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
-          uint32_t gr[32], ur[32];
-          tmem_ld32(tb + c, gr);
-          tmem_ld32(tb + BN / 2 + c, ur);
-          tmem_ld_wait();
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = silu_f(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
-          if (valid) store_row32(orow + n * (BN / 2) + c, v);
-        }
-      } else if (EPI == EPI_PAIRSUM_F32) {
-        // columns [0, BN/2) and [BN/2, BN) of the tile are two parts of one value
-        float* frow = p.outf + (size_t)(row0 + (valid ? r : 0)) * p.ldo;
-#pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
-          uint32_t hr[32], lr[32];
-          tmem_ld32(tb + c, hr);
-          tmem_ld32(tb + BN / 2 + c, lr);
-          tmem_ld_wait();
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(hr[i]) + __uint_as_float(lr[i]);
-          if (valid) store_row32_f32(frow + n * (BN / 2) + c, v);
-        }
+      if (!half) {
+        // M = 256: this CTA's 128 rows in TMEM lanes 0..127, all 256 columns
+        const int row0 = base + (int)rank * kTileM;
+        const int r = q * 32 + lane;
+        epilogue_row<EPI>(p, tb, BN, (int64_t)row0 + r, paired ? n * (BN / 2) : n * BN,
+                          r < off[g + 1] - row0);
       } else {
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t hr[32];
-          tmem_ld32(tb + c, hr);
-          tmem_ld_wait();
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float h = __uint_as_float(hr[i]);
-            v[i] = (EPI == EPI_GELU) ? gelu_f(h) : h;
-          }
-          if (valid) store_row32(orow + n * BN + c, v);
-        }
+        // M = 128: this CTA's 64 rows; lanes 0..63 hold tile columns [0, 128) and
+        // lanes 64..127 columns [128, 256), each in TMEM columns 0..127
+        const int row0 = base + (int)rank * (kTileM / 2);
+        const int r = (q & 1) * 32 + lane, ch = q >> 1;
+        epilogue_row<EPI>(p, tb, BN / 2, (int64_t)row0 + r,
+                          paired ? n * (BN / 2) + ch * (BN / 4) : n * BN + ch * (BN / 2),
+                          r < off[g + 1] - row0);
       }
       tc_fence_before();
       __syncwarp();
@@ -809,6 +984,12 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
   a.outf = p.outf;
   a.ldo = p.ldo;
   a.status = p.status;
+  a.counter = p.counter;
+  {
+    const char* env = getenv("MOE_GEMM_L2HINT");
+    a.l2hint = (env && env[0] == '1') ? 1 : 0;
+  }
+  if (p.counter == nullptr) return cudaErrorInvalidValue;
   const int64_t tiles = p.max_tiles > 0 ? p.max_tiles : 1;
   if (p.pair) {                 // 256 x 256 tiles on CTA pairs
     if (BN != 256) return cudaErrorInvalidValue;

@@ -23,6 +23,7 @@ WsLayout ws_layout(const moe_config& c) {
   L.r_split = o;      o = align256(o + 2 * Epad * (size_t)c.D * sizeof(bf16));
   L.r_wmax = o;       o = align256(o + (size_t)c.D * sizeof(float));
   L.r_approx = o;     o = align256(o + T * Epad * sizeof(float));
+  L.counters = o;     o = align256(o + 8 * sizeof(int32_t));
   L.total = o;
   return L;
 }
@@ -139,6 +140,7 @@ moe_status moe_route(const moe_config* cfg, const void* x, const float* w_router
   rs.approx = (float*)(ws + L.r_approx);
   rs.pair = !(pair_env && pair_env[0] == '0');
   rs.status = nullptr;
+  rs.counter = (int32_t*)(ws + L.counters);
   return cuda_status(launch_route(c, x, w_router, expert_bias, logits, logits_out != nullptr,
                                   topk_idx, topk_w, rs, as_stream(stream)));
 }
@@ -213,6 +215,9 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   const int32_t* mt256 = mt128 + (c.E + 1);
   const int64_t R = (int64_t)c.T * c.top_k;
   const int nup = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
+  // tile counters of the four GEMM launches below start at zero
+  int32_t* ctr = (int32_t*)(ws + W.counters);
+  if (cudaMemsetAsync(ctr + 1, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
 
   // Routed experts, gate_up (+ activation) then down, over the rank-major rows.
   GemmProblem up;
@@ -228,6 +233,7 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   up.out = (bf16*)act; up.ldo = c.F;
   up.epi = c.act == MOE_ACT_SWIGLU ? EPI_SWIGLU : EPI_GELU;
   up.status = status;
+  up.counter = ctr + 1;
   cudaError_t err = launch_grouped_gemm(up, s);
   if (err != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -241,6 +247,7 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   dn.max_tiles = (R / (dn.pair ? 2 * kTileM : kTileM) + c.E) * (int64_t)(c.D / dn.tile_n);
   dn.out = (bf16*)y_perm; dn.ldo = c.D;
   dn.epi = EPI_STORE;
+  dn.counter = ctr + 2;
   err = launch_grouped_gemm(dn, s);
   if (err != cudaSuccess || c.n_shared == 0) return cuda_status(err);
 
@@ -260,6 +267,7 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   su.out = act_s; su.ldo = Fc;
   su.epi = EPI_SWIGLU;
   su.status = status;
+  su.counter = ctr + 3;
   err = launch_grouped_gemm(su, s);
   if (err != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -273,6 +281,7 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   sd.max_tiles = ((int64_t)(c.T + tm_sd - 1) / tm_sd) * (c.D / sd.tile_n);
   sd.out = (bf16*)shared_out; sd.ldo = c.D;
   sd.epi = EPI_STORE;
+  sd.counter = ctr + 4;
   return cuda_status(launch_grouped_gemm(sd, s));
 }
 

@@ -34,6 +34,7 @@ struct WsLayout {
   size_t r_split;       // bf16 [2*Epad, D]: tensor-core router weights
   size_t r_wmax;        // fp32 [D]
   size_t r_approx;      // fp32 [T, Epad]
+  size_t counters;      // int32 [8]: GEMM tile counters (router, routed up/down, shared up/down)
   size_t total;
   int nblk;
 };
@@ -59,11 +60,12 @@ int down_tile_n(const moe_config& c);
 // ---------------------------------------------------------------------------
 // Workspace buffers of the tensor-core router (bf16 x).
 struct RouterScratch {
-  bf16* bsplit;     // [2 * Epad, D]: W_r hi / mid rows, 128-expert interleave
+  bf16* bsplit;     // [2 * Epad, D]: W_r hi / mid rows in 64-expert groups
   float* wmax;      // [D]: max_e |W_r[e, d]|
   float* approx;    // [T, Epad]: tensor-core logits (hi + mid)
   int pair;         // GEMM on CTA pairs
   int32_t* status;
+  int32_t* counter; // GEMM tile counter (zeroed by the router before its launch)
 };
 // logits: where the tiled path stores fp32 logits (caller's buffer or workspace);
 // keep_logits: the caller asked for them (the fused few-expert path then writes them).
@@ -103,6 +105,7 @@ struct GemmProblem {
   int epi; int tile_n;
   int pair;                               // 1: 256-row tiles on CTA pairs (mt_start per 256 rows)
   int32_t* status;
+  int32_t* counter;                       // device tile counter, zero when the launch starts
 };
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s);
 

@@ -6,12 +6,15 @@
 // [*, rows = K, cols = N] (n contiguous), through a 64 x 64 shared-memory tile so
 // both the read (along n) and the write (along kk) are coalesced.
 //   GU_SWIGLU   routed gate_up -> [E, 2F, D]; output column block b (256 wide)
-//               holds gate columns b*128..b*128+127 then the matching up columns,
-//               so one 128x256 accumulator tile carries both halves of SwiGLU.
+//               holds, for intermediate columns b*128 + [0, 64): gate then up, and
+//               for b*128 + [64, 128): gate then up.  Every 128-row half of a block
+//               therefore carries both factors of 64 SwiGLU outputs, so a 256-wide
+//               accumulator tile (one CTA, or a CTA pair whose CTAs each hold a
+//               128-row half of B) keeps each gate column beside its up column.
 //   TRANSPOSE   W1 [E, D, F] -> [E, F, D];  down [E, F, D] -> [E, D, F].
 //   GU_SHARED   S shared gate_up [S, D, 2Fs] -> one [2*S*Fs, D] expert whose gate
 //               (and up) columns are the S experts' gates (ups) concatenated,
-//               interleaved in 128-blocks like GU_SWIGLU.
+//               interleaved in 64-column groups like GU_SWIGLU.
 //   DOWN_SHARED S shared down [S, Fs, D] -> one [D, S*Fs] expert (rows concatenated).
 // Summing S SwiGLU experts equals one SwiGLU expert with the concatenated
 // intermediate dim, so the shared experts run as a single GEMM pair.
@@ -28,16 +31,17 @@ __device__ __forceinline__ size_t pack_src(int mode, int g, int n, int kk, int N
   switch (mode) {
     case GU_SWIGLU: {
       const int blk = n >> 8, w = n & 255;
-      const int col = (w < 128) ? blk * 128 + w : P + blk * 128 + (w - 128);
+      const int f = blk * 128 + (w >> 7) * 64 + (w & 63);     // intermediate column
+      const int col = ((w >> 6) & 1) ? P + f : f;             // up : gate
       return ((size_t)g * K + kk) * (size_t)(2 * P) + col;
     }
     case TRANSPOSE:
       return ((size_t)g * K + kk) * (size_t)N + n;
     case GU_SHARED: {
       const int blk = n >> 8, w = n & 255;
-      const int c = blk * 128 + (w & 127);      // column of the concatenated half
-      const int i = c / P;                      // shared expert
-      const int col = (w >> 7) * P + (c - i * P);
+      const int c = blk * 128 + (w >> 7) * 64 + (w & 63);   // concatenated column
+      const int i = c / P;                                  // shared expert
+      const int col = ((w >> 6) & 1) * P + (c - i * P);
       return ((size_t)i * K + kk) * (size_t)(2 * P) + col;
     }
     default: {                                  // DOWN_SHARED, input [S, Fs, D]

@@ -25,18 +25,12 @@ namespace moe {
 
 namespace {
 
-constexpr uint64_t kBarrierLimitNs = 1000000000ull;
+constexpr long long kBarrierLimitCycles = 2000000000ll;   // ~1 s at 2 GHz
 constexpr int kPreWarps = kPreThreads / 32;
-
-__device__ __forceinline__ uint64_t pre_global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
 
 // Grid-wide barrier for a cooperative launch.  bar[0] counts arrivals, bar[1] is a
 // generation the last arrival bumps; both start at zero (set on the stream before
-// the launch).  Bounded: after kBarrierLimitNs a waiting block reports
+// the launch).  Bounded: after kBarrierLimitCycles a waiting block reports
 // MOE_ERR_TIMEOUT and the kernel returns without touching the outputs further.
 __device__ bool grid_barrier(unsigned* bar, unsigned nblocks, int32_t* status) {
   __threadfence();
@@ -50,9 +44,9 @@ __device__ bool grid_barrier(unsigned* bar, unsigned nblocks, int32_t* status) {
       __threadfence();
       atomicAdd(bar + 1, 1u);
     } else {
-      const uint64_t t0 = pre_global_ns();
+      const long long t0 = clock64();
       while (*gen == g) {
-        if (pre_global_ns() - t0 > kBarrierLimitNs) {
+        if (clock64() - t0 > kBarrierLimitCycles) {
           atomicCAS(status, 0, (int)MOE_ERR_TIMEOUT);
           ok = 0;
           break;

@@ -347,8 +347,9 @@ cudaError_t launch_route_t(const moe_config& c, const XT* x, const float* w_rout
 // ---------------------------------------------------------------------------
 // 1. router_split_kernel: W_r (fp32) = hi + mid + lo with hi = bf16(W_r),
 //    mid = bf16(W_r - hi), |lo| <= 2^-18 |W_r|.  hi and mid rows are packed K-major
-//    for the grouped GEMM, interleaved per 128 experts (a 256-row block holds the
-//    hi rows then the mid rows of the same 128 experts); wmax[d] = max_e |W_r[e,d]|.
+//    for the grouped GEMM in 64-expert groups (a 256-row block holds, for experts
+//    128b + [0, 64), the hi rows then the mid rows, then the same for 128b + [64,
+//    128)), the layout the GEMM's paired epilogue reads; wmax[d] = max_e |W_r[e,d]|.
 // 2. The grouped GEMM (dense group, EPI_PAIRSUM_F32) gives approx[t,e] = x.hi + x.mid
 //    in fp32 on the tensor cores (x is bf16, so every product is exact; only the
 //    fp32 accumulation and the dropped lo part differ from the exact value).
@@ -391,9 +392,10 @@ router_split_kernel(const float* __restrict__ w, int E, int Epad, int D, bf16* _
       m[i] = __float2bfloat16_rn(v[i] - __bfloat162float(h[i]));
       mx[i] = fmaxf(mx[i], fabsf(v[i]));
     }
-    const size_t row_hi = (size_t)(e / kRouterRowBlock) * (2 * kRouterRowBlock) + (e % kRouterRowBlock);
+    const int j = e % kRouterRowBlock;
+    const size_t row_hi = (size_t)(e / kRouterRowBlock) * (2 * kRouterRowBlock) + (j / 64) * 128 + (j % 64);
     *reinterpret_cast<uint4*>(bsplit + row_hi * D + d) = hi;
-    *reinterpret_cast<uint4*>(bsplit + (row_hi + kRouterRowBlock) * D + d) = mid;
+    *reinterpret_cast<uint4*>(bsplit + (row_hi + 64) * D + d) = mid;
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) atomicMax(wmax_bits + d + i, __float_as_uint(mx[i]));   // |w| >= 0
@@ -555,6 +557,8 @@ cudaError_t launch_route_tc(const moe_config& c, const bf16* x, const float* w, 
   const int Epad = (c.E + kRouterRowBlock - 1) / kRouterRowBlock * kRouterRowBlock;
   cudaError_t err = cudaMemsetAsync(rs.wmax, 0, (size_t)c.D * sizeof(float), s);
   if (err != cudaSuccess) return err;
+  err = cudaMemsetAsync(rs.counter, 0, sizeof(int32_t), s);
+  if (err != cudaSuccess) return err;
   dim3 sgrid((c.D / 8 + 127) / 128, (Epad + 15) / 16);
   router_split_kernel<<<sgrid, 128, 0, s>>>(w, c.E, Epad, c.D, rs.bsplit,
                                             reinterpret_cast<unsigned*>(rs.wmax));
@@ -573,6 +577,7 @@ cudaError_t launch_route_tc(const moe_config& c, const bf16* x, const float* w, 
   g.outf = rs.approx; g.ldo = Epad;
   g.epi = EPI_PAIRSUM_F32;
   g.status = rs.status;
+  g.counter = rs.counter;
   err = launch_grouped_gemm(g, s);
   if (err != cudaSuccess) return err;
   // every approximate logit is within coef * S_t of the exact one (see above)

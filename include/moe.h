@@ -93,8 +93,9 @@ MOE_API size_t moe_workspace_size(const moe_config* cfg);
 MOE_API size_t moe_packed_weights_size(const moe_config* cfg);
 
 /* Repack expert weights once into the layout the grouped GEMMs read (K-major
- * tiles; for SwiGLU, gate and up columns interleaved in blocks of 128 so each
- * 256-wide output tile holds matching gate/up columns).  Not part of the forward.
+ * tiles; for SwiGLU, gate and up columns interleaved in groups of 64 so every
+ * 128-wide half of a 256-wide output tile holds matching gate/up columns).  Not
+ * part of the forward.
  *   w_gate_up  device bf16 [E, D, 2F] (SwiGLU: columns [0,F) gate, [F,2F) up)
  *              or [E, D, F] (GELU: W1)  -- "Expert Parallel (EP)", Requirements:
  *              tensor-style gate_up_proj / down_proj experts

@@ -1,6 +1,7 @@
 """GPU edge cases: ragged batches, skewed and empty experts, k = E, ties, the
 worked example's closed form, device error reporting and determinism."""
 import math
+import os
 
 import numpy as np
 import pytest
@@ -11,7 +12,7 @@ import moe_workloads as W
 import oracle
 from conftest import read_golden
 from parity_helpers import (assert_layer_close, compare_routing, f64, make_layer, oracle_layer,
-                            oracle_route)
+                            oracle_route, up_weights)
 
 pytestmark = pytest.mark.gpu
 
@@ -202,3 +203,59 @@ def test_ties_on_the_tensor_core_router(E, k):
                 assert a_ in r and r.index(a_) < r.index(b_)
     ref = oracle_route(wl, inp)
     compare_routing(idx, layer.buf["topk_w"].cpu().numpy(), ref)
+
+
+# per-expert row counts around the 128- and 256-row tile edges: empty, one row, a
+# last tile with <= 64 rows (only the first CTA of a pair holds rows), 65..128 rows
+# (both CTAs of an M = 128 pair tile), 129..255, exactly 256, and 256 + a few
+UNEVEN_COUNTS = [0, 1, 64, 65, 100, 128, 129, 200, 256, 257, 320, 384, 385, 115, 0, 3]
+
+
+@pytest.mark.parametrize("act", ["swiglu", "gelu"])
+def test_uneven_expert_tiles(act):
+    """Every routed row (and every shared-expert token) of the expert FFN stage
+    against the oracle, with hand-set expert sizes that put the last M tile of
+    each expert in every tiling case of both GEMM kernels."""
+    counts = np.array(UNEVEN_COUNTS)
+    E, T = counts.size, int(counts.sum())            # top-1: one row per token
+    shared = act == "swiglu"
+    wl = BASE.with_(T=T, D=256, E=E, ep_size=4, top_k=1, F=256, act=act,
+                    n_shared=1 if shared else 0, F_shared=256 if shared else 0)
+    inp = W.make_inputs(wl, device="cuda")
+    layer = make_layer(wl, inp)
+    b = layer.allocate(T)
+    cfg = layer.config(T)
+    # token t goes to the expert whose block of the (shuffled) assignment holds t
+    rng = np.random.default_rng(11)
+    assign = rng.permutation(np.repeat(np.arange(E), counts)).astype(np.int32)
+    idx = torch.from_numpy(assign.reshape(T, 1)).cuda()
+    b["status"].zero_()
+    M.moe_preprocess(cfg, idx, b["counts"], b["expert_offsets"], b["rank_splits"],
+                     b["rank_offsets"], b["pos"], b["src"], b["workspace"], b["status"])
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    x_perm = torch.randn((T, wl.D), generator=g, device="cuda").to(torch.bfloat16)
+    x_bf = inp["x"].to(torch.bfloat16) if shared else None
+    for flag in ("1", "0"):                          # CTA-pair kernel, then one-CTA kernel
+        os.environ["MOE_GEMM_CTA_PAIR"] = flag
+        try:
+            b["y_perm"].zero_()
+            M.moe_expert_ffn(cfg, x_perm, x_bf, b["expert_offsets"], layer.packed, b["act"],
+                             b["y_perm"], b["shared_out"], b["workspace"], b["status"])
+            torch.cuda.synchronize()
+        finally:
+            del os.environ["MOE_GEMM_CTA_PAIR"]
+        assert int(b["status"].item()) == 0
+        off = b["expert_offsets"].cpu().numpy()
+        assert np.array_equal(np.diff(off), counts)
+        wup = up_weights(wl, inp)
+        xp, yp = f64(x_perm), f64(b["y_perm"])
+        for e in range(E):
+            lo, hi = int(off[e]), int(off[e + 1])
+            if hi == lo:
+                continue
+            ref = oracle.expert_ffn(xp[lo:hi], f64(wup[e]), f64(inp["w_down"][e]), act)
+            assert_layer_close(yp[lo:hi], ref, np.zeros_like(ref), f"y_perm expert {e} ({hi - lo} rows)")
+        if shared:
+            s_ref = oracle.shared_experts(f64(x_bf), f64(inp["ws_gate_up"]), f64(inp["ws_down"]))
+            assert_layer_close(f64(b["shared_out"]), s_ref, np.zeros_like(s_ref), "shared_out")
