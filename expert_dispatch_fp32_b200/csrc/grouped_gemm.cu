@@ -60,7 +60,6 @@ struct GemmArgs {
   int32_t ldo;
   int32_t* status;
   int32_t* counter;          // tile counter, zero at launch
-  int32_t l2hint;            // 1: TMA loads carry L2 evict_last (A) / evict_first (B) policies
 };
 
 // ---------------------------------------------------------------------------
@@ -281,52 +280,6 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
-// The same loads with an L2 cache policy (createpolicy): A rows are re-read by
-// every N block of their band (evict_last), each weight tile only by the M tiles
-// running beside it (evict_first).
-__device__ __forceinline__ uint64_t l2_policy_evict_last() {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
-__device__ __forceinline__ uint64_t l2_policy_evict_first() {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
-__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                                 int c0, int c1, uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "l"(pol)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                                 int c0, int c1, int c2, uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "l"(pol)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_2d_pair_hint(uint32_t dst, const CUtensorMap* map,
-                                                      uint32_t leader_bar, int c0, int c1, uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c0), "r"(c1), "l"(pol)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_3d_pair_hint(uint32_t dst, const CUtensorMap* map,
-                                                      uint32_t leader_bar, int c0, int c1, int c2,
-                                                      uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c0), "r"(c1), "r"(c2), "l"(pol)
-      : "memory");
-}
 __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                             uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -543,7 +496,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       int stage = 0;
       uint32_t phase = 0;
       int next = atomicAdd(p.counter, 1);
-      const uint64_t pol_a = l2_policy_evict_last(), pol_b = l2_policy_evict_first();
       for (int qi = 0;; ++qi) {
         const int tile = tq_post<false>(p.counter, next, total, qi, qfull0, qempty0, tq, abort_flag, p.status);
         if (tile < 0) break;
@@ -555,13 +507,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
           const uint32_t fb = full0 + 8 * stage;
           mbar_arrive_expect_tx(fb, C::kStageBytes);
-          if (p.l2hint) {
-            tma_load_2d_hint(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * kTileK, row0, pol_a);
-            tma_load_3d_hint(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * kTileK, n * BN, g, pol_b);
-          } else {
-            tma_load_2d(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * kTileK, row0);
-            tma_load_3d(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * kTileK, n * BN, g);
-          }
+          tma_load_2d(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * kTileK, row0);
+          tma_load_3d(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * kTileK, n * BN, g);
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -755,7 +702,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
       int stage = 0;
       uint32_t phase = 0;
       int next = leader ? atomicAdd(p.counter, 1) : 0;
-      const uint64_t pol_a = l2_policy_evict_last(), pol_b = l2_policy_evict_first();
       for (int qi = 0;; ++qi) {
         const int tile = leader
             ? tq_post<true>(p.counter, next, total, qi, qfull0, qempty0, tq, abort_flag, p.status)
@@ -772,13 +718,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
           if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * C::kStageBytes);
           const uint32_t fb = full0_leader + 8 * stage;
-          if (p.l2hint) {
-            tma_load_2d_pair_hint(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * kTileK, arow, pol_a);
-            tma_load_3d_pair_hint(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * kTileK, brow, g, pol_b);
-          } else {
-            tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * kTileK, arow);
-            tma_load_3d_pair(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * kTileK, brow, g);
-          }
+          tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * kTileK, arow);
+          tma_load_3d_pair(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * kTileK, brow, g);
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -985,10 +926,6 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
   a.ldo = p.ldo;
   a.status = p.status;
   a.counter = p.counter;
-  {
-    const char* env = getenv("MOE_GEMM_L2HINT");
-    a.l2hint = (env && env[0] == '1') ? 1 : 0;
-  }
   if (p.counter == nullptr) return cudaErrorInvalidValue;
   const int64_t tiles = p.max_tiles > 0 ? p.max_tiles : 1;
   if (p.pair) {                 // 256 x 256 tiles on CTA pairs

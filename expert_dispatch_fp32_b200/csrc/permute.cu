@@ -5,18 +5,13 @@
 // Tracing a Token Through Expert Parallelism", Step 2 (each chosen expert gets a
 // copy of the token), Step 4 (weighted sum of the expert outputs) and Step 5
 // (residual add).  On one GPU the exchange is the gather itself.
-//
-// Both kernels run one warp per token over 16-byte vectors (8 bf16 or 8 fp32
-// elements), so each warp instruction touches 512 contiguous bytes of one row,
-// with several vectors in flight per lane.
 #include "moe_internal.cuh"
 
 namespace moe {
 
 namespace {
 
-constexpr int kUnroll = 4;
-constexpr int kThreads = 256;
+constexpr int kCombineThreads = 256;
 
 struct Vec8 { float v[8]; };
 
@@ -50,39 +45,25 @@ __device__ __forceinline__ void st8(float* p, const Vec8& o) {
   reinterpret_cast<float4*>(p)[1] = make_float4(o.v[4], o.v[5], o.v[6], o.v[7]);
 }
 
-// Token pre-all-to-all as a scatter in token order: warp w owns token t, reads
-// x[t, :] once (16-byte vectors, 512 contiguous bytes per warp instruction) and
-// writes the bf16 row to its k destinations x_perm[pos[t*k + j], :].  Every byte
-// of x is read from HBM once and every byte of x_perm written once.
+// Token pre-all-to-all as a scatter in token order.  Block b handles token t = b
+// (strided by the grid) and each thread one 16-byte chunk of the row: the chunk
+// of x[t, :] is read once and written, as bf16, to its k destinations
+// x_perm[pos[t*k + j], :] (a warp touches 512 contiguous bytes per store).  Every
+// byte of x is read from HBM once and every byte of x_perm written once.
 template <typename XT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(1024)
 dispatch_kernel(const XT* __restrict__ x, const int32_t* __restrict__ pos, bf16* __restrict__ x_perm,
                 int T, int D, int k, uint32_t R) {
-  const int lane = threadIdx.x & 31;
-  const int wpb = blockDim.x >> 5;
-  for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
-    const uint32_t my_pos = lane < k ? (uint32_t)__ldg(pos + (size_t)t * k + lane) : 0u;
-    const XT* xrow = x + (size_t)t * D;
-    for (int c0 = lane * 8; c0 < D; c0 += 256 * kUnroll) {
-      uint4 v[kUnroll];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int c = c0 + u * 256;
-        if (c < D) {
-          Vec8 f;
-          ld8(xrow + c, f);
-          v[u] = pack_bf16(f);
-        }
-      }
+  const int cpr = D >> 3;
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    const int32_t* pr = pos + (size_t)t * k;
+    for (int ch = threadIdx.x; ch < cpr; ch += blockDim.x) {
+      Vec8 f;
+      ld8(x + (size_t)t * D + ch * 8, f);
+      const uint4 v = pack_bf16(f);
       for (int j = 0; j < k; ++j) {
-        const uint32_t p = __shfl_sync(0xffffffffu, my_pos, j);
-        if (p >= R) continue;                    // a pair the preprocess skipped
-        bf16* dst = x_perm + (size_t)p * D;
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-          const int c = c0 + u * 256;
-          if (c < D) *reinterpret_cast<uint4*>(dst + c) = v[u];
-        }
+        const uint32_t p = (uint32_t)__ldg(pr + j);
+        if (p < R) *reinterpret_cast<uint4*>(x_perm + (size_t)p * D + ch * 8) = v;   // else skipped pair
       }
     }
   }
@@ -95,7 +76,7 @@ dispatch_kernel(const XT* __restrict__ x, const int32_t* __restrict__ pos, bf16*
 // indices are clamped to [0, R): pos is only undefined after the preprocess
 // reported an out-of-range expert, and then the output is unspecified anyway.
 template <typename XT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kCombineThreads)
 combine_kernel(const bf16* __restrict__ y_perm, const int32_t* __restrict__ pos,
                const float* __restrict__ topk_w, const XT* __restrict__ x,
                const bf16* __restrict__ shared, XT* __restrict__ out, int T, int D, int k,
@@ -141,12 +122,21 @@ combine_kernel(const bf16* __restrict__ y_perm, const int32_t* __restrict__ pos,
   }
 }
 
-int warp_grid(int T) {
-  const int wpb = kThreads / 32;
+int combine_grid(int T) {
+  const int wpb = kCombineThreads / 32;
   const int need = (T + wpb - 1) / wpb;
   const int cap = sm_count() * 8;
   return need < cap ? (need > 0 ? need : 1) : cap;
 }
+
+// Dispatch: one block per token row (strided when T exceeds the grid limit); the
+// block covers the row's D/8 chunks with up to 1024 threads.
+dim3 row_block(int D) {
+  const int cpr = D >> 3;
+  const int th = cpr < 1024 ? ((cpr + 31) / 32) * 32 : 1024;
+  return dim3(th);
+}
+dim3 row_grid(int T) { return dim3(T < 65535 ? (T > 0 ? T : 1) : 65535); }
 
 }  // namespace
 
@@ -154,10 +144,10 @@ cudaError_t launch_dispatch(const moe_config& c, const void* x, const int32_t* p
                             cudaStream_t s) {
   const uint32_t R = (uint32_t)c.T * c.top_k;
   if (c.x_dtype == MOE_DT_F32)
-    dispatch_kernel<float><<<warp_grid(c.T), kThreads, 0, s>>>(static_cast<const float*>(x), pos,
+    dispatch_kernel<float><<<row_grid(c.T), row_block(c.D), 0, s>>>(static_cast<const float*>(x), pos,
                                                                x_perm, c.T, c.D, c.top_k, R);
   else
-    dispatch_kernel<bf16><<<warp_grid(c.T), kThreads, 0, s>>>(static_cast<const bf16*>(x), pos,
+    dispatch_kernel<bf16><<<row_grid(c.T), row_block(c.D), 0, s>>>(static_cast<const bf16*>(x), pos,
                                                               x_perm, c.T, c.D, c.top_k, R);
   return cudaGetLastError();
 }
@@ -167,11 +157,11 @@ cudaError_t launch_combine(const moe_config& c, const bf16* y_perm, const int32_
                            cudaStream_t s) {
   const uint32_t R = (uint32_t)c.T * c.top_k;
   if (c.x_dtype == MOE_DT_F32)
-    combine_kernel<float><<<warp_grid(c.T), kThreads, 0, s>>>(
+    combine_kernel<float><<<combine_grid(c.T), kCombineThreads, 0, s>>>(
         y_perm, pos, topk_w, static_cast<const float*>(x), shared_out, static_cast<float*>(out),
         c.T, c.D, c.top_k, R);
   else
-    combine_kernel<bf16><<<warp_grid(c.T), kThreads, 0, s>>>(
+    combine_kernel<bf16><<<combine_grid(c.T), kCombineThreads, 0, s>>>(
         y_perm, pos, topk_w, static_cast<const bf16*>(x), shared_out, static_cast<bf16*>(out), c.T,
         c.D, c.top_k, R);
   return cudaGetLastError();

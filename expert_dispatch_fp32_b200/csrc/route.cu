@@ -30,7 +30,6 @@ namespace moe {
 
 namespace {
 
-constexpr int kRouteBM = 128;
 constexpr int kRouteBK = 32;
 constexpr int kRouteThreads = 256;
 
