@@ -62,6 +62,33 @@ struct GemmArgs {
   int32_t* counter;          // tile counter, zero at launch
 };
 
+// The CTA-pair kernel runs up to kMaxPhases GEMMs ("phases") in one persistent
+// launch: tiles are numbered phase after phase and taken in that order.  A
+// phase may depend on an earlier one (the down projection reads the activation
+// rows the gate_up phase writes): its tile waits, before its first A load, until
+// every tile of the matching 256-row band of the earlier phase has been stored.
+constexpr int kMaxPhases = 4;
+struct PhaseArgs {
+  CUtensorMap tmap_a;        // A [rows, K]
+  CUtensorMap tmap_b;        // B [G, N, K]
+  bf16* out;
+  float* outf;               // EPI_PAIRSUM_F32 output
+  int32_t ldo, N, K, epi;
+  int32_t dense_rows;        // > 0: one dense group of this many rows; 0: the expert groups
+  int32_t dep;               // phase whose band must be complete before A is read, or -1
+  int32_t signal;            // 1: the epilogue counts stored tiles per band in done[]
+  int32_t done_base;         // first done[] slot of this phase's bands (signal or dep source)
+};
+struct PairArgs {
+  PhaseArgs ph[kMaxPhases];
+  const int32_t* group_offsets;   // [G + 1] (grouped phases)
+  const int32_t* mt_start;        // [G + 1] prefix of ceil(rows / 256)
+  int32_t G, nph;
+  int32_t* status;
+  int32_t* counter;          // tile counter, zero at launch
+  int32_t* done;             // band completion counts, zero at launch
+};
+
 // ---------------------------------------------------------------------------
 // PTX wrappers
 // ---------------------------------------------------------------------------
@@ -369,8 +396,8 @@ __device__ __forceinline__ void store_row32_f32(float* dst, const float (&v)[32]
 //   EPI_STORE / EPI_GELU: output column col0 + c = value (or its GELU).
 // tcgen05.ld is warp-collective, so every lane runs the loads.
 template <int EPI>
-__device__ __forceinline__ void epilogue_row(const GemmArgs& p, uint32_t tb, int tcols, int64_t row,
-                                             int col0, bool valid) {
+__device__ __forceinline__ void epilogue_row(bf16* out, float* outf, int ldo, uint32_t tb, int tcols,
+                                             int64_t row, int col0, bool valid) {
   if (EPI == EPI_SWIGLU || EPI == EPI_PAIRSUM_F32) {
 #pragma unroll 1
     for (int c = 0; c < tcols / 2; c += 32) {
@@ -386,8 +413,8 @@ __device__ __forceinline__ void epilogue_row(const GemmArgs& p, uint32_t tb, int
         v[i] = (EPI == EPI_SWIGLU) ? silu_f(x) * y : x + y;
       }
       if (valid) {
-        if (EPI == EPI_SWIGLU) store_row32(p.out + row * p.ldo + col0 + c, v);
-        else store_row32_f32(p.outf + row * p.ldo + col0 + c, v);
+        if (EPI == EPI_SWIGLU) store_row32(out + row * ldo + col0 + c, v);
+        else store_row32_f32(outf + row * ldo + col0 + c, v);
       }
     }
   } else {
@@ -402,8 +429,19 @@ __device__ __forceinline__ void epilogue_row(const GemmArgs& p, uint32_t tb, int
         const float x = __uint_as_float(h[i]);
         v[i] = (EPI == EPI_GELU) ? gelu_f(x) : x;
       }
-      if (valid) store_row32(p.out + row * p.ldo + col0 + c, v);
+      if (valid) store_row32(out + row * ldo + col0 + c, v);
     }
+  }
+}
+
+// Runtime choice of the epilogue (the phases of one launch differ).
+__device__ __forceinline__ void epilogue_row_rt(int epi, bf16* out, float* outf, int ldo, uint32_t tb,
+                                                int tcols, int64_t row, int col0, bool valid) {
+  switch (epi) {
+    case EPI_SWIGLU: epilogue_row<EPI_SWIGLU>(out, outf, ldo, tb, tcols, row, col0, valid); break;
+    case EPI_GELU: epilogue_row<EPI_GELU>(out, outf, ldo, tb, tcols, row, col0, valid); break;
+    case EPI_PAIRSUM_F32: epilogue_row<EPI_PAIRSUM_F32>(out, outf, ldo, tb, tcols, row, col0, valid); break;
+    default: epilogue_row<EPI_STORE>(out, outf, ldo, tb, tcols, row, col0, valid); break;
   }
 }
 
@@ -565,7 +603,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       const bool valid = r < rows_valid;
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       const bool paired = EPI == EPI_SWIGLU || EPI == EPI_PAIRSUM_F32;
-      epilogue_row<EPI>(p, tb, BN, (int64_t)row0 + r, paired ? n * (BN / 2) : n * BN, valid);
+      epilogue_row<EPI>(p.out, p.outf, p.ldo, tb, BN, (int64_t)row0 + r, paired ? n * (BN / 2) : n * BN, valid);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
@@ -622,8 +660,47 @@ struct PairCfg {
   }
 };
 
-template <int EPI>
-__global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(const __grid_constant__ GemmArgs p) {
+// Where a pair tile sits: phase, group, M tile (256 rows), N block, its first row,
+// the group's end row, and its band slot (the M tile's index across the phase).
+struct PairTile {
+  int ph, g, m, n, base, end, band;
+};
+
+__device__ __forceinline__ void decode_pair_tile(int tile, const int* pstart, int nph, const int* mt,
+                                                 const int* off, int G, const int* dmt,
+                                                 const int* doff, const PairArgs& p, PairTile& t) {
+  int ph = 0;
+  while (ph + 1 < nph && tile >= pstart[ph + 1]) ++ph;
+  const int nb = p.ph[ph].N / PairCfg::BN;
+  const bool dense = p.ph[ph].dense_rows > 0;
+  const int* pm = dense ? dmt + 2 * ph : mt;
+  const int* po = dense ? doff + 2 * ph : off;
+  decode_tile(tile - pstart[ph], pm, dense ? 1 : G, nb, t.g, t.m, t.n);
+  t.ph = ph;
+  t.base = po[t.g] + t.m * 2 * kTileM;
+  t.end = po[t.g + 1];
+  t.band = pm[t.g] + t.m;
+}
+
+// Bounded wait (cycle count) until *cnt >= need, read with acquire semantics.
+__device__ __noinline__ bool wait_count(const int32_t* cnt, int need, volatile int* abort_flag,
+                                        int32_t* status) {
+  const long long t0 = clock64();
+  for (uint32_t it = 0;; ++it) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+    if (v >= need) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      *abort_flag = 1;
+      if (status != nullptr) atomicCAS(status, 0, (int32_t)MOE_ERR_TIMEOUT);
+      return false;
+    }
+    __nanosleep(64);
+  }
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(const __grid_constant__ PairArgs p) {
   using C = PairCfg;
   constexpr int S = C::kStages, BN = C::BN, TM2 = 2 * kTileM;
   extern __shared__ uint8_t smem_raw[];
@@ -636,10 +713,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
   volatile int* tq = reinterpret_cast<volatile int*>(bars + 2 * S + 4 + 2 * kTileQ);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(tq) + kTileQ);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* pstart = reinterpret_cast<int*>(tmem_slot + 2);          // [kMaxPhases + 1]
+  int* dmt = pstart + kMaxPhases + 1;                           // [kMaxPhases][2]
+  int* doff = dmt + 2 * kMaxPhases;                             // [kMaxPhases][2]
   int* mt = reinterpret_cast<int*>(smem + S * C::kStageBytes + kCtrlBytes);
-  const bool dense = p.group_offsets == nullptr;
-  const int G = dense ? 1 : p.G;
+  const int G = p.G > 0 ? p.G : 1;
   int* off = mt + (G + 1);
+  const int nph = p.nph;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -664,15 +744,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    prefetch_tmap(&p.tmap_a);
-    prefetch_tmap(&p.tmap_b);
-  }
-  if (dense) {
-    if (threadIdx.x == 0) {
-      mt[0] = 0; mt[1] = (p.dense_rows + TM2 - 1) / TM2;
-      off[0] = 0; off[1] = p.dense_rows;
+    for (int ph = 0; ph < nph; ++ph) {
+      prefetch_tmap(&p.ph[ph].tmap_a);
+      prefetch_tmap(&p.ph[ph].tmap_b);
+      const int rows = p.ph[ph].dense_rows;
+      dmt[2 * ph] = 0; dmt[2 * ph + 1] = (rows + TM2 - 1) / TM2;
+      doff[2 * ph] = 0; doff[2 * ph + 1] = rows;
     }
-  } else {
+  }
+  if (p.group_offsets != nullptr) {
     for (int i = threadIdx.x; i <= G; i += blockDim.x) {
       mt[i] = p.mt_start[i];
       off[i] = p.group_offsets[i];
@@ -685,14 +765,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
+  __syncthreads();
+  if (threadIdx.x == 0) {          // tile numbering: phase after phase
+    int acc_t = 0;
+    for (int ph = 0; ph < nph; ++ph) {
+      pstart[ph] = acc_t;
+      const int mtiles = p.ph[ph].dense_rows > 0 ? dmt[2 * ph + 1] : mt[G];
+      acc_t += mtiles * (p.ph[ph].N / BN);
+    }
+    pstart[nph] = acc_t;
+  }
   tc_fence_before();
   cluster_sync();               // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-
-  const int nb = p.N / BN;
-  const int total = mt[G] * nb;
-  const int ksteps = p.K / kTileK;
+  const int total = pstart[nph];
   const uint32_t qempty_sched = map_to_cta(qempty0, 0);
 
   if (warp == 0) {
@@ -707,19 +794,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
             ? tq_post<true>(p.counter, next, total, qi, qfull0, qempty0, tq, abort_flag, p.status)
             : tq_take<false>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
         if (tile < 0) break;
-        int g, m, n;
-        decode_tile(tile, mt, G, nb, g, m, n);
-        const int base = off[g] + m * TM2;
-        const bool half = off[g + 1] - base <= kTileM;     // M = 128: 64 rows per CTA
-        const int arow = base + (int)rank * (half ? kTileM / 2 : kTileM);
-        const int brow = n * BN + (int)rank * (BN / 2);
+        PairTile t;
+        decode_pair_tile(tile, pstart, nph, mt, off, G, dmt, doff, p, t);
+        const PhaseArgs& P = p.ph[t.ph];
+        const bool half = t.end - t.base <= kTileM;     // M = 128: 64 rows per CTA
+        const int arow = t.base + (int)rank * (half ? kTileM / 2 : kTileM);
+        const int brow = t.n * BN + (int)rank * (BN / 2);
+        if (P.dep >= 0) {
+          // A rows of this band are written by phase P.dep: wait until all of its
+          // N blocks (8 epilogue warps each) are stored, then order those generic-proxy
+          // stores before this thread's TMA (async-proxy) reads
+          const PhaseArgs& Q = p.ph[P.dep];
+          if (!wait_count(p.done + Q.done_base + t.band, 8 * (Q.N / BN), abort_flag, p.status)) break;
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
+        const int ksteps = P.K / kTileK;
         bool ok = true;
         for (int kb = 0; kb < ksteps; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
           if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * C::kStageBytes);
           const uint32_t fb = full0_leader + 8 * stage;
-          tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * kTileK, arow);
-          tma_load_3d_pair(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * kTileK, brow, g);
+          tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), &P.tmap_a, fb, kb * kTileK, arow);
+          tma_load_3d_pair(smem_u32(b_smem + stage * C::kBBytes), &P.tmap_b, fb, kb * kTileK, brow,
+                           P.dense_rows > 0 ? 0 : t.g);
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -735,10 +832,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
       for (int qi = 0;; ++qi) {
         const int tile = tq_take<false>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
         if (tile < 0) break;
-        int g, m, n;
-        decode_tile(tile, mt, G, nb, g, m, n);
-        const bool half = off[g + 1] - (off[g] + m * TM2) <= kTileM;
+        PairTile t;
+        decode_pair_tile(tile, pstart, nph, mt, off, G, dmt, doff, p, t);
+        const bool half = t.end - t.base <= kTileM;
         const uint32_t idesc = half ? C::kIdescHalf : C::kIdesc;
+        const int ksteps = p.ph[t.ph].K / kTileK;
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -769,32 +867,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
     for (int qi = 0;; ++qi) {
       const int tile = tq_take<true>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
       if (__any_sync(0xffffffffu, tile < 0)) break;
-      int g, m, n;
-      decode_tile(tile, mt, G, nb, g, m, n);
-      const int base = off[g] + m * TM2;
-      const bool half = off[g + 1] - base <= kTileM;
+      PairTile t;
+      decode_pair_tile(tile, pstart, nph, mt, off, G, dmt, doff, p, t);
+      const PhaseArgs& P = p.ph[t.ph];
+      const bool half = t.end - t.base <= kTileM;
       bool ok = true;
       if (lane == 0) ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const bool paired = EPI == EPI_SWIGLU || EPI == EPI_PAIRSUM_F32;
+      const bool paired = P.epi == EPI_SWIGLU || P.epi == EPI_PAIRSUM_F32;
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       if (!half) {
         // M = 256: this CTA's 128 rows in TMEM lanes 0..127, all 256 columns
-        const int row0 = base + (int)rank * kTileM;
+        const int row0 = t.base + (int)rank * kTileM;
         const int r = q * 32 + lane;
-        epilogue_row<EPI>(p, tb, BN, (int64_t)row0 + r, paired ? n * (BN / 2) : n * BN,
-                          r < off[g + 1] - row0);
+        epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, BN, (int64_t)row0 + r,
+                        paired ? t.n * (BN / 2) : t.n * BN, r < t.end - row0);
       } else {
         // M = 128: this CTA's 64 rows; lanes 0..63 hold tile columns [0, 128) and
         // lanes 64..127 columns [128, 256), each in TMEM columns 0..127
-        const int row0 = base + (int)rank * (kTileM / 2);
+        const int row0 = t.base + (int)rank * (kTileM / 2);
         const int r = (q & 1) * 32 + lane, ch = q >> 1;
-        epilogue_row<EPI>(p, tb, BN / 2, (int64_t)row0 + r,
-                          paired ? n * (BN / 2) + ch * (BN / 4) : n * BN + ch * (BN / 2),
-                          r < off[g + 1] - row0);
+        epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, BN / 2, (int64_t)row0 + r,
+                        paired ? t.n * (BN / 2) + ch * (BN / 4) : t.n * BN + ch * (BN / 2),
+                        r < t.end - row0);
       }
       tc_fence_before();
+      if (P.signal) {
+        // count this warp's stores of the band for the phase that reads them back
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(p.done + P.done_base + t.band, 1);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader + 8 * acc);
       acc ^= 1;
@@ -858,10 +963,9 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t K, uint64_t N, uint6
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI>
-cudaError_t launch_tc_pair(const GemmArgs& a, int clusters, cudaStream_t s) {
+cudaError_t launch_tc_pair(const PairArgs& a, int clusters, cudaStream_t s) {
   const size_t smem = PairCfg::smem_bytes(a.group_offsets ? a.G : 1);
-  auto kern = grouped_gemm_pair_kernel<EPI>;
+  auto kern = grouped_gemm_pair_kernel;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg;
@@ -906,6 +1010,80 @@ int sm_count() {
   return n;
 }
 
+int64_t pair_band_bound(const GemmProblem& p) {
+  // 256-row bands of a phase: ceil(rows / 256) for a dense group; for the expert
+  // groups at most rows / 256 + G (each group adds at most one partial band)
+  if (p.group_offsets == nullptr) return (p.dense_rows + 2 * kTileM - 1) / (2 * kTileM);
+  return p.a_rows / (2 * kTileM) + p.G;
+}
+
+int64_t pair_done_slots(const GemmProblem* probs, int n) {
+  int64_t slots = 0;
+  for (int i = 0; i < n; ++i)
+    for (int j = i + 1; j < n; ++j)
+      if (probs[j].dep == i) { slots += pair_band_bound(probs[i]); break; }
+  return slots;
+}
+
+cudaError_t launch_grouped_pair(const GemmProblem* probs, int n, int32_t* counter, int32_t* done,
+                                cudaStream_t s) {
+  if (n < 1 || n > kMaxPhases || counter == nullptr) return cudaErrorInvalidValue;
+  PairArgs a;
+  memset(&a, 0, sizeof(a));
+  a.nph = n;
+  a.status = probs[0].status;
+  a.counter = counter;
+  a.done = done;
+  int64_t tiles = 0, slot = 0;
+  for (int i = 0; i < n; ++i) {
+    const GemmProblem& p = probs[i];
+    PhaseArgs& P = a.ph[i];
+    if (p.tile_n != 256 || p.N % 256 != 0 || p.K % kTileK != 0) return cudaErrorInvalidValue;
+    if (!make_map_2d(&P.tmap_a, p.A, (uint64_t)p.K, (uint64_t)p.a_rows, kTileM)) return cudaErrorInvalidValue;
+    // each CTA of a pair loads its 128-row half of the 256-row B tile
+    if (!make_map_3d(&P.tmap_b, p.B, (uint64_t)p.K, (uint64_t)p.N, (uint64_t)p.G, 128))
+      return cudaErrorInvalidValue;
+    if (p.group_offsets != nullptr) {
+      if (a.group_offsets != nullptr && (a.group_offsets != p.group_offsets || a.G != p.G))
+        return cudaErrorInvalidValue;          // grouped phases share one grouping
+      a.group_offsets = p.group_offsets;
+      a.mt_start = p.mt_start;
+      a.G = p.G;
+      P.dense_rows = 0;
+    } else {
+      if (p.dense_rows <= 0) return cudaErrorInvalidValue;
+      P.dense_rows = p.dense_rows;
+    }
+    P.out = p.out;
+    P.outf = p.outf;
+    P.ldo = p.ldo;
+    P.N = p.N;
+    P.K = p.K;
+    P.epi = p.epi;
+    P.dep = p.dep;
+    P.signal = 0;
+    P.done_base = 0;
+    if (p.dep >= 0) {
+      // the phase read back must come first, share this phase's row tiling and count its bands
+      if (p.dep >= i || done == nullptr) return cudaErrorInvalidValue;
+      const GemmProblem& q = probs[p.dep];
+      if ((q.group_offsets == nullptr) != (p.group_offsets == nullptr) ||
+          (p.group_offsets == nullptr && q.dense_rows != p.dense_rows))
+        return cudaErrorInvalidValue;
+      PhaseArgs& Q = a.ph[p.dep];
+      if (!Q.signal) {
+        Q.signal = 1;
+        Q.done_base = (int32_t)slot;
+        slot += pair_band_bound(q);
+      }
+    }
+    tiles += (p.max_tiles > 0 ? p.max_tiles : 1);
+  }
+  const int64_t pairs = sm_count() / 2;
+  const int clusters = (int)(tiles < pairs ? tiles : pairs);
+  return launch_tc_pair(a, clusters, s);
+}
+
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
   GemmArgs a;
   memset(&a, 0, sizeof(a));
@@ -928,14 +1106,10 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
   a.counter = p.counter;
   if (p.counter == nullptr) return cudaErrorInvalidValue;
   const int64_t tiles = p.max_tiles > 0 ? p.max_tiles : 1;
-  if (p.pair) {                 // 256 x 256 tiles on CTA pairs
-    if (BN != 256) return cudaErrorInvalidValue;
-    const int64_t pairs = sm_count() / 2;
-    const int clusters = (int)(tiles < pairs ? tiles : pairs);
-    if (p.epi == EPI_SWIGLU) return launch_tc_pair<EPI_SWIGLU>(a, clusters, s);
-    if (p.epi == EPI_GELU) return launch_tc_pair<EPI_GELU>(a, clusters, s);
-    if (p.epi == EPI_PAIRSUM_F32) return launch_tc_pair<EPI_PAIRSUM_F32>(a, clusters, s);
-    return launch_tc_pair<EPI_STORE>(a, clusters, s);
+  if (p.pair) {                 // 256 x 256 tiles on CTA pairs: a one-phase pair launch
+    GemmProblem q = p;
+    q.dep = -1;
+    return launch_grouped_pair(&q, 1, p.counter, nullptr, s);
   }
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   if (BN == 256) {

@@ -23,7 +23,10 @@ WsLayout ws_layout(const moe_config& c) {
   L.r_split = o;      o = align256(o + 2 * Epad * (size_t)c.D * sizeof(bf16));
   L.r_wmax = o;       o = align256(o + (size_t)c.D * sizeof(float));
   L.r_approx = o;     o = align256(o + T * Epad * sizeof(float));
-  L.counters = o;     o = align256(o + 8 * sizeof(int32_t));
+  // band counts of the fused FFN launch: routed gate_up bands (<= R/256 + E) and the
+  // shared gate_up bands (ceil(T/256))
+  const size_t done_slots = (size_t)(T * c.top_k) / 256 + E + (T + 255) / 256 + 2;
+  L.counters = o;     o = align256(o + (8 + done_slots) * sizeof(int32_t));
   L.total = o;
   return L;
 }
@@ -215,9 +218,7 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   const int32_t* mt256 = mt128 + (c.E + 1);
   const int64_t R = (int64_t)c.T * c.top_k;
   const int nup = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
-  // tile counters of the four GEMM launches below start at zero
   int32_t* ctr = (int32_t*)(ws + W.counters);
-  if (cudaMemsetAsync(ctr + 1, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
 
   // Routed experts, gate_up (+ activation) then down, over the rank-major rows.
   GemmProblem up;
@@ -234,8 +235,7 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   up.epi = c.act == MOE_ACT_SWIGLU ? EPI_SWIGLU : EPI_GELU;
   up.status = status;
   up.counter = ctr + 1;
-  cudaError_t err = launch_grouped_gemm(up, s);
-  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  up.dep = -1;
 
   GemmProblem dn = up;
   dn.A = (const bf16*)act; dn.a_rows = R;
@@ -248,40 +248,69 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   dn.out = (bf16*)y_perm; dn.ldo = c.D;
   dn.epi = EPI_STORE;
   dn.counter = ctr + 2;
-  err = launch_grouped_gemm(dn, s);
-  if (err != cudaSuccess || c.n_shared == 0) return cuda_status(err);
 
   // Shared experts: one dense SwiGLU expert of intermediate S*Fs over all tokens.
   const int Fc = c.n_shared * c.F_shared;
   bf16* act_s = (bf16*)(ws + W.act_shared);
-  GemmProblem su;
+  GemmProblem su, sd;
   memset(&su, 0, sizeof(su));
-  su.A = (const bf16*)x; su.a_rows = c.T;
-  su.B = (const bf16*)(pk + P.ws_up); su.G = 1;
-  su.N = 2 * Fc; su.K = c.D;
-  su.group_offsets = nullptr; su.mt_start = nullptr; su.dense_rows = c.T;
-  su.tile_n = 256;
-  su.pair = use_pair;
-  const int tm_s = su.pair ? 2 * kTileM : kTileM;
-  su.max_tiles = ((int64_t)(c.T + tm_s - 1) / tm_s) * (2 * Fc / 256);
-  su.out = act_s; su.ldo = Fc;
-  su.epi = EPI_SWIGLU;
-  su.status = status;
-  su.counter = ctr + 3;
+  if (c.n_shared > 0) {
+    su.A = (const bf16*)x; su.a_rows = c.T;
+    su.B = (const bf16*)(pk + P.ws_up); su.G = 1;
+    su.N = 2 * Fc; su.K = c.D;
+    su.group_offsets = nullptr; su.mt_start = nullptr; su.dense_rows = c.T;
+    su.tile_n = 256;
+    su.pair = use_pair;
+    const int tm_s = su.pair ? 2 * kTileM : kTileM;
+    su.max_tiles = ((int64_t)(c.T + tm_s - 1) / tm_s) * (2 * Fc / 256);
+    su.out = act_s; su.ldo = Fc;
+    su.epi = EPI_SWIGLU;
+    su.status = status;
+    su.counter = ctr + 3;
+    su.dep = -1;
+
+    sd = su;
+    sd.A = act_s; sd.a_rows = c.T;
+    sd.B = (const bf16*)(pk + P.ws_down);
+    sd.N = c.D; sd.K = Fc;
+    sd.tile_n = down_tile_n(c);
+    sd.pair = use_pair && sd.tile_n == 256;
+    const int tm_sd = sd.pair ? 2 * kTileM : kTileM;
+    sd.max_tiles = ((int64_t)(c.T + tm_sd - 1) / tm_sd) * (c.D / sd.tile_n);
+    sd.out = (bf16*)shared_out; sd.ldo = c.D;
+    sd.epi = EPI_STORE;
+    sd.counter = ctr + 4;
+  }
+
+  // MOE_GEMM_FUSED=0 selects one launch per GEMM (read at each call; for comparison)
+  const char* fused_env = getenv("MOE_GEMM_FUSED");
+  const bool fused = !(fused_env && fused_env[0] == '0');
+  if (fused && up.pair && dn.pair && (c.n_shared == 0 || sd.pair)) {
+    // One persistent launch: routed gate_up, shared gate_up, routed down, shared down.
+    // Each down tile waits only for the gate_up band it reads, so the down phase
+    // starts while the last gate_up tiles finish (no launch gap, one tail).
+    GemmProblem ph[4];
+    int n = 0;
+    ph[n++] = up;
+    if (c.n_shared > 0) ph[n++] = su;
+    ph[n] = dn; ph[n].dep = 0; ++n;
+    if (c.n_shared > 0) { ph[n] = sd; ph[n].dep = 1; ++n; }
+    const int64_t slots = pair_done_slots(ph, n);
+    if (cudaMemsetAsync(ctr, 0, (size_t)(8 + slots) * sizeof(int32_t), s) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return cuda_status(launch_grouped_pair(ph, n, ctr, ctr + 8, s));
+  }
+
+  // Otherwise one launch per GEMM, each with its own tile counter.
+  if (cudaMemsetAsync(ctr + 1, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  dn.dep = -1;
+  sd.dep = -1;
+  cudaError_t err = launch_grouped_gemm(up, s);
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  err = launch_grouped_gemm(dn, s);
+  if (err != cudaSuccess || c.n_shared == 0) return cuda_status(err);
   err = launch_grouped_gemm(su, s);
   if (err != cudaSuccess) return MOE_ERR_CUDA;
-
-  GemmProblem sd = su;
-  sd.A = act_s; sd.a_rows = c.T;
-  sd.B = (const bf16*)(pk + P.ws_down);
-  sd.N = c.D; sd.K = Fc;
-  sd.tile_n = down_tile_n(c);
-  sd.pair = use_pair && sd.tile_n == 256;
-  const int tm_sd = sd.pair ? 2 * kTileM : kTileM;
-  sd.max_tiles = ((int64_t)(c.T + tm_sd - 1) / tm_sd) * (c.D / sd.tile_n);
-  sd.out = (bf16*)shared_out; sd.ldo = c.D;
-  sd.epi = EPI_STORE;
-  sd.counter = ctr + 4;
   return cuda_status(launch_grouped_gemm(sd, s));
 }
 

@@ -34,7 +34,8 @@ struct WsLayout {
   size_t r_split;       // bf16 [2*Epad, D]: tensor-core router weights
   size_t r_wmax;        // fp32 [D]
   size_t r_approx;      // fp32 [T, Epad]
-  size_t counters;      // int32 [8]: GEMM tile counters (router, routed up/down, shared up/down)
+  size_t counters;      // int32 [8]: GEMM tile counters (router, routed up/down, shared up/down),
+                        // followed directly by the fused FFN launch's band counts int32 [done_slots]
   size_t total;
   int nblk;
 };
@@ -106,7 +107,16 @@ struct GemmProblem {
   int pair;                               // 1: 256-row tiles on CTA pairs (mt_start per 256 rows)
   int32_t* status;
   int32_t* counter;                       // device tile counter, zero when the launch starts
+  int dep;                                // launch_grouped_pair: index of the phase whose output
+                                          // rows this phase reads as A, or -1
 };
+// Up to 4 GEMMs (all 256-wide tiles) in one persistent CTA-pair launch, tiles taken
+// phase after phase; probs[i].dep = j (j < i) makes phase i read phase j's output
+// rows only after each 256-row band of them is stored.  `counter` (one int) and
+// `done` (pair_done_slots ints) must be zero when the launch starts.
+cudaError_t launch_grouped_pair(const GemmProblem* probs, int n, int32_t* counter, int32_t* done,
+                                cudaStream_t s);
+int64_t pair_done_slots(const GemmProblem* probs, int n);
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s);
 
 int sm_count();

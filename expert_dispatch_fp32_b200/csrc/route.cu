@@ -577,6 +577,7 @@ cudaError_t launch_route_tc(const moe_config& c, const bf16* x, const float* w, 
   g.epi = EPI_PAIRSUM_F32;
   g.status = rs.status;
   g.counter = rs.counter;
+  g.dep = -1;
   err = launch_grouped_gemm(g, s);
   if (err != cudaSuccess) return err;
   // every approximate logit is within coef * S_t of the exact one (see above)

@@ -259,3 +259,21 @@ def test_uneven_expert_tiles(act):
         if shared:
             s_ref = oracle.shared_experts(f64(x_bf), f64(inp["ws_gate_up"]), f64(inp["ws_down"]))
             assert_layer_close(f64(b["shared_out"]), s_ref, np.zeros_like(s_ref), "shared_out")
+
+
+def test_fused_and_separate_ffn_launches_agree(monkeypatch):
+    """The single persistent launch (gate_up, shared gate_up, down, shared down with
+    band dependencies) gives the same bits as one launch per GEMM, and both match
+    the oracle (ragged expert ends and a partial last band of the shared expert)."""
+    wl = BASE.with_(T=700, D=512, E=16, ep_size=4, top_k=3, F=512, n_shared=2, F_shared=256, seed=9)
+    inp = W.make_inputs(wl, device="cuda")
+    outs = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("MOE_GEMM_FUSED", flag)
+        layer = make_layer(wl, inp)
+        outs.append(layer.forward(inp["x"]).clone())
+        torch.cuda.synchronize()
+        layer.check_status()
+    assert torch.equal(outs[0], outs[1])
+    res = oracle_layer(wl, inp)
+    assert_layer_close(f64(outs[0]), res["out"], f64(inp["x"]))
