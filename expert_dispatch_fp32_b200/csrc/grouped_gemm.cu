@@ -69,7 +69,8 @@ struct GemmArgs {
 // every tile of the matching 256-row band of the earlier phase has been stored.
 constexpr int kMaxPhases = 4;
 struct PhaseArgs {
-  CUtensorMap tmap_a;        // A [rows, K]
+  CUtensorMap tmap_a;        // A [rows, K], 128-row box
+  CUtensorMap tmap_a64;      // the same A with a 64-row box (M = 128 remainder tiles)
   CUtensorMap tmap_b;        // B [G, N, K]
   bf16* out;
   float* outf;               // EPI_PAIRSUM_F32 output
@@ -746,6 +747,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     for (int ph = 0; ph < nph; ++ph) {
       prefetch_tmap(&p.ph[ph].tmap_a);
+      prefetch_tmap(&p.ph[ph].tmap_a64);
       prefetch_tmap(&p.ph[ph].tmap_b);
       const int rows = p.ph[ph].dense_rows;
       dmt[2 * ph] = 0; dmt[2 * ph + 1] = (rows + TM2 - 1) / TM2;
@@ -799,6 +801,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         const PhaseArgs& P = p.ph[t.ph];
         const bool half = t.end - t.base <= kTileM;     // M = 128: 64 rows per CTA
         const int arow = t.base + (int)rank * (half ? kTileM / 2 : kTileM);
+        const CUtensorMap* amap = half ? &P.tmap_a64 : &P.tmap_a;
+        const uint32_t stage_tx = 2u * (uint32_t)((half ? C::kABytes / 2 : C::kABytes) + C::kBBytes);
         const int brow = t.n * BN + (int)rank * (BN / 2);
         if (P.dep >= 0) {
           // A rows of this band are written by phase P.dep: wait until all of its
@@ -812,9 +816,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         bool ok = true;
         for (int kb = 0; kb < ksteps; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
-          if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, 2 * C::kStageBytes);
+          if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, stage_tx);
           const uint32_t fb = full0_leader + 8 * stage;
-          tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), &P.tmap_a, fb, kb * kTileK, arow);
+          tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), amap, fb, kb * kTileK, arow);
           tma_load_3d_pair(smem_u32(b_smem + stage * C::kBBytes), &P.tmap_b, fb, kb * kTileK, brow,
                            P.dense_rows > 0 ? 0 : t.g);
           if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -1039,7 +1043,9 @@ cudaError_t launch_grouped_pair(const GemmProblem* probs, int n, int32_t* counte
     const GemmProblem& p = probs[i];
     PhaseArgs& P = a.ph[i];
     if (p.tile_n != 256 || p.N % 256 != 0 || p.K % kTileK != 0) return cudaErrorInvalidValue;
-    if (!make_map_2d(&P.tmap_a, p.A, (uint64_t)p.K, (uint64_t)p.a_rows, kTileM)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&P.tmap_a, p.A, (uint64_t)p.K, (uint64_t)p.a_rows, kTileM) ||
+        !make_map_2d(&P.tmap_a64, p.A, (uint64_t)p.K, (uint64_t)p.a_rows, kTileM / 2))
+      return cudaErrorInvalidValue;
     // each CTA of a pair loads its 128-row half of the 256-row B tile
     if (!make_map_3d(&P.tmap_b, p.B, (uint64_t)p.K, (uint64_t)p.N, (uint64_t)p.G, 128))
       return cudaErrorInvalidValue;
