@@ -71,6 +71,7 @@ constexpr int kMaxPhases = 4;
 struct PhaseArgs {
   CUtensorMap tmap_a;        // A [rows, K], 128-row box
   CUtensorMap tmap_a64;      // the same A with a 64-row box (M = 128 remainder tiles)
+  CUtensorMap tmap_a32;      // the same A with a 32-row box (skinny remainder tiles)
   CUtensorMap tmap_b;        // B [G, N, K]
   bf16* out;
   float* outf;               // EPI_PAIRSUM_F32 output
@@ -85,6 +86,7 @@ struct PairArgs {
   const int32_t* group_offsets;   // [G + 1] (grouped phases)
   const int32_t* mt_start;        // [G + 1] prefix of ceil(rows / 256)
   int32_t G, nph;
+  int32_t skinny;            // 1: remainders of <= 64 rows run as skinny (weights-as-M) tiles
   int32_t* status;
   int32_t* counter;          // tile counter, zero at launch
   int32_t* done;             // band completion counts, zero at launch
@@ -667,6 +669,25 @@ struct PairTile {
   int ph, g, m, n, base, end, band;
 };
 
+// Shape of a pair tile from the rows it has left: > 128 rows: M = 256 (128 rows per
+// CTA); 65..128 rows: M = 128 (64 rows per CTA).  A group of at most 64 rows in all
+// (a decode-sized batch) runs skinny when enabled: the weights take the M side
+// (M = 128: 64 weight rows per CTA, twice) and the rows the N side, N = rows
+// rounded up to 32 (N/2 rows per CTA; a multiple of 32 is a valid N for every
+// 2-CTA MMA shape), for 2N/256 of an M = 128 tile's MMA work.  The remainder band
+// of a larger group stays M = 128: as its own skinny tile it would race ahead of
+// the group's full tile that streams the same weights, and on deepseek_v3 that
+// cost 2.2 GB of extra HBM reads per layer (ncu: 26.6 vs 24.4 GB, 7.39 vs 7.25 ms).
+enum TileKind { TK_FULL = 0, TK_HALF = 1, TK_SKINNY = 2 };
+__device__ __forceinline__ int tile_kind(const PairTile& t, int skinny, int& ns) {
+  const int left = t.end - t.base;
+  ns = 0;
+  if (left > kTileM) return TK_FULL;
+  if (!skinny || left > kTileM / 2 || t.m != 0) return TK_HALF;
+  ns = (left + 31) & ~31;
+  return TK_SKINNY;
+}
+
 __device__ __forceinline__ void decode_pair_tile(int tile, const int* pstart, int nph, const int* mt,
                                                  const int* off, int G, const int* dmt,
                                                  const int* doff, const PairArgs& p, PairTile& t) {
@@ -681,6 +702,44 @@ __device__ __forceinline__ void decode_pair_tile(int tile, const int* pstart, in
   t.base = po[t.g] + t.m * 2 * kTileM;
   t.end = po[t.g + 1];
   t.band = pm[t.g] + t.m;
+}
+
+// Epilogue of a skinny tile.  The accumulators hold weights-rows x tile-rows: in
+// CTA r, TMEM lane i (i < 64) has weight row i of the CTA's slab for tile rows
+// [0, ns/2), lane 64 + i the same weight row for tile rows [ns/2, ns), at columns
+// 0.. (first 64 slab rows) and 128.. (second 64).  Warp q reads lanes 32q..32q+31.
+// The slab's rows are, per 256-wide N block n: SwiGLU / router pairs: the first and
+// second factor of outputs n*128 + 64r + i; plain outputs: columns n*256 + 128r + i
+// and + 64.  One output element per store (a warp writes 32 consecutive columns).
+__device__ __forceinline__ void epilogue_skinny(int epi, bf16* out, float* outf, int ldo, uint32_t tb,
+                                                const PairTile& t, int rank, int q, int lane, int ns) {
+  uint32_t r0[32], r1[32];
+  tmem_ld32(tb, r0);
+  tmem_ld32(tb + 128, r1);
+  tmem_ld_wait();
+  const int i = (q & 1) * 32 + lane;
+  const int nh = ns >> 1;
+  const int j0 = (q >> 1) * nh;                    // first tile row of this lane half
+  const bool paired = epi == EPI_SWIGLU || epi == EPI_PAIRSUM_F32;
+  const int col = paired ? t.n * 128 + rank * 64 + i : t.n * 256 + rank * 128 + i;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    if (c >= nh) break;
+    const int64_t row = (int64_t)t.base + j0 + c;
+    if (row >= t.end) break;
+    const float a = __uint_as_float(r0[c]), b = __uint_as_float(r1[c]);
+    if (epi == EPI_SWIGLU) {
+      out[row * ldo + col] = __float2bfloat16_rn(silu_f(a) * b);
+    } else if (epi == EPI_PAIRSUM_F32) {
+      outf[row * ldo + col] = a + b;
+    } else if (epi == EPI_GELU) {
+      out[row * ldo + col] = __float2bfloat16_rn(gelu_f(a));
+      out[row * ldo + col + 64] = __float2bfloat16_rn(gelu_f(b));
+    } else {
+      out[row * ldo + col] = __float2bfloat16_rn(a);
+      out[row * ldo + col + 64] = __float2bfloat16_rn(b);
+    }
+  }
 }
 
 // Bounded wait (cycle count) until *cnt >= need, read with acquire semantics.
@@ -748,6 +807,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
     for (int ph = 0; ph < nph; ++ph) {
       prefetch_tmap(&p.ph[ph].tmap_a);
       prefetch_tmap(&p.ph[ph].tmap_a64);
+      prefetch_tmap(&p.ph[ph].tmap_a32);
       prefetch_tmap(&p.ph[ph].tmap_b);
       const int rows = p.ph[ph].dense_rows;
       dmt[2 * ph] = 0; dmt[2 * ph + 1] = (rows + TM2 - 1) / TM2;
@@ -799,10 +859,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         PairTile t;
         decode_pair_tile(tile, pstart, nph, mt, off, G, dmt, doff, p, t);
         const PhaseArgs& P = p.ph[t.ph];
-        const bool half = t.end - t.base <= kTileM;     // M = 128: 64 rows per CTA
-        const int arow = t.base + (int)rank * (half ? kTileM / 2 : kTileM);
-        const CUtensorMap* amap = half ? &P.tmap_a64 : &P.tmap_a;
-        const uint32_t stage_tx = 2u * (uint32_t)((half ? C::kABytes / 2 : C::kABytes) + C::kBBytes);
+        int ns;
+        const int kind = tile_kind(t, p.skinny, ns);
+        // rows of A this CTA loads: 128 (full), its 64 (half), or its ns/2 of a 32-row box
+        const int arow = t.base + (int)rank * (kind == TK_FULL ? kTileM : kind == TK_HALF ? kTileM / 2 : ns / 2);
+        const CUtensorMap* amap = kind == TK_FULL ? &P.tmap_a : kind == TK_HALF ? &P.tmap_a64 : &P.tmap_a32;
+        const int abytes = kind == TK_FULL ? C::kABytes : kind == TK_HALF ? C::kABytes / 2 : C::kABytes / 4;
+        const uint32_t stage_tx = 2u * (uint32_t)(abytes + C::kBBytes);
         const int brow = t.n * BN + (int)rank * (BN / 2);
         if (P.dep >= 0) {
           // A rows of this band are written by phase P.dep: wait until all of its
@@ -838,8 +901,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         if (tile < 0) break;
         PairTile t;
         decode_pair_tile(tile, pstart, nph, mt, off, G, dmt, doff, p, t);
-        const bool half = t.end - t.base <= kTileM;
-        const uint32_t idesc = half ? C::kIdescHalf : C::kIdesc;
+        int ns;
+        const int kind = tile_kind(t, p.skinny, ns);
+        const uint32_t idesc = kind == TK_FULL ? C::kIdesc : kind == TK_HALF ? C::kIdescHalf
+                                                                             : make_idesc(kTileM, ns);
         const int ksteps = p.ph[t.ph].K / kTileK;
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.status)) break;
         tc_fence_after();
@@ -850,9 +915,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
           tc_fence_after();
           const uint64_t ad = sw128_desc(smem_u32(a_smem + stage * C::kABytes));
           const uint64_t bd = sw128_desc(smem_u32(b_smem + stage * C::kBBytes));
+          if (kind != TK_SKINNY) {
 #pragma unroll
-          for (int kk = 0; kk < kTileK / 16; ++kk)
-            tc_mma_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+            for (int kk = 0; kk < kTileK / 16; ++kk)
+              tc_mma_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+          } else {
+            // weights as the M operand: rows 0..63 of each CTA's B slab into columns
+            // [0, ns/2), rows 64..127 into columns [128, 128 + ns/2); the rows as N
+            const uint64_t bd_hi = sw128_desc(smem_u32(b_smem + stage * C::kBBytes + C::kBBytes / 2));
+#pragma unroll
+            for (int kk = 0; kk < kTileK / 16; ++kk) {
+              tc_mma_pair(d_tmem, bd + 2 * kk, ad + 2 * kk, idesc, (kb | kk) != 0);
+              tc_mma_pair(d_tmem + 128, bd_hi + 2 * kk, ad + 2 * kk, idesc, (kb | kk) != 0);
+            }
+          }
           tc_commit_pair_both(empty0 + 8 * stage);
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
@@ -874,14 +950,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
       PairTile t;
       decode_pair_tile(tile, pstart, nph, mt, off, G, dmt, doff, p, t);
       const PhaseArgs& P = p.ph[t.ph];
-      const bool half = t.end - t.base <= kTileM;
+      int ns;
+      const int kind = tile_kind(t, p.skinny, ns);
       bool ok = true;
       if (lane == 0) ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const bool paired = P.epi == EPI_SWIGLU || P.epi == EPI_PAIRSUM_F32;
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      if (!half) {
+      if (kind == TK_SKINNY) {
+        epilogue_skinny(P.epi, P.out, P.outf, P.ldo, tb, t, (int)rank, q, lane, ns);
+      } else if (kind == TK_FULL) {
         // M = 256: this CTA's 128 rows in TMEM lanes 0..127, all 256 columns
         const int row0 = t.base + (int)rank * kTileM;
         const int r = q * 32 + lane;
@@ -1035,6 +1114,11 @@ cudaError_t launch_grouped_pair(const GemmProblem* probs, int n, int32_t* counte
   PairArgs a;
   memset(&a, 0, sizeof(a));
   a.nph = n;
+  {
+    // MOE_GEMM_SKINNY=0 runs groups of <= 64 rows as M = 128 tiles too
+    const char* env = getenv("MOE_GEMM_SKINNY");
+    a.skinny = (env && env[0] == '0') ? 0 : 1;
+  }
   a.status = probs[0].status;
   a.counter = counter;
   a.done = done;
@@ -1044,7 +1128,8 @@ cudaError_t launch_grouped_pair(const GemmProblem* probs, int n, int32_t* counte
     PhaseArgs& P = a.ph[i];
     if (p.tile_n != 256 || p.N % 256 != 0 || p.K % kTileK != 0) return cudaErrorInvalidValue;
     if (!make_map_2d(&P.tmap_a, p.A, (uint64_t)p.K, (uint64_t)p.a_rows, kTileM) ||
-        !make_map_2d(&P.tmap_a64, p.A, (uint64_t)p.K, (uint64_t)p.a_rows, kTileM / 2))
+        !make_map_2d(&P.tmap_a64, p.A, (uint64_t)p.K, (uint64_t)p.a_rows, kTileM / 2) ||
+        !make_map_2d(&P.tmap_a32, p.A, (uint64_t)p.K, (uint64_t)p.a_rows, kTileM / 4))
       return cudaErrorInvalidValue;
     // each CTA of a pair loads its 128-row half of the 256-row B tile
     if (!make_map_3d(&P.tmap_b, p.B, (uint64_t)p.K, (uint64_t)p.N, (uint64_t)p.G, 128))

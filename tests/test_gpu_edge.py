@@ -49,6 +49,14 @@ def test_tile_widths(D, F, act):
     run_and_compare(BASE.with_(T=300, D=D, F=F, act=act, x_dtype="f32" if act == "gelu" else "bf16"))
 
 
+@pytest.mark.parametrize("T", [5, 40])
+def test_decode_batch_with_shared_experts(T):
+    """Decode-sized batches: every expert group and the shared expert's single band
+    hold at most 64 rows, so every tile of the FFN launch is skinny."""
+    run_and_compare(BASE.with_(T=T, D=256, E=16, ep_size=4, top_k=2, F=256, n_shared=1,
+                               F_shared=256, seed=T))
+
+
 def test_k_equals_e_and_no_renormalisation():
     run_and_compare(BASE.with_(T=200, E=8, top_k=8, ep_size=4))
     run_and_compare(BASE.with_(T=200, renormalize=False))
@@ -211,12 +219,14 @@ def test_ties_on_the_tensor_core_router(E, k):
 UNEVEN_COUNTS = [0, 1, 64, 65, 100, 128, 129, 200, 256, 257, 320, 384, 385, 115, 0, 3]
 
 
-@pytest.mark.parametrize("act", ["swiglu", "gelu"])
-def test_uneven_expert_tiles(act):
+@pytest.mark.parametrize("act,extra", [("swiglu", []), ("gelu", []), ("swiglu", [189, 0, 0, 0])])
+def test_uneven_expert_tiles(act, extra):
     """Every routed row (and every shared-expert token) of the expert FFN stage
     against the oracle, with hand-set expert sizes that put the last M tile of
-    each expert in every tiling case of both GEMM kernels."""
-    counts = np.array(UNEVEN_COUNTS)
+    each expert in every tiling case of both GEMM kernels (groups of <= 64 rows run
+    as skinny tiles; with 189 more rows the shared expert's last 256-row band
+    holds 36 rows)."""
+    counts = np.array(UNEVEN_COUNTS + extra)
     E, T = counts.size, int(counts.sum())            # top-1: one row per token
     shared = act == "swiglu"
     wl = BASE.with_(T=T, D=256, E=E, ep_size=4, top_k=1, F=256, act=act,
@@ -236,8 +246,11 @@ def test_uneven_expert_tiles(act):
     g.manual_seed(5)
     x_perm = torch.randn((T, wl.D), generator=g, device="cuda").to(torch.bfloat16)
     x_bf = inp["x"].to(torch.bfloat16) if shared else None
-    for flag in ("1", "0"):                          # CTA-pair kernel, then one-CTA kernel
-        os.environ["MOE_GEMM_CTA_PAIR"] = flag
+    # CTA-pair kernel with skinny remainder tiles, with M = 128 remainders only, then
+    # the one-CTA kernel
+    for pair, skinny in (("1", "1"), ("1", "0"), ("0", "1")):
+        os.environ["MOE_GEMM_CTA_PAIR"] = pair
+        os.environ["MOE_GEMM_SKINNY"] = skinny
         try:
             b["y_perm"].zero_()
             M.moe_expert_ffn(cfg, x_perm, x_bf, b["expert_offsets"], layer.packed, b["act"],
@@ -245,6 +258,7 @@ def test_uneven_expert_tiles(act):
             torch.cuda.synchronize()
         finally:
             del os.environ["MOE_GEMM_CTA_PAIR"]
+            del os.environ["MOE_GEMM_SKINNY"]
         assert int(b["status"].item()) == 0
         off = b["expert_offsets"].cpu().numpy()
         assert np.array_equal(np.diff(off), counts)
