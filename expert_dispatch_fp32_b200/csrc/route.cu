@@ -213,7 +213,20 @@ route_small_kernel(const XT* __restrict__ x, const float* __restrict__ w,
   extern __shared__ float4 w_s4[];
   const float* w_s = reinterpret_cast<const float*>(w_s4);
   const int n4 = E * D / 4;
-  for (int i = threadIdx.x; i < n4; i += blockDim.x) w_s4[i] = __ldg(reinterpret_cast<const float4*>(w) + i);
+  {
+    // stage W_r with 8 independent 16-byte loads in flight per thread (a plain
+    // load-store loop waits out one L2 round trip per vector)
+    constexpr int U = 8;
+    for (int i0 = threadIdx.x; i0 < n4; i0 += blockDim.x * U) {
+      float4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (i0 + u * (int)blockDim.x < n4) v[u] = __ldg(reinterpret_cast<const float4*>(w) + i0 + u * blockDim.x);
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (i0 + u * (int)blockDim.x < n4) w_s4[i0 + u * blockDim.x] = v[u];
+    }
+  }
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
