@@ -11,8 +11,8 @@ from ._binding import (  # noqa: F401
     MOE_ERR_INDEX_OOB, MOE_ERR_INVALID_ARG, MOE_ERR_SCRATCH_LIMIT, MOE_ERR_TIMEOUT,
     MOE_ERR_UNSUPPORTED, MOE_OK,
     MoeConfig, MoeError, lib, moe_abi_version, moe_combine_unpermute, moe_dispatch_permute,
-    moe_expert_ffn, moe_forward, moe_packed_weights_size, moe_prepare_weights, moe_preprocess,
-    moe_preprocess_noalloc,
+    moe_ep_local_ids, moe_expert_ffn, moe_forward, moe_gather_rows, moe_packed_weights_size,
+    moe_prepare_weights, moe_preprocess, moe_preprocess_noalloc, moe_shared_ffn,
     moe_route, moe_status_string, moe_validate_config, moe_workspace_size,
 )
 from .layer import MoELayer, make_config  # noqa: F401

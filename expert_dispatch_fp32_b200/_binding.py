@@ -55,6 +55,10 @@ _SIGS = {
                                    _vp]),
     "moe_preprocess_noalloc": (ctypes.c_int, [_cfgp, _i32p, _i32p, _i32p, _i32p, _i32p, _i32p, _i32p,
                                               _i32p, _vp]),
+    "moe_shared_ffn": (ctypes.c_int, [_cfgp, _vp, _vp, _vp, _vp, _i32p, _vp]),
+    "moe_ep_local_ids": (ctypes.c_int, [_cfgp, _i32p, _i32p, _i32p, _vp]),
+    "moe_gather_rows": (ctypes.c_int, [_vp, _i32p, _vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                       _vp]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_abi_version": (ctypes.c_int32, []),
 }
@@ -151,6 +155,19 @@ def moe_expert_ffn(cfg, x_perm, x, expert_offsets, packed, act, y_perm, shared_o
                    status, stream=None):
     _call("moe_expert_ffn", ctypes.byref(cfg), _p(x_perm), _p(x), _p(expert_offsets), _p(packed),
           _p(act), _p(y_perm), _p(shared_out), _p(workspace), _p(status), _s(stream))
+
+
+def moe_shared_ffn(cfg, x, packed, shared_out, workspace, status, stream=None):
+    _call("moe_shared_ffn", ctypes.byref(cfg), _p(x), _p(packed), _p(shared_out), _p(workspace),
+          _p(status), _s(stream))
+
+
+def moe_ep_local_ids(cfg, topk_idx, src, ids, stream=None):
+    _call("moe_ep_local_ids", ctypes.byref(cfg), _p(topk_idx), _p(src), _p(ids), _s(stream))
+
+
+def moe_gather_rows(src, index, dst, n, n_src, D, stream=None):
+    _call("moe_gather_rows", _p(src), _p(index), _p(dst), n, n_src, D, _s(stream))
 
 
 def moe_combine_unpermute(cfg, y_perm, pos, topk_w, x, shared_out, out, stream=None):

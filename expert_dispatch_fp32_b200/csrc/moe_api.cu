@@ -186,22 +186,31 @@ moe_status moe_dispatch_permute(const moe_config* cfg, const void* x, const int3
   return cuda_status(launch_dispatch(c, x, pos, (bf16*)x_perm, as_stream(stream)));
 }
 
-moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void* x,
-                          const int32_t* expert_offsets, const void* packed, void* act,
-                          void* y_perm, void* shared_out, void* workspace, int32_t* status,
-                          void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The expert-FFN stage: the routed experts over x_perm (`routed`) and/or the shared
+// experts over x (`shared`), one persistent launch when all tiles are 256 wide.
+moe_status ffn_run(const moe_config* cfg, const void* x_perm, const void* x,
+                   const int32_t* expert_offsets, const void* packed, void* act, void* y_perm,
+                   void* shared_out, void* workspace, int32_t* status, void* stream, bool routed,
+                   bool shared) {
   moe_status st = moe_validate_config(cfg);
   if (st != MOE_OK) return st;
   const moe_config& c = *cfg;
-  if (c.T == 0) return MOE_OK;
-  MOE_CHECK_PTR(x_perm);
-  MOE_CHECK_PTR(expert_offsets);
+  if (shared && c.n_shared == 0) return MOE_ERR_INVALID_ARG;
+  if (c.T == 0 || (!routed && !shared)) return MOE_OK;
+  if (routed) {
+    MOE_CHECK_PTR(x_perm);
+    MOE_CHECK_PTR(expert_offsets);
+    MOE_CHECK_PTR(act);
+    MOE_CHECK_PTR(y_perm);
+  }
   MOE_CHECK_PTR(packed);
-  MOE_CHECK_PTR(act);
-  MOE_CHECK_PTR(y_perm);
   MOE_CHECK_PTR(workspace);
   MOE_CHECK_PTR(status);
-  if (c.n_shared > 0) {
+  if (shared) {
     MOE_CHECK_PTR(x);
     MOE_CHECK_PTR(shared_out);
   }
@@ -254,7 +263,8 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   bf16* act_s = (bf16*)(ws + W.act_shared);
   GemmProblem su, sd;
   memset(&su, 0, sizeof(su));
-  if (c.n_shared > 0) {
+  memset(&sd, 0, sizeof(sd));
+  if (shared) {
     su.A = (const bf16*)x; su.a_rows = c.T;
     su.B = (const bf16*)(pk + P.ws_up); su.G = 1;
     su.N = 2 * Fc; su.K = c.D;
@@ -285,16 +295,16 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   // MOE_GEMM_FUSED=0 selects one launch per GEMM (read at each call; for comparison)
   const char* fused_env = getenv("MOE_GEMM_FUSED");
   const bool fused = !(fused_env && fused_env[0] == '0');
-  if (fused && up.pair && dn.pair && (c.n_shared == 0 || sd.pair)) {
+  if (fused && (!routed || (up.pair && dn.pair)) && (!shared || (su.pair && sd.pair))) {
     // One persistent launch: routed gate_up, shared gate_up, routed down, shared down.
     // Each down tile waits only for the gate_up band it reads, so the down phase
     // starts while the last gate_up tiles finish (no launch gap, one tail).
     GemmProblem ph[4];
     int n = 0;
-    ph[n++] = up;
-    if (c.n_shared > 0) ph[n++] = su;
-    ph[n] = dn; ph[n].dep = 0; ++n;
-    if (c.n_shared > 0) { ph[n] = sd; ph[n].dep = 1; ++n; }
+    if (routed) ph[n++] = up;
+    if (shared) ph[n++] = su;
+    if (routed) { ph[n] = dn; ph[n].dep = 0; ++n; }
+    if (shared) { ph[n] = sd; ph[n].dep = routed ? 1 : 0; ++n; }
     const int64_t slots = pair_done_slots(ph, n);
     if (cudaMemsetAsync(ctr, 0, (size_t)(8 + slots) * sizeof(int32_t), s) != cudaSuccess)
       return MOE_ERR_CUDA;
@@ -305,13 +315,34 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void*
   if (cudaMemsetAsync(ctr + 1, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
   dn.dep = -1;
   sd.dep = -1;
-  cudaError_t err = launch_grouped_gemm(up, s);
-  if (err != cudaSuccess) return MOE_ERR_CUDA;
-  err = launch_grouped_gemm(dn, s);
-  if (err != cudaSuccess || c.n_shared == 0) return cuda_status(err);
-  err = launch_grouped_gemm(su, s);
-  if (err != cudaSuccess) return MOE_ERR_CUDA;
-  return cuda_status(launch_grouped_gemm(sd, s));
+  if (routed) {
+    if (launch_grouped_gemm(up, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_grouped_gemm(dn, s) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  if (shared) {
+    if (launch_grouped_gemm(su, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_grouped_gemm(sd, s) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void* x,
+                          const int32_t* expert_offsets, const void* packed, void* act,
+                          void* y_perm, void* shared_out, void* workspace, int32_t* status,
+                          void* stream) {
+  const bool shared = cfg != nullptr && cfg->n_shared > 0 && shared_out != nullptr;
+  return ffn_run(cfg, x_perm, x, expert_offsets, packed, act, y_perm, shared_out, workspace, status,
+                 stream, true, shared);
+}
+
+moe_status moe_shared_ffn(const moe_config* cfg, const void* x, const void* packed, void* shared_out,
+                          void* workspace, int32_t* status, void* stream) {
+  return ffn_run(cfg, nullptr, x, nullptr, packed, nullptr, nullptr, shared_out, workspace, status,
+                 stream, false, true);
 }
 
 moe_status moe_combine_unpermute(const moe_config* cfg, const void* y_perm, const int32_t* pos,
@@ -352,6 +383,30 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_rout
                       status, stream);
   if (st != MOE_OK) return st;
   return moe_combine_unpermute(cfg, y_perm, pos, topk_w, x, shared_out, out, stream);
+}
+
+moe_status moe_ep_local_ids(const moe_config* cfg, const int32_t* topk_idx, const int32_t* src,
+                            int32_t* ids, void* stream) {
+  moe_status st = moe_validate_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (c.T == 0) return MOE_OK;
+  MOE_CHECK_PTR(topk_idx);
+  MOE_CHECK_PTR(src);
+  MOE_CHECK_PTR(ids);
+  return cuda_status(launch_local_ids(topk_idx, src, ids, c.T * c.top_k, c.E / c.ep_size,
+                                      as_stream(stream)));
+}
+
+moe_status moe_gather_rows(const void* src, const int32_t* index, void* dst, int32_t n,
+                           int32_t n_src, int32_t D, void* stream) {
+  if (n < 0 || n_src < 0 || D <= 0 || D % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  MOE_CHECK_PTR(index);
+  MOE_CHECK_PTR(dst);
+  if (n_src > 0) MOE_CHECK_PTR(src);
+  return cuda_status(launch_gather_rows((const bf16*)src, index, (bf16*)dst, n, n_src, D,
+                                        as_stream(stream)));
 }
 
 const char* moe_status_string(moe_status s) {

@@ -81,6 +81,11 @@ cudaError_t launch_preprocess(const moe_config& c, const int32_t* topk_idx, int3
                               int32_t* rank_offsets, int32_t* pos, int32_t* src,
                               int32_t* block_counts, int max_blocks, int32_t* mt_start,
                               unsigned* barrier, int32_t* status, cudaStream_t s);
+// Multi-rank helpers (ep.cu).
+cudaError_t launch_local_ids(const int32_t* topk_idx, const int32_t* src, int32_t* ids, int R, int El,
+                             cudaStream_t s);
+cudaError_t launch_gather_rows(const bf16* src, const int32_t* index, bf16* dst, int n, int n_src,
+                               int D, cudaStream_t s);
 cudaError_t launch_dispatch(const moe_config& c, const void* x, const int32_t* pos,
                             bf16* x_perm, cudaStream_t s);
 cudaError_t launch_combine(const moe_config& c, const bf16* y_perm, const int32_t* pos,

@@ -166,13 +166,22 @@ MOE_API moe_status moe_dispatch_permute(const moe_config* cfg, const void* x, co
  *   packed         device, from moe_prepare_weights
  *   act            device bf16 [R, F], written (intermediate)
  *   y_perm         device bf16 [R, D], written
- *   shared_out     device bf16 [T, D], written when S > 0, else may be NULL
+ *   shared_out     device bf16 [T, D], written when S > 0; NULL skips the shared
+ *                  experts (moe_shared_ffn runs them alone)
  *   workspace      the buffer moe_preprocess wrote its tile prefix into
  *   status         device int32, MOE_ERR_TIMEOUT if a bounded wait expired */
 MOE_API moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void* x,
                           const int32_t* expert_offsets, const void* packed, void* act,
                           void* y_perm, void* shared_out, void* workspace, int32_t* status,
                           void* stream);
+
+/* The shared experts alone (S > 0): shared_out[t] = sum_i SwiGLU_i(x[t]) for the T
+ * tokens of cfg, from the shared part of `packed` (moe_prepare_weights of any config
+ * with the same E, D, F, act, S and Fs).  Used by the multi-rank forward, where a
+ * rank runs the routed experts on rows received from other ranks but the shared
+ * experts on its own tokens.  Arguments as moe_expert_ffn. */
+MOE_API moe_status moe_shared_ffn(const moe_config* cfg, const void* x, const void* packed,
+                                  void* shared_out, void* workspace, int32_t* status, void* stream);
 
 /* Stage 3, combine (token post-all-to-all, unpermute, routing weights, residual).
  * "Expert Parallel (EP)", Communication Pattern, step 4; "Worked Example ...",
@@ -228,6 +237,29 @@ MOE_API moe_status moe_preprocess_noalloc(const moe_config* cfg, const int32_t* 
                                           int32_t* rank_splits, int32_t* rank_offsets,
                                           int32_t* pos, int32_t* src, int32_t* status,
                                           void* stream);
+
+/* Multi-rank expert parallelism ("Expert Parallel (EP)", Communication Pattern
+ * steps 2-4): with ep_size = number of ranks, rank r owns experts
+ * [r*El, (r+1)*El).  Each rank routes, preprocesses and dispatches its own tokens;
+ * x_perm is then rank-major, and rows [rank_offsets[r], rank_offsets[r+1]) go to
+ * rank r in the token pre-all-to-all (performed by the caller's communication
+ * library).  These two calls do the row bookkeeping around the exchanges.
+ *
+ * ids[row] = local expert, on its destination rank, of dispatch row `row`:
+ *   topk_idx[src[row]] % El  (-1 where src is outside [0, T*k)).
+ *   topk_idx, src device int32 [T*k] (from moe_route / moe_preprocess of cfg);
+ *   ids device int32 [T*k], written.  Sent along with the rows so the receiver can
+ *   group its rows by local expert (moe_preprocess with k = 1 over them). */
+MOE_API moe_status moe_ep_local_ids(const moe_config* cfg, const int32_t* topk_idx, const int32_t* src,
+                                    int32_t* ids, void* stream);
+
+/* dst[i, :] = src[index[i], :] for i in [0, n): bf16 rows of D elements (D % 8 == 0).
+ * Rows whose index is outside [0, n_src) are left unwritten.  Used on the
+ * receiving rank to put the local experts' output rows back in received order
+ * (index = the pos of its k = 1 preprocess) for the token post-all-to-all.
+ *   src device bf16 [n_src, D]; index device int32 [n]; dst device bf16 [n, D]. */
+MOE_API moe_status moe_gather_rows(const void* src, const int32_t* index, void* dst, int32_t n,
+                                   int32_t n_src, int32_t D, void* stream);
 
 /* Static description of a status code. */
 MOE_API const char* moe_status_string(moe_status s);
