@@ -215,17 +215,22 @@ def test_ties_on_the_tensor_core_router(E, k):
 
 # per-expert row counts around the 128- and 256-row tile edges: empty, one row, a
 # last tile with <= 64 rows (only the first CTA of a pair holds rows), 65..128 rows
-# (both CTAs of an M = 128 pair tile), 129..255, exactly 256, and 256 + a few
-UNEVEN_COUNTS = [0, 1, 64, 65, 100, 128, 129, 200, 256, 257, 320, 384, 385, 115, 0, 3]
+# (both CTAs of an M = 128 pair tile), 129..255, exactly 256, 256 + a few (1, 32,
+# 33, 64, 128, 129 rows; after two full tiles; in the second band of an expert of
+# nine full tiles)
+UNEVEN_COUNTS = [0, 1, 64, 65, 100, 128, 129, 200, 256, 257, 320, 384, 385, 115, 0, 3,
+                 288, 289, 529, 2344]
 
 
-@pytest.mark.parametrize("act,extra", [("swiglu", []), ("gelu", []), ("swiglu", [189, 0, 0, 0])])
+@pytest.mark.parametrize("act,extra", [("swiglu", []), ("gelu", []), ("swiglu", [47, 0, 0, 0]),
+                                       ("swiglu", [134, 0, 0, 0])])
 def test_uneven_expert_tiles(act, extra):
     """Every routed row (and every shared-expert token) of the expert FFN stage
     against the oracle, with hand-set expert sizes that put the last M tile of
     each expert in every tiling case of both GEMM kernels (groups of <= 64 rows run
-    as skinny tiles; with 189 more rows the shared expert's last 256-row band
-    holds 36 rows)."""
+    as skinny tiles).  The shared expert runs over all T tokens: T = 5857 leaves
+    225 rows in its last 256-row band, T + 47 leaves 16 and T + 134 leaves 103
+    (M = 128 tiles, the first with rows in one CTA only)."""
     counts = np.array(UNEVEN_COUNTS + extra)
     E, T = counts.size, int(counts.sum())            # top-1: one row per token
     shared = act == "swiglu"
