@@ -297,16 +297,19 @@ route_small_kernel(const XT* __restrict__ x, const float* __restrict__ w,
 template <int EP, int TW, typename XT>
 cudaError_t launch_small(const moe_config& c, const XT* x, const float* w, const float* bias,
                          float* logits_out, int32_t* topk_idx, float* topk_w, cudaStream_t s) {
+  const int threads = kSmallThreads;
   const size_t smem = (size_t)c.E * c.D * sizeof(float);
   auto kern = route_small_kernel<EP, TW, XT>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  const int per_sm = (int)((227u << 10) / (smem + 1024));
-  const int warps = kSmallThreads / 32;
+  const int warps = threads / 32;
   const int need = (c.T + warps * TW - 1) / (warps * TW);
-  const int cap = sm_count() * (per_sm > 0 ? per_sm : 1);
-  kern<<<need < cap ? need : cap, kSmallThreads, smem, s>>>(x, w, bias, logits_out, topk_idx, topk_w,
-                                                            c.T, c.D, c.E, c.top_k, c.renormalize);
+  int occ = 1;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, smem);
+  if (err != cudaSuccess) return err;
+  const int cap = sm_count() * (occ > 0 ? occ : 1);
+  kern<<<need < cap ? need : cap, threads, smem, s>>>(x, w, bias, logits_out, topk_idx, topk_w,
+                                                      c.T, c.D, c.E, c.top_k, c.renormalize);
   return cudaGetLastError();
 }
 
@@ -341,6 +344,11 @@ cudaError_t launch_route_t(const moe_config& c, const XT* x, const float* w_rout
   const size_t wbytes = (size_t)c.E * c.D * sizeof(float);
   if (c.E <= 32 && wbytes <= kSmallRouterSmem) {
     float* lo = keep_logits ? logits : nullptr;
+    // Four tokens per warp read W_r from shared memory half as often as two, which pays
+    // once the 64-token blocks still cover most SMs (mixtral_8x7b: 45 vs 59 us); with
+    // fewer tokens the two-token form keeps more SMs busy (small_e8_d2048: 22.5 vs 28.7 us)
+    if (c.E <= 8 && 4 * ((c.T + 63) / 64) >= 3 * sm_count())
+      return launch_small<8, 4, XT>(c, x, w_router, bias, lo, topk_idx, topk_w, s);
     if (c.E <= 8) return launch_small<8, 2, XT>(c, x, w_router, bias, lo, topk_idx, topk_w, s);
     if (c.E <= 16) return launch_small<16, 1, XT>(c, x, w_router, bias, lo, topk_idx, topk_w, s);
     return launch_small<32, 1, XT>(c, x, w_router, bias, lo, topk_idx, topk_w, s);

@@ -83,6 +83,13 @@ def test_zipf_skew_small():
     run_and_compare(W.get("zipf_skew_e64").with_(T=2000, D=256, F=256, F_shared=128))
 
 
+@pytest.mark.parametrize("T", [7043, 9000])
+def test_few_expert_router_four_tokens_per_warp(T):
+    """Batches large enough for the four-tokens-per-warp router (with a ragged last
+    group of tokens): routing and the whole layer against the oracle."""
+    run_and_compare(BASE.with_(T=T, D=512, E=8, top_k=2, F=128, seed=3))
+
+
 def test_ties_go_to_the_lower_index():
     wl = BASE.with_(T=512, E=8, top_k=2)
     inp = W.make_inputs(wl, device="cuda")
