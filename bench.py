@@ -318,10 +318,27 @@ def run_ours(args):
                                 b["out"], stream)
         ev[5].record(stream)
 
+    def stages_fused(ev):
+        # the three launches moe_forward runs: router + preprocess + dispatch in one
+        ev[0].record(stream)
+        M.moe_route_dispatch(cfg, x, layer.w_router, layer.expert_bias, None, b["topk_idx"],
+                             b["topk_w"], b["counts"], b["expert_offsets"], b["rank_splits"],
+                             b["rank_offsets"], b["pos"], b["src"], b["x_perm"], b["workspace"],
+                             b["status"], stream)
+        ev[1].record(stream)
+        M.moe_expert_ffn(cfg, b["x_perm"], x_bf, b["expert_offsets"], layer.packed, b["act"],
+                         b["y_perm"], b["shared_out"], b["workspace"], b["status"], stream)
+        ev[2].record(stream)
+        M.moe_combine_unpermute(cfg, b["y_perm"], b["pos"], b["topk_w"], x, b["shared_out"],
+                                b["out"], stream)
+        ev[3].record(stream)
+
     def fwd(ev):
         ev[0].record(stream)
         layer.forward(x, stream)
         ev[1].record(stream)
+
+    fused = M.moe_route_dispatch_is_fused(cfg)
 
     mk = lambda n=6: [torch.cuda.Event(enable_timing=True) for _ in range(n)]
     # the stage-by-stage step is moe_forward: check once that both give the same bits
@@ -359,6 +376,17 @@ def run_ours(args):
     stage_ms = np.zeros(5)
     for ev in sevs:
         stage_ms += [ev[j].elapsed_time(ev[j + 1]) for j in range(5)]
+    fused_ms = None
+    if fused:
+        fevs = [mk(4) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush_l2()
+            stages_fused(fevs[i])
+        torch.cuda.synchronize()
+        layer.check_status()
+        fused_ms = np.zeros(3)
+        for ev in fevs:
+            fused_ms += [ev[j].elapsed_time(ev[j + 1]) for j in range(3)]
     total_ms_max = max_over_ranks(total_ms, ws)
     value = replica_value(T, ws, args.steps, total_ms_max)
 
@@ -443,7 +471,7 @@ def run_ours(args):
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     disp_gbs = disp_b / (stage_ms[2] / args.steps / 1e3) / 1e9
     comb_gbs = comb_b / (stage_ms[4] / args.steps / 1e3) / 1e9
-    launches_per_step = route_launches(wl) + 1 + 1 + ffn_launches(wl) + 1
+    launches_per_step = (1 if fused else route_launches(wl) + 1 + 1) + ffn_launches(wl) + 1
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
@@ -469,6 +497,9 @@ def run_ours(args):
         "clocks": clk.summary(),
         "stages_us": {n: 1e3 * float(v) / args.steps for n, v in
                       zip(("route", "preprocess", "dispatch", "expert_ffn", "combine"), stage_ms)},
+        "forward_stages_us": ({n: 1e3 * float(v) / args.steps for n, v in
+                               zip(("route_preprocess_dispatch", "expert_ffn", "combine"), fused_ms)}
+                              if fused else None),
         "ffn_tflops": ffn_tflops,
         "dispatch_gbs": disp_gbs, "dispatch_frac_hbm": disp_gbs / hbm,
         "combine_gbs": comb_gbs, "combine_frac_hbm": comb_gbs / hbm,

@@ -4,7 +4,8 @@ The compute path is libmoe.so (hand-written CUDA behind a C ABI, include/moe.h);
 this package holds its ctypes binding and a small layer object that allocates
 buffers with PyTorch.  Stages, after "Expert Parallel (EP)", Communication
 Pattern: moe_route -> moe_preprocess -> moe_dispatch_permute -> moe_expert_ffn
--> moe_combine_unpermute (or moe_forward for all five).
+-> moe_combine_unpermute (moe_route_dispatch for the first three in one launch where
+it applies, moe_forward for all five).
 """
 from ._binding import (  # noqa: F401
     LIB_PATH, MOE_ACT_GELU, MOE_ACT_SWIGLU, MOE_DT_BF16, MOE_DT_F32, MOE_ERR_CUDA,
@@ -13,6 +14,6 @@ from ._binding import (  # noqa: F401
     MoeConfig, MoeError, lib, moe_abi_version, moe_combine_unpermute, moe_dispatch_permute,
     moe_ep_local_ids, moe_expert_ffn, moe_forward, moe_gather_rows, moe_packed_weights_size,
     moe_prepare_weights, moe_preprocess, moe_preprocess_noalloc, moe_shared_ffn,
-    moe_route, moe_status_string, moe_validate_config, moe_workspace_size,
+    moe_route, moe_route_dispatch, moe_route_dispatch_is_fused, moe_status_string, moe_validate_config, moe_workspace_size,
 )
 from .layer import MoELayer, make_config  # noqa: F401

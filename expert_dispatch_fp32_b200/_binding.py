@@ -48,6 +48,9 @@ _SIGS = {
     "moe_preprocess": (ctypes.c_int, [_cfgp, _i32p, _i32p, _i32p, _i32p, _i32p, _i32p, _i32p, _vp,
                                       _i32p, _vp]),
     "moe_dispatch_permute": (ctypes.c_int, [_cfgp, _vp, _i32p, _vp, _vp]),
+    "moe_route_dispatch_is_fused": (ctypes.c_int32, [_cfgp]),
+    "moe_route_dispatch": (ctypes.c_int, [_cfgp, _vp, _f32p, _f32p, _f32p, _i32p, _f32p, _i32p, _i32p,
+                                          _i32p, _i32p, _i32p, _i32p, _vp, _vp, _i32p, _vp]),
     "moe_expert_ffn": (ctypes.c_int, [_cfgp, _vp, _vp, _i32p, _vp, _vp, _vp, _vp, _vp, _i32p, _vp]),
     "moe_combine_unpermute": (ctypes.c_int, [_cfgp, _vp, _i32p, _f32p, _vp, _vp, _vp, _vp]),
     "moe_forward": (ctypes.c_int, [_cfgp, _vp, _f32p, _f32p, _vp, _f32p, _i32p, _f32p, _i32p, _i32p,
@@ -149,6 +152,18 @@ def moe_preprocess_noalloc(cfg, topk_idx, counts, expert_offsets, rank_splits, r
 
 def moe_dispatch_permute(cfg, x, pos, x_perm, stream=None):
     _call("moe_dispatch_permute", ctypes.byref(cfg), _p(x), _p(pos), _p(x_perm), _s(stream))
+
+
+def moe_route_dispatch(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w, counts,
+                       expert_offsets, rank_splits, rank_offsets, pos, src, x_perm, workspace, status,
+                       stream=None):
+    _call("moe_route_dispatch", ctypes.byref(cfg), _p(x), _p(w_router), _p(expert_bias),
+          _p(logits_out), _p(topk_idx), _p(topk_w), _p(counts), _p(expert_offsets), _p(rank_splits),
+          _p(rank_offsets), _p(pos), _p(src), _p(x_perm), _p(workspace), _p(status), _s(stream))
+
+
+def moe_route_dispatch_is_fused(cfg) -> bool:
+    return bool(lib().moe_route_dispatch_is_fused(ctypes.byref(cfg)))
 
 
 def moe_expert_ffn(cfg, x_perm, x, expert_offsets, packed, act, y_perm, shared_out, workspace,

@@ -12,7 +12,10 @@ WsLayout ws_layout(const moe_config& c) {
   WsLayout L;
   const size_t T = (size_t)c.T, E = (size_t)c.E;
   const size_t R = T * (size_t)c.top_k;
-  L.nblk = preprocess_blocks((int64_t)R);
+  // one histogram row per preprocess block (at most kPreMaxBlocks; the fused router +
+  // preprocess + dispatch launch uses one block per SM)
+  L.nblk = kPreMaxBlocks;
+  (void)R;
   size_t o = 0;
   L.logits = o;       o = align256(o + T * E * sizeof(float));
   L.block_counts = o; o = align256(o + (size_t)L.nblk * E * sizeof(int32_t));
@@ -364,6 +367,54 @@ moe_status moe_combine_unpermute(const moe_config* cfg, const void* y_perm, cons
                                     as_stream(stream)));
 }
 
+int32_t moe_route_dispatch_is_fused(const moe_config* cfg) {
+  if (moe_validate_config(cfg) != MOE_OK) return 0;
+  const char* env = getenv("MOE_ROUTE_FUSED");
+  if (env && env[0] == '0') return 0;
+  return route_pre_dispatch_applies(*cfg, ws_layout(*cfg).nblk) ? 1 : 0;
+}
+
+moe_status moe_route_dispatch(const moe_config* cfg, const void* x, const float* w_router,
+                              const float* expert_bias, float* logits_out, int32_t* topk_idx,
+                              float* topk_w, int32_t* counts, int32_t* expert_offsets,
+                              int32_t* rank_splits, int32_t* rank_offsets, int32_t* pos,
+                              int32_t* src, void* x_perm, void* workspace, int32_t* status,
+                              void* stream) {
+  moe_status st = moe_validate_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  const WsLayout L = ws_layout(c);
+  // MOE_ROUTE_FUSED=0 runs the three stage calls (read at each call; for comparison)
+  const bool fused = moe_route_dispatch_is_fused(cfg) != 0;
+  if (!fused) {
+    st = moe_route(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w, workspace, stream);
+    if (st != MOE_OK) return st;
+    st = moe_preprocess(cfg, topk_idx, counts, expert_offsets, rank_splits, rank_offsets, pos, src,
+                        workspace, status, stream);
+    if (st != MOE_OK) return st;
+    return moe_dispatch_permute(cfg, x, pos, x_perm, stream);
+  }
+  MOE_CHECK_PTR(x);
+  MOE_CHECK_PTR(w_router);
+  MOE_CHECK_PTR(topk_idx);
+  MOE_CHECK_PTR(topk_w);
+  MOE_CHECK_PTR(counts);
+  MOE_CHECK_PTR(expert_offsets);
+  MOE_CHECK_PTR(rank_splits);
+  MOE_CHECK_PTR(rank_offsets);
+  MOE_CHECK_PTR(pos);
+  MOE_CHECK_PTR(src);
+  MOE_CHECK_PTR(x_perm);
+  MOE_CHECK_PTR(workspace);
+  MOE_CHECK_PTR(status);
+  if (logits_out != nullptr && !aligned16(logits_out)) return MOE_ERR_INVALID_ARG;
+  uint8_t* ws = (uint8_t*)workspace;
+  return cuda_status(launch_route_pre_dispatch(
+      c, x, w_router, expert_bias, logits_out, topk_idx, topk_w, counts, expert_offsets, rank_splits,
+      rank_offsets, pos, src, (int32_t*)(ws + L.block_counts), L.nblk, (int32_t*)(ws + L.mt_start),
+      (unsigned*)(ws + L.barrier), (bf16*)x_perm, status, as_stream(stream)));
+}
+
 moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_router,
                        const float* expert_bias, const void* packed, float* logits_out,
                        int32_t* topk_idx, float* topk_w, int32_t* counts,
@@ -371,13 +422,9 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_rout
                        int32_t* pos, int32_t* src, void* x_perm, void* act, void* y_perm,
                        void* shared_out, void* out, void* workspace, int32_t* status,
                        void* stream) {
-  moe_status st = moe_route(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w,
-                            workspace, stream);
-  if (st != MOE_OK) return st;
-  st = moe_preprocess(cfg, topk_idx, counts, expert_offsets, rank_splits, rank_offsets, pos, src,
-                      workspace, status, stream);
-  if (st != MOE_OK) return st;
-  st = moe_dispatch_permute(cfg, x, pos, x_perm, stream);
+  moe_status st = moe_route_dispatch(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w,
+                                     counts, expert_offsets, rank_splits, rank_offsets, pos, src,
+                                     x_perm, workspace, status, stream);
   if (st != MOE_OK) return st;
   st = moe_expert_ffn(cfg, x_perm, x, expert_offsets, packed, act, y_perm, shared_out, workspace,
                       status, stream);

@@ -86,6 +86,16 @@ cudaError_t launch_local_ids(const int32_t* topk_idx, const int32_t* src, int32_
                              cudaStream_t s);
 cudaError_t launch_gather_rows(const bf16* src, const int32_t* index, bf16* dst, int n, int n_src,
                                int D, cudaStream_t s);
+// Router + preprocess + dispatch in one cooperative launch (few experts; see
+// route_dispatch.cu).  route_pre_dispatch_applies: whether the configuration fits it.
+bool route_pre_dispatch_applies(const moe_config& c, int max_blocks);
+cudaError_t launch_route_pre_dispatch(const moe_config& c, const void* x, const float* w,
+                                      const float* bias, float* logits_out, int32_t* topk_idx,
+                                      float* topk_w, int32_t* counts, int32_t* expert_offsets,
+                                      int32_t* rank_splits, int32_t* rank_offsets, int32_t* pos,
+                                      int32_t* src, int32_t* block_counts, int max_blocks,
+                                      int32_t* mt_start, unsigned* barrier, bf16* x_perm,
+                                      int32_t* status, cudaStream_t s);
 cudaError_t launch_dispatch(const moe_config& c, const void* x, const int32_t* pos,
                             bf16* x_perm, cudaStream_t s);
 cudaError_t launch_combine(const moe_config& c, const bf16* y_perm, const int32_t* pos,

@@ -24,7 +24,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-#include "moe_internal.cuh"
+#include "device_util.cuh"
 
 namespace moe {
 
@@ -168,37 +168,6 @@ route_topk_kernel(const float* __restrict__ logits, int32_t* __restrict__ topk_i
   if (lane < k) {
     topk_idx[(size_t)t * k + lane] = my_idx;
     topk_w[(size_t)t * k + lane] = num / den;
-  }
-}
-
-// Warp argmax top-k over one logit per lane (lanes >= E hold none).
-__device__ __forceinline__ void warp_topk_write(float l, int E, int k, int renorm, size_t t,
-                                                int32_t* __restrict__ topk_idx,
-                                                float* __restrict__ topk_w) {
-  const int lane = threadIdx.x & 31;
-  bool avail = lane < E;
-  int my_idx = 0;
-  float my_val = 0.f, top = 0.f;
-  for (int j = 0; j < k; ++j) {
-    float bv = avail ? l : -INFINITY;
-    int bi = avail ? lane : 0x7fffffff;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-    }
-    if (lane == bi) avail = false;
-    if (lane == j) { my_idx = bi; my_val = bv; }
-    if (j == 0) top = bv;
-  }
-  const float num = (lane < k) ? expf(my_val - top) : 0.f;
-  float den = renorm ? num : (lane < E ? expf(l - top) : 0.f);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-  if (lane < k) {
-    topk_idx[t * k + lane] = my_idx;
-    topk_w[t * k + lane] = num / den;
   }
 }
 

@@ -1,0 +1,286 @@
+// Router, preprocess and dispatch in one cooperative launch, for few experts.
+//
+// "Expert Parallel (EP)", Communication Pattern steps 1-2 (gate + top-k, per-expert
+// counts and split sizes, tokens permuted by expert assignment); "Worked Example:
+// Tracing a Token Through Expert Parallelism", Steps 1-2.
+//
+// Block b owns tokens [b * tpb, (b + 1) * tpb) and, for the preprocess, the flat
+// (token, slot) pairs of those tokens:
+//  1. W_r and the block's x rows are loaded into shared memory;
+//  2. each warp routes TW tokens at a time with the arithmetic of the few-expert
+//     router (fp32 8-term slices folded into fp64, lane-parallel over D, exact
+//     argmax top-k, renormalised softmax weights) and keeps the selections;
+//  3. the block's per-expert histogram goes out, then one grid barrier;
+//  4. the totals, expert offsets, rank splits and tile prefixes, and the in-order
+//     rows of the block's pairs, exactly as the preprocess computes them;
+//  5. each pair's x row is written to x_perm from shared memory (bf16).
+// Every output is bit-identical to moe_route + moe_preprocess +
+// moe_dispatch_permute; x is read from HBM once.
+#include "device_util.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kFuseThreads = 512;
+constexpr int kFuseWarps = kFuseThreads / 32;
+
+struct FuseArgs {
+  const void* x;
+  const float* w;
+  const float* bias;
+  float* logits_out;
+  int32_t* topk_idx;
+  float* topk_w;
+  int T, D, E, k, renorm, ep, tpb;
+  int32_t* block_counts;   // [gridDim.x][E]
+  unsigned* barrier;       // [2], zero at launch
+  int32_t *counts, *expert_offsets, *rank_splits, *rank_offsets, *mt_start, *pos, *src, *status;
+  bf16* x_perm;
+};
+
+__device__ __forceinline__ void x8(const bf16* p, float (&v)[8]) {
+  const uint4 t = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&t);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float2 f = __bfloat1622float2(h[q]);
+    v[2 * q] = f.x; v[2 * q + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void x8(const float* p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// Shared-memory slot of the 16-byte unit u of W_r (row-major [E, D] fp32, D % 8 == 0).
+// Lane l reads W_r[e, d0 .. d0+7] with d0 = 256 c + 8 l as two units; storing, per row
+// and 256-column chunk, the first units of all lanes, then the second units, makes
+// each of the two reads of a warp 512 contiguous bytes (no bank conflict).  A row's
+// last partial chunk (D % 256) keeps the same split over its lanes.
+__device__ __forceinline__ int w_slot(int u, int D) {
+  const int upr = D >> 2;                    // units per row
+  const int row = u / upr, r = u - row * upr;
+  const int c = r >> 6, j = r & 63;          // chunk of 64 units, unit within it
+  const int cw = min(64, upr - c * 64);      // units in this chunk (even)
+  return row * upr + c * 64 + (j & 1) * (cw >> 1) + (j >> 1);
+}
+
+template <int EP, int TW, typename XT>
+__global__ void __launch_bounds__(kFuseThreads, 1) route_pre_dispatch_kernel(const FuseArgs a) {
+  extern __shared__ uint4 fsm[];
+  const int E = a.E, D = a.D, k = a.k;
+  const int t_lo = blockIdx.x * a.tpb;
+  const int ntok = max(min(t_lo + a.tpb, a.T) - t_lo, 0);
+  float* w_s = reinterpret_cast<float*>(fsm);                          // [E * D], see w_slot
+  const float4* fsm4 = reinterpret_cast<const float4*>(fsm);
+  XT* x_s = reinterpret_cast<XT*>(w_s + (size_t)E * D);               // [tpb * D]
+  int* sel = reinterpret_cast<int*>(x_s + (size_t)a.tpb * D);         // [tpb * k]
+  int* pos_s = sel + a.tpb * k;                                       // [tpb * k]
+  int* cnt = pos_s + a.tpb * k;                                       // [E]
+  int* tmp = cnt + E;                                                 // [E]
+  int* warp_cnt = tmp + E;                                            // [kFuseWarps * E]
+  __shared__ int warp_sums[32];
+  __shared__ int total;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  // 1. W_r and the block's x rows into shared memory, 16-byte loads, U in flight
+  {
+    const int nw = E * D / 4;                                         // 16-byte units of W_r
+    const int nx = ntok * D * (int)sizeof(XT) / 16;                   // of the x rows
+    const uint4* wg = reinterpret_cast<const uint4*>(a.w);
+    const uint4* xg = reinterpret_cast<const uint4*>(static_cast<const XT*>(a.x) + (size_t)t_lo * D);
+    uint4* xs = reinterpret_cast<uint4*>(x_s);
+    constexpr int U = 8;
+    for (int i0 = tid; i0 < nw + nx; i0 += kFuseThreads * U) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = i0 + u * kFuseThreads;
+        if (i < nw) v[u] = __ldg(wg + i);
+        else if (i < nw + nx) v[u] = __ldg(xg + (i - nw));
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int i = i0 + u * kFuseThreads;
+        if (i < nw) fsm[w_slot(i, D)] = v[u];
+        else if (i < nw + nx) xs[i - nw] = v[u];
+      }
+    }
+  }
+  __syncthreads();
+
+  // 2. route: the few-expert router's arithmetic, x from shared memory
+  for (int g0 = warp * TW; g0 < ntok; g0 += kFuseWarps * TW) {
+    double acc[TW][EP];
+#pragma unroll
+    for (int i = 0; i < TW; ++i)
+#pragma unroll
+      for (int e = 0; e < EP; ++e) acc[i][e] = 0.0;
+    const int upr = D >> 2;
+    for (int d0 = lane * 8, c64 = 0; d0 < D; d0 += 256, c64 += 64) {
+      // this lane's two W_r units of the chunk (see w_slot): c64 + lane, and half the
+      // chunk's units further
+      const int u0 = c64 + lane, u1 = u0 + (min(64, upr - c64) >> 1);
+      float xv[TW][8];
+#pragma unroll
+      for (int i = 0; i < TW; ++i) {
+        if (g0 + i < ntok) {
+          x8(x_s + (size_t)(g0 + i) * D + d0, xv[i]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) xv[i][q] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < EP; ++e) {
+        if (e < E) {
+          // W_r[e, d0 .. d0+3] and [d0+4 .. d0+7]
+          const float4 w0 = fsm4[e * upr + u0];
+          const float4 w1 = fsm4[e * upr + u1];
+#pragma unroll
+          for (int i = 0; i < TW; ++i) {
+            float p = xv[i][0] * w0.x;
+            p = fmaf(xv[i][1], w0.y, p);
+            p = fmaf(xv[i][2], w0.z, p);
+            p = fmaf(xv[i][3], w0.w, p);
+            p = fmaf(xv[i][4], w1.x, p);
+            p = fmaf(xv[i][5], w1.y, p);
+            p = fmaf(xv[i][6], w1.z, p);
+            p = fmaf(xv[i][7], w1.w, p);
+            acc[i][e] += (double)p;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < TW; ++i)
+#pragma unroll
+      for (int e = 0; e < EP; ++e)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[i][e] += __shfl_xor_sync(0xffffffffu, acc[i][e], o);
+#pragma unroll
+    for (int i = 0; i < TW; ++i) {
+      if (g0 + i >= ntok) break;
+      const int t = t_lo + g0 + i;
+      float l = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < EP; ++e)
+        if (lane == e) l = (float)acc[i][e];
+      if (lane < E && a.bias != nullptr) l = l + a.bias[lane];
+      if (a.logits_out != nullptr && lane < E) a.logits_out[(size_t)t * E + lane] = l;
+      const int s = warp_topk_write(l, E, k, a.renorm, (size_t)t, a.topk_idx, a.topk_w);
+      if (lane < k) {
+        // an expert id out of range (only NaN logits give one) is what the preprocess
+        // reports as MOE_ERR_INDEX_OOB and skips; so here
+        const bool ok = (unsigned)s < (unsigned)E;
+        sel[(g0 + i) * k + lane] = ok ? s : -1;
+        if (!ok) atomicCAS(a.status, 0, (int)MOE_ERR_INDEX_OOB);
+      }
+    }
+  }
+  __syncthreads();
+
+  // 3. this block's histogram, then every block's
+  for (int e = tid; e < E; e += kFuseThreads) cnt[e] = 0;
+  __syncthreads();
+  for (int f = tid; f < ntok * k; f += kFuseThreads)
+    if (sel[f] >= 0) atomicAdd(&cnt[sel[f]], 1);
+  __syncthreads();
+  for (int e = tid; e < E; e += kFuseThreads) a.block_counts[(size_t)blockIdx.x * E + e] = cnt[e];
+  if (!grid_barrier(a.barrier, gridDim.x, a.status)) return;
+
+  // 4. totals and block-0 outputs, then the in-order rows of the block's pairs
+  pre_totals<kFuseThreads>(a.block_counts, E, a.ep, cnt, tmp, warp_cnt, warp_sums, &total, a.counts,
+                           a.expert_offsets, a.rank_splits, a.rank_offsets, a.mt_start);
+  const int base = t_lo * k;
+  pre_positions<kFuseThreads>(base, base + ntok * k, [&](int f) { return sel[f - base]; }, E, cnt,
+                              warp_cnt, a.pos, a.src, pos_s);
+
+  // 5. dispatch from shared memory: one 16-byte chunk of one pair's row per thread
+  const int cpr = D >> 3;
+  for (int i = tid; i < ntok * k * cpr; i += kFuseThreads) {
+    const int f = i / cpr, ch = i - f * cpr;
+    if (sel[f] < 0) continue;                        // no row (reported above)
+    float v[8];
+    x8(x_s + (size_t)(f / k) * D + ch * 8, v);
+    uint4 o;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) h[q] = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+    *reinterpret_cast<uint4*>(a.x_perm + (size_t)pos_s[f] * D + ch * 8) = o;
+  }
+}
+
+size_t fuse_smem(const moe_config& c, int tpb) {
+  const size_t sx = c.x_dtype == MOE_DT_F32 ? 4 : 2;
+  return (size_t)c.E * c.D * 4 + (size_t)tpb * c.D * sx + 2 * (size_t)tpb * c.top_k * 4 +
+         (size_t)(2 + kFuseWarps) * c.E * 4;
+}
+
+template <int EP, int TW, typename XT>
+cudaError_t launch_fused(const FuseArgs& a, int grid, size_t smem, cudaStream_t s) {
+  auto kern = route_pre_dispatch_kernel<EP, TW, XT>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  int occ = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kFuseThreads, smem);
+  if (err != cudaSuccess) return err;
+  if ((int64_t)occ * sm_count() < grid) return cudaErrorCooperativeLaunchTooLarge;
+  FuseArgs args = a;
+  void* p[] = {&args};
+  err = cudaLaunchCooperativeKernel((const void*)kern, dim3(grid), dim3(kFuseThreads), p, smem, s);
+  if (err != cudaSuccess) return err;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// Shared-memory budget of the fused kernel (W_r, the block's x rows, selections, rows).
+constexpr size_t kFuseSmemLimit = 200u << 10;
+
+bool route_pre_dispatch_applies(const moe_config& c, int max_blocks) {
+  if (c.T <= 0 || c.E > 32) return false;
+  int grid = sm_count();
+  if (grid > max_blocks) grid = max_blocks;
+  if (grid > c.T) grid = c.T;
+  const int tpb = (c.T + grid - 1) / grid;
+  return fuse_smem(c, tpb) <= kFuseSmemLimit;
+}
+
+cudaError_t launch_route_pre_dispatch(const moe_config& c, const void* x, const float* w,
+                                      const float* bias, float* logits_out, int32_t* topk_idx,
+                                      float* topk_w, int32_t* counts, int32_t* expert_offsets,
+                                      int32_t* rank_splits, int32_t* rank_offsets, int32_t* pos,
+                                      int32_t* src, int32_t* block_counts, int max_blocks,
+                                      int32_t* mt_start, unsigned* barrier, bf16* x_perm,
+                                      int32_t* status, cudaStream_t s) {
+  int grid = sm_count();
+  if (grid > max_blocks) grid = max_blocks;
+  if (grid > c.T) grid = c.T;
+  if (grid < 1) return cudaErrorInvalidValue;
+  const int tpb = (c.T + grid - 1) / grid;
+  grid = (c.T + tpb - 1) / tpb;                    // no empty block
+  const size_t smem = fuse_smem(c, tpb);
+  if (smem > kFuseSmemLimit || c.E > 32) return cudaErrorInvalidValue;
+  cudaError_t err = cudaMemsetAsync(barrier, 0, 2 * sizeof(unsigned), s);
+  if (err != cudaSuccess) return err;
+  FuseArgs a;
+  a.x = x; a.w = w; a.bias = bias; a.logits_out = logits_out; a.topk_idx = topk_idx; a.topk_w = topk_w;
+  a.T = c.T; a.D = c.D; a.E = c.E; a.k = c.top_k; a.renorm = c.renormalize; a.ep = c.ep_size;
+  a.tpb = tpb;
+  a.block_counts = block_counts; a.barrier = barrier;
+  a.counts = counts; a.expert_offsets = expert_offsets; a.rank_splits = rank_splits;
+  a.rank_offsets = rank_offsets; a.mt_start = mt_start; a.pos = pos; a.src = src; a.status = status;
+  a.x_perm = x_perm;
+  const bool f32 = c.x_dtype == MOE_DT_F32;
+  if (c.E <= 8)
+    return f32 ? launch_fused<8, 2, float>(a, grid, smem, s) : launch_fused<8, 2, bf16>(a, grid, smem, s);
+  if (c.E <= 16)
+    return f32 ? launch_fused<16, 1, float>(a, grid, smem, s) : launch_fused<16, 1, bf16>(a, grid, smem, s);
+  return f32 ? launch_fused<32, 1, float>(a, grid, smem, s) : launch_fused<32, 1, bf16>(a, grid, smem, s);
+}
+
+}  // namespace moe

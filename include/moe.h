@@ -195,9 +195,31 @@ MOE_API moe_status moe_combine_unpermute(const moe_config* cfg, const void* y_pe
                                  const float* topk_w, const void* x, const void* shared_out,
                                  void* out, void* stream);
 
-/* The whole layer: moe_route, moe_preprocess, moe_dispatch_permute,
- * moe_expert_ffn and moe_combine_unpermute enqueued in that order on `stream`,
- * with the same arguments as above.  logits_out and expert_bias may be NULL. */
+/* Router, preprocess and dispatch together ("Expert Parallel (EP)", Communication
+ * Pattern steps 1-2; "Worked Example: Tracing a Token Through Expert Parallelism",
+ * Steps 1-2): the outputs of moe_route, moe_preprocess and moe_dispatch_permute,
+ * bit for bit, with the same arguments as those calls.  With at most 32 experts and
+ * W_r plus one SM's share of the x rows fitting in 200 KB of shared memory this is
+ * ONE cooperative launch that reads x once (each block routes its tokens, publishes
+ * its expert histogram, passes one grid barrier, writes its pairs' rows and copies
+ * its x rows into x_perm); otherwise (or with MOE_ROUTE_FUSED=0 in the environment)
+ * it enqueues the three calls.  Errors: those of the three calls; a grid barrier that
+ * does not complete within about a second sets MOE_ERR_TIMEOUT in *status. */
+MOE_API moe_status moe_route_dispatch(const moe_config* cfg, const void* x, const float* w_router,
+                              const float* expert_bias, float* logits_out, int32_t* topk_idx,
+                              float* topk_w, int32_t* counts, int32_t* expert_offsets,
+                              int32_t* rank_splits, int32_t* rank_offsets, int32_t* pos,
+                              int32_t* src, void* x_perm, void* workspace, int32_t* status,
+                              void* stream);
+
+/* 1 if moe_route_dispatch runs as one launch for this configuration (on the current
+ * device, with the current environment), else 0 (also for an invalid configuration). */
+MOE_API int32_t moe_route_dispatch_is_fused(const moe_config* cfg);
+
+/* The whole layer: moe_route_dispatch (moe_route, moe_preprocess and
+ * moe_dispatch_permute), moe_expert_ffn and moe_combine_unpermute enqueued in that
+ * order on `stream`, with the same arguments as above.  logits_out and expert_bias
+ * may be NULL. */
 MOE_API moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_router,
                        const float* expert_bias, const void* packed, float* logits_out,
                        int32_t* topk_idx, float* topk_w, int32_t* counts,

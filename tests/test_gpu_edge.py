@@ -90,6 +90,45 @@ def test_few_expert_router_four_tokens_per_warp(T):
     run_and_compare(BASE.with_(T=T, D=512, E=8, top_k=2, F=128, seed=3))
 
 
+@pytest.mark.parametrize("T,D,E,k,xdt,renorm,logits,shared", [
+    (1, 128, 8, 2, "bf16", True, False, False),
+    (3, 256, 8, 8, "bf16", True, True, False),          # k = E
+    (129, 512, 16, 4, "f32", False, True, False),        # fp32 x, no renormalisation
+    (1000, 256, 32, 6, "bf16", True, True, True),
+    (4096, 2048, 8, 2, "bf16", True, False, False),      # the default workload's shape
+    (300, 64, 16, 2, "f32", True, False, False),
+])
+def test_fused_route_dispatch_matches_stage_calls(T, D, E, k, xdt, renorm, logits, shared):
+    """moe_route_dispatch as one cooperative launch gives the bits of moe_route +
+    moe_preprocess + moe_dispatch_permute (routing, weights, logits, counts, offsets,
+    splits, rows, x_perm) and the same layer output (so the same GEMM tile prefix)."""
+    wl = BASE.with_(T=T, D=D, E=E, ep_size=2 if E % 2 == 0 else 1, top_k=k, F=128, x_dtype=xdt,
+                    renormalize=renorm, n_shared=1 if shared else 0, F_shared=128 if shared else 0,
+                    seed=7)
+    inp = W.make_inputs(wl, device="cuda")
+    layer = make_layer(wl, inp, keep_logits=logits)
+    layer.allocate(T)
+    assert M.moe_route_dispatch_is_fused(layer.config(T))
+    keys = ["topk_idx", "topk_w", "counts", "expert_offsets", "rank_splits", "rank_offsets", "pos",
+            "src", "x_perm", "out"] + (["logits"] if logits else [])
+    res = {}
+    for fused in ("0", "1"):
+        os.environ["MOE_ROUTE_FUSED"] = fused
+        try:
+            for key in keys:
+                layer.buf[key].fill_(-3)
+            layer.forward(inp["x"])
+            torch.cuda.synchronize()
+            layer.check_status()
+        finally:
+            del os.environ["MOE_ROUTE_FUSED"]
+        res[fused] = {key: layer.buf[key].clone() for key in keys}
+    for key in keys:
+        assert torch.equal(res["0"][key], res["1"][key]), key
+    ref = oracle_route(wl, inp)
+    compare_routing(res["1"]["topk_idx"].cpu().numpy(), res["1"]["topk_w"].cpu().numpy(), ref)
+
+
 def test_ties_go_to_the_lower_index():
     wl = BASE.with_(T=512, E=8, top_k=2)
     inp = W.make_inputs(wl, device="cuda")
