@@ -86,6 +86,28 @@ __device__ int block_scan_array(int* vals, int n, int* warp_sums, int* total) {
   return *total;
 }
 
+// Exclusive scan of vals[0..n) in place, returns the total (the whole block calls):
+// one warp's shuffles for n <= 32, else block_scan_array.
+__device__ __forceinline__ int scan_array(int* vals, int n, int* warp_sums, int* total) {
+  if (n > 32) return block_scan_array(vals, n, warp_sums, total);
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x < 32) {
+    const int v = lane < n ? vals[lane] : 0;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += t;
+    }
+    if (lane < n) vals[lane] = inc - v;
+    if (lane == 31) *total = inc;
+  }
+  __syncthreads();
+  const int t = *total;
+  __syncthreads();            // every thread has read *total before a next call rewrites it
+  return t;
+}
+
 // After the grid barrier of a cooperative preprocess over NB = gridDim.x blocks, each
 // holding a contiguous chunk of the flat (token, slot) pairs and having published its
 // per-expert histogram row in block_counts[blockIdx.x][E]: cnt[e] becomes the first
@@ -135,7 +157,7 @@ __device__ void pre_totals(const int32_t* block_counts, int E, int ep, int* cnt,
   __syncthreads();
   if (blockIdx.x == 0)
     for (int e = tid; e < E; e += NT) counts[e] = tmp[e];
-  const int R_all = block_scan_array(tmp, E, warp_sums, total);   // tmp = expert offsets
+  const int R_all = scan_array(tmp, E, warp_sums, total);          // tmp = expert offsets
   for (int e = tid; e < E; e += NT) cnt[e] += tmp[e];              // running row of e
   if (blockIdx.x == 0) {
     for (int e = tid; e < E; e += NT) expert_offsets[e] = tmp[e];
@@ -158,7 +180,7 @@ __device__ void pre_totals(const int32_t* block_counts, int E, int ep, int* cnt,
         warp_cnt[e] = (ce + tm - 1) / tm;
       }
       __syncthreads();
-      const int tiles = block_scan_array(warp_cnt, E, warp_sums, total);
+      const int tiles = scan_array(warp_cnt, E, warp_sums, total);
       for (int e = tid; e < E; e += NT) outp[e] = warp_cnt[e];
       if (tid == 0) outp[E] = tiles;
     }

@@ -6,7 +6,8 @@
 //
 // Block b owns tokens [b * tpb, (b + 1) * tpb) and, for the preprocess, the flat
 // (token, slot) pairs of those tokens:
-//  1. W_r and the block's x rows are loaded into shared memory;
+//  1. W_r and the block's x rows are brought into shared memory by bulk copies, each
+//     warp's rows on a barrier of its own, so routing starts as its rows land;
 //  2. each warp routes TW tokens at a time with the arithmetic of the few-expert
 //     router (fp32 8-term slices folded into fp64, lane-parallel over D, exact
 //     argmax top-k, renormalised softmax weights) and keeps the selections;
@@ -55,17 +56,46 @@ __device__ __forceinline__ void x8(const float* p, float (&v)[8]) {
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-// Shared-memory slot of the 16-byte unit u of W_r (row-major [E, D] fp32, D % 8 == 0).
-// Lane l reads W_r[e, d0 .. d0+7] with d0 = 256 c + 8 l as two units; storing, per row
-// and 256-column chunk, the first units of all lanes, then the second units, makes
-// each of the two reads of a warp 512 contiguous bytes (no bank conflict).  A row's
-// last partial chunk (D % 256) keeps the same split over its lanes.
-__device__ __forceinline__ int w_slot(int u, int D) {
-  const int upr = D >> 2;                    // units per row
-  const int row = u / upr, r = u - row * upr;
-  const int c = r >> 6, j = r & 63;          // chunk of 64 units, unit within it
-  const int cw = min(64, upr - c * 64);      // units in this chunk (even)
-  return row * upr + c * 64 + (j & 1) * (cw >> 1) + (j >> 1);
+constexpr long long kFuseWaitLimitCycles = 2000000000ll;   // about 1 s at 2 GHz
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for phase 0 of a staging barrier: false (and MOE_ERR_TIMEOUT) on expiry.
+__device__ __noinline__ bool mbar_wait0(uint32_t bar, int32_t* status) {
+  const long long t0 = clock64();
+  while (!mbar_test(bar, 0)) {
+    if (clock64() - t0 > kFuseWaitLimitCycles) {
+      atomicCAS(status, 0, (int)MOE_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+// Bulk copy (the copy engine) of `bytes` from global to shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
 }
 
 template <int EP, int TW, typename XT>
@@ -74,8 +104,7 @@ __global__ void __launch_bounds__(kFuseThreads, 1) route_pre_dispatch_kernel(con
   const int E = a.E, D = a.D, k = a.k;
   const int t_lo = blockIdx.x * a.tpb;
   const int ntok = max(min(t_lo + a.tpb, a.T) - t_lo, 0);
-  float* w_s = reinterpret_cast<float*>(fsm);                          // [E * D], see w_slot
-  const float4* fsm4 = reinterpret_cast<const float4*>(fsm);
+  float* w_s = reinterpret_cast<float*>(fsm);                          // [E * D]
   XT* x_s = reinterpret_cast<XT*>(w_s + (size_t)E * D);               // [tpb * D]
   int* sel = reinterpret_cast<int*>(x_s + (size_t)a.tpb * D);         // [tpb * k]
   int* pos_s = sel + a.tpb * k;                                       // [tpb * k]
@@ -84,33 +113,38 @@ __global__ void __launch_bounds__(kFuseThreads, 1) route_pre_dispatch_kernel(con
   int* warp_cnt = tmp + E;                                            // [kFuseWarps * E]
   __shared__ int warp_sums[32];
   __shared__ int total;
+  __shared__ __align__(8) uint64_t bars[1 + kFuseWarps];              // W_r, each warp's x rows
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  // 1. W_r and the block's x rows into shared memory, 16-byte loads, U in flight
-  {
-    const int nw = E * D / 4;                                         // 16-byte units of W_r
-    const int nx = ntok * D * (int)sizeof(XT) / 16;                   // of the x rows
-    const uint4* wg = reinterpret_cast<const uint4*>(a.w);
-    const uint4* xg = reinterpret_cast<const uint4*>(static_cast<const XT*>(a.x) + (size_t)t_lo * D);
-    uint4* xs = reinterpret_cast<uint4*>(x_s);
-    constexpr int U = 8;
-    for (int i0 = tid; i0 < nw + nx; i0 += kFuseThreads * U) {
-      uint4 v[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int i = i0 + u * kFuseThreads;
-        if (i < nw) v[u] = __ldg(wg + i);
-        else if (i < nw + nx) v[u] = __ldg(xg + (i - nw));
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int i = i0 + u * kFuseThreads;
-        if (i < nw) fsm[w_slot(i, D)] = v[u];
-        else if (i < nw + nx) xs[i - nw] = v[u];
-      }
-    }
+  // 1. bulk copies into shared memory: W_r on bars[0], warp w's token rows on bars[1 + w],
+  //    so a warp starts routing once W_r and its own rows are in
+  if (tid == 0) {
+    for (int i = 0; i <= kFuseWarps; ++i) mbar_init(smem_addr(&bars[i]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  const uint32_t xrow = (uint32_t)D * (uint32_t)sizeof(XT);
+  if (tid == 0) {
+    mbar_expect(smem_addr(&bars[0]), (uint32_t)E * D * 4);
+    bulk_g2s(w_s, a.w, (uint32_t)E * D * 4, smem_addr(&bars[0]));
+    const XT* xg = static_cast<const XT*>(a.x) + (size_t)t_lo * D;
+    for (int w = 0; w < kFuseWarps; ++w) {
+      uint32_t n = 0;
+      for (int g0 = w * TW; g0 < ntok; g0 += kFuseWarps * TW) n += (uint32_t)min(TW, ntok - g0);
+      const uint32_t bar = smem_addr(&bars[1 + w]);
+      mbar_expect(bar, n * xrow);
+      for (int g0 = w * TW; g0 < ntok; g0 += kFuseWarps * TW)
+        for (int i = 0; i < TW && g0 + i < ntok; ++i)
+          bulk_g2s(x_s + (size_t)(g0 + i) * D, xg + (size_t)(g0 + i) * D, xrow, bar);
+    }
+  }
+  {
+    bool ok = true;
+    if (lane == 0) ok = mbar_wait0(smem_addr(&bars[0]), a.status) && mbar_wait0(smem_addr(&bars[1 + warp]), a.status);
+    // on a timeout (reported) the warp goes on with whatever shared memory holds
+    __syncwarp();
+    (void)ok;
+  }
 
   // 2. route: the few-expert router's arithmetic, x from shared memory
   for (int g0 = warp * TW; g0 < ntok; g0 += kFuseWarps * TW) {
@@ -119,11 +153,7 @@ __global__ void __launch_bounds__(kFuseThreads, 1) route_pre_dispatch_kernel(con
     for (int i = 0; i < TW; ++i)
 #pragma unroll
       for (int e = 0; e < EP; ++e) acc[i][e] = 0.0;
-    const int upr = D >> 2;
-    for (int d0 = lane * 8, c64 = 0; d0 < D; d0 += 256, c64 += 64) {
-      // this lane's two W_r units of the chunk (see w_slot): c64 + lane, and half the
-      // chunk's units further
-      const int u0 = c64 + lane, u1 = u0 + (min(64, upr - c64) >> 1);
+    for (int d0 = lane * 8; d0 < D; d0 += 256) {
       float xv[TW][8];
 #pragma unroll
       for (int i = 0; i < TW; ++i) {
@@ -137,9 +167,8 @@ __global__ void __launch_bounds__(kFuseThreads, 1) route_pre_dispatch_kernel(con
 #pragma unroll
       for (int e = 0; e < EP; ++e) {
         if (e < E) {
-          // W_r[e, d0 .. d0+3] and [d0+4 .. d0+7]
-          const float4 w0 = fsm4[e * upr + u0];
-          const float4 w1 = fsm4[e * upr + u1];
+          const float4 w0 = *reinterpret_cast<const float4*>(w_s + (size_t)e * D + d0);
+          const float4 w1 = *reinterpret_cast<const float4*>(w_s + (size_t)e * D + d0 + 4);
 #pragma unroll
           for (int i = 0; i < TW; ++i) {
             float p = xv[i][0] * w0.x;
@@ -199,18 +228,21 @@ __global__ void __launch_bounds__(kFuseThreads, 1) route_pre_dispatch_kernel(con
   pre_positions<kFuseThreads>(base, base + ntok * k, [&](int f) { return sel[f - base]; }, E, cnt,
                               warp_cnt, a.pos, a.src, pos_s);
 
-  // 5. dispatch from shared memory: one 16-byte chunk of one pair's row per thread
+  // 5. dispatch from shared memory: a warp per pair, 16 bytes of its row per lane
   const int cpr = D >> 3;
-  for (int i = tid; i < ntok * k * cpr; i += kFuseThreads) {
-    const int f = i / cpr, ch = i - f * cpr;
+  for (int f = warp; f < ntok * k; f += kFuseWarps) {
     if (sel[f] < 0) continue;                        // no row (reported above)
-    float v[8];
-    x8(x_s + (size_t)(f / k) * D + ch * 8, v);
-    uint4 o;
-    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
+    const XT* row = x_s + (size_t)(f / k) * D;
+    bf16* dst = a.x_perm + (size_t)pos_s[f] * D;
+    for (int ch = lane; ch < cpr; ch += 32) {
+      float v[8];
+      x8(row + ch * 8, v);
+      uint4 o;
+      __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) h[q] = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
-    *reinterpret_cast<uint4*>(a.x_perm + (size_t)pos_s[f] * D + ch * 8) = o;
+      for (int q = 0; q < 4; ++q) h[q] = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+      *reinterpret_cast<uint4*>(dst + ch * 8) = o;
+    }
   }
 }
 
