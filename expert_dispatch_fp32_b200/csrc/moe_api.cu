@@ -409,10 +409,22 @@ moe_status moe_route_dispatch(const moe_config* cfg, const void* x, const float*
   MOE_CHECK_PTR(status);
   if (logits_out != nullptr && !aligned16(logits_out)) return MOE_ERR_INVALID_ARG;
   uint8_t* ws = (uint8_t*)workspace;
-  return cuda_status(launch_route_pre_dispatch(
+  const cudaError_t err = launch_route_pre_dispatch(
       c, x, w_router, expert_bias, logits_out, topk_idx, topk_w, counts, expert_offsets, rank_splits,
       rank_offsets, pos, src, (int32_t*)(ws + L.block_counts), L.nblk, (int32_t*)(ws + L.mt_start),
-      (unsigned*)(ws + L.barrier), (bf16*)x_perm, status, as_stream(stream)));
+      (unsigned*)(ws + L.barrier), (bf16*)x_perm, status, as_stream(stream));
+  if (err == cudaErrorCooperativeLaunchTooLarge) {
+    // fewer SMs available than the one-block-per-SM grid needs (a partitioned GPU):
+    // the stage calls compute the same outputs
+    (void)cudaGetLastError();
+    st = moe_route(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w, workspace, stream);
+    if (st != MOE_OK) return st;
+    st = moe_preprocess(cfg, topk_idx, counts, expert_offsets, rank_splits, rank_offsets, pos, src,
+                        workspace, status, stream);
+    if (st != MOE_OK) return st;
+    return moe_dispatch_permute(cfg, x, pos, x_perm, stream);
+  }
+  return cuda_status(err);
 }
 
 moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_router,

@@ -203,8 +203,9 @@ MOE_API moe_status moe_combine_unpermute(const moe_config* cfg, const void* y_pe
  * ONE cooperative launch that reads x once (each block routes its tokens, publishes
  * its expert histogram, passes one grid barrier, writes its pairs' rows and copies
  * its x rows into x_perm); otherwise (or with MOE_ROUTE_FUSED=0 in the environment)
- * it enqueues the three calls.  Errors: those of the three calls; a grid barrier that
- * does not complete within about a second sets MOE_ERR_TIMEOUT in *status. */
+ * it enqueues the three calls, as it also does when the cooperative launch is refused
+ * for want of SMs.  Errors: those of the three calls; a grid barrier that does not
+ * complete within about a second sets MOE_ERR_TIMEOUT in *status. */
 MOE_API moe_status moe_route_dispatch(const moe_config* cfg, const void* x, const float* w_router,
                               const float* expert_bias, float* logits_out, int32_t* topk_idx,
                               float* topk_w, int32_t* counts, int32_t* expert_offsets,
