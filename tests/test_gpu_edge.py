@@ -129,6 +129,29 @@ def test_fused_route_dispatch_matches_stage_calls(T, D, E, k, xdt, renorm, logit
     compare_routing(res["1"]["topk_idx"].cpu().numpy(), res["1"]["topk_w"].cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("k,D,shared", [(6, 320, True), (7, 512, False), (8, 1088, True)])
+def test_combine_forms_agree(k, D, shared):
+    """The combine that loads every routed row of a step before its multiply-adds (used
+    for k = 6..8) gives the bits of the slot-by-slot form, and the layer matches the
+    oracle (D not a multiple of 256: a ragged last column chunk)."""
+    wl = BASE.with_(T=333, D=D, E=16, ep_size=4, top_k=k, F=128,
+                    n_shared=1 if shared else 0, F_shared=128 if shared else 0, seed=4)
+    inp = W.make_inputs(wl, device="cuda")
+    layer = make_layer(wl, inp)
+    outs = []
+    for form in ("0", "1"):
+        os.environ["MOE_PERMUTE_V"] = form
+        try:
+            outs.append(layer.forward(inp["x"]).clone())
+            torch.cuda.synchronize()
+        finally:
+            del os.environ["MOE_PERMUTE_V"]
+    layer.check_status()
+    assert torch.equal(outs[0], outs[1])
+    res = oracle_layer(wl, inp)
+    assert_layer_close(f64(outs[1]), res["out"], f64(inp["x"]))
+
+
 def test_ties_go_to_the_lower_index():
     wl = BASE.with_(T=512, E=8, top_k=2)
     inp = W.make_inputs(wl, device="cuda")
