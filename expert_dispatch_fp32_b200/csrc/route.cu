@@ -352,26 +352,35 @@ cudaError_t launch_route_t(const moe_config& c, const XT* x, const float* w_rout
 constexpr int kRouterRowBlock = 128;      // experts per 256-row (hi, mid) block
 constexpr int kRefineWarps = 4;
 
+constexpr int kSplitRows = 8;       // expert rows per thread of the W_r split
 __global__ void __launch_bounds__(128)
 router_split_kernel(const float* __restrict__ w, int E, int Epad, int D, bf16* __restrict__ bsplit,
                     unsigned* __restrict__ wmax_bits) {
   const int dq = blockIdx.x * blockDim.x + threadIdx.x;     // 8-column chunk
   if (dq * 8 >= D) return;
   const int d = dq * 8;
-  const int e0 = blockIdx.y * 16;
+  const int e0 = blockIdx.y * kSplitRows;
   float mx[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) mx[i] = 0.f;
-  for (int e = e0; e < e0 + 16 && e < Epad; ++e) {
-    float v[8];
-    if (e < E) {
-      const float4 a = __ldg(reinterpret_cast<const float4*>(w + (size_t)e * D + d));
-      const float4 b = __ldg(reinterpret_cast<const float4*>(w + (size_t)e * D + d + 4));
-      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-    } else {
+  // all kSplitRows rows' loads first (in flight together), then split and store
+  float4 va[kSplitRows], vb[kSplitRows];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+  for (int r = 0; r < kSplitRows; ++r) {
+    const int e = e0 + r;
+    if (e < E) {
+      va[r] = __ldg(reinterpret_cast<const float4*>(w + (size_t)e * D + d));
+      vb[r] = __ldg(reinterpret_cast<const float4*>(w + (size_t)e * D + d + 4));
+    } else {
+      va[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+      vb[r] = va[r];
     }
+  }
+#pragma unroll
+  for (int r = 0; r < kSplitRows; ++r) {
+    const int e = e0 + r;
+    if (e >= Epad) break;
+    const float v[8] = {va[r].x, va[r].y, va[r].z, va[r].w, vb[r].x, vb[r].y, vb[r].z, vb[r].w};
     uint4 hi, mid;
     __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(&hi);
     __nv_bfloat16* m = reinterpret_cast<__nv_bfloat16*>(&mid);
@@ -548,8 +557,8 @@ cudaError_t launch_route_tc(const moe_config& c, const bf16* x, const float* w, 
   if (err != cudaSuccess) return err;
   err = cudaMemsetAsync(rs.counter, 0, sizeof(int32_t), s);
   if (err != cudaSuccess) return err;
-  dim3 sgrid((c.D / 8 + 127) / 128, (Epad + 15) / 16);
-  router_split_kernel<<<sgrid, 128, 0, s>>>(w, c.E, Epad, c.D, rs.bsplit,
+  dim3 sgrid((c.D / 8 + 63) / 64, (Epad + kSplitRows - 1) / kSplitRows);
+  router_split_kernel<<<sgrid, 64, 0, s>>>(w, c.E, Epad, c.D, rs.bsplit,
                                             reinterpret_cast<unsigned*>(rs.wmax));
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
