@@ -97,6 +97,9 @@ def test_few_expert_router_four_tokens_per_warp(T):
     (1000, 256, 32, 6, "bf16", True, True, True),
     (4096, 2048, 8, 2, "bf16", True, False, False),      # the default workload's shape
     (300, 64, 16, 2, "f32", True, False, False),
+    (148, 256, 1, 1, "bf16", True, False, False),       # one expert; one token per block
+    (445, 128, 4, 4, "bf16", False, True, False),        # k = E, four tokens per block
+    (20, 128, 32, 32, "bf16", True, True, True),         # k = E = 32: every lane selects
 ])
 def test_fused_route_dispatch_matches_stage_calls(T, D, E, k, xdt, renorm, logits, shared):
     """moe_route_dispatch as one cooperative launch gives the bits of moe_route +
