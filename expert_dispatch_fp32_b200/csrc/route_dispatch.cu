@@ -89,6 +89,12 @@ __device__ __noinline__ bool mbar_wait0(uint32_t bar, int32_t* status) {
   }
   return true;
 }
+// Bulk copy (the copy engine) of `bytes` from shared to global memory (bulk group).
+__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_addr(src)), "r"(bytes)
+               : "memory");
+}
 // Bulk copy (the copy engine) of `bytes` from global to shared memory, completing on `bar`.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
@@ -228,7 +234,25 @@ __global__ void __launch_bounds__(kFuseThreads, 1) route_pre_dispatch_kernel(con
   pre_positions<kFuseThreads>(base, base + ntok * k, [&](int f) { return sel[f - base]; }, E, cnt,
                               warp_cnt, a.pos, a.src, pos_s);
 
-  // 5. dispatch from shared memory: a warp per pair, 16 bytes of its row per lane
+  // 5. dispatch from shared memory.  bf16 x: the row is already x_perm's bytes, one bulk
+  //    copy per pair (issued by lane 0 of a warp, which waits until its copies have read
+  //    shared memory before the block may exit); fp32 x: a warp per pair converts.
+  if (sizeof(XT) == 2) {
+    if (lane == 0) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      int issued = 0;
+      for (int f = warp; f < ntok * k; f += kFuseWarps) {
+        if (sel[f] < 0) continue;                    // no row (reported above)
+        bulk_s2g(a.x_perm + (size_t)pos_s[f] * D, x_s + (size_t)(f / k) * D, (uint32_t)D * 2);
+        ++issued;
+      }
+      if (issued) {
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      }
+    }
+    return;
+  }
   const int cpr = D >> 3;
   for (int f = warp; f < ntok * k; f += kFuseWarps) {
     if (sel[f] < 0) continue;                        // no row (reported above)
