@@ -761,6 +761,9 @@ __device__ __noinline__ bool wait_count(const int32_t* cnt, int need, volatile i
 }
 
 __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(const __grid_constant__ PairArgs p) {
+  // launched as a programmatic dependent of the previous kernel on the stream: wait until
+  // that kernel has completed and its writes are visible (a no-op otherwise)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   using C = PairCfg;
   constexpr int S = C::kStages, BN = C::BN, TM2 = 2 * kTileM;
   extern __shared__ uint8_t smem_raw[];
@@ -855,7 +858,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         const int tile = leader
             ? tq_post<true>(p.counter, next, total, qi, qfull0, qempty0, tq, abort_flag, p.status)
             : tq_take<false>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
-        if (tile < 0) break;
+        if (tile < 0) {
+          // no tile left for this CTA: the next kernel on the stream may start launching
+          // (it waits for this grid's completion before it reads anything)
+          asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+          break;
+        }
         PairTile t;
         decode_pair_tile(tile, pstart, nph, mt, off, G, dmt, doff, p, t);
         const PhaseArgs& P = p.ph[t.ph];
@@ -1057,13 +1065,19 @@ cudaError_t launch_tc_pair(const PairArgs& a, int clusters, cudaStream_t s) {
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: the grid may be scheduled while the previous kernel
+  // finishes (the kernel's first instruction waits for that kernel's completion)
+  // (MOE_PDL=0 in the environment: plain stream order; read at each call, for comparison)
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  const char* pdl_env = getenv("MOE_PDL");
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = (pdl_env && pdl_env[0] == '0') ? 1 : 2;
   err = cudaLaunchKernelEx(&cfg, kern, a);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();

@@ -8,6 +8,9 @@
 
 namespace moe {
 
+// Counter word of the fused FFN launch (words 0..4: the router GEMM and the separate GEMMs).
+constexpr int kFfnCounter = 5;
+
 WsLayout ws_layout(const moe_config& c) {
   WsLayout L;
   const size_t T = (size_t)c.T, E = (size_t)c.E;
@@ -30,6 +33,7 @@ WsLayout ws_layout(const moe_config& c) {
   // shared gate_up bands (ceil(T/256))
   const size_t done_slots = (size_t)(T * c.top_k) / 256 + E + (T + 255) / 256 + 2;
   L.counters = o;     o = align256(o + (8 + done_slots) * sizeof(int32_t));
+  L.done_slots = done_slots;
   L.total = o;
   return L;
 }
@@ -198,7 +202,7 @@ namespace {
 moe_status ffn_run(const moe_config* cfg, const void* x_perm, const void* x,
                    const int32_t* expert_offsets, const void* packed, void* act, void* y_perm,
                    void* shared_out, void* workspace, int32_t* status, void* stream, bool routed,
-                   bool shared) {
+                   bool shared, bool counters_zeroed = false) {
   moe_status st = moe_validate_config(cfg);
   if (st != MOE_OK) return st;
   const moe_config& c = *cfg;
@@ -308,10 +312,15 @@ moe_status ffn_run(const moe_config* cfg, const void* x_perm, const void* x,
     if (shared) ph[n++] = su;
     if (routed) { ph[n] = dn; ph[n].dep = 0; ++n; }
     if (shared) { ph[n] = sd; ph[n].dep = routed ? 1 : 0; ++n; }
+    // tile counter: word kFfnCounter; band counts from word 8.  Zeroed here unless the
+    // caller (moe_forward) zeroed them earlier on the stream, so that the launch directly
+    // follows the previous kernel (programmatic dependent launch needs no memset between)
     const int64_t slots = pair_done_slots(ph, n);
-    if (cudaMemsetAsync(ctr, 0, (size_t)(8 + slots) * sizeof(int32_t), s) != cudaSuccess)
+    if (!counters_zeroed &&
+        cudaMemsetAsync(ctr + kFfnCounter, 0, (size_t)(8 - kFfnCounter + slots) * sizeof(int32_t), s) !=
+            cudaSuccess)
       return MOE_ERR_CUDA;
-    return cuda_status(launch_grouped_pair(ph, n, ctr, ctr + 8, s));
+    return cuda_status(launch_grouped_pair(ph, n, ctr + kFfnCounter, ctr + 8, s));
   }
 
   // Otherwise one launch per GEMM, each with its own tile counter.
@@ -434,12 +443,25 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_rout
                        int32_t* pos, int32_t* src, void* x_perm, void* act, void* y_perm,
                        void* shared_out, void* out, void* workspace, int32_t* status,
                        void* stream) {
-  moe_status st = moe_route_dispatch(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w,
-                                     counts, expert_offsets, rank_splits, rank_offsets, pos, src,
-                                     x_perm, workspace, status, stream);
+  moe_status st = moe_validate_config(cfg);
   if (st != MOE_OK) return st;
-  st = moe_expert_ffn(cfg, x_perm, x, expert_offsets, packed, act, y_perm, shared_out, workspace,
-                      status, stream);
+  MOE_CHECK_PTR(workspace);
+  {
+    // the expert FFN's tile counter and band counts, zeroed before the router so that
+    // the FFN launch follows the dispatch directly
+    const WsLayout L = ws_layout(*cfg);
+    int32_t* ctr = (int32_t*)((uint8_t*)workspace + L.counters);
+    if (cfg->T > 0 && cudaMemsetAsync(ctr + kFfnCounter, 0,
+                                      (8 - kFfnCounter + L.done_slots) * sizeof(int32_t),
+                                      as_stream(stream)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  st = moe_route_dispatch(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w, counts,
+                          expert_offsets, rank_splits, rank_offsets, pos, src, x_perm, workspace,
+                          status, stream);
+  if (st != MOE_OK) return st;
+  st = ffn_run(cfg, x_perm, x, expert_offsets, packed, act, y_perm, shared_out, workspace, status,
+               stream, true, cfg->n_shared > 0 && shared_out != nullptr, true);
   if (st != MOE_OK) return st;
   return moe_combine_unpermute(cfg, y_perm, pos, topk_w, x, shared_out, out, stream);
 }

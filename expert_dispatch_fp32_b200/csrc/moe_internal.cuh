@@ -34,8 +34,10 @@ struct WsLayout {
   size_t r_split;       // bf16 [2*Epad, D]: tensor-core router weights
   size_t r_wmax;        // fp32 [D]
   size_t r_approx;      // fp32 [T, Epad]
-  size_t counters;      // int32 [8]: GEMM tile counters (router, routed up/down, shared up/down),
-                        // followed directly by the fused FFN launch's band counts int32 [done_slots]
+  size_t counters;      // int32 [8]: GEMM tile counters (router, routed up/down, shared up/down,
+                        // the fused FFN launch), followed directly by the fused FFN launch's
+                        // band counts int32 [done_slots]
+  size_t done_slots;
   size_t total;
   int nblk;
 };

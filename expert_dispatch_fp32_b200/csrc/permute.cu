@@ -5,6 +5,8 @@
 // Tracing a Token Through Expert Parallelism", Step 2 (each chosen expert gets a
 // copy of the token), Step 4 (weighted sum of the expert outputs) and Step 5
 // (residual add).  On one GPU the exchange is the gather itself.
+#include <string.h>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -81,6 +83,7 @@ combine_kernel(const bf16* __restrict__ y_perm, const int32_t* __restrict__ pos,
                const float* __restrict__ topk_w, const XT* __restrict__ x,
                const bf16* __restrict__ shared, XT* __restrict__ out, int T, int D, int k,
                uint32_t R) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // see launch_pdl
   constexpr int U = 2;
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
@@ -130,6 +133,7 @@ __global__ void __launch_bounds__(kCombineThreads)
 combine_k_kernel(const bf16* __restrict__ y_perm, const int32_t* __restrict__ pos,
                  const float* __restrict__ topk_w, const XT* __restrict__ x,
                  const bf16* __restrict__ shared, XT* __restrict__ out, int T, int D, uint32_t R) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // see launch_pdl
   const int lane = threadIdx.x & 31;
   const int wpb = blockDim.x >> 5;
   for (int t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
@@ -157,6 +161,25 @@ combine_k_kernel(const bf16* __restrict__ y_perm, const int32_t* __restrict__ po
       st8(out + (size_t)t * D + c, acc);
     }
   }
+}
+
+// Launch as a programmatic dependent of the previous kernel on the stream: the grid may
+// be scheduled while that kernel finishes; the kernel's first instruction
+// (griddepcontrol.wait) waits until it has completed and its writes are visible.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  const char* pdl_env = getenv("MOE_PDL");       // MOE_PDL=0: plain stream order
+  cfg.attrs = attr;
+  cfg.numAttrs = (pdl_env && pdl_env[0] == '0') ? 0 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
 int combine_grid(int T) {
@@ -198,25 +221,21 @@ cudaError_t launch_combine(const moe_config& c, const bf16* y_perm, const int32_
   const char* env = getenv("MOE_PERMUTE_V");
   const bool hoist = !(env && env[0] == '0') && c.x_dtype == MOE_DT_BF16;
 #define MOE_COMBINE_K(KC)                                                                       \
-  if (hoist && c.top_k == KC) {                                                                 \
-    combine_k_kernel<bf16, KC><<<combine_grid(c.T), kCombineThreads, 0, s>>>(                   \
-        y_perm, pos, topk_w, static_cast<const bf16*>(x), shared_out, static_cast<bf16*>(out),  \
-        c.T, c.D, R);                                                                           \
-    return cudaGetLastError();                                                                  \
-  }
+  if (hoist && c.top_k == KC)                                                                   \
+    return launch_pdl(combine_k_kernel<bf16, KC>, combine_grid(c.T), kCombineThreads, s, y_perm, \
+                      pos, topk_w, static_cast<const bf16*>(x), shared_out,                      \
+                      static_cast<bf16*>(out), c.T, c.D, R);
   MOE_COMBINE_K(6)
   MOE_COMBINE_K(7)
   MOE_COMBINE_K(8)
 #undef MOE_COMBINE_K
   if (c.x_dtype == MOE_DT_F32)
-    combine_kernel<float><<<combine_grid(c.T), kCombineThreads, 0, s>>>(
-        y_perm, pos, topk_w, static_cast<const float*>(x), shared_out, static_cast<float*>(out),
-        c.T, c.D, c.top_k, R);
-  else
-    combine_kernel<bf16><<<combine_grid(c.T), kCombineThreads, 0, s>>>(
-        y_perm, pos, topk_w, static_cast<const bf16*>(x), shared_out, static_cast<bf16*>(out), c.T,
-        c.D, c.top_k, R);
-  return cudaGetLastError();
+    return launch_pdl(combine_kernel<float>, combine_grid(c.T), kCombineThreads, s, y_perm, pos,
+                      topk_w, static_cast<const float*>(x), shared_out, static_cast<float*>(out),
+                      c.T, c.D, c.top_k, R);
+  return launch_pdl(combine_kernel<bf16>, combine_grid(c.T), kCombineThreads, s, y_perm, pos, topk_w,
+                    static_cast<const bf16*>(x), shared_out, static_cast<bf16*>(out), c.T, c.D,
+                    c.top_k, R);
 }
 
 }  // namespace moe

@@ -234,6 +234,9 @@ __global__ void __launch_bounds__(kFuseThreads, 1) route_pre_dispatch_kernel(con
   pre_positions<kFuseThreads>(base, base + ntok * k, [&](int f) { return sel[f - base]; }, E, cnt,
                               warp_cnt, a.pos, a.src, pos_s);
 
+  // the expert FFN (launched as a programmatic dependent) may start launching now
+  if (tid == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
   // 5. dispatch from shared memory.  bf16 x: the row is already x_perm's bytes, one bulk
   //    copy per pair (issued by lane 0 of a warp, which waits until its copies have read
   //    shared memory before the block may exit); fp32 x: a warp per pair converts.
