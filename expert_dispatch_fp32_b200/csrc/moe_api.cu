@@ -73,6 +73,62 @@ inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK 
     if ((p) == nullptr || !aligned16(p)) return MOE_ERR_INVALID_ARG; \
   } while (0)
 
+// moe_route_dispatch; barrier_zeroed: grid-barrier words the caller zeroed on the stream
+// already (moe_forward's one memset), else the workspace's words, zeroed here.
+moe_status route_dispatch_run(const moe_config* cfg, const void* x, const float* w_router,
+                              const float* expert_bias, float* logits_out, int32_t* topk_idx,
+                              float* topk_w, int32_t* counts, int32_t* expert_offsets,
+                              int32_t* rank_splits, int32_t* rank_offsets, int32_t* pos,
+                              int32_t* src, void* x_perm, void* workspace, int32_t* status,
+                              void* stream, unsigned* barrier_zeroed) {
+  moe_status st = moe_validate_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  const WsLayout L = ws_layout(c);
+  // MOE_ROUTE_FUSED=0 runs the three stage calls (read at each call; for comparison)
+  const bool fused = moe_route_dispatch_is_fused(cfg) != 0;
+  if (!fused) {
+    st = moe_route(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w, workspace, stream);
+    if (st != MOE_OK) return st;
+    st = moe_preprocess(cfg, topk_idx, counts, expert_offsets, rank_splits, rank_offsets, pos, src,
+                        workspace, status, stream);
+    if (st != MOE_OK) return st;
+    return moe_dispatch_permute(cfg, x, pos, x_perm, stream);
+  }
+  MOE_CHECK_PTR(x);
+  MOE_CHECK_PTR(w_router);
+  MOE_CHECK_PTR(topk_idx);
+  MOE_CHECK_PTR(topk_w);
+  MOE_CHECK_PTR(counts);
+  MOE_CHECK_PTR(expert_offsets);
+  MOE_CHECK_PTR(rank_splits);
+  MOE_CHECK_PTR(rank_offsets);
+  MOE_CHECK_PTR(pos);
+  MOE_CHECK_PTR(src);
+  MOE_CHECK_PTR(x_perm);
+  MOE_CHECK_PTR(workspace);
+  MOE_CHECK_PTR(status);
+  if (logits_out != nullptr && !aligned16(logits_out)) return MOE_ERR_INVALID_ARG;
+  uint8_t* ws = (uint8_t*)workspace;
+  const cudaError_t err = launch_route_pre_dispatch(
+      c, x, w_router, expert_bias, logits_out, topk_idx, topk_w, counts, expert_offsets, rank_splits,
+      rank_offsets, pos, src, (int32_t*)(ws + L.block_counts), L.nblk, (int32_t*)(ws + L.mt_start),
+      barrier_zeroed != nullptr ? barrier_zeroed : (unsigned*)(ws + L.barrier), barrier_zeroed != nullptr,
+      (bf16*)x_perm, status, as_stream(stream));
+  if (err == cudaErrorCooperativeLaunchTooLarge) {
+    // fewer SMs available than the one-block-per-SM grid needs (a partitioned GPU):
+    // the stage calls compute the same outputs
+    (void)cudaGetLastError();
+    st = moe_route(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w, workspace, stream);
+    if (st != MOE_OK) return st;
+    st = moe_preprocess(cfg, topk_idx, counts, expert_offsets, rank_splits, rank_offsets, pos, src,
+                        workspace, status, stream);
+    if (st != MOE_OK) return st;
+    return moe_dispatch_permute(cfg, x, pos, x_perm, stream);
+  }
+  return cuda_status(err);
+}
+
 }  // namespace
 
 extern "C" {
@@ -389,51 +445,9 @@ moe_status moe_route_dispatch(const moe_config* cfg, const void* x, const float*
                               int32_t* rank_splits, int32_t* rank_offsets, int32_t* pos,
                               int32_t* src, void* x_perm, void* workspace, int32_t* status,
                               void* stream) {
-  moe_status st = moe_validate_config(cfg);
-  if (st != MOE_OK) return st;
-  const moe_config& c = *cfg;
-  const WsLayout L = ws_layout(c);
-  // MOE_ROUTE_FUSED=0 runs the three stage calls (read at each call; for comparison)
-  const bool fused = moe_route_dispatch_is_fused(cfg) != 0;
-  if (!fused) {
-    st = moe_route(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w, workspace, stream);
-    if (st != MOE_OK) return st;
-    st = moe_preprocess(cfg, topk_idx, counts, expert_offsets, rank_splits, rank_offsets, pos, src,
-                        workspace, status, stream);
-    if (st != MOE_OK) return st;
-    return moe_dispatch_permute(cfg, x, pos, x_perm, stream);
-  }
-  MOE_CHECK_PTR(x);
-  MOE_CHECK_PTR(w_router);
-  MOE_CHECK_PTR(topk_idx);
-  MOE_CHECK_PTR(topk_w);
-  MOE_CHECK_PTR(counts);
-  MOE_CHECK_PTR(expert_offsets);
-  MOE_CHECK_PTR(rank_splits);
-  MOE_CHECK_PTR(rank_offsets);
-  MOE_CHECK_PTR(pos);
-  MOE_CHECK_PTR(src);
-  MOE_CHECK_PTR(x_perm);
-  MOE_CHECK_PTR(workspace);
-  MOE_CHECK_PTR(status);
-  if (logits_out != nullptr && !aligned16(logits_out)) return MOE_ERR_INVALID_ARG;
-  uint8_t* ws = (uint8_t*)workspace;
-  const cudaError_t err = launch_route_pre_dispatch(
-      c, x, w_router, expert_bias, logits_out, topk_idx, topk_w, counts, expert_offsets, rank_splits,
-      rank_offsets, pos, src, (int32_t*)(ws + L.block_counts), L.nblk, (int32_t*)(ws + L.mt_start),
-      (unsigned*)(ws + L.barrier), (bf16*)x_perm, status, as_stream(stream));
-  if (err == cudaErrorCooperativeLaunchTooLarge) {
-    // fewer SMs available than the one-block-per-SM grid needs (a partitioned GPU):
-    // the stage calls compute the same outputs
-    (void)cudaGetLastError();
-    st = moe_route(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w, workspace, stream);
-    if (st != MOE_OK) return st;
-    st = moe_preprocess(cfg, topk_idx, counts, expert_offsets, rank_splits, rank_offsets, pos, src,
-                        workspace, status, stream);
-    if (st != MOE_OK) return st;
-    return moe_dispatch_permute(cfg, x, pos, x_perm, stream);
-  }
-  return cuda_status(err);
+  return route_dispatch_run(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w, counts,
+                            expert_offsets, rank_splits, rank_offsets, pos, src, x_perm, workspace,
+                            status, stream, nullptr);
 }
 
 moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_router,
@@ -447,8 +461,9 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_rout
   if (st != MOE_OK) return st;
   MOE_CHECK_PTR(workspace);
   {
-    // the expert FFN's tile counter and band counts, zeroed before the router so that
-    // the FFN launch follows the dispatch directly
+    // the expert FFN's tile counter and band counts (and, in words 6-7, the fused router's
+    // grid barrier), zeroed before the router so that the FFN launch follows the dispatch
+    // directly
     const WsLayout L = ws_layout(*cfg);
     int32_t* ctr = (int32_t*)((uint8_t*)workspace + L.counters);
     if (cfg->T > 0 && cudaMemsetAsync(ctr + kFfnCounter, 0,
@@ -456,9 +471,14 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const float* w_rout
                                       as_stream(stream)) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
-  st = moe_route_dispatch(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w, counts,
-                          expert_offsets, rank_splits, rank_offsets, pos, src, x_perm, workspace,
-                          status, stream);
+  {
+    // the fused router's grid-barrier words: two words of the block zeroed above
+    const WsLayout L = ws_layout(*cfg);
+    int32_t* ctr = (int32_t*)((uint8_t*)workspace + L.counters);
+    st = route_dispatch_run(cfg, x, w_router, expert_bias, logits_out, topk_idx, topk_w, counts,
+                            expert_offsets, rank_splits, rank_offsets, pos, src, x_perm, workspace,
+                            status, stream, reinterpret_cast<unsigned*>(ctr + kFfnCounter + 1));
+  }
   if (st != MOE_OK) return st;
   st = ffn_run(cfg, x_perm, x, expert_offsets, packed, act, y_perm, shared_out, workspace, status,
                stream, true, cfg->n_shared > 0 && shared_out != nullptr, true);

@@ -96,8 +96,8 @@ cudaError_t launch_route_pre_dispatch(const moe_config& c, const void* x, const 
                                       float* topk_w, int32_t* counts, int32_t* expert_offsets,
                                       int32_t* rank_splits, int32_t* rank_offsets, int32_t* pos,
                                       int32_t* src, int32_t* block_counts, int max_blocks,
-                                      int32_t* mt_start, unsigned* barrier, bf16* x_perm,
-                                      int32_t* status, cudaStream_t s);
+                                      int32_t* mt_start, unsigned* barrier, bool barrier_zeroed,
+                                      bf16* x_perm, int32_t* status, cudaStream_t s);
 cudaError_t launch_dispatch(const moe_config& c, const void* x, const int32_t* pos,
                             bf16* x_perm, cudaStream_t s);
 cudaError_t launch_combine(const moe_config& c, const bf16* y_perm, const int32_t* pos,

@@ -314,8 +314,8 @@ cudaError_t launch_route_pre_dispatch(const moe_config& c, const void* x, const 
                                       float* topk_w, int32_t* counts, int32_t* expert_offsets,
                                       int32_t* rank_splits, int32_t* rank_offsets, int32_t* pos,
                                       int32_t* src, int32_t* block_counts, int max_blocks,
-                                      int32_t* mt_start, unsigned* barrier, bf16* x_perm,
-                                      int32_t* status, cudaStream_t s) {
+                                      int32_t* mt_start, unsigned* barrier, bool barrier_zeroed,
+                                      bf16* x_perm, int32_t* status, cudaStream_t s) {
   int grid = sm_count();
   if (grid > max_blocks) grid = max_blocks;
   if (grid > c.T) grid = c.T;
@@ -324,8 +324,10 @@ cudaError_t launch_route_pre_dispatch(const moe_config& c, const void* x, const 
   grid = (c.T + tpb - 1) / tpb;                    // no empty block
   const size_t smem = fuse_smem(c, tpb);
   if (smem > kFuseSmemLimit || c.E > 32) return cudaErrorInvalidValue;
-  cudaError_t err = cudaMemsetAsync(barrier, 0, 2 * sizeof(unsigned), s);
-  if (err != cudaSuccess) return err;
+  if (!barrier_zeroed) {
+    const cudaError_t err = cudaMemsetAsync(barrier, 0, 2 * sizeof(unsigned), s);
+    if (err != cudaSuccess) return err;
+  }
   FuseArgs a;
   a.x = x; a.w = w; a.bias = bias; a.logits_out = logits_out; a.topk_idx = topk_idx; a.topk_w = topk_w;
   a.T = c.T; a.D = c.D; a.E = c.E; a.k = c.top_k; a.renorm = c.renormalize; a.ep = c.ep_size;
