@@ -207,6 +207,10 @@ moe_status moe_route(const moe_config* cfg, const void* x, const float* w_router
   rs.pair = !(pair_env && pair_env[0] == '0');
   rs.status = nullptr;
   rs.counter = (int32_t*)(ws + L.counters);
+  // the split logits path and the tensor-core path never run in one call: the split
+  // path's fp64 slice totals reuse the W_r split region
+  rs.part = (double*)(ws + L.r_split);
+  rs.part_bytes = L.r_wmax - L.r_split;
   return cuda_status(launch_route(c, x, w_router, expert_bias, logits, logits_out != nullptr,
                                   topk_idx, topk_w, rs, as_stream(stream)));
 }

@@ -69,6 +69,8 @@ struct RouterScratch {
   int pair;         // GEMM on CTA pairs
   int32_t* status;
   int32_t* counter; // GEMM tile counter (zeroed by the router before its launch)
+  double* part;     // fp64 slice totals of a split logits launch (aliases bsplit), or null
+  size_t part_bytes;
 };
 // logits: where the tiled path stores fp32 logits (caller's buffer or workspace);
 // keep_logits: the caller asked for them (the fused few-expert path then writes them).

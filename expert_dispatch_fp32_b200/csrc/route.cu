@@ -9,7 +9,9 @@
 // 32-wide K slices of both operands through shared memory.  Each thread sums a
 // 32-term K slice in fp32 and folds the slice into an fp64 running total, so the
 // stored fp32 logit is the dot product rounded once, to within fp32 round-off of
-// a 32-term partial (~1e-8 relative), far inside the 1e-5 near-tie margin.
+// a 32-term partial (~1e-8 relative), far inside the 1e-5 near-tie margin.  With few
+// tokens the K range is split across blocks (fp64 slice totals, added in order by a
+// second kernel before the single rounding).
 //
 // Top-k kernel: one warp per token; selection j is an exact warp argmax on
 // (logit, -index), so ties go to the lower expert index; lane j keeps pick j.
@@ -49,7 +51,7 @@ template <int BN, int BM, typename XT>
 __global__ void __launch_bounds__(kRouteThreads)
 route_logits_kernel(const XT* __restrict__ x, const float* __restrict__ w,
                     const float* __restrict__ bias, float* __restrict__ logits, int T, int D,
-                    int E) {
+                    int E, int kchunk, double* __restrict__ part) {
   constexpr int BK = kRouteBK;
   constexpr int NTN = BN / 4;                 // thread columns, 4 experts each
   constexpr int NTM = kRouteThreads / NTN;    // thread rows
@@ -68,7 +70,9 @@ route_logits_kernel(const XT* __restrict__ x, const float* __restrict__ w,
 #pragma unroll
     for (int j = 0; j < 4; ++j) tot[i][j] = 0.0;
 
-  for (int k0 = 0; k0 < D; k0 += BK) {
+  // K range of this block: all of D, or slice blockIdx.z of a split launch
+  const int kbeg = blockIdx.z * kchunk, kend = kbeg + kchunk;
+  for (int k0 = kbeg; k0 < kend; k0 += BK) {
     for (int i = tid; i < BM * (BK / 4); i += kRouteThreads) {
       const int r = i / (BK / 4), c4 = (i % (BK / 4)) * 4;
       const int t = m0 + r;
@@ -119,6 +123,11 @@ route_logits_kernel(const XT* __restrict__ x, const float* __restrict__ w,
     for (int j = 0; j < 4; ++j) {
       const int e = n0 + tx * 4 + j;
       if (e >= E) continue;
+      if (part != nullptr) {
+        // split launch: the slice's fp64 total; route_reduce_kernel adds the slices
+        part[((size_t)blockIdx.z * T + t) * E + e] = tot[i][j];
+        continue;
+      }
       float l = (float)tot[i][j];
       if (bias != nullptr) l = l + bias[e];
       logits[(size_t)t * E + e] = l;
@@ -168,6 +177,23 @@ route_topk_kernel(const float* __restrict__ logits, int32_t* __restrict__ topk_i
   if (lane < k) {
     topk_idx[(size_t)t * k + lane] = my_idx;
     topk_w[(size_t)t * k + lane] = num / den;
+  }
+}
+
+// Split logits launch, second step: one thread per (token, expert) adds the fp64 slice
+// totals in slice order, rounds once and adds the bias, as the unsplit kernel does.
+__global__ void __launch_bounds__(256)
+route_reduce_kernel(const double* __restrict__ part, int nsplit, const float* __restrict__ bias,
+                    float* __restrict__ logits, int T, int E) {
+  const size_t n = (size_t)T * E;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    double sum = 0.0;
+#pragma unroll 8
+    for (int z = 0; z < nsplit; ++z) sum += __ldg(part + (size_t)z * n + i);
+    float l = (float)sum;
+    if (bias != nullptr) l = l + bias[i % E];
+    logits[i] = l;
   }
 }
 
@@ -284,32 +310,77 @@ cudaError_t launch_small(const moe_config& c, const XT* x, const float* w, const
 
 constexpr size_t kSmallRouterSmem = 200u << 10;
 
+// Tile shape of the logits kernel: BN experts x BM tokens per block.
+struct LogitsTiles {
+  int bn, bm, m_blocks, n_blocks;
+};
+LogitsTiles logits_tiles(const moe_config& c) {
+  LogitsTiles g;
+  g.bn = c.E >= 64 ? 64 : c.E > 16 ? 32 : c.E > 8 ? 16 : 8;
+  const int m_blocks128 = (c.T + 127) / 128;
+  g.n_blocks = (c.E + g.bn - 1) / g.bn;
+  // 64-token tiles when 128-token tiles leave SMs idle (needs >= 2 tokens per thread row)
+  const bool small_m = g.bn >= 32 && (int64_t)m_blocks128 * g.n_blocks < 2 * sm_count();
+  g.bm = small_m ? 64 : 128;
+  g.m_blocks = (c.T + g.bm - 1) / g.bm;
+  return g;
+}
+
+// With few tokens the logits kernel has too few blocks to stream W_r (and the
+// tensor-core filter GEMM too few tiles: 2 for deepseek_v3's 256 x 7168 router, ~150 us
+// for 32 tokens), so the K range is split over blockIdx.z: each block stores the fp64
+// total of its 32-wide slices and route_reduce_kernel adds the slices in order.  Split
+// count: the largest divisor of D/32 that brings the grid to ~2 blocks per SM and whose
+// slice totals (nsplit * T * E doubles) fit in `cap` bytes.  The kernel does not overlap
+// one slice's loads with the previous slice's math, so a block costs a few us per slice:
+// the split is taken only when every block has at most kSplitMaxSlices slices (measured,
+// 256 x 7168 router: 46 vs 150 us for 32 tokens (4 slices per block), 65 vs 131 us for
+// 128 (8); 64 x 2048 router: 28 vs 53 us for 32 tokens (1), 44 vs 53 for 256 (8), 116 vs
+// 53 for 1024 (32)), and never past kSplitRouteMaxFma multiply-adds (T * E * D).
+constexpr int kSplitMaxSlices = 8;
+constexpr double kSplitRouteMaxFma = 5.0e8;
+int split_route_count(const moe_config& c, size_t cap) {
+  // MOE_ROUTE_SPLIT=0 keeps the unsplit paths (read at each call; for comparison)
+  const char* env = getenv("MOE_ROUTE_SPLIT");
+  if (env && env[0] == '0') return 1;
+  if (cap == 0 || (double)c.T * c.E * c.D > kSplitRouteMaxFma) return 1;
+  const LogitsTiles g = logits_tiles(c);
+  const int64_t blocks = (int64_t)g.m_blocks * g.n_blocks;
+  const int64_t target = (2 * sm_count() + blocks - 1) / blocks;
+  const int slices = c.D / kRouteBK;
+  int best = 1;
+  for (int d = 2; d <= slices && d <= target; ++d)
+    if (slices % d == 0 && (size_t)d * c.T * c.E * sizeof(double) <= cap) best = d;
+  return slices / best <= kSplitMaxSlices ? best : 1;
+}
+
 template <typename XT>
 cudaError_t launch_logits(const moe_config& c, const XT* x, const float* w, const float* bias,
-                          float* logits, cudaStream_t s) {
-  const int bn = c.E >= 64 ? 64 : c.E > 16 ? 32 : c.E > 8 ? 16 : 8;
-  const int m_blocks128 = (c.T + 127) / 128, n_blocks = (c.E + bn - 1) / bn;
-  // 64-token tiles when 128-token tiles leave SMs idle (needs >= 2 tokens per thread row)
-  const bool small_m = bn >= 32 && (int64_t)m_blocks128 * n_blocks < 2 * sm_count();
-  const int bm = small_m ? 64 : 128;
-  dim3 grid((c.T + bm - 1) / bm, n_blocks);
+                          float* logits, int nsplit, double* part, cudaStream_t s) {
+  const LogitsTiles g = logits_tiles(c);
+  const bool small_m = g.bm == 64;
+  const int kchunk = c.D / nsplit;
+  if (nsplit < 2) part = nullptr;
+  dim3 grid(g.m_blocks, g.n_blocks, nsplit);
+#define MOE_ROUTE_ARGS x, w, bias, logits, c.T, c.D, c.E, kchunk, part
 #define MOE_ROUTE_TILE(BN_)                                                                        \
-  if (small_m) route_logits_kernel<BN_, 64, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E); \
-  else route_logits_kernel<BN_, 128, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E);
-  switch (bn) {
+  if (small_m) route_logits_kernel<BN_, 64, XT><<<grid, kRouteThreads, 0, s>>>(MOE_ROUTE_ARGS); \
+  else route_logits_kernel<BN_, 128, XT><<<grid, kRouteThreads, 0, s>>>(MOE_ROUTE_ARGS);
+  switch (g.bn) {
     case 64: MOE_ROUTE_TILE(64) break;
     case 32: MOE_ROUTE_TILE(32) break;
-    case 16: route_logits_kernel<16, 128, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E); break;
-    default: route_logits_kernel<8, 128, XT><<<grid, kRouteThreads, 0, s>>>(x, w, bias, logits, c.T, c.D, c.E); break;
+    case 16: route_logits_kernel<16, 128, XT><<<grid, kRouteThreads, 0, s>>>(MOE_ROUTE_ARGS); break;
+    default: route_logits_kernel<8, 128, XT><<<grid, kRouteThreads, 0, s>>>(MOE_ROUTE_ARGS); break;
   }
 #undef MOE_ROUTE_TILE
+#undef MOE_ROUTE_ARGS
   return cudaGetLastError();
 }
 
 template <typename XT>
 cudaError_t launch_route_t(const moe_config& c, const XT* x, const float* w_router,
                            const float* bias, float* logits, bool keep_logits, int32_t* topk_idx,
-                           float* topk_w, cudaStream_t s) {
+                           float* topk_w, double* part, size_t part_bytes, cudaStream_t s) {
   const size_t wbytes = (size_t)c.E * c.D * sizeof(float);
   if (c.E <= 32 && wbytes <= kSmallRouterSmem) {
     float* lo = keep_logits ? logits : nullptr;
@@ -322,8 +393,16 @@ cudaError_t launch_route_t(const moe_config& c, const XT* x, const float* w_rout
     if (c.E <= 16) return launch_small<16, 1, XT>(c, x, w_router, bias, lo, topk_idx, topk_w, s);
     return launch_small<32, 1, XT>(c, x, w_router, bias, lo, topk_idx, topk_w, s);
   }
-  cudaError_t err = launch_logits(c, x, w_router, bias, logits, s);
+  const int nsplit = part != nullptr ? split_route_count(c, part_bytes) : 1;
+  cudaError_t err = launch_logits(c, x, w_router, bias, logits, nsplit, part, s);
   if (err != cudaSuccess) return err;
+  if (nsplit > 1) {
+    const int64_t n = (int64_t)c.T * c.E;
+    const int64_t rb = (n + 255) / 256, cap = 8 * (int64_t)sm_count();
+    route_reduce_kernel<<<(int)(rb < cap ? rb : cap), 256, 0, s>>>(part, nsplit, bias, logits, c.T, c.E);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
   const int warps_per_block = 8;
   const int blocks = (c.T + warps_per_block - 1) / warps_per_block;
   route_topk_kernel<<<blocks, warps_per_block * 32, 0, s>>>(logits, topk_idx, topk_w, c.T, c.E,
@@ -594,17 +673,19 @@ cudaError_t launch_route(const moe_config& c, const void* x, const float* w_rout
                          float* topk_w, const RouterScratch& rs, cudaStream_t s) {
   if (c.x_dtype == MOE_DT_F32)
     return launch_route_t(c, static_cast<const float*>(x), w_router, bias, logits, keep_logits,
-                          topk_idx, topk_w, s);
+                          topk_idx, topk_w, rs.part, rs.part_bytes, s);
   // bf16 x with renormalised weights and no logits to return, too many experts for the
   // fused shared-memory router: tensor-core filter and exact refine (MOE_ROUTER_TC=0
   // selects the SIMT paths, which compute every logit exactly)
   const char* env = getenv("MOE_ROUTER_TC");
   const bool tc_ok = !(env && env[0] == '0');
   const bool few = c.E <= 32 && (size_t)c.E * c.D * sizeof(float) <= kSmallRouterSmem;
-  if (tc_ok && !few && c.renormalize && !keep_logits && rs.bsplit != nullptr)
+  // few tokens: the split SIMT logits (exact) beat the tensor-core filter's fixed cost
+  const bool split = !few && split_route_count(c, rs.part_bytes) > 1;
+  if (tc_ok && !few && !split && c.renormalize && !keep_logits && rs.bsplit != nullptr)
     return launch_route_tc(c, static_cast<const bf16*>(x), w_router, bias, rs, topk_idx, topk_w, s);
   return launch_route_t(c, static_cast<const bf16*>(x), w_router, bias, logits, keep_logits,
-                        topk_idx, topk_w, s);
+                        topk_idx, topk_w, rs.part, rs.part_bytes, s);
 }
 
 }  // namespace moe

@@ -285,6 +285,43 @@ def test_ties_on_the_tensor_core_router(E, k):
     compare_routing(idx, layer.buf["topk_w"].cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("T,D,E,k,xdt,zipf", [(32, 2048, 64, 6, "bf16", True),
+                                               (40, 1024, 48, 4, "bf16", False),
+                                               (100, 512, 256, 8, "bf16", False),
+                                               (7, 7168, 256, 8, "bf16", False),
+                                               (32, 1024, 64, 2, "f32", False)])
+def test_split_k_router(T, D, E, k, xdt, zipf):
+    """Few tokens and more than 32 experts: the logits kernel splits D across blocks
+    (fp64 slice totals added in order before the single rounding).  Routing against
+    the oracle with and without returned logits, and against the unsplit paths
+    (tensor-core filter + refine, or the unsplit SIMT kernel)."""
+    wl = BASE.with_(T=T, D=D, E=E, ep_size=8 if E % 8 == 0 else 1, top_k=k, F=128, x_dtype=xdt,
+                    zipf_bias=zipf)
+    inp = W.make_inputs(wl, device="cuda")
+    layer = make_layer(wl, inp)
+    b = layer.allocate(T)
+    cfg = layer.config(T)
+    ref = oracle_route(wl, inp)
+    runs = []
+    for split in ("1", "0"):
+        os.environ["MOE_ROUTE_SPLIT"] = split
+        try:
+            for keep in (True, False):
+                b["logits"] = torch.full((T, E), float("nan"), device="cuda") if keep else None
+                M.moe_route(cfg, inp["x"], inp["w_router"], inp["bias"], b["logits"], b["topk_idx"],
+                            b["topk_w"], b["workspace"])
+                torch.cuda.synchronize()
+                if keep:
+                    assert np.allclose(b["logits"].cpu().numpy(), ref["logits"], rtol=2e-6, atol=2e-6)
+                idx, w = b["topk_idx"].cpu().numpy(), b["topk_w"].cpu().numpy()
+                compare_routing(idx, w, ref)
+                runs.append(idx)
+        finally:
+            del os.environ["MOE_ROUTE_SPLIT"]
+    for r in runs[1:]:
+        assert np.array_equal(r, runs[0])
+
+
 # per-expert row counts around the 128- and 256-row tile edges: empty, one row, a
 # last tile with <= 64 rows (only the first CTA of a pair holds rows), 65..128 rows
 # (both CTAs of an M = 128 pair tile), 129..255, exactly 256, 256 + a few (1, 32,
