@@ -125,10 +125,29 @@ combine_kernel(const bf16* __restrict__ y_perm, const int32_t* __restrict__ pos,
   }
 }
 
+// Raw 8-element bf16 chunks, converted to fp32 only where they are used (half the
+// registers of converting at the load, so more loads stay in flight per lane).
+template <typename T> struct Raw8;
+template <> struct Raw8<bf16> { uint4 a; };
+__device__ __forceinline__ void ldr(const bf16* p, Raw8<bf16>& r) {
+  r.a = __ldg(reinterpret_cast<const uint4*>(p));
+}
+__device__ __forceinline__ void cvt(const Raw8<bf16>& r, Vec8& o) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r.a);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(h[i]);
+    o.v[2 * i] = f.x; o.v[2 * i + 1] = f.y;
+  }
+}
+
 // Combine with every row chunk of a step in flight: x, shared and the KC routed rows,
-// one 256-column chunk each, loaded before the first multiply-add; the arithmetic and
-// its order are those of combine_kernel.
-template <typename XT, int KC>
+// U 256-column chunks each, loaded before the first multiply-add; the arithmetic and
+// its order are those of combine_kernel.  Measured after an L2 flush (same bits as the
+// slot-by-slot walk): mixtral_8x7b (k = 2, U = 2) 57.4 -> 45.1 us (5.96 TB/s),
+// small_e8_d2048 18.4 -> 14.3 us, deepseek_v3 (k = 8, U = 1) 227 -> 205 us, zipf_skew_e64
+// 111 -> 98 us; U = 4 at k = 2 (90 registers, half the resident warps) was slower than 2.
+template <typename XT, int KC, int U>
 __global__ void __launch_bounds__(kCombineThreads)
 combine_k_kernel(const bf16* __restrict__ y_perm, const int32_t* __restrict__ pos,
                  const float* __restrict__ topk_w, const XT* __restrict__ x,
@@ -142,23 +161,41 @@ combine_k_kernel(const bf16* __restrict__ y_perm, const int32_t* __restrict__ po
     uint32_t p[KC];
 #pragma unroll
     for (int j = 0; j < KC; ++j) p[j] = __shfl_sync(0xffffffffu, my_pos, j);
-    for (int c = lane * 8; c < D; c += 256) {
-      Vec8 acc, sh, y[KC];
-      ld8(x + (size_t)t * D + c, acc);
-      if (shared != nullptr) ld8(shared + (size_t)t * D + c, sh);
+    for (int c0 = lane * 8; c0 < D; c0 += 256 * U) {
+      Raw8<XT> xr[U];
+      Raw8<bf16> sr[U], yr[KC][U];
 #pragma unroll
-      for (int j = 0; j < KC; ++j) ld8(y_perm + (size_t)p[j] * D + c, y[j]);
-      if (shared != nullptr) {
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + u * 256;
+        if (c < D) {
+          ldr(x + (size_t)t * D + c, xr[u]);
+          if (shared != nullptr) ldr(shared + (size_t)t * D + c, sr[u]);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc.v[i] += sh.v[i];
+          for (int j = 0; j < KC; ++j) ldr(y_perm + (size_t)p[j] * D + c, yr[j][u]);
+        }
       }
 #pragma unroll
-      for (int j = 0; j < KC; ++j) {
-        const float w = __shfl_sync(0xffffffffu, my_w, j);
+      for (int u = 0; u < U; ++u) {
+        if (c0 + u * 256 < D) {
+          Vec8 acc;
+          cvt(xr[u], acc);
+          if (shared != nullptr) {
+            Vec8 sv;
+            cvt(sr[u], sv);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc.v[i] = fmaf(w, y[j].v[i], acc.v[i]);
+            for (int i = 0; i < 8; ++i) acc.v[i] += sv.v[i];
+          }
+#pragma unroll
+          for (int j = 0; j < KC; ++j) {
+            const float w = __shfl_sync(0xffffffffu, my_w, j);
+            Vec8 yv;
+            cvt(yr[j][u], yv);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc.v[i] = fmaf(w, yv.v[i], acc.v[i]);
+          }
+          st8(out + (size_t)t * D + c0 + u * 256, acc);
+        }
       }
-      st8(out + (size_t)t * D + c, acc);
     }
   }
 }
@@ -216,18 +253,23 @@ cudaError_t launch_combine(const moe_config& c, const bf16* y_perm, const int32_
                            const float* topk_w, const void* x, const bf16* shared_out, void* out,
                            cudaStream_t s) {
   const uint32_t R = (uint32_t)c.T * c.top_k;
-  // k = 6..8 (bf16 x): every row of a step in flight (deepseek_v3: 263 -> 228 us after the FFN);
-  // for k <= 4 the two-chunk walk over the slots measured as fast
+  // bf16 x: every row chunk of a step in flight, U chunks per row (k = 1: 4; k <= 4: 2;
+  // else 1); MOE_PERMUTE_V=0 selects the slot-by-slot walk (for comparison)
   const char* env = getenv("MOE_PERMUTE_V");
   const bool hoist = !(env && env[0] == '0') && c.x_dtype == MOE_DT_BF16;
-#define MOE_COMBINE_K(KC)                                                                       \
-  if (hoist && c.top_k == KC)                                                                   \
-    return launch_pdl(combine_k_kernel<bf16, KC>, combine_grid(c.T), kCombineThreads, s, y_perm, \
-                      pos, topk_w, static_cast<const bf16*>(x), shared_out,                      \
+#define MOE_COMBINE_K(KC, U)                                                                       \
+  if (hoist && c.top_k == KC)                                                                      \
+    return launch_pdl(combine_k_kernel<bf16, KC, U>, combine_grid(c.T), kCombineThreads, s, y_perm, \
+                      pos, topk_w, static_cast<const bf16*>(x), shared_out,                         \
                       static_cast<bf16*>(out), c.T, c.D, R);
-  MOE_COMBINE_K(6)
-  MOE_COMBINE_K(7)
-  MOE_COMBINE_K(8)
+  MOE_COMBINE_K(1, 4)
+  MOE_COMBINE_K(2, 2)
+  MOE_COMBINE_K(3, 2)
+  MOE_COMBINE_K(4, 2)
+  MOE_COMBINE_K(5, 1)
+  MOE_COMBINE_K(6, 1)
+  MOE_COMBINE_K(7, 1)
+  MOE_COMBINE_K(8, 1)
 #undef MOE_COMBINE_K
   if (c.x_dtype == MOE_DT_F32)
     return launch_pdl(combine_kernel<float>, combine_grid(c.T), kCombineThreads, s, y_perm, pos,

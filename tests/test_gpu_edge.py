@@ -132,11 +132,14 @@ def test_fused_route_dispatch_matches_stage_calls(T, D, E, k, xdt, renorm, logit
     compare_routing(res["1"]["topk_idx"].cpu().numpy(), res["1"]["topk_w"].cpu().numpy(), ref)
 
 
-@pytest.mark.parametrize("k,D,shared", [(6, 320, True), (7, 512, False), (8, 1088, True)])
+@pytest.mark.parametrize("k,D,shared", [(1, 704, False), (2, 320, True), (2, 1600, False),
+                                        (3, 576, True), (4, 1088, False), (5, 512, True),
+                                        (6, 320, True), (7, 512, False), (8, 1088, True)])
 def test_combine_forms_agree(k, D, shared):
-    """The combine that loads every routed row of a step before its multiply-adds (used
-    for k = 6..8) gives the bits of the slot-by-slot form, and the layer matches the
-    oracle (D not a multiple of 256: a ragged last column chunk)."""
+    """The combine that loads every routed row of a step before its multiply-adds (U
+    column chunks per row: 4 for k = 1, 2 for k <= 4, 1 above) gives the bits of the
+    slot-by-slot form, and the layer matches the oracle (D not a multiple of 256 * U: a
+    ragged last step)."""
     wl = BASE.with_(T=333, D=D, E=16, ep_size=4, top_k=k, F=128,
                     n_shared=1 if shared else 0, F_shared=128 if shared else 0, seed=4)
     inp = W.make_inputs(wl, device="cuda")
