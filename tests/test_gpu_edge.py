@@ -132,6 +132,43 @@ def test_fused_route_dispatch_matches_stage_calls(T, D, E, k, xdt, renorm, logit
     compare_routing(res["1"]["topk_idx"].cpu().numpy(), res["1"]["topk_w"].cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("k", [2, 6])
+def test_long_batch_grid_stride(k):
+    """More tokens than the dispatch grid's 65535-block cap (two rows per block for k <= 4,
+    one for k = 6): the grid-stride loops of the stage kernels, the fused launch's
+    ~950 tokens per block, and the combine's capped grid.  Stage calls and the fused launch
+    give the same bits; routing for every token and the layer on sampled tokens against
+    the oracle."""
+    T = 140001
+    wl = BASE.with_(T=T, D=64, E=8, ep_size=2, top_k=k, F=128, seed=13)
+    inp = W.make_inputs(wl, device="cuda")
+    layer = make_layer(wl, inp)
+    layer.allocate(T)
+    keys = ["topk_idx", "topk_w", "pos", "src", "x_perm", "out"]
+    res = {}
+    for fused in ("0", "1"):
+        os.environ["MOE_ROUTE_FUSED"] = fused
+        try:
+            for key in keys:
+                layer.buf[key].fill_(-3)
+            layer.forward(inp["x"])
+            torch.cuda.synchronize()
+            layer.check_status()
+        finally:
+            del os.environ["MOE_ROUTE_FUSED"]
+        res[fused] = {key: layer.buf[key].clone() for key in keys}
+    for key in keys:
+        assert torch.equal(res["0"][key], res["1"][key]), key
+    ref = oracle_route(wl, inp)
+    compare_routing(res["1"]["topk_idx"].cpu().numpy(), res["1"]["topk_w"].cpu().numpy(), ref)
+    tokens = np.unique(np.concatenate([np.arange(4), [65534, 65535, 65536, 131069, 131070, 131071],
+                                       np.random.default_rng(2).choice(T, 300, replace=False),
+                                       [T - 2, T - 1]]))
+    part = oracle_layer(wl, inp, tokens)
+    got = f64(res["1"]["out"][torch.from_numpy(tokens).cuda()])
+    assert_layer_close(got, part["out"], f64(inp["x"][torch.from_numpy(tokens).cuda()]))
+
+
 @pytest.mark.parametrize("k,D,shared", [(1, 704, False), (2, 320, True), (2, 1600, False),
                                         (3, 576, True), (4, 1088, False), (5, 512, True),
                                         (6, 320, True), (7, 512, False), (8, 1088, True)])
