@@ -214,11 +214,17 @@ def cpu_threads():
 
 def pick_sample(wl, host, budget_s):
     """Tokens per oracle sample so one sample costs about budget_s on the host:
-    time a 64-token probe and scale (tokens are independent, cost is linear)."""
+    time a 64-token probe and scale (tokens are independent, cost is linear), then
+    re-time a quarter of that estimate and scale again (the small probe carries the
+    per-call costs, so by itself it undersizes the sample by a factor of 2-3)."""
     probe = min(64, wl.T)
     cpu_oracle_time(wl, host, probe, seed=99)            # warm the BLAS threads
     t = cpu_oracle_time(wl, host, probe, seed=98)
-    return int(max(probe, min(16 * wl.T, budget_s * probe / max(t, 1e-6))))
+    cap = 16 * wl.T
+    n = int(max(probe, min(cap, budget_s * probe / max(t, 1e-6))))
+    n2 = max(probe, n // 4)
+    t2 = cpu_oracle_time(wl, host, n2, seed=97)
+    return int(max(probe, min(cap, budget_s * n2 / max(t2, 1e-6))))
 
 
 # ---------------------------------------------------------------------------
@@ -505,7 +511,9 @@ def run_ours(args):
         "combine_gbs": comb_gbs, "combine_frac_hbm": comb_gbs / hbm,
     }
     if want_cpu:
-        n_tok = args.cpu_sample or pick_sample(wl, cpu_host, 12.0)
+        # sized for ~12 s of oracle work (the calibration still undersizes it by ~1/3:
+        # larger samples run the BLAS steps more efficiently per token)
+        n_tok = args.cpu_sample or pick_sample(wl, cpu_host, 18.0)
         t = cpu_oracle_time(wl, cpu_host, n_tok, seed=1)
         line["cpu_baseline"] = {"value": n_tok / t, "unit": "tokens/s", "cores": cpu_threads(),
                                 "kind": "oracle",
