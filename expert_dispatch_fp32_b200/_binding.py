@@ -62,6 +62,7 @@ _SIGS = {
     "moe_ep_local_ids": (ctypes.c_int, [_cfgp, _i32p, _i32p, _i32p, _vp]),
     "moe_gather_rows": (ctypes.c_int, [_vp, _i32p, _vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                        _vp]),
+    "moe_check_wait_timeout": (ctypes.c_int, [_vp, _i32p, _vp]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_abi_version": (ctypes.c_int32, []),
 }
@@ -102,6 +103,10 @@ def _call(name, *args):
     st = getattr(lib(), name)(*args)
     if st != MOE_OK:
         raise MoeError(name, st)
+
+
+def moe_check_wait_timeout(barrier, status, stream=None):
+    _call("moe_check_wait_timeout", _p(barrier), _p(status), _s(stream))
 
 
 def moe_status_string(status: int) -> str:

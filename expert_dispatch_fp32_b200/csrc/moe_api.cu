@@ -514,6 +514,12 @@ moe_status moe_gather_rows(const void* src, const int32_t* index, void* dst, int
                                         as_stream(stream)));
 }
 
+moe_status moe_check_wait_timeout(uint32_t* barrier, int32_t* status, void* stream) {
+  MOE_CHECK_PTR(barrier);
+  MOE_CHECK_PTR(status);
+  return cuda_status(launch_barrier_timeout_check(barrier, status, as_stream(stream)));
+}
+
 const char* moe_status_string(moe_status s) {
   switch (s) {
     case MOE_OK: return "ok";

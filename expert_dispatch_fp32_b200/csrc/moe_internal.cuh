@@ -85,6 +85,8 @@ cudaError_t launch_preprocess(const moe_config& c, const int32_t* topk_idx, int3
                               int32_t* rank_offsets, int32_t* pos, int32_t* src,
                               int32_t* block_counts, int max_blocks, int32_t* mt_start,
                               unsigned* barrier, int32_t* status, cudaStream_t s);
+// Self-check of the bounded grid-barrier wait (preprocess.cu): one block, barrier for two.
+cudaError_t launch_barrier_timeout_check(unsigned* barrier, int32_t* status, cudaStream_t s);
 // Multi-rank helpers (ep.cu).
 cudaError_t launch_local_ids(const int32_t* topk_idx, const int32_t* src, int32_t* ids, int R, int El,
                              cudaStream_t s);

@@ -79,7 +79,21 @@ pre_fused_kernel(const PreArgs a) {
       E, cnt, warp_cnt, a.pos, a.src, nullptr);
 }
 
+// One block waits at a grid barrier sized for two blocks: nothing completes it, so the
+// bounded wait of grid_barrier (the one the cooperative kernels use) runs out, records
+// MOE_ERR_TIMEOUT in *status and the kernel returns.
+__global__ void barrier_timeout_check_kernel(unsigned* bar, int32_t* status) {
+  grid_barrier(bar, 2u, status);
+}
+
 }  // namespace
+
+cudaError_t launch_barrier_timeout_check(unsigned* barrier, int32_t* status, cudaStream_t s) {
+  cudaError_t err = cudaMemsetAsync(barrier, 0, 2 * sizeof(unsigned), s);
+  if (err != cudaSuccess) return err;
+  barrier_timeout_check_kernel<<<1, 32, 0, s>>>(barrier, status);
+  return cudaGetLastError();
+}
 
 int preprocess_blocks(int64_t R) {
   const int64_t want = (R + kPreThreads - 1) / kPreThreads;

@@ -284,6 +284,18 @@ MOE_API moe_status moe_ep_local_ids(const moe_config* cfg, const int32_t* topk_i
 MOE_API moe_status moe_gather_rows(const void* src, const int32_t* index, void* dst, int32_t n,
                                    int32_t n_src, int32_t D, void* stream);
 
+/* Self-check of device-side failure detection.  The cooperative kernels (moe_preprocess,
+ * moe_route_dispatch) synchronise their blocks at a grid barrier whose wait is bounded
+ * (~1 s of SM cycles); a block that gives up writes MOE_ERR_TIMEOUT to the status word
+ * and the kernel returns, so the CUDA context stays usable and the caller reads the
+ * status when convenient (the error convention of every call above).  This call runs
+ * that barrier with one block where two are expected, so nothing completes it and the
+ * wait runs out: after the stream reaches it, *status holds MOE_ERR_TIMEOUT (if it was
+ * MOE_OK before).  Takes ~1 s of device time.
+ *   barrier: two device uint32 words of scratch (zeroed by the call);
+ *   status: device int32, not reset by the call. */
+MOE_API moe_status moe_check_wait_timeout(uint32_t* barrier, int32_t* status, void* stream);
+
 /* Static description of a status code. */
 MOE_API const char* moe_status_string(moe_status s);
 

@@ -102,6 +102,8 @@ def test_null_and_misaligned_pointers_rejected_on_host(B):
     assert lib.moe_route(by, fake + 4, fake, None, None, fake, fake, fake, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_preprocess(by, fake, fake, fake, fake, fake, fake, fake, fake, None, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_dispatch_permute(by, fake, None, fake, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_check_wait_timeout(None, fake, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_check_wait_timeout(fake, None, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_expert_ffn(by, fake, None, fake, None, fake, fake, None, fake, fake, None) == B.MOE_ERR_INVALID_ARG
     # out may not alias the residual
     assert lib.moe_combine_unpermute(by, fake, fake, fake, fake, None, fake, None) == B.MOE_ERR_INVALID_ARG

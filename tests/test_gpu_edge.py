@@ -264,6 +264,18 @@ def test_out_of_range_index_sets_status():
     assert int(status.item()) == M.MOE_ERR_INDEX_OOB
 
 
+def test_bounded_wait_reports_timeout():
+    """A grid-barrier wait that nothing completes runs out (~1 s), the kernel records
+    MOE_ERR_TIMEOUT in the status word and returns; the context stays usable (a forward
+    afterwards still matches the oracle)."""
+    bar = torch.zeros(2, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    M.moe_check_wait_timeout(bar, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == M.MOE_ERR_TIMEOUT
+    run_and_compare(BASE.with_(T=64, seed=21))
+
+
 def test_empty_batch_forward():
     wl = BASE.with_(T=0)
     inp = W.make_inputs(BASE, device="cuda")
