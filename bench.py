@@ -479,6 +479,30 @@ def run_ours(args):
     comb_gbs = comb_b / (stage_ms[4] / args.steps / 1e3) / 1e9
     launches_per_step = (1 if fused else route_launches(wl) + 1 + 1) + ffn_launches(wl) + 1
 
+    # layer roofline: the sum of every stage's ideal time over the measured step.  Ideal
+    # times: route = max(bytes / HBM, flop / fp32 peak), the fp32 peak from the unit counts
+    # (148 SMs x 128 FP32 lanes x 2 flop x the max SM clock); preprocess and dispatch and
+    # combine = bytes / HBM; FFN = max(flop / the bf16 peak used above, bytes of the hit
+    # experts' weights / HBM)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    fp32_tf = sms * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    hit = int((b["counts"][:wl.E] > 0).sum().item())
+    mats = 3 if wl.act == "swiglu" else 2
+    w_bytes = hit * mats * wl.D * wl.F * 2 + wl.n_shared * 3 * wl.D * wl.F_shared * 2
+    hbm_bs = hbm * 1e9
+    ideal_us = {
+        "route": 1e6 * max((wl.T * wl.D * sx + wl.E * wl.D * 4 + wl.R * 8) / hbm_bs,
+                           2.0 * wl.T * wl.D * wl.E / (fp32_tf * 1e12)),
+        "preprocess": 1e6 * wl.R * 12 / hbm_bs,
+        "dispatch": 1e6 * disp_b / hbm_bs,
+        "expert_ffn": 1e6 * max(wl.ffn_flop() / (peak_tf * 1e12), w_bytes / hbm_bs),
+        "combine": 1e6 * comb_b / hbm_bs,
+    }
+    step_us = 1e3 * total_ms_max / args.steps
+    layer_roofline = {"ideal_us": ideal_us, "sum_ideal_us": sum(ideal_us.values()),
+                      "measured_us": step_us, "frac": sum(ideal_us.values()) / step_us,
+                      "fp32_peak_tflops": fp32_tf, "ffn_peak": peak_key}
+
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
@@ -507,6 +531,7 @@ def run_ours(args):
                                zip(("route_preprocess_dispatch", "expert_ffn", "combine"), fused_ms)}
                               if fused else None),
         "ffn_tflops": ffn_tflops,
+        "layer_roofline": layer_roofline,
         "dispatch_gbs": disp_gbs, "dispatch_frac_hbm": disp_gbs / hbm,
         "combine_gbs": comb_gbs, "combine_frac_hbm": comb_gbs / hbm,
     }
