@@ -70,26 +70,54 @@ route_logits_kernel(const XT* __restrict__ x, const float* __restrict__ w,
 #pragma unroll
     for (int j = 0; j < 4; ++j) tot[i][j] = 0.0;
 
-  // K range of this block: all of D, or slice blockIdx.z of a split launch
+  // K range of this block: all of D, or slice blockIdx.z of a split launch.  The next
+  // slice's global loads go to registers before the current slice's math, so their
+  // latency overlaps it (the values and the arithmetic are those of a plain loop).
   const int kbeg = blockIdx.z * kchunk, kend = kbeg + kchunk;
-  for (int k0 = kbeg; k0 < kend; k0 += BK) {
-    for (int i = tid; i < BM * (BK / 4); i += kRouteThreads) {
-      const int r = i / (BK / 4), c4 = (i % (BK / 4)) * 4;
-      const int t = m0 + r;
-      float v[4] = {0.f, 0.f, 0.f, 0.f};
-      if (t < T) load4(x + (size_t)t * D + k0 + c4, v);
+  constexpr int XN = BM * (BK / 4), WN = BN * (BK / 4);
+  constexpr int XL = (XN + kRouteThreads - 1) / kRouteThreads;
+  constexpr int WL = (WN + kRouteThreads - 1) / kRouteThreads;
+  float xr[XL][4], wr[WL][4];
+  auto load_slice = [&](int k0) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) xs[c4 + q][r] = v[q];
+    for (int l = 0; l < XL; ++l) {
+      const int i = tid + l * kRouteThreads;
+      const int r = i / (BK / 4), c4 = (i % (BK / 4)) * 4;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) xr[l][q] = 0.f;
+      if (i < XN && m0 + r < T) load4(x + (size_t)(m0 + r) * D + k0 + c4, xr[l]);
     }
-    for (int i = tid; i < BN * (BK / 4); i += kRouteThreads) {
-      const int r = i / (BK / 4), c4 = (i % (BK / 4)) * 4;
-      const int e = n0 + r;
-      float v[4] = {0.f, 0.f, 0.f, 0.f};
-      if (e < E) load4(w + (size_t)e * D + k0 + c4, v);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) ws[c4 + q][r] = v[q];
+    for (int l = 0; l < WL; ++l) {
+      const int i = tid + l * kRouteThreads;
+      const int r = i / (BK / 4), c4 = (i % (BK / 4)) * 4;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) wr[l][q] = 0.f;
+      if (i < WN && n0 + r < E) load4(w + (size_t)(n0 + r) * D + k0 + c4, wr[l]);
+    }
+  };
+  if (kbeg < kend) load_slice(kbeg);
+  for (int k0 = kbeg; k0 < kend; k0 += BK) {
+#pragma unroll
+    for (int l = 0; l < XL; ++l) {
+      const int i = tid + l * kRouteThreads;
+      const int r = i / (BK / 4), c4 = (i % (BK / 4)) * 4;
+      if (i < XN) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xs[c4 + q][r] = xr[l][q];
+      }
+    }
+#pragma unroll
+    for (int l = 0; l < WL; ++l) {
+      const int i = tid + l * kRouteThreads;
+      const int r = i / (BK / 4), c4 = (i % (BK / 4)) * 4;
+      if (i < WN) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) ws[c4 + q][r] = wr[l][q];
+      }
     }
     __syncthreads();
+    if (k0 + BK < kend) load_slice(k0 + BK);
     float acc[TM][4];
 #pragma unroll
     for (int i = 0; i < TM; ++i)
@@ -331,14 +359,14 @@ LogitsTiles logits_tiles(const moe_config& c) {
 // for 32 tokens), so the K range is split over blockIdx.z: each block stores the fp64
 // total of its 32-wide slices and route_reduce_kernel adds the slices in order.  Split
 // count: the largest divisor of D/32 that brings the grid to ~2 blocks per SM and whose
-// slice totals (nsplit * T * E doubles) fit in `cap` bytes.  The kernel does not overlap
-// one slice's loads with the previous slice's math, so a block costs a few us per slice:
-// the split is taken only when every block has at most kSplitMaxSlices slices (measured,
-// 256 x 7168 router: 46 vs 150 us for 32 tokens (4 slices per block), 65 vs 131 us for
-// 128 (8); 64 x 2048 router: 28 vs 53 us for 32 tokens (1), 44 vs 53 for 256 (8), 116 vs
-// 53 for 1024 (32)), and never past kSplitRouteMaxFma multiply-adds (T * E * D).
-constexpr int kSplitMaxSlices = 8;
-constexpr double kSplitRouteMaxFma = 5.0e8;
+// slice totals (nsplit * T * E doubles) fit in `cap` bytes.  Taken when every block has
+// at most kSplitMaxSlices slices, or twice that with at least one block per SM, and never
+// past kSplitRouteMaxFma multiply-adds (T * E * D).  Measured against the tensor-core
+// router: 256 x 7168 router 42 vs 150 us for 32 tokens, 52 vs 131 for 128, 71 vs 131 for
+// 256, 114 vs 143 for 512 (32 slices, 224 blocks); 64 x 2048 router 28 vs 53 us for 32
+// tokens, 34 vs 53 for 256, 48 vs 53 for 512, but 77 vs 53 for 1024 (32 slices, 32 blocks).
+constexpr int kSplitMaxSlices = 16;
+constexpr double kSplitRouteMaxFma = 1.0e9;
 int split_route_count(const moe_config& c, size_t cap) {
   // MOE_ROUTE_SPLIT=0 keeps the unsplit paths (read at each call; for comparison)
   const char* env = getenv("MOE_ROUTE_SPLIT");
@@ -351,7 +379,10 @@ int split_route_count(const moe_config& c, size_t cap) {
   int best = 1;
   for (int d = 2; d <= slices && d <= target; ++d)
     if (slices % d == 0 && (size_t)d * c.T * c.E * sizeof(double) <= cap) best = d;
-  return slices / best <= kSplitMaxSlices ? best : 1;
+  const int per_block = slices / best;
+  const bool ok = per_block <= kSplitMaxSlices ||
+                  (per_block <= 2 * kSplitMaxSlices && blocks * best >= sm_count());
+  return ok ? best : 1;
 }
 
 template <typename XT>
