@@ -57,6 +57,15 @@ def test_decode_batch_with_shared_experts(T):
                                F_shared=256, seed=T))
 
 
+@pytest.mark.parametrize("T,E,k,zipf", [(24, 64, 6, True), (9, 256, 8, False)])
+def test_decode_batch_many_experts(T, E, k, zipf):
+    """A decode-sized forward with more than 32 experts: the split-K router, skinny FFN
+    tiles (every group holds a few rows), shared experts and the hoisted combine, against
+    the oracle."""
+    run_and_compare(BASE.with_(T=T, D=512, E=E, ep_size=8, top_k=k, F=256, n_shared=1,
+                               F_shared=256, zipf_bias=zipf, seed=T))
+
+
 def test_k_equals_e_and_no_renormalisation():
     run_and_compare(BASE.with_(T=200, E=8, top_k=8, ep_size=4))
     run_and_compare(BASE.with_(T=200, renormalize=False))
