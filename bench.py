@@ -53,7 +53,17 @@ def parse_args():
     ap.add_argument("--cpu-sample", type=int, default=0,
                     help="tokens per CPU-oracle sample (0 = sized for ~12 s of host time)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run the workload's shapes with this many tokens instead of its T "
+                         "(serving-sized batches; the line's workload name gets a _t<N> suffix)")
     return ap.parse_args()
+
+
+def pick_workload(args):
+    wl = W.get(args.workload)
+    if args.tokens > 0:
+        wl = wl.with_(T=args.tokens, name=f"{wl.name}_t{args.tokens}")
+    return wl
 
 
 def load_peaks():
@@ -235,7 +245,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    wl = W.get(args.workload)
+    wl = pick_workload(args)
     inp = W.make_inputs(wl, device="cpu")
     host = host_inputs_f64(wl, inp)
     del inp
@@ -272,7 +282,7 @@ def run_ours(args):
     torch.cuda.set_device(local)
     import expert_dispatch_fp32_b200 as M
 
-    wl = W.get(args.workload)
+    wl = pick_workload(args)
     peaks, peak_src = load_peaks()
     inp = W.make_inputs(wl, device="cuda")
     if rank > 0:
