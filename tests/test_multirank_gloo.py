@@ -67,3 +67,16 @@ def test_reference_arm_line_on_rank0():
     line = json.loads(p.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_reference_arm_tokens_override():
+    """--tokens runs the workload's shapes at another token count and names it so."""
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "worked_example_t64", "--tokens", "9", "--steps", "1",
+                        "--warmup", "1"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert p.returncode == 0, p.stderr
+    line = json.loads(p.stdout.strip().splitlines()[-1])
+    assert line["config"]["workload"] == "worked_example_t64_t9" and line["config"]["T"] == 9
+    assert line["value"] > 0
