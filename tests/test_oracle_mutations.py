@@ -14,7 +14,7 @@ from test_oracle_pins import ALL_CHECKS
 
 _orig = {name: getattr(O, name) for name in
          ("combine", "expert_ffn", "topk_select", "gelu", "expert_placement", "preprocess",
-          "router_logits", "shared_experts", "bf16_round", "permute")}
+          "router_logits", "shared_experts", "bf16_round", "permute", "route_gaps")}
 
 
 def _combine_no_residual(y_tok, topk_w, residual, shared=None):
@@ -98,6 +98,30 @@ def _permute_off_by_one(x_rows, src, k):
     return np.asarray(x_rows)[(np.asarray(src, dtype=np.int64) + 1) % (len(src)) // k]
 
 
+def _gaps_one_neighbour_early(logits, k):
+    s = -np.sort(-np.asarray(logits, dtype=np.float64), axis=1)
+    gap, inner = _orig["route_gaps"](logits, k)
+    if 2 <= k:
+        gap = s[:, k - 2] - s[:, k - 1]
+    return gap, inner
+
+
+def _gaps_inner_includes_next(logits, k):
+    s = -np.sort(-np.asarray(logits, dtype=np.float64), axis=1)
+    gap, inner = _orig["route_gaps"](logits, k)
+    if k < s.shape[1]:
+        inner = np.diff(-s[:, :k + 1], axis=1).min(axis=1)
+    return gap, inner
+
+
+def _gaps_unsorted(logits, k):
+    l = np.asarray(logits, dtype=np.float64)
+    T, E = l.shape
+    gap = l[:, k - 1] - l[:, k] if k < E else np.full(T, np.inf)
+    inner = np.abs(np.diff(l[:, :k], axis=1)).min(axis=1) if k > 1 else np.full(T, np.inf)
+    return gap, inner
+
+
 MUTATIONS = {
     "combine drops the residual": ("combine", _combine_no_residual),
     "SwiGLU gate/up halves swapped": ("expert_ffn", _ffn_swapped),
@@ -112,6 +136,9 @@ MUTATIONS = {
     "shared experts weighted by 1/2": ("shared_experts", _shared_half),
     "bf16 by truncation": ("bf16_round", _bf16_truncate),
     "permute gathers the wrong row": ("permute", _permute_off_by_one),
+    "set gap taken one neighbour early": ("route_gaps", _gaps_one_neighbour_early),
+    "inner gap includes the (k+1)-th logit": ("route_gaps", _gaps_inner_includes_next),
+    "gaps read from unsorted logits": ("route_gaps", _gaps_unsorted),
 }
 
 

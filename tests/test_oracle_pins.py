@@ -81,10 +81,12 @@ def check_worked_example_placement(O):
     E = GOLD["num_experts"][0]
     ep = GOLD["num_devices"][0]
     assert E // ep == GOLD["experts_per_device"][0]
-    for e, dev, loc in zip(GOLD["chosen_experts"], GOLD["device_of_chosen"],
-                           GOLD["local_index_of_chosen"]):
-        r, l = O.expert_placement(e, E, ep)
-        assert (int(r), int(l)) == (dev, loc)
+    for e, dev in zip(GOLD["chosen_experts"], GOLD["device_of_chosen"]):
+        r, _ = O.expert_placement(e, E, ep)
+        assert int(r) == dev
+    # Step 2 prints the remote entry's tag: expert 11 is local expert 11 mod 4 = 3
+    _, l = O.expert_placement(GOLD["chosen_experts"][1], E, ep)
+    assert int(l) == GOLD["local_index_of_remote"][0]
     ranks, _ = O.expert_placement(np.arange(E), E, ep)
     assert list(np.nonzero(ranks == 0)[0]) == GOLD["experts_on_device_0"]
     assert list(np.nonzero(ranks == 2)[0]) == GOLD["experts_on_device_2"]
@@ -180,6 +182,44 @@ def check_ties_lower_index(O):
     idx, w = O.topk_select(logits, 2)
     assert idx.tolist() == [[0, 1], [3, 6], [2, 5]]
     assert np.allclose(w, 0.5)
+
+
+def check_route_gaps(O):
+    """The margins that decide which tokens the parity tests exempt, on logits whose
+    sorted values are built from powers of two, so every gap is an exact fp32
+    number known in advance.  Each row lists its logits out of order; the k-th/(k+1)-th
+    gap, the gaps around it and the gaps inside the top-k all differ, so taking the
+    wrong neighbour, forgetting to sort, or letting the (k+1)-th into the inner gap
+    each gives a different number."""
+    h = 2.0 ** -17                          # ~7.6e-6: below the 1e-5 exemption threshold
+    H = 2.0 ** -16                          # ~1.5e-5: above it
+    # sorted descending: 4, 3.5, 3.25, 3.25 - h, 3 ... ; gaps 0.5, 0.25, h, 0.25 - h ...
+    desc = np.array([4.0, 3.5, 3.25, 3.25 - h, 3.0, 1.0], dtype=np.float32)
+    perm = [3, 0, 5, 1, 4, 2]
+    rows = np.stack([desc[perm], desc[perm[::-1]]])
+    # k = 3: gap_k = 3.25 - (3.25 - h) = h; inner = min(0.5, 0.25) = 0.25
+    g, inner = O.route_gaps(rows, 3)
+    assert g.tolist() == [h, h] and inner.tolist() == [0.25, 0.25]
+    # k = 2: gap_k = 3.5 - 3.25 = 0.25; inner = 0.5
+    g, inner = O.route_gaps(rows, 2)
+    assert g.tolist() == [0.25, 0.25] and inner.tolist() == [0.5, 0.5]
+    # k = 4: gap_k = (3.25 - h) - 3 = 0.25 - h; inner = h (the 3rd/4th pair)
+    g, inner = O.route_gaps(rows, 4)
+    assert g.tolist() == [0.25 - h, 0.25 - h] and inner.tolist() == [h, h]
+    # k = 1: the set margin is the top two's gap; no order inside a single pick
+    g, inner = O.route_gaps(rows, 1)
+    assert g.tolist() == [0.5, 0.5] and np.all(np.isinf(inner))
+    # k = E: every expert is chosen, the set has no margin to lose
+    g, inner = O.route_gaps(rows, 6)
+    assert np.all(np.isinf(g)) and inner.tolist() == [h, h]
+    # exact ties give a zero gap, and one of 2^-16 stays above the threshold
+    ties = np.array([[1.0, 2.0, 2.0, 0.0], [2.0, 2.0 - H, 0.0, 2.0 - H - 0.5]], dtype=np.float32)
+    g, inner = O.route_gaps(ties, 1)
+    assert g.tolist() == [0.0, H]
+    g, inner = O.route_gaps(ties, 2)
+    assert g.tolist() == [1.0, 0.5] and inner.tolist() == [0.0, H]
+    # the rows' margins against the 1e-5 threshold the tests apply
+    assert h < 1e-5 < H
 
 
 def check_softmax_library(O):
@@ -405,7 +445,8 @@ def check_bruteforce_layer(O):
 
 ALL_CHECKS = [
     check_worked_example_placement, check_worked_example_routing, check_worked_example_output,
-    check_logits_exact, check_topk_bruteforce, check_ties_lower_index, check_softmax_library,
+    check_logits_exact, check_topk_bruteforce, check_ties_lower_index, check_route_gaps,
+    check_softmax_library,
     check_preprocess_invariants, check_permute_roundtrip, check_activation_closed_forms,
     check_swiglu_gate_up_order, check_ffn_library, check_bf16_round_library,
     check_identical_experts_is_dense, check_single_expert_is_dense, check_zero_experts_is_shared,
