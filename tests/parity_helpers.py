@@ -49,11 +49,26 @@ def oracle_route(wl, inp, tokens=None):
     return dict(logits=logits, idx=idx, w=w, gap=gap, inner=inner)
 
 
-def compare_routing(gpu_idx, gpu_w, ref):
-    """Assert routing parity; returns (n_exempt, n_exempt_that_differ)."""
+MAX_EXEMPT_FRAC = 0.005   # near-tie tokens allowed before a test calls the exemption suspect
+
+
+def compare_routing(gpu_idx, gpu_w, ref, max_exempt="default"):
+    """Assert routing parity; returns (n_exempt, n_exempt_that_differ).
+
+    The exemption must stay rare: random logits put a k-th/(k+1)-th gap below 1e-5
+    on about 1e-4 of tokens, so more than MAX_EXEMPT_FRAC of T (at least 2 tokens)
+    means the gaps are wrong, not the routing.  Tests built on exact ties pass
+    max_exempt=None."""
     idx, w = ref["idx"], ref["w"]
     exempt = ref["gap"] < GAP
     order_exempt = (ref["inner"] < GAP) & ~exempt
+    if max_exempt == "default":
+        max_exempt = max(2, int(MAX_EXEMPT_FRAC * len(idx)))
+    n_ex = int(exempt.sum() + order_exempt.sum())
+    print(f"[routing] tokens {len(idx)}, set-exempt {int(exempt.sum())}, "
+          f"order-exempt {int(order_exempt.sum())}")
+    if max_exempt is not None:
+        assert n_ex <= max_exempt, f"{n_ex} exempt tokens of {len(idx)} (bound {max_exempt})"
     strict = ~exempt & ~order_exempt
     bad = np.nonzero(~np.all(gpu_idx[strict] == idx[strict], axis=1))[0]
     assert bad.size == 0, f"{bad.size} non-exempt tokens route differently, e.g. {np.nonzero(strict)[0][bad[:5]]}"
