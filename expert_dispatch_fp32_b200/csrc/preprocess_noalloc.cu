@@ -29,21 +29,55 @@ static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchInts];
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 int32_t* g_scratch_ptr[kMaxDevices] = {nullptr};
+unsigned long long g_scratch_ctx[kMaxDevices] = {0};   // context id the address belongs to
+
+// Unique id of the calling thread's current context (0 if none is current yet).  Ids
+// are never reused in a process, so a device reset, which destroys the context and
+// reloads the library's device array when the next one is made, shows as a new id.
+unsigned long long current_context_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = []() -> GetCurrentFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<GetCurrentFn>(p);
+  }();
+  static GetIdFn get_id = []() -> GetIdFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<GetIdFn>(p);
+  }();
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS ||
+      ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 // Device address of g_noalloc_scratch on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address must come from
-// cudaGetSymbolAddress, once per device, with that device current.
+// cudaGetSymbolAddress, with the device current: once per device, and again only if
+// the device's context has changed since (the array then lives in the new context).
 cudaError_t scratch_for_current_device(int32_t** out) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (g_scratch_ptr[dev] == nullptr || ctx == 0 || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
-    err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    err = cudaGetSymbolAddress(&p, g_noalloc_scratch);   // makes the context current if needed
     if (err != cudaSuccess) return err;
     g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+    g_scratch_ctx[dev] = current_context_id();
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;

@@ -168,7 +168,10 @@ MOE_API moe_status moe_dispatch_permute(const moe_config* cfg, const void* x, co
  *   y_perm         device bf16 [R, D], written
  *   shared_out     device bf16 [T, D], written when S > 0; NULL skips the shared
  *                  experts (moe_shared_ffn runs them alone)
- *   workspace      the buffer moe_preprocess wrote its tile prefix into
+ *   workspace      the buffer moe_preprocess (or moe_route_dispatch) wrote its tile
+ *                  prefix into, for this same routing: moe_preprocess_noalloc writes no
+ *                  prefix, so its outputs need a moe_preprocess of the same topk_idx
+ *                  before this call, or the tiles follow an earlier routing
  *   status         device int32, MOE_ERR_TIMEOUT if a bounded wait expired */
 MOE_API moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void* x,
                           const int32_t* expert_offsets, const void* packed, void* act,
@@ -245,12 +248,16 @@ MOE_API moe_status moe_forward(const moe_config* cfg, const void* x, const float
  * moe_preprocess (bit-identical results); it does not write the GEMM tile prefix
  * that moe_expert_ffn reads from a workspace, so it is a drop-in for the
  * bookkeeping outputs only.
- *   Limit: min(160, ceil(T*k / 256)) * E + 2*(E + 1) + 2 int32 values must fit in
- *   the scratch; larger configurations return MOE_ERR_SCRATCH_LIMIT before anything
- *   is enqueued.
+ *   Limit: max(1, min(160, ceil(T*k / 256))) * E + 2*(E + 1) + 2 int32 values must
+ *   fit in the scratch (the check uses this count; the launch may then use fewer
+ *   blocks on a GPU with fewer SMs); larger configurations return
+ *   MOE_ERR_SCRATCH_LIMIT before anything is enqueued.
  *   First call on each device: finds the scratch array's device address with
  *   cudaGetSymbolAddress (once per device, with that device current), so make that
- *   first call before any stream capture.
+ *   first call before any stream capture.  The address is looked up again when the
+ *   device's context is not the one it was found in (after cudaDeviceReset, the
+ *   library's device array is loaded anew); that lookup, too, must not fall inside a
+ *   stream capture.
  *   Concurrency: every call shares the one array and leaves its contents behind
  *   (each call rewrites all it reads); calls that may overlap on the GPU, e.g. on
  *   two streams without ordering between them, race and must not be issued. */

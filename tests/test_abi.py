@@ -97,7 +97,12 @@ def test_null_and_misaligned_pointers_rejected_on_host(B):
     c = good_cfg(B)
     lib = B.lib()
     by = ctypes.byref(c)
-    fake = 1 << 20                    # never dereferenced: validation fails first
+    # a real, 256-byte-aligned host buffer stands in for every non-null argument: the
+    # calls must reject before they enqueue anything, and if one ever did not, it would
+    # hand the runtime an address it can reject, never an arbitrary one
+    import numpy as np
+    buf = np.zeros(1 << 16, dtype=np.uint8)
+    fake = (buf.ctypes.data + 255) // 256 * 256
     assert lib.moe_route(by, None, fake, None, None, fake, fake, fake, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_route(by, fake + 4, fake, None, None, fake, fake, fake, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_preprocess(by, fake, fake, fake, fake, fake, fake, fake, fake, None, None) == B.MOE_ERR_INVALID_ARG

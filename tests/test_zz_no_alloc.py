@@ -55,10 +55,40 @@ def test_noalloc_preprocess_matches_workspace_preprocess_twice():
         for key in KEYS:
             assert torch.equal(got[key], ref[key]), (call, key)
         assert int(got["counts"].sum().item()) == wl.R
+        # and against the oracle's definition of the same bookkeeping
+        pre = oracle.preprocess(idx.cpu().numpy(), wl.E, wl.ep_size)
+        for key in KEYS:
+            assert np.array_equal(got[key].cpu().numpy(), pre[key]), (call, key)
 
 
 @pytest.mark.gpu
 def test_noalloc_rejects_configs_beyond_its_scratch():
-    cfg = M.make_config(1 << 20, 64, 1024, 8, 8, 128)      # 8192 blocks x 1024 experts
-    st = M.lib().moe_preprocess_noalloc(ctypes.byref(cfg), *([1 << 20] * 8), None)
+    # 2048 tokens x top-8 over 1024 experts: 64 histogram blocks x 1024 experts plus the
+    # prefixes need 67 588 int32, more than the 65 536 the scratch holds.  Real buffers of
+    # the right sizes, so nothing would fault even if a launch were enqueued.
+    wl = W.Workload(name="wide", T=2048, D=64, E=1024, ep_size=8, top_k=8, F=128)
+    cfg = M.make_config(wl.T, wl.D, wl.E, wl.ep_size, wl.top_k, wl.F)
+    idx = torch.zeros((wl.T, wl.top_k), dtype=torch.int32, device="cuda")
+    got = _buffers(wl)
+    st = M.lib().moe_preprocess_noalloc(
+        ctypes.byref(cfg), idx.data_ptr(), got["counts"].data_ptr(), got["expert_offsets"].data_ptr(),
+        got["rank_splits"].data_ptr(), got["rank_offsets"].data_ptr(), got["pos"].data_ptr(),
+        got["src"].data_ptr(), got["status"].data_ptr(), None)
     assert st == M.MOE_ERR_SCRATCH_LIMIT
+    torch.cuda.synchronize()
+    assert int(got["counts"][0].item()) == -7          # nothing was written
+    # just under the limit: 1920 tokens -> 60 histogram blocks -> 63 492 int32 (1984 tokens
+    # would need 62 blocks, 65 540 int32, four too many)
+    wl2 = wl.with_(T=1920)
+    cfg2 = M.make_config(wl2.T, wl2.D, wl2.E, wl2.ep_size, wl2.top_k, wl2.F)
+    g = torch.Generator(device="cpu").manual_seed(5)
+    idx2 = torch.rand((wl2.T, wl2.E), generator=g).argsort(dim=1)[:, :wl2.top_k]
+    idx2 = idx2.to(torch.int32).contiguous().cuda()       # k distinct experts per token
+    got2 = _buffers(wl2)
+    M.moe_preprocess_noalloc(cfg2, idx2, got2["counts"], got2["expert_offsets"], got2["rank_splits"],
+                             got2["rank_offsets"], got2["pos"], got2["src"], got2["status"])
+    torch.cuda.synchronize()
+    assert int(got2["status"].item()) == 0
+    pre = oracle.preprocess(idx2.cpu().numpy(), wl2.E, wl2.ep_size)
+    for key in KEYS:
+        assert np.array_equal(got2[key].cpu().numpy(), pre[key]), key
