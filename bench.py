@@ -37,7 +37,7 @@ sys.path.insert(0, ROOT)
 
 import moe_workloads as W  # noqa: E402
 
-DEFAULT_WORKLOAD = "small_e8_d2048"
+DEFAULT_WORKLOAD = "deepseek_v3"
 METRIC = "MoE-layer fwd tokens/s on 1 B200; grouped-FFN % BF16 peak; permute/combine GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
@@ -184,8 +184,29 @@ def ffn_launches(wl):
     return 4 if wl.n_shared else 2
 
 
-def cpu_oracle_time(wl, inp_host, n_tok, seed=0):
-    """Time the oracle's layer forward on a token sample (weights already float64 on the host)."""
+class HostOracleInputs:
+    """The oracle's view of a workload's inputs: x and the router on the host in
+    float64, expert weights fetched one expert at a time (bf16 -> float64) from
+    wherever the drawn tensors live, so a 256-expert layer never needs its ~90 GB of
+    float64 weights at once.  The fetch is part of the oracle's work as timed."""
+
+    def __init__(self, wl, inp):
+        f = lambda t: None if t is None else t.detach().cpu().to(torch.float64).numpy()
+        self.wl = wl
+        self.x = f(inp["x"])
+        self.w_router = inp["w_router"].cpu().numpy()
+        self.bias = None if inp["bias"] is None else inp["bias"].cpu().numpy()
+        self._up = inp["w_gate_up"] if wl.act == "swiglu" else inp["w1"]
+        self._down = inp["w_down"]
+        self.ws_up, self.ws_down = f(inp["ws_gate_up"]), f(inp["ws_down"])
+
+    def expert(self, e):
+        f = lambda t: t.detach().cpu().to(torch.float64).numpy()
+        return f(self._up[e]), f(self._down[e])
+
+
+def cpu_oracle_time(wl, host, n_tok, seed=0):
+    """Time the oracle's layer forward on a token sample (weights streamed per expert)."""
     import oracle
     rng = np.random.default_rng(seed)
     # a sample larger than the batch runs the oracle over several random draws of it
@@ -193,22 +214,14 @@ def cpu_oracle_time(wl, inp_host, n_tok, seed=0):
     t = 0.0
     for n in sizes:
         toks = np.sort(rng.choice(wl.T, size=n, replace=False))
-        x = inp_host["x"][toks]
+        x = host.x[toks]
         t0 = time.perf_counter()
-        oracle.moe_layer(x, inp_host["w_router"], inp_host["bias"], inp_host["w_up"], inp_host["w_down"],
-                         inp_host["ws_up"], inp_host["ws_down"], E=wl.E, ep_size=wl.ep_size,
-                         top_k=wl.top_k, act=wl.act, renormalize=wl.renormalize,
-                         x_is_f32=(wl.x_dtype == "f32"))
+        oracle.moe_layer(x, host.w_router, host.bias, None, None, host.ws_up, host.ws_down,
+                         E=wl.E, ep_size=wl.ep_size, top_k=wl.top_k, act=wl.act,
+                         renormalize=wl.renormalize, x_is_f32=(wl.x_dtype == "f32"),
+                         expert_weights=host.expert)
         t += time.perf_counter() - t0
     return t
-
-
-def host_inputs_f64(wl, inp):
-    f = lambda t: None if t is None else t.detach().cpu().to(torch.float64).numpy()
-    return dict(x=f(inp["x"]), w_router=inp["w_router"].cpu().numpy(),
-                bias=None if inp["bias"] is None else inp["bias"].cpu().numpy(),
-                w_up=f(inp["w_gate_up"] if wl.act == "swiglu" else inp["w1"]), w_down=f(inp["w_down"]),
-                ws_up=f(inp["ws_gate_up"]), ws_down=f(inp["ws_down"]))
 
 
 def cpu_threads():
@@ -223,11 +236,11 @@ def cpu_threads():
 
 
 def pick_sample(wl, host, budget_s):
-    """Tokens per oracle sample so one sample costs about budget_s on the host:
-    time a 64-token probe and scale (tokens are independent, cost is linear), then
-    re-time a quarter of that estimate and scale again (the small probe carries the
-    per-call costs, so by itself it undersizes the sample by a factor of 2-3)."""
-    probe = min(64, wl.T)
+    """Tokens per oracle sample so one sample costs about budget_s on the host: time a
+    small probe and scale (tokens are independent; with few tokens per expert the cost
+    grows with the experts they touch, about linearly in the tokens), then re-time a
+    quarter of that estimate and scale again (the probe carries the per-call costs)."""
+    probe = min(2 if wl.E * wl.D * wl.F >= 1 << 30 else 64, wl.T)
     cpu_oracle_time(wl, host, probe, seed=99)            # warm the BLAS threads
     t = cpu_oracle_time(wl, host, probe, seed=98)
     cap = 16 * wl.T
@@ -246,9 +259,12 @@ def run_reference(args):
     if rank != 0:
         return 0
     wl = pick_workload(args)
-    inp = W.make_inputs(wl, device="cpu")
-    host = host_inputs_f64(wl, inp)
-    del inp
+    # the same seeded draws as the GPU arm (drawn on the GPU where there is one: a
+    # 256-expert layer's weights take minutes to draw on the host); the oracle itself
+    # runs on the host cores only
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = W.make_inputs(wl, device=dev)
+    host = HostOracleInputs(wl, inp)
     n_tok = args.cpu_sample or pick_sample(wl, host, min(10.0, max(0.5, 120.0 / max(1, args.steps))))
     for i in range(args.warmup):
         cpu_oracle_time(wl, host, min(n_tok, 16), seed=i)
@@ -266,7 +282,8 @@ def run_reference(args):
                    "tokens_per_step": n_tok},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"{n_tok} random tokens of the {wl.name} batch per step "
-                                   f"(tokens are independent: dropless routing)"},
+                                   f"(tokens are independent: dropless routing); expert weights "
+                                   f"fetched and widened to float64 one expert at a time"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -290,7 +307,8 @@ def run_ours(args):
     cpu_host = None
     want_cpu = (rank == 0 and ws == 1 and not args.no_cpu_baseline)
     if want_cpu:
-        cpu_host = host_inputs_f64(wl, inp)
+        # keeps the drawn weights (bf16, on the device) for the oracle to fetch per expert
+        cpu_host = HostOracleInputs(wl, inp)
     up = inp["w_gate_up"] if wl.act == "swiglu" else inp["w1"]
     layer = M.MoELayer(D=wl.D, E=wl.E, ep_size=wl.ep_size, top_k=wl.top_k, F=wl.F,
                        w_router=inp["w_router"], w_gate_up=up, w_down=inp["w_down"],
@@ -461,15 +479,14 @@ def run_ours(args):
     e2e_value = replica_value(T, ws, args.steps, e2e_ms)
     sx = 4 if wl.x_dtype == "f32" else 2
 
-    # roofline of the dominant kernel: the grouped expert FFN (tcgen05 GEMMs)
+    # roofline of the dominant kernel: the grouped expert FFN (tcgen05 GEMMs), against the
+    # measured bf16 burst peak (a kernel of a few ms, timed alone in the stage pass); the
+    # ratio to the seconds-long sustained figure is reported beside it
     ffn_ms = stage_ms[3] / args.steps
     ffn_tflops = wl.ffn_flop() / (ffn_ms / 1e3) / 1e12
-    # a step of several ms keeps the tensor cores busy long enough to meet the power cap:
-    # compare against the sustained figure there, the burst figure for short steps
-    long_step = total_ms_max / args.steps > 2.0
-    peak_key = "bf16_tflops_sustained" if long_step else "bf16_tflops"
+    peak_key = "bf16_tflops"
     peak_tf = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
-    burst_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    sust_tf = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "ffn_traffic.json")
     if os.path.exists(tpath):
@@ -529,8 +546,8 @@ def run_ours(args):
                                + (", shared gate_up+down" if wl.n_shared else "") + ")",
                      "timed": "CUDA events around the FFN stage call in a stage-by-stage pass "
                               "of the same kernels, after an L2 flush per step",
-                     "peak_source": f"{peak_src} bf16 " + ("sustained (step > 2 ms)" if long_step else "burst"),
-                     "frac_of_burst": ffn_tflops / burst_tf},
+                     "peak_source": f"{peak_src} bf16 burst (cuBLAS 8192^3, best of 10)",
+                     "frac_of_sustained": ffn_tflops / sust_tf},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * wl.D * sx,
                 "d2h_bytes_per_step": T * wl.D * sx},
         "gpu_launches": launches_per_step * args.steps,
