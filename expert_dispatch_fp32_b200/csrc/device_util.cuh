@@ -9,6 +9,26 @@ namespace {
 
 constexpr long long kBarrierLimitCycles = 2000000000ll;   // ~1 s at 2 GHz
 
+// Eight terms of a router dot product, added to `acc` in order.  x (bf16 or fp32) and
+// w (fp32) convert exactly to fp64 and their product needs at most 48 significant
+// bits, so every term is exact and only the fp64 sums round: the logit, rounded once
+// to fp32 at the end, is the exact dot product's fp32 value unless the fp64 rounding
+// (relative 2^-53 of the largest partial sum) moves it across an fp32 rounding
+// boundary.  With fp32 partial products, inputs whose partial sums are orders of
+// magnitude above the logit (heavy cancellation) lost the digits that rank experts.
+__device__ __forceinline__ double dot8_exact(const float (&x)[8], const float4& w0, const float4& w1,
+                                             double acc) {
+  acc = fma((double)x[0], (double)w0.x, acc);
+  acc = fma((double)x[1], (double)w0.y, acc);
+  acc = fma((double)x[2], (double)w0.z, acc);
+  acc = fma((double)x[3], (double)w0.w, acc);
+  acc = fma((double)x[4], (double)w1.x, acc);
+  acc = fma((double)x[5], (double)w1.y, acc);
+  acc = fma((double)x[6], (double)w1.z, acc);
+  acc = fma((double)x[7], (double)w1.w, acc);
+  return acc;
+}
+
 // Grid-wide barrier for a cooperative launch.  bar[0] counts arrivals, bar[1] is a
 // generation the last arrival bumps; both start at zero (set on the stream before
 // the launch).  Bounded: after kBarrierLimitCycles a waiting block reports
@@ -112,13 +132,12 @@ __device__ __forceinline__ int scan_array(int* vals, int n, int* warp_sums, int*
 // holding a contiguous chunk of the flat (token, slot) pairs and having published its
 // per-expert histogram row in block_counts[blockIdx.x][E]: cnt[e] becomes the first
 // row of expert e for this block's pairs (expert offset + pairs of e in earlier
-// blocks); block 0 also writes counts, expert offsets, rank splits / offsets and the
-// GEMM M-tile prefixes.  tmp[E] and warp_cnt[>= E] are scratch.
+// blocks); block 0 also writes counts, expert offsets and rank splits / offsets.
+// tmp[E] is scratch.
 template <int NT>
 __device__ void pre_totals(const int32_t* block_counts, int E, int ep, int* cnt, int* tmp,
-                           int* warp_cnt, int* warp_sums, int* total, int32_t* counts,
-                           int32_t* expert_offsets, int32_t* rank_splits, int32_t* rank_offsets,
-                           int32_t* mt_start) {
+                           int* warp_sums, int* total, int32_t* counts,
+                           int32_t* expert_offsets, int32_t* rank_splits, int32_t* rank_offsets) {
   const int tid = threadIdx.x;
   // rows of other blocks are read past L1, which is not coherent across SMs.  With
   // E < NT the blocks' rows of an expert are split over NT / E threads (their partial
@@ -170,20 +189,6 @@ __device__ void pre_totals(const int32_t* block_counts, int E, int ep, int* cnt,
       rank_offsets[r] = lo;
     }
     if (tid == 0) rank_offsets[ep] = R_all;
-    // GEMM M-tile prefixes: [0, E] for 128-row tiles, [E+1, 2E+1] for 256-row tiles
-    for (int half = 0; half < 2; ++half) {
-      const int tm = half ? 2 * kTileM : kTileM;
-      int* outp = mt_start + half * (E + 1);
-      __syncthreads();
-      for (int e = tid; e < E; e += NT) {
-        const int ce = (e + 1 < E ? tmp[e + 1] : R_all) - tmp[e];
-        warp_cnt[e] = (ce + tm - 1) / tm;
-      }
-      __syncthreads();
-      const int tiles = scan_array(warp_cnt, E, warp_sums, total);
-      for (int e = tid; e < E; e += NT) outp[e] = warp_cnt[e];
-      if (tid == 0) outp[E] = tiles;
-    }
   }
   __syncthreads();
 }

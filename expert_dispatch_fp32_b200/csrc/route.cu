@@ -4,22 +4,25 @@
 // scores all E experts for the token, softmax-normalises, keeps the top-k.
 // "Expert Parallel (EP)", Configuration: router_dtype 'fp32'.
 //
-// Logits kernel: a token-tiled SIMT fp32 GEMM (x[T,D] . W_r[E,D]^T).  W_r does not
-// fit in shared memory for large E*D, so tiles of BM tokens x BN experts stream
-// 32-wide K slices of both operands through shared memory.  Each thread sums a
-// 32-term K slice in fp32 and folds the slice into an fp64 running total, so the
-// stored fp32 logit is the dot product rounded once, to within fp32 round-off of
-// a 32-term partial (~1e-8 relative), far inside the 1e-5 near-tie margin.  With few
-// tokens the K range is split across blocks (fp64 slice totals, added in order by a
-// second kernel before the single rounding).
+// Every router path forms each term x_d * W_r[e,d] exactly in fp64 (both operands
+// convert exactly and the product needs at most 48 bits), sums the terms in fp64 and
+// rounds the total once to fp32 (dot8_exact in device_util.cuh): the stored logit is
+// the exact dot product's fp32 value up to the fp64 sums' rounding, whatever the
+// magnitudes and cancellation in x.
+//
+// Logits kernel: a token-tiled SIMT GEMM (x[T,D] . W_r[E,D]^T).  W_r does not fit in
+// shared memory for large E*D, so tiles of BM tokens x BN experts stream 32-wide K
+// slices of both operands through shared memory; each thread keeps fp64 totals of its
+// register tile.  With few tokens the K range is split across blocks (fp64 slice
+// totals, added in order by a second kernel before the single rounding).
 //
 // Top-k kernel: one warp per token; selection j is an exact warp argmax on
 // (logit, -index), so ties go to the lower expert index; lane j keeps pick j.
 //
 // Few experts (E <= 32 and W_r small enough for shared memory): one fused kernel.
 // W_r is staged in shared memory once per block; each warp streams TW tokens of x
-// with coalesced 16-byte loads (lane l holds columns 8l..8l+7 of every 256), sums
-// each 8-column slice in fp32 and folds it into an fp64 per-lane accumulator, then
+// with coalesced 16-byte loads (lane l holds columns 8l..8l+7 of every 256), adds
+// their exact terms to an fp64 per-lane accumulator, then
 // an fp64 butterfly leaves every lane with all E dot products; lane e keeps logit
 // e and the warp runs the same exact argmax top-k without a logits round trip.
 #include <math.h>
@@ -118,29 +121,22 @@ route_logits_kernel(const XT* __restrict__ x, const float* __restrict__ w,
     }
     __syncthreads();
     if (k0 + BK < kend) load_slice(k0 + BK);
-    float acc[TM][4];
-#pragma unroll
-    for (int i = 0; i < TM; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 8
+    // every term exact in fp64 (see dot8_exact), summed in K order
+#pragma unroll 4
     for (int kk = 0; kk < BK; ++kk) {
-      float a[TM];
+      double a[TM];
 #pragma unroll
-      for (int i = 0; i < TM; ++i) a[i] = xs[kk][ty * TM + i];
+      for (int i = 0; i < TM; ++i) a[i] = (double)xs[kk][ty * TM + i];
       const float4 b = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
+      const double b0 = b.x, b1 = b.y, b2 = b.z, b3 = b.w;
 #pragma unroll
       for (int i = 0; i < TM; ++i) {
-        acc[i][0] = fmaf(a[i], b.x, acc[i][0]);
-        acc[i][1] = fmaf(a[i], b.y, acc[i][1]);
-        acc[i][2] = fmaf(a[i], b.z, acc[i][2]);
-        acc[i][3] = fmaf(a[i], b.w, acc[i][3]);
+        tot[i][0] = fma(a[i], b0, tot[i][0]);
+        tot[i][1] = fma(a[i], b1, tot[i][1]);
+        tot[i][2] = fma(a[i], b2, tot[i][2]);
+        tot[i][3] = fma(a[i], b3, tot[i][3]);
       }
     }
-#pragma unroll
-    for (int i = 0; i < TM; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) tot[i][j] += (double)acc[i][j];
     __syncthreads();
   }
 #pragma unroll
@@ -283,15 +279,7 @@ route_small_kernel(const XT* __restrict__ x, const float* __restrict__ w,
           const float4 w1 = *reinterpret_cast<const float4*>(w_s + (size_t)e * D + d0 + 4);
 #pragma unroll
           for (int i = 0; i < TW; ++i) {
-            float p = xv[i][0] * w0.x;
-            p = fmaf(xv[i][1], w0.y, p);
-            p = fmaf(xv[i][2], w0.z, p);
-            p = fmaf(xv[i][3], w0.w, p);
-            p = fmaf(xv[i][4], w1.x, p);
-            p = fmaf(xv[i][5], w1.y, p);
-            p = fmaf(xv[i][6], w1.z, p);
-            p = fmaf(xv[i][7], w1.w, p);
-            acc[i][e] += (double)p;
+            acc[i][e] = dot8_exact(xv[i], w0, w1, acc[i][e]);
           }
         }
       }
@@ -457,8 +445,8 @@ cudaError_t launch_route_t(const moe_config& c, const XT* x, const float* w_rout
 //    one fp32 rounding per MMA instruction in each of the two chains plus the lo
 //    part, with a factor 2 of margin).  Experts whose approx is below the k-th
 //    largest approx minus 2 eps_t cannot be in the exact top-k; the others
-//    (usually k plus one or two) get an exact logit (fp32 8-term slices folded into
-//    fp64, as in the SIMT paths), and the top-k and weights are taken from those.
+//    (usually k plus one or two) get an exact logit (exact fp64 terms summed in fp64,
+//    as in the SIMT paths), and the top-k and weights are taken from those.
 constexpr int kRouterRowBlock = 128;      // experts per 256-row (hi, mid) block
 constexpr int kRefineWarps = 4;
 
@@ -596,15 +584,7 @@ route_refine_kernel(const bf16* __restrict__ x, const float* __restrict__ w,
         const float* wr = w + (size_t)ce[q] * D + d0;
         const float4 w0 = __ldg(reinterpret_cast<const float4*>(wr));
         const float4 w1 = __ldg(reinterpret_cast<const float4*>(wr + 4));
-        float p = xf[0] * w0.x;
-        p = fmaf(xf[1], w0.y, p);
-        p = fmaf(xf[2], w0.z, p);
-        p = fmaf(xf[3], w0.w, p);
-        p = fmaf(xf[4], w1.x, p);
-        p = fmaf(xf[5], w1.y, p);
-        p = fmaf(xf[6], w1.z, p);
-        p = fmaf(xf[7], w1.w, p);
-        acc[q] += (double)p;
+        acc[q] = dot8_exact(xf, w0, w1, acc[q]);
       }
     }
 #pragma unroll
@@ -677,7 +657,7 @@ cudaError_t launch_route_tc(const moe_config& c, const bf16* x, const float* w, 
   g.A = x; g.a_rows = c.T;
   g.B = rs.bsplit; g.G = 1;
   g.N = 2 * Epad; g.K = c.D;
-  g.group_offsets = nullptr; g.mt_start = nullptr; g.dense_rows = c.T;
+  g.group_offsets = nullptr; g.dense_rows = c.T;
   g.tile_n = 256;
   g.pair = rs.pair;
   const int tm = g.pair ? 2 * kTileM : kTileM;
@@ -690,7 +670,7 @@ cudaError_t launch_route_tc(const moe_config& c, const bf16* x, const float* w, 
   err = launch_grouped_gemm(g, s);
   if (err != cudaSuccess) return err;
   // every approximate logit is within coef * S_t of the exact one (see above)
-  const float coef = (float)(4.0 * (c.D / 16 + 2) * 0x1p-23 + 0x1p-17);
+  const float coef = route_filter_coef(c.D);
   const size_t smem = (size_t)kRefineWarps * 2 * c.E * sizeof(int);
   route_refine_kernel<<<(c.T + kRefineWarps - 1) / kRefineWarps, 32 * kRefineWarps, smem, s>>>(
       x, w, bias, rs.approx, Epad, rs.wmax, coef, topk_idx, topk_w, c.T, c.D, c.E, c.top_k);
@@ -698,6 +678,23 @@ cudaError_t launch_route_tc(const moe_config& c, const bf16* x, const float* w, 
 }
 
 }  // namespace
+
+float route_filter_coef(int D) {
+  // per D: one fp32 rounding (<= 2^-23 relative, doubled) of a magnitude <= S_t per
+  // 16-deep MMA instruction in each of the hi and mid chains, two more for their sum,
+  // plus the dropped lo part (<= 2^-18 S_t, doubled)
+  return (float)(4.0 * (D / 16 + 2) * 0x1p-23 + 0x1p-17);
+}
+
+bool route_takes_filter(const moe_config& c, size_t part_bytes, bool keep_logits) {
+  if (c.x_dtype != MOE_DT_BF16) return false;
+  const char* env = getenv("MOE_ROUTER_TC");
+  const bool tc_ok = !(env && env[0] == '0');
+  const bool few = c.E <= 32 && (size_t)c.E * c.D * sizeof(float) <= kSmallRouterSmem;
+  // few tokens: the split SIMT logits (exact) beat the tensor-core filter's fixed cost
+  const bool split = !few && split_route_count(c, part_bytes) > 1;
+  return tc_ok && !few && !split && c.renormalize && !keep_logits;
+}
 
 cudaError_t launch_route(const moe_config& c, const void* x, const float* w_router,
                          const float* bias, float* logits, bool keep_logits, int32_t* topk_idx,
@@ -708,12 +705,7 @@ cudaError_t launch_route(const moe_config& c, const void* x, const float* w_rout
   // bf16 x with renormalised weights and no logits to return, too many experts for the
   // fused shared-memory router: tensor-core filter and exact refine (MOE_ROUTER_TC=0
   // selects the SIMT paths, which compute every logit exactly)
-  const char* env = getenv("MOE_ROUTER_TC");
-  const bool tc_ok = !(env && env[0] == '0');
-  const bool few = c.E <= 32 && (size_t)c.E * c.D * sizeof(float) <= kSmallRouterSmem;
-  // few tokens: the split SIMT logits (exact) beat the tensor-core filter's fixed cost
-  const bool split = !few && split_route_count(c, rs.part_bytes) > 1;
-  if (tc_ok && !few && !split && c.renormalize && !keep_logits && rs.bsplit != nullptr)
+  if (route_takes_filter(c, rs.part_bytes, keep_logits) && rs.bsplit != nullptr)
     return launch_route_tc(c, static_cast<const bf16*>(x), w_router, bias, rs, topk_idx, topk_w, s);
   return launch_route_t(c, static_cast<const bf16*>(x), w_router, bias, logits, keep_logits,
                         topk_idx, topk_w, rs.part, rs.part_bytes, s);

@@ -9,10 +9,10 @@
 //  1. W_r and the block's x rows are brought into shared memory by bulk copies, each
 //     warp's rows on a barrier of its own, so routing starts as its rows land;
 //  2. each warp routes TW tokens at a time with the arithmetic of the few-expert
-//     router (fp32 8-term slices folded into fp64, lane-parallel over D, exact
+//     router (exact fp64 terms summed in fp64, lane-parallel over D, exact
 //     argmax top-k, renormalised softmax weights) and keeps the selections;
 //  3. the block's per-expert histogram goes out, then one grid barrier;
-//  4. the totals, expert offsets, rank splits and tile prefixes, and the in-order
+//  4. the totals, expert offsets and rank splits, and the in-order
 //     rows of the block's pairs, exactly as the preprocess computes them;
 //  5. each pair's x row is written to x_perm from shared memory (bf16).
 // Every output is bit-identical to moe_route + moe_preprocess +
@@ -36,7 +36,7 @@ struct FuseArgs {
   int T, D, E, k, renorm, ep, tpb;
   int32_t* block_counts;   // [gridDim.x][E]
   unsigned* barrier;       // [2], zero at launch
-  int32_t *counts, *expert_offsets, *rank_splits, *rank_offsets, *mt_start, *pos, *src, *status;
+  int32_t *counts, *expert_offsets, *rank_splits, *rank_offsets, *pos, *src, *status;
   bf16* x_perm;
 };
 
@@ -177,15 +177,7 @@ __global__ void __launch_bounds__(kFuseThreads, 1) route_pre_dispatch_kernel(con
           const float4 w1 = *reinterpret_cast<const float4*>(w_s + (size_t)e * D + d0 + 4);
 #pragma unroll
           for (int i = 0; i < TW; ++i) {
-            float p = xv[i][0] * w0.x;
-            p = fmaf(xv[i][1], w0.y, p);
-            p = fmaf(xv[i][2], w0.z, p);
-            p = fmaf(xv[i][3], w0.w, p);
-            p = fmaf(xv[i][4], w1.x, p);
-            p = fmaf(xv[i][5], w1.y, p);
-            p = fmaf(xv[i][6], w1.z, p);
-            p = fmaf(xv[i][7], w1.w, p);
-            acc[i][e] += (double)p;
+            acc[i][e] = dot8_exact(xv[i], w0, w1, acc[i][e]);
           }
         }
       }
@@ -228,8 +220,8 @@ __global__ void __launch_bounds__(kFuseThreads, 1) route_pre_dispatch_kernel(con
   if (!grid_barrier(a.barrier, gridDim.x, a.status)) return;
 
   // 4. totals and block-0 outputs, then the in-order rows of the block's pairs
-  pre_totals<kFuseThreads>(a.block_counts, E, a.ep, cnt, tmp, warp_cnt, warp_sums, &total, a.counts,
-                           a.expert_offsets, a.rank_splits, a.rank_offsets, a.mt_start);
+  pre_totals<kFuseThreads>(a.block_counts, E, a.ep, cnt, tmp, warp_sums, &total, a.counts,
+                           a.expert_offsets, a.rank_splits, a.rank_offsets);
   const int base = t_lo * k;
   pre_positions<kFuseThreads>(base, base + ntok * k, [&](int f) { return sel[f - base]; }, E, cnt,
                               warp_cnt, a.pos, a.src, pos_s);
@@ -314,7 +306,7 @@ cudaError_t launch_route_pre_dispatch(const moe_config& c, const void* x, const 
                                       float* topk_w, int32_t* counts, int32_t* expert_offsets,
                                       int32_t* rank_splits, int32_t* rank_offsets, int32_t* pos,
                                       int32_t* src, int32_t* block_counts, int max_blocks,
-                                      int32_t* mt_start, unsigned* barrier, bool barrier_zeroed,
+                                      unsigned* barrier, bool barrier_zeroed,
                                       bf16* x_perm, int32_t* status, cudaStream_t s) {
   int grid = sm_count();
   if (grid > max_blocks) grid = max_blocks;
@@ -334,7 +326,7 @@ cudaError_t launch_route_pre_dispatch(const moe_config& c, const void* x, const 
   a.tpb = tpb;
   a.block_counts = block_counts; a.barrier = barrier;
   a.counts = counts; a.expert_offsets = expert_offsets; a.rank_splits = rank_splits;
-  a.rank_offsets = rank_offsets; a.mt_start = mt_start; a.pos = pos; a.src = src; a.status = status;
+  a.rank_offsets = rank_offsets; a.pos = pos; a.src = src; a.status = status;
   a.x_perm = x_perm;
   const bool f32 = c.x_dtype == MOE_DT_F32;
   if (c.E <= 8)

@@ -160,6 +160,19 @@ def make_inputs(wl: Workload, device="cpu") -> dict:
     return out
 
 
+def make_router_inputs(wl: Workload, device="cpu") -> dict:
+    """x, w_router and bias only: the first two draws of ``make_inputs`` (same
+    generator, same order, so the same bits), without drawing the expert weights."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(wl.seed)
+    xdt = torch.float32 if wl.x_dtype == "f32" else torch.bfloat16
+    x = _draw(gen, (wl.T, wl.D), wl.x_std, device, xdt)
+    w_router = _draw(gen, (wl.E, wl.D), wl.w_router_std, device, torch.float32)
+    b = router_bias(wl)
+    return {"x": x, "w_router": w_router, "bias": None if b is None else b.to(device)}
+
+
 def make_x(wl: Workload, device="cpu", seed: int | None = None) -> torch.Tensor:
     """A fresh activation batch only (same distribution as ``make_inputs``' x)."""
     device = torch.device(device)

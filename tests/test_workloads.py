@@ -55,3 +55,11 @@ def test_oracle_full_tiny_workload():
     assert res["out"].shape == (64, 64)
     assert res["counts"].sum() == wl.R
     assert np.all(np.isfinite(res["out"]))
+
+
+def test_router_inputs_are_the_first_draws():
+    wl = W.get("zipf_skew_e64").with_(T=96, D=128, F=128, F_shared=128)
+    full = W.make_inputs(wl)
+    part = W.make_router_inputs(wl)
+    for key in ("x", "w_router", "bias"):
+        assert torch.equal(full[key], part[key]), key
