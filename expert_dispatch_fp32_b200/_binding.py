@@ -37,6 +37,15 @@ class MoeError(RuntimeError):
         self.status = status
 
 
+class MoeEpPeers(ctypes.Structure):
+    """Mirror of ``moe_ep_peers`` (include/moe.h): P, cap and six device pointers to
+    device arrays of P device pointers."""
+    _fields_ = [("P", ctypes.c_int32), ("cap", ctypes.c_int32),
+                ("cnt", ctypes.c_void_p), ("flags", ctypes.c_void_p), ("recv_x", ctypes.c_void_p),
+                ("recv_src", ctypes.c_void_p), ("recv_rank", ctypes.c_void_p),
+                ("y_back", ctypes.c_void_p)]
+
+
 _lib = None
 _vp, _i32p, _f32p, _cfgp = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(MoeConfig)
 _SIGS = {
@@ -63,6 +72,20 @@ _SIGS = {
     "moe_gather_rows": (ctypes.c_int, [_vp, _i32p, _vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                        _vp]),
     "moe_check_wait_timeout": (ctypes.c_int, [_vp, _i32p, _vp]),
+    "moe_ep_send_counts": (ctypes.c_int, [_cfgp, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, _i32p,
+                                          ctypes.c_uint32, _vp]),
+    "moe_ep_send_rows": (ctypes.c_int, [_cfgp, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, _vp,
+                                        _i32p, _i32p, _i32p, ctypes.c_uint32, _i32p, _i32p, _vp]),
+    "moe_ep_recv_layout": (ctypes.c_int, [_cfgp, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, _i32p,
+                                          ctypes.c_uint32, _i32p, _vp]),
+    "moe_ep_return_rows": (ctypes.c_int, [_cfgp, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, _vp,
+                                          _i32p, ctypes.c_uint32, _i32p, _i32p, _vp]),
+    "moe_ep_wait_returned": (ctypes.c_int, [_cfgp, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                            ctypes.c_uint32, _i32p, _vp]),
+    "moe_router_filter_view": (ctypes.c_int, [_cfgp, ctypes.POINTER(ctypes.c_size_t),
+                                              ctypes.POINTER(ctypes.c_int32),
+                                              ctypes.POINTER(ctypes.c_size_t),
+                                              ctypes.POINTER(ctypes.c_float)]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_abi_version": (ctypes.c_int32, []),
 }
@@ -107,6 +130,45 @@ def _call(name, *args):
 
 def moe_check_wait_timeout(barrier, status, stream=None):
     _call("moe_check_wait_timeout", _p(barrier), _p(status), _s(stream))
+
+
+def moe_ep_send_counts(cfg, peers, rank0, nlocal, counts, epoch, stream=None):
+    _call("moe_ep_send_counts", ctypes.byref(cfg), ctypes.addressof(peers), rank0, nlocal, _p(counts),
+          epoch, _s(stream))
+
+
+def moe_ep_send_rows(cfg, peers, rank0, nlocal, x, topk_idx, pos, expert_offsets, epoch, done, status,
+                     stream=None):
+    _call("moe_ep_send_rows", ctypes.byref(cfg), ctypes.addressof(peers), rank0, nlocal, _p(x),
+          _p(topk_idx), _p(pos), _p(expert_offsets), epoch, _p(done), _p(status), _s(stream))
+
+
+def moe_ep_recv_layout(cfg, peers, rank0, nlocal, local_offsets, epoch, status, stream=None):
+    _call("moe_ep_recv_layout", ctypes.byref(cfg), ctypes.addressof(peers), rank0, nlocal,
+          _p(local_offsets), epoch, _p(status), _s(stream))
+
+
+def moe_ep_return_rows(cfg, peers, rank0, nlocal, y_recv, local_offsets, epoch, done, status, stream=None):
+    _call("moe_ep_return_rows", ctypes.byref(cfg), ctypes.addressof(peers), rank0, nlocal, _p(y_recv),
+          _p(local_offsets), epoch, _p(done), _p(status), _s(stream))
+
+
+def moe_ep_wait_returned(cfg, peers, rank0, nlocal, epoch, status, stream=None):
+    _call("moe_ep_wait_returned", ctypes.byref(cfg), ctypes.addressof(peers), rank0, nlocal, epoch,
+          _p(status), _s(stream))
+
+
+def moe_router_filter_view(cfg):
+    """(approx_offset, approx_ld, wmax_offset, coef) of the tensor-core router's values
+    in the workspace after moe_route, or None when cfg takes another router path."""
+    ao, ld, wo, cf = ctypes.c_size_t(), ctypes.c_int32(), ctypes.c_size_t(), ctypes.c_float()
+    st = lib().moe_router_filter_view(ctypes.byref(cfg), ctypes.byref(ao), ctypes.byref(ld),
+                                      ctypes.byref(wo), ctypes.byref(cf))
+    if st == MOE_ERR_UNSUPPORTED:
+        return None
+    if st != MOE_OK:
+        raise MoeError("moe_router_filter_view", st)
+    return ao.value, ld.value, wo.value, cf.value
 
 
 def moe_status_string(status: int) -> str:

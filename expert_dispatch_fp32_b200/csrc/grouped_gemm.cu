@@ -16,10 +16,10 @@
 // on one CTA and serves the narrower N tiles.  In both, the tile list is
 // expert-major, then N block, then M tile fastest, so the CTAs that run at the
 // same time share each weight tile through L2 and stream every weight from HBM
-// about once.  The per-expert M-tile prefix (mt_start) comes from the preprocess
-// stage on the device: the host never learns the counts, so grid = #SMs and each
-// CTA walks tiles blockIdx.x, blockIdx.x + gridDim.x, ...  Empty experts own no
-// tiles, so their weights are never read.
+// about once.  Each CTA derives the per-expert M-tile prefix from the group offsets
+// (a block scan at launch): the host never learns the counts, so the grid is sized
+// for the worst case and the CTAs take tiles from a device counter.  Empty experts
+// own no tiles, so their weights are never read.
 //
 // One-CTA kernel: one CTA per SM, 6 warps:
 //   warp 0      TMA producer: A tile [128 x 64] and B tile [BN x 64] per K step
@@ -52,8 +52,7 @@ constexpr int kCtrlBytes = 512;     // barriers, tile queue, TMEM slot, abort fl
 struct GemmArgs {
   CUtensorMap tmap_a;
   CUtensorMap tmap_b;
-  const int32_t* group_offsets;
-  const int32_t* mt_start;
+  const int32_t* group_offsets;   // the kernel derives the M tiles from these
   int32_t G, N, K, dense_rows;
   bf16* out;
   float* outf;               // EPI_PAIRSUM_F32 output
@@ -83,10 +82,10 @@ struct PhaseArgs {
 };
 struct PairArgs {
   PhaseArgs ph[kMaxPhases];
-  const int32_t* group_offsets;   // [G + 1] (grouped phases)
-  const int32_t* mt_start;        // [G + 1] prefix of ceil(rows / 256)
+  const int32_t* group_offsets;   // [G + 1] (grouped phases); the kernel derives the M tiles
   int32_t G, nph;
-  int32_t skinny;            // 1: remainders of <= 64 rows run as skinny (weights-as-M) tiles
+  int32_t skinny;            // 1: groups of <= 64 rows run as skinny (weights-as-M) tiles
+  int32_t fold;              // 1: a last band of 257..320 rows runs as one folded tile
   int32_t* status;
   int32_t* counter;          // tile counter, zero at launch
   int32_t* done;             // band completion counts, zero at launch
@@ -391,19 +390,22 @@ __device__ __forceinline__ void store_row32_f32(float* dst, const float (&v)[32]
   for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 }
 
-// Epilogue of one output row: this thread's `tcols` TMEM columns at `tb` hold
-// accumulator values of row `row` (`valid` false: read, store nothing).
+// Epilogue of one output row: this thread's TMEM columns at `tb` hold accumulator
+// values of row `row` (`valid` false: read, store nothing); output columns
+// col0 + [cb, ce) are done (a range, so a caller can release the TMEM columns read so
+// far before doing the rest).
 //   EPI_SWIGLU / EPI_PAIRSUM_F32: every 128 columns are [first 64 | second 64] of
 //     64 outputs (packed gate/up or router hi/mid groups); output column
-//     col0 + 64 * group + c = silu(first) * second, or first + second in fp32.
-//   EPI_STORE / EPI_GELU: output column col0 + c = value (or its GELU).
+//     col0 + 64 * group + c = silu(first) * second, or first + second in fp32
+//     (output columns [0, 64) read TMEM columns [0, 128)).
+//   EPI_STORE / EPI_GELU: output column col0 + c = value (or its GELU), TMEM column c.
 // tcgen05.ld is warp-collective, so every lane runs the loads.
 template <int EPI>
-__device__ __forceinline__ void epilogue_row(bf16* out, float* outf, int ldo, uint32_t tb, int tcols,
-                                             int64_t row, int col0, bool valid) {
+__device__ __forceinline__ void epilogue_row(bf16* out, float* outf, int ldo, uint32_t tb, int cb,
+                                             int ce, int64_t row, int col0, bool valid) {
   if (EPI == EPI_SWIGLU || EPI == EPI_PAIRSUM_F32) {
 #pragma unroll 1
-    for (int c = 0; c < tcols / 2; c += 32) {
+    for (int c = cb; c < ce; c += 32) {
       const int tc = (c >> 6) * 128 + (c & 63);
       uint32_t a[32], b[32];
       tmem_ld32(tb + tc, a);
@@ -422,7 +424,7 @@ __device__ __forceinline__ void epilogue_row(bf16* out, float* outf, int ldo, ui
     }
   } else {
 #pragma unroll 1
-    for (int c = 0; c < tcols; c += 32) {
+    for (int c = cb; c < ce; c += 32) {
       uint32_t h[32];
       tmem_ld32(tb + c, h);
       tmem_ld_wait();
@@ -439,12 +441,12 @@ __device__ __forceinline__ void epilogue_row(bf16* out, float* outf, int ldo, ui
 
 // Runtime choice of the epilogue (the phases of one launch differ).
 __device__ __forceinline__ void epilogue_row_rt(int epi, bf16* out, float* outf, int ldo, uint32_t tb,
-                                                int tcols, int64_t row, int col0, bool valid) {
+                                                int cb, int ce, int64_t row, int col0, bool valid) {
   switch (epi) {
-    case EPI_SWIGLU: epilogue_row<EPI_SWIGLU>(out, outf, ldo, tb, tcols, row, col0, valid); break;
-    case EPI_GELU: epilogue_row<EPI_GELU>(out, outf, ldo, tb, tcols, row, col0, valid); break;
-    case EPI_PAIRSUM_F32: epilogue_row<EPI_PAIRSUM_F32>(out, outf, ldo, tb, tcols, row, col0, valid); break;
-    default: epilogue_row<EPI_STORE>(out, outf, ldo, tb, tcols, row, col0, valid); break;
+    case EPI_SWIGLU: epilogue_row<EPI_SWIGLU>(out, outf, ldo, tb, cb, ce, row, col0, valid); break;
+    case EPI_GELU: epilogue_row<EPI_GELU>(out, outf, ldo, tb, cb, ce, row, col0, valid); break;
+    case EPI_PAIRSUM_F32: epilogue_row<EPI_PAIRSUM_F32>(out, outf, ldo, tb, cb, ce, row, col0, valid); break;
+    default: epilogue_row<EPI_STORE>(out, outf, ldo, tb, cb, ce, row, col0, valid); break;
   }
 }
 
@@ -461,6 +463,37 @@ struct GemmCfg {
   }
 };
 
+// Per-group M tiles and their prefix, from the group offsets in shared memory:
+// mt[g] = first tile of group g, mt[G] = all tiles.  Each thread sums a run of
+// consecutive groups, a block scan of the run totals gives each run's first tile.
+// Called by every thread of the block (it holds block barriers); wsum holds one int
+// per warp.
+template <class TilesFn>
+__device__ void group_tile_prefix(const int* off, int G, int* mt, int* wsum, TilesFn tiles) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int per = (G + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int g0 = min(G, (int)threadIdx.x * per), g1 = min(G, g0 + per);
+  int run = 0;
+  for (int g = g0; g < g1; ++g) run += tiles(off[g + 1] - off[g]);
+  int inc = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += v;
+  }
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();
+  int before = 0;
+  for (int w = 0; w < warp; ++w) before += wsum[w];
+  int pre = before + inc - run;
+  for (int g = g0; g < g1; ++g) {
+    mt[g] = pre;
+    pre += tiles(off[g + 1] - off[g]);
+  }
+  if (threadIdx.x == blockDim.x - 1) mt[G] = before + inc;
+  __syncthreads();
+}
+
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs p) {
   using C = GemmCfg<BN>;
@@ -475,6 +508,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
   volatile int* tq = reinterpret_cast<volatile int*>(bars + 2 * S + 4 + 2 * kTileQ);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(tq) + kTileQ);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* wsum = const_cast<int*>(abort_flag) + 1;                 // [kGemmThreads / 32]
   int* mt = reinterpret_cast<int*>(smem + S * C::kStageBytes + kCtrlBytes);
   const bool dense = p.group_offsets == nullptr;
   const int G = dense ? 1 : p.G;
@@ -509,10 +543,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       off[0] = 0; off[1] = p.dense_rows;
     }
   } else {
-    for (int i = threadIdx.x; i <= G; i += blockDim.x) {
-      mt[i] = p.mt_start[i];
-      off[i] = p.group_offsets[i];
-    }
+    for (int i = threadIdx.x; i <= G; i += blockDim.x) off[i] = p.group_offsets[i];
+    __syncthreads();
+    group_tile_prefix(off, G, mt, wsum, [](int rows) { return (rows + kTileM - 1) / kTileM; });
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -606,7 +639,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_kernel(const __g
       const bool valid = r < rows_valid;
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       const bool paired = EPI == EPI_SWIGLU || EPI == EPI_PAIRSUM_F32;
-      epilogue_row<EPI>(p.out, p.outf, p.ldo, tb, BN, (int64_t)row0 + r, paired ? n * (BN / 2) : n * BN, valid);
+      epilogue_row<EPI>(p.out, p.outf, p.ldo, tb, 0, paired ? BN / 2 : BN, (int64_t)row0 + r,
+                        paired ? n * (BN / 2) : n * BN, valid);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
@@ -654,7 +688,9 @@ struct PairCfg {
   static constexpr int kStages = 6;
   static constexpr int kABytes = kTileM * kTileK * 2;            // this CTA's A half
   static constexpr int kBBytes = (BN / 2) * kTileK * 2;          // this CTA's B half
-  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kRemRows = 32;                           // folded rows per CTA (box)
+  static constexpr int kRemBytes = kRemRows * kTileK * 2;        // this CTA's folded rows
+  static constexpr int kStageBytes = kABytes + kBBytes + kRemBytes;
   static constexpr int kTmemCols = 2 * BN;
   static constexpr uint32_t kIdesc = make_idesc(2 * kTileM, BN);
   static constexpr uint32_t kIdescHalf = make_idesc(kTileM, BN);
@@ -662,6 +698,8 @@ struct PairCfg {
     return 1024 + (size_t)kStages * kStageBytes + kCtrlBytes + 2 * (size_t)(G + 1) * sizeof(int);
   }
 };
+// Largest remainder folded into a single-band group's tile (rows beyond 256).
+constexpr int kFoldMax = PairCfg::kRemRows;
 
 // Where a pair tile sits: phase, group, M tile (256 rows), N block, its first row,
 // the group's end row, and its band slot (the M tile's index across the phase).
@@ -669,23 +707,46 @@ struct PairTile {
   int ph, g, m, n, base, end, band;
 };
 
-// Shape of a pair tile from the rows it has left: > 128 rows: M = 256 (128 rows per
-// CTA); 65..128 rows: M = 128 (64 rows per CTA).  A group of at most 64 rows in all
-// (a decode-sized batch) runs skinny when enabled: the weights take the M side
-// (M = 128: 64 weight rows per CTA, twice) and the rows the N side, N = rows
-// rounded up to 32 (N/2 rows per CTA; a multiple of 32 is a valid N for every
-// 2-CTA MMA shape), for 2N/256 of an M = 128 tile's MMA work.  The remainder band
-// of a larger group stays M = 128: as its own skinny tile it would race ahead of
-// the group's full tile that streams the same weights, and on deepseek_v3 that
-// cost 2.2 GB of extra HBM reads per layer (ncu: 26.6 vs 24.4 GB, 7.39 vs 7.25 ms).
-enum TileKind { TK_FULL = 0, TK_HALF = 1, TK_SKINNY = 2 };
-__device__ __forceinline__ int tile_kind(const PairTile& t, int skinny, int& ns) {
+// Shape of a pair tile from the rows it has left:
+//   > 128 rows: M = 256 (128 rows per CTA), TK_FULL;
+//   65..128 rows: M = 128 (64 rows per CTA), TK_HALF;
+//   a group of at most 64 rows in all (a decode-sized batch), when enabled: TK_SKINNY,
+//     the weights on the M side (M = 128: 64 weight rows per CTA, twice) and the rows
+//     on the N side, N = rows rounded up to 32 (N/2 rows per CTA; a multiple of 32 is
+//     a valid N for every 2-CTA MMA shape), for 2N/256 of an M = 128 tile's MMA work;
+//   with folding enabled, a group of 257..320 rows in all: TK_FOLD, the M = 256 tile
+//     of the first 256 rows plus, on every K step and from the same weight slab in
+//     shared memory, the skinny product of the remainder rows.  The remainder then
+//     costs two small MMAs per K step instead of a second tile that streams the whole
+//     weight panel again for a few rows (on deepseek_v3's routing, 256 +- 18 rows per
+//     expert, half the experts have one).  Measured on 256 experts of 272 rows each
+//     (deepseek_v3 shapes): the folded tile costs 1.46 full tiles, a full tile plus an
+//     M = 128 tile 1.51; with 320 rows (N = 64) folding was slower (1.61 vs 1.51), as it
+//     was for the last band of larger groups (small_e8_d2048, 1035..1096 rows: 0.503 vs
+//     0.475 ms), where the folded tile falls behind the group's other tiles that share
+//     its weight tiles through L2.  So only single-band groups with a remainder of at
+//     most 32 rows fold.
+// ns: the skinny (or folded) product's N, the row count rounded up to 32.
+enum TileKind { TK_FULL = 0, TK_HALF = 1, TK_SKINNY = 2, TK_FOLD = 3 };
+__device__ __forceinline__ int tile_kind(const PairTile& t, int skinny, int fold, int& ns) {
   const int left = t.end - t.base;
   ns = 0;
+  if (fold && t.m == 0 && left > 2 * kTileM && left <= 2 * kTileM + kFoldMax) {
+    ns = (left - 2 * kTileM + 31) & ~31;
+    return TK_FOLD;
+  }
   if (left > kTileM) return TK_FULL;
   if (!skinny || left > kTileM / 2 || t.m != 0) return TK_HALF;
   ns = (left + 31) & ~31;
   return TK_SKINNY;
+}
+
+// M tiles of a group of `rows` rows: 256 rows each; with folding, a group of 257..
+// 256 + kFoldMax rows is one tile.
+__device__ __forceinline__ int pair_mtiles(int rows, int fold) {
+  if (rows <= 0) return 0;
+  if (fold && rows > 2 * kTileM && rows <= 2 * kTileM + kFoldMax) return 1;
+  return (rows + 2 * kTileM - 1) / (2 * kTileM);
 }
 
 __device__ __forceinline__ void decode_pair_tile(int tile, const int* pstart, int nph, const int* mt,
@@ -704,18 +765,21 @@ __device__ __forceinline__ void decode_pair_tile(int tile, const int* pstart, in
   t.band = pm[t.g] + t.m;
 }
 
-// Epilogue of a skinny tile.  The accumulators hold weights-rows x tile-rows: in
-// CTA r, TMEM lane i (i < 64) has weight row i of the CTA's slab for tile rows
-// [0, ns/2), lane 64 + i the same weight row for tile rows [ns/2, ns), at columns
-// 0.. (first 64 slab rows) and 128.. (second 64).  Warp q reads lanes 32q..32q+31.
+// Epilogue of a skinny product (a skinny tile, or the remainder of a folded one).  The
+// accumulators hold weights-rows x tile-rows: in CTA r, TMEM lane i (i < 64) has
+// weight row i of the CTA's slab for tile rows [0, ns/2), lane 64 + i the same weight
+// row for tile rows [ns/2, ns), at columns tb.. (first 64 slab rows) and tb + 32..
+// (second 64).  Warp q reads lanes 32q..32q+31.  The tile rows start at row `rbase`.
 // The slab's rows are, per 256-wide N block n: SwiGLU / router pairs: the first and
 // second factor of outputs n*128 + 64r + i; plain outputs: columns n*256 + 128r + i
 // and + 64.  One output element per store (a warp writes 32 consecutive columns).
+constexpr int kSkinnyHi = 32;     // TMEM column offset of the second 64 slab rows' product
 __device__ __forceinline__ void epilogue_skinny(int epi, bf16* out, float* outf, int ldo, uint32_t tb,
-                                                const PairTile& t, int rank, int q, int lane, int ns) {
+                                                const PairTile& t, int rbase, int rank, int q,
+                                                int lane, int ns) {
   uint32_t r0[32], r1[32];
   tmem_ld32(tb, r0);
-  tmem_ld32(tb + 128, r1);
+  tmem_ld32(tb + kSkinnyHi, r1);
   tmem_ld_wait();
   const int i = (q & 1) * 32 + lane;
   const int nh = ns >> 1;
@@ -725,7 +789,7 @@ __device__ __forceinline__ void epilogue_skinny(int epi, bf16* out, float* outf,
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
     if (c >= nh) break;
-    const int64_t row = (int64_t)t.base + j0 + c;
+    const int64_t row = (int64_t)rbase + j0 + c;
     if (row >= t.end) break;
     const float a = __uint_as_float(r0[c]), b = __uint_as_float(r1[c]);
     if (epi == EPI_SWIGLU) {
@@ -760,25 +824,36 @@ __device__ __noinline__ bool wait_count(const int32_t* cnt, int need, volatile i
   }
 }
 
+// TMEM of a pair CTA: two 256-column accumulators (buffers 0 and 1), each tracked as
+// two regions: its head (columns 0..63) and its tail (64..255).  A tile with its main
+// accumulator in buffer b occupies b's head and (unless skinny: its products fit in the
+// head) b's tail; a folded tile also puts its remainder product in the OTHER buffer's
+// head.  The MMA issuer waits, per region, until the region's previous occupant has
+// been read out; the epilogue releases each region as soon as it has read it, a
+// folded tile's remainder first and a main accumulator's head before its tail, so a
+// folded tile waits only for the first part of the previous tile's epilogue.
+// Barrier index of a region: head of b = b, tail of b = 2 + b.
 __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(const __grid_constant__ PairArgs p) {
   // launched as a programmatic dependent of the previous kernel on the stream: wait until
   // that kernel has completed and its writes are visible (a no-op otherwise)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   using C = PairCfg;
-  constexpr int S = C::kStages, BN = C::BN, TM2 = 2 * kTileM;
+  constexpr int S = C::kStages, BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* a_smem = smem;
   uint8_t* b_smem = smem + S * C::kABytes;
+  uint8_t* r_smem = smem + S * (C::kABytes + C::kBBytes);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
-  // bars: full[S], empty[S], tmem_full[2], tmem_empty[2], qfull[Q], qempty[Q]
-  volatile int* tq = reinterpret_cast<volatile int*>(bars + 2 * S + 4 + 2 * kTileQ);
+  // bars: full[S], empty[S], tmem_full[2], tmem_free[4], qfull[Q], qempty[Q]
+  volatile int* tq = reinterpret_cast<volatile int*>(bars + 2 * S + 6 + 2 * kTileQ);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(tq) + kTileQ);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* pstart = reinterpret_cast<int*>(tmem_slot + 2);          // [kMaxPhases + 1]
   int* dmt = pstart + kMaxPhases + 1;                           // [kMaxPhases][2]
   int* doff = dmt + 2 * kMaxPhases;                             // [kMaxPhases][2]
+  int* wsum = doff + 2 * kMaxPhases;                            // [kGemmThreads / 32]
   int* mt = reinterpret_cast<int*>(smem + S * C::kStageBytes + kCtrlBytes);
   const int G = p.G > 0 ? p.G : 1;
   int* off = mt + (G + 1);
@@ -788,18 +863,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
-  const uint32_t tfull0 = smem_u32(bars + 2 * S), tempty0 = smem_u32(bars + 2 * S + 2);
-  const uint32_t qfull0 = smem_u32(bars + 2 * S + 4), qempty0 = smem_u32(bars + 2 * S + 4 + kTileQ);
+  const uint32_t tfull0 = smem_u32(bars + 2 * S), tfree0 = smem_u32(bars + 2 * S + 2);
+  const uint32_t qfull0 = smem_u32(bars + 2 * S + 6), qempty0 = smem_u32(bars + 2 * S + 6 + kTileQ);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(full0 + 8 * i, 1);
       mbar_init(empty0 + 8 * i, 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(tfull0 + 8 * i, 1);
-      mbar_init(tempty0 + 8 * i, 8);
-    }
+    for (int i = 0; i < 2; ++i) mbar_init(tfull0 + 8 * i, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(tfree0 + 8 * i, 8);     // 4 epilogue warps x 2 CTAs
     for (int i = 0; i < kTileQ; ++i) {
       mbar_init(qfull0 + 8 * i, 1);
       // leader: MMA issuer + 4 epilogue warps; peer: producer + 4 epilogue warps
@@ -813,15 +886,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
       prefetch_tmap(&p.ph[ph].tmap_a32);
       prefetch_tmap(&p.ph[ph].tmap_b);
       const int rows = p.ph[ph].dense_rows;
-      dmt[2 * ph] = 0; dmt[2 * ph + 1] = (rows + TM2 - 1) / TM2;
+      dmt[2 * ph] = 0; dmt[2 * ph + 1] = pair_mtiles(rows, p.fold);
       doff[2 * ph] = 0; doff[2 * ph + 1] = rows;
     }
   }
   if (p.group_offsets != nullptr) {
-    for (int i = threadIdx.x; i <= G; i += blockDim.x) {
-      mt[i] = p.mt_start[i];
-      off[i] = p.group_offsets[i];
-    }
+    for (int i = threadIdx.x; i <= G; i += blockDim.x) off[i] = p.group_offsets[i];
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -831,6 +901,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   __syncthreads();
+  if (p.group_offsets != nullptr) {
+    const int fold = p.fold;
+    group_tile_prefix(off, G, mt, wsum, [fold](int rows) { return pair_mtiles(rows, fold); });
+  }
   if (threadIdx.x == 0) {          // tile numbering: phase after phase
     int acc_t = 0;
     for (int ph = 0; ph < nph; ++ph) {
@@ -868,12 +942,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         decode_pair_tile(tile, pstart, nph, mt, off, G, dmt, doff, p, t);
         const PhaseArgs& P = p.ph[t.ph];
         int ns;
-        const int kind = tile_kind(t, p.skinny, ns);
+        const int kind = tile_kind(t, p.skinny, p.fold, ns);
+        const bool m256 = kind == TK_FULL || kind == TK_FOLD;
         // rows of A this CTA loads: 128 (full), its 64 (half), or its ns/2 of a 32-row box
-        const int arow = t.base + (int)rank * (kind == TK_FULL ? kTileM : kind == TK_HALF ? kTileM / 2 : ns / 2);
-        const CUtensorMap* amap = kind == TK_FULL ? &P.tmap_a : kind == TK_HALF ? &P.tmap_a64 : &P.tmap_a32;
-        const int abytes = kind == TK_FULL ? C::kABytes : kind == TK_HALF ? C::kABytes / 2 : C::kABytes / 4;
-        const uint32_t stage_tx = 2u * (uint32_t)(abytes + C::kBBytes);
+        const int arow = t.base + (int)rank * (m256 ? kTileM : kind == TK_HALF ? kTileM / 2 : ns / 2);
+        const CUtensorMap* amap = m256 ? &P.tmap_a : kind == TK_HALF ? &P.tmap_a64 : &P.tmap_a32;
+        const int abytes = m256 ? C::kABytes : kind == TK_HALF ? C::kABytes / 2 : C::kABytes / 4;
+        // a folded tile also loads its remainder rows: this CTA's ns/2 of a 32-row box
+        const bool fold = kind == TK_FOLD;
+        const int rrow = t.base + 2 * kTileM + (int)rank * (ns / 2);
+        const uint32_t stage_tx = 2u * (uint32_t)(abytes + C::kBBytes + (fold ? C::kRemBytes : 0));
         const int brow = t.n * BN + (int)rank * (BN / 2);
         if (P.dep >= 0) {
           // A rows of this band are written by phase P.dep: wait until all of its
@@ -892,6 +970,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
           tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), amap, fb, kb * kTileK, arow);
           tma_load_3d_pair(smem_u32(b_smem + stage * C::kBBytes), &P.tmap_b, fb, kb * kTileK, brow,
                            P.dense_rows > 0 ? 0 : t.g);
+          if (fold)
+            tma_load_2d_pair(smem_u32(r_smem + stage * C::kRemBytes), &P.tmap_a32, fb, kb * kTileK, rrow);
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -903,39 +983,59 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
-      uint32_t acc_phase = 0;
+      uint32_t freeph = 0;       // bit i: parity of the next wait on TMEM region i
       for (int qi = 0;; ++qi) {
         const int tile = tq_take<false>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
         if (tile < 0) break;
         PairTile t;
         decode_pair_tile(tile, pstart, nph, mt, off, G, dmt, doff, p, t);
         int ns;
-        const int kind = tile_kind(t, p.skinny, ns);
-        const uint32_t idesc = kind == TK_FULL ? C::kIdesc : kind == TK_HALF ? C::kIdescHalf
-                                                                             : make_idesc(kTileM, ns);
+        const int kind = tile_kind(t, p.skinny, p.fold, ns);
+        const uint32_t idesc = kind == TK_FULL || kind == TK_FOLD ? C::kIdesc
+                               : kind == TK_HALF ? C::kIdescHalf : make_idesc(kTileM, ns);
+        const uint32_t idesc_s = make_idesc(kTileM, ns);        // skinny / folded remainder
         const int ksteps = p.ph[t.ph].K / kTileK;
-        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.status)) break;
+        // the TMEM regions this tile writes: this buffer's head, its tail unless skinny,
+        // the other buffer's head if folded
+        const uint32_t need = (1u << acc) | (kind != TK_SKINNY ? 4u << acc : 0u) |
+                              (kind == TK_FOLD ? 1u << (acc ^ 1) : 0u);
+        bool ok = true;
+        for (int i = 0; i < 4 && ok; ++i) {
+          if (!((need >> i) & 1u)) continue;
+          ok = mbar_wait(tfree0 + 8 * i, ((freeph >> i) & 1u) ^ 1u, abort_flag, p.status);
+          freeph ^= 1u << i;
+        }
+        if (!ok) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        bool ok = true;
+        // skinny products (and a folded remainder, in the other buffer's head): the
+        // first 64 weight rows into columns [0, ns/2), the second 64 into [32, 32 + ns/2)
+        const uint32_t s_tmem = kind == TK_FOLD ? tmem_base + (uint32_t)((acc ^ 1) * BN) : d_tmem;
         for (int kb = 0; kb < ksteps; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ad = sw128_desc(smem_u32(a_smem + stage * C::kABytes));
           const uint64_t bd = sw128_desc(smem_u32(b_smem + stage * C::kBBytes));
-          if (kind != TK_SKINNY) {
+          const uint64_t bd_hi = sw128_desc(smem_u32(b_smem + stage * C::kBBytes + C::kBBytes / 2));
+          if (kind == TK_SKINNY) {
+            // weights as the M operand (each CTA's B slab as two 64-row halves), rows as N
+#pragma unroll
+            for (int kk = 0; kk < kTileK / 16; ++kk) {
+              tc_mma_pair(s_tmem, bd + 2 * kk, ad + 2 * kk, idesc_s, (kb | kk) != 0);
+              tc_mma_pair(s_tmem + kSkinnyHi, bd_hi + 2 * kk, ad + 2 * kk, idesc_s, (kb | kk) != 0);
+            }
+          } else if (kind == TK_FOLD) {
+            const uint64_t rd = sw128_desc(smem_u32(r_smem + stage * C::kRemBytes));
+#pragma unroll
+            for (int kk = 0; kk < kTileK / 16; ++kk) {
+              tc_mma_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+              tc_mma_pair(s_tmem, bd + 2 * kk, rd + 2 * kk, idesc_s, (kb | kk) != 0);
+              tc_mma_pair(s_tmem + kSkinnyHi, bd_hi + 2 * kk, rd + 2 * kk, idesc_s, (kb | kk) != 0);
+            }
+          } else {
 #pragma unroll
             for (int kk = 0; kk < kTileK / 16; ++kk)
               tc_mma_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
-          } else {
-            // weights as the M operand: rows 0..63 of each CTA's B slab into columns
-            // [0, ns/2), rows 64..127 into columns [128, 128 + ns/2); the rows as N
-            const uint64_t bd_hi = sw128_desc(smem_u32(b_smem + stage * C::kBBytes + C::kBBytes / 2));
-#pragma unroll
-            for (int kk = 0; kk < kTileK / 16; ++kk) {
-              tc_mma_pair(d_tmem, bd + 2 * kk, ad + 2 * kk, idesc, (kb | kk) != 0);
-              tc_mma_pair(d_tmem + 128, bd_hi + 2 * kk, ad + 2 * kk, idesc, (kb | kk) != 0);
-            }
           }
           tc_commit_pair_both(empty0 + 8 * stage);
           if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -943,15 +1043,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         if (!ok) break;
         tc_commit_pair_both(tfull0 + 8 * acc);
         acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
       }
     }
   } else {
     // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
     const int q = warp & 3;
-    const uint32_t tempty_leader = map_to_cta(tempty0, 0);
+    const uint32_t tfree_leader = map_to_cta(tfree0, 0);
     int acc = 0;
     uint32_t acc_phase = 0;
+    // release TMEM region i: this warp has read all of its columns
+    auto release = [&](int i) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tfree_leader + 8 * i);
+    };
     for (int qi = 0;; ++qi) {
       const int tile = tq_take<true>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
       if (__any_sync(0xffffffffu, tile < 0)) break;
@@ -959,31 +1064,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
       decode_pair_tile(tile, pstart, nph, mt, off, G, dmt, doff, p, t);
       const PhaseArgs& P = p.ph[t.ph];
       int ns;
-      const int kind = tile_kind(t, p.skinny, ns);
+      const int kind = tile_kind(t, p.skinny, p.fold, ns);
       bool ok = true;
       if (lane == 0) ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const bool paired = P.epi == EPI_SWIGLU || P.epi == EPI_PAIRSUM_F32;
-      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      const uint32_t lanes = (uint32_t)(q * 32) << 16;
+      const uint32_t tb = tmem_base + lanes + (uint32_t)(acc * BN);
+      if (kind == TK_FOLD) {
+        // the remainder rows (after the first 256), from the other buffer's head
+        epilogue_skinny(P.epi, P.out, P.outf, P.ldo, tmem_base + lanes + (uint32_t)((acc ^ 1) * BN), t,
+                        t.base + 2 * kTileM, (int)rank, q, lane, ns);
+        release(acc ^ 1);
+      }
       if (kind == TK_SKINNY) {
-        epilogue_skinny(P.epi, P.out, P.outf, P.ldo, tb, t, (int)rank, q, lane, ns);
-      } else if (kind == TK_FULL) {
-        // M = 256: this CTA's 128 rows in TMEM lanes 0..127, all 256 columns
+        epilogue_skinny(P.epi, P.out, P.outf, P.ldo, tb, t, t.base, (int)rank, q, lane, ns);
+        release(acc);
+      } else if (kind != TK_HALF) {
+        // M = 256: this CTA's 128 rows in TMEM lanes 0..127, all 256 columns; output
+        // columns [0, 64) read the head (and, paired, columns 64..127)
         const int row0 = t.base + (int)rank * kTileM;
         const int r = q * 32 + lane;
-        epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, BN, (int64_t)row0 + r,
-                        paired ? t.n * (BN / 2) : t.n * BN, r < t.end - row0);
+        const int col0 = paired ? t.n * (BN / 2) : t.n * BN;
+        const bool valid = r < min(t.end - row0, kTileM);
+        epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, 0, 64, (int64_t)row0 + r, col0, valid);
+        release(acc);
+        epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, 64, paired ? BN / 2 : BN, (int64_t)row0 + r,
+                        col0, valid);
+        release(2 + acc);
       } else {
         // M = 128: this CTA's 64 rows; lanes 0..63 hold tile columns [0, 128) and
         // lanes 64..127 columns [128, 256), each in TMEM columns 0..127
         const int row0 = t.base + (int)rank * (kTileM / 2);
         const int r = (q & 1) * 32 + lane, ch = q >> 1;
-        epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, BN / 2, (int64_t)row0 + r,
-                        paired ? t.n * (BN / 2) + ch * (BN / 4) : t.n * BN + ch * (BN / 2),
-                        r < t.end - row0);
+        const int col0 = paired ? t.n * (BN / 2) + ch * (BN / 4) : t.n * BN + ch * (BN / 2);
+        const bool valid = r < t.end - row0;
+        epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, 0, paired ? BN / 4 : 64, (int64_t)row0 + r,
+                        col0, valid);
+        release(acc);
+        if (!paired)
+          epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, 64, BN / 2, (int64_t)row0 + r, col0, valid);
+        release(2 + acc);
       }
-      tc_fence_before();
       if (P.signal) {
         // count this warp's stores of the band for the phase that reads them back
         asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -992,7 +1115,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         if (lane == 0) atomicAdd(p.done + P.done_base + t.band, 1);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty_leader + 8 * acc);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -1129,9 +1251,12 @@ cudaError_t launch_grouped_pair(const GemmProblem* probs, int n, int32_t* counte
   memset(&a, 0, sizeof(a));
   a.nph = n;
   {
-    // MOE_GEMM_SKINNY=0 runs groups of <= 64 rows as M = 128 tiles too
+    // MOE_GEMM_SKINNY=0 runs groups of <= 64 rows as M = 128 tiles too; MOE_GEMM_FOLD=0
+    // runs a group's remainder of <= 64 rows past a full band as its own M = 128 tile
     const char* env = getenv("MOE_GEMM_SKINNY");
     a.skinny = (env && env[0] == '0') ? 0 : 1;
+    env = getenv("MOE_GEMM_FOLD");
+    a.fold = (env && env[0] == '0') ? 0 : 1;
   }
   a.status = probs[0].status;
   a.counter = counter;
@@ -1152,7 +1277,6 @@ cudaError_t launch_grouped_pair(const GemmProblem* probs, int n, int32_t* counte
       if (a.group_offsets != nullptr && (a.group_offsets != p.group_offsets || a.G != p.G))
         return cudaErrorInvalidValue;          // grouped phases share one grouping
       a.group_offsets = p.group_offsets;
-      a.mt_start = p.mt_start;
       a.G = p.G;
       P.dense_rows = 0;
     } else {
@@ -1199,7 +1323,6 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
   if (!make_map_3d(&a.tmap_b, p.B, (uint64_t)p.K, (uint64_t)p.N, (uint64_t)p.G, b_box))
     return cudaErrorInvalidValue;
   a.group_offsets = p.group_offsets;
-  a.mt_start = p.mt_start;
   a.G = p.G;
   a.N = p.N;
   a.K = p.K;

@@ -23,7 +23,6 @@ WsLayout ws_layout(const moe_config& c) {
   L.logits = o;       o = align256(o + T * E * sizeof(float));
   L.block_counts = o; o = align256(o + (size_t)L.nblk * E * sizeof(int32_t));
   L.barrier = o;      o = align256(o + 2 * sizeof(uint32_t));
-  L.mt_start = o;     o = align256(o + 2 * (E + 1) * sizeof(int32_t));
   L.act_shared = o;   o = align256(o + T * (size_t)c.n_shared * c.F_shared * sizeof(bf16));
   const size_t Epad = (E + 127) / 128 * 128;
   L.r_split = o;      o = align256(o + 2 * Epad * (size_t)c.D * sizeof(bf16));
@@ -112,7 +111,7 @@ moe_status route_dispatch_run(const moe_config* cfg, const void* x, const float*
   uint8_t* ws = (uint8_t*)workspace;
   const cudaError_t err = launch_route_pre_dispatch(
       c, x, w_router, expert_bias, logits_out, topk_idx, topk_w, counts, expert_offsets, rank_splits,
-      rank_offsets, pos, src, (int32_t*)(ws + L.block_counts), L.nblk, (int32_t*)(ws + L.mt_start),
+      rank_offsets, pos, src, (int32_t*)(ws + L.block_counts), L.nblk,
       barrier_zeroed != nullptr ? barrier_zeroed : (unsigned*)(ws + L.barrier), barrier_zeroed != nullptr,
       (bf16*)x_perm, status, as_stream(stream));
   if (err == cudaErrorCooperativeLaunchTooLarge) {
@@ -237,7 +236,7 @@ moe_status moe_preprocess(const moe_config* cfg, const int32_t* topk_idx, int32_
   uint8_t* ws = (uint8_t*)workspace;
   return cuda_status(launch_preprocess(c, topk_idx, counts, expert_offsets, rank_splits,
                                        rank_offsets, pos, src, (int32_t*)(ws + L.block_counts),
-                                       L.nblk, (int32_t*)(ws + L.mt_start),
+                                       L.nblk,
                                        (unsigned*)(ws + L.barrier), status, as_stream(stream)));
 }
 
@@ -290,8 +289,6 @@ moe_status ffn_run(const moe_config* cfg, const void* x_perm, const void* x,
   const PackLayout P = pack_layout(c);
   const uint8_t* pk = (const uint8_t*)packed;
   uint8_t* ws = (uint8_t*)workspace;
-  const int32_t* mt128 = (const int32_t*)(ws + W.mt_start);
-  const int32_t* mt256 = mt128 + (c.E + 1);
   const int64_t R = (int64_t)c.T * c.top_k;
   const int nup = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
   int32_t* ctr = (int32_t*)(ws + W.counters);
@@ -305,7 +302,6 @@ moe_status ffn_run(const moe_config* cfg, const void* x_perm, const void* x,
   up.group_offsets = expert_offsets;
   up.tile_n = up_tile_n(c);
   up.pair = use_pair && up.tile_n == 256;
-  up.mt_start = up.pair ? mt256 : mt128;
   up.max_tiles = (R / (up.pair ? 2 * kTileM : kTileM) + c.E) * (int64_t)(nup / up.tile_n);
   up.out = (bf16*)act; up.ldo = c.F;
   up.epi = c.act == MOE_ACT_SWIGLU ? EPI_SWIGLU : EPI_GELU;
@@ -319,7 +315,6 @@ moe_status ffn_run(const moe_config* cfg, const void* x_perm, const void* x,
   dn.N = c.D; dn.K = c.F;
   dn.tile_n = down_tile_n(c);
   dn.pair = use_pair && dn.tile_n == 256;
-  dn.mt_start = dn.pair ? mt256 : mt128;
   dn.max_tiles = (R / (dn.pair ? 2 * kTileM : kTileM) + c.E) * (int64_t)(c.D / dn.tile_n);
   dn.out = (bf16*)y_perm; dn.ldo = c.D;
   dn.epi = EPI_STORE;
@@ -335,7 +330,7 @@ moe_status ffn_run(const moe_config* cfg, const void* x_perm, const void* x,
     su.A = (const bf16*)x; su.a_rows = c.T;
     su.B = (const bf16*)(pk + P.ws_up); su.G = 1;
     su.N = 2 * Fc; su.K = c.D;
-    su.group_offsets = nullptr; su.mt_start = nullptr; su.dense_rows = c.T;
+    su.group_offsets = nullptr; su.dense_rows = c.T;
     su.tile_n = 256;
     su.pair = use_pair;
     const int tm_s = su.pair ? 2 * kTileM : kTileM;
@@ -514,10 +509,100 @@ moe_status moe_gather_rows(const void* src, const int32_t* index, void* dst, int
                                         as_stream(stream)));
 }
 
+// Host checks shared by the peer-exchange calls: a valid config, a peers table whose
+// P is the config's ep_size, and a covered rank range inside [0, P).
+static moe_status ep_check(const moe_config* cfg, const moe_ep_peers* peers, int32_t rank0,
+                           int32_t nlocal) {
+  moe_status st = moe_validate_config(cfg);
+  if (st != MOE_OK) return st;
+  if (peers == nullptr || peers->P != cfg->ep_size || peers->P < 1 || peers->cap < 0) return MOE_ERR_INVALID_ARG;
+  if (peers->cnt == nullptr || peers->flags == nullptr || peers->recv_x == nullptr ||
+      peers->recv_src == nullptr || peers->recv_rank == nullptr || peers->y_back == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (nlocal < 1 || rank0 < 0 || rank0 + nlocal > peers->P) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+moe_status moe_ep_send_counts(const moe_config* cfg, const moe_ep_peers* peers, int32_t rank0,
+                              int32_t nlocal, const int32_t* counts, uint32_t epoch, void* stream) {
+  moe_status st = ep_check(cfg, peers, rank0, nlocal);
+  if (st != MOE_OK) return st;
+  MOE_CHECK_PTR(counts);
+  return cuda_status(launch_ep_send_counts(*peers, rank0, nlocal, counts, cfg->E, epoch, as_stream(stream)));
+}
+
+moe_status moe_ep_send_rows(const moe_config* cfg, const moe_ep_peers* peers, int32_t rank0,
+                            int32_t nlocal, const void* x, const int32_t* topk_idx, const int32_t* pos,
+                            const int32_t* expert_offsets, uint32_t epoch, int32_t* done,
+                            int32_t* status, void* stream) {
+  moe_status st = ep_check(cfg, peers, rank0, nlocal);
+  if (st != MOE_OK) return st;
+  MOE_CHECK_PTR(expert_offsets);
+  MOE_CHECK_PTR(done);
+  MOE_CHECK_PTR(status);
+  if (cfg->T > 0) {
+    MOE_CHECK_PTR(x);
+    MOE_CHECK_PTR(topk_idx);
+    MOE_CHECK_PTR(pos);
+  }
+  return cuda_status(launch_ep_send_rows(*cfg, *peers, rank0, nlocal, x, topk_idx, pos, expert_offsets,
+                                         done, status, epoch, as_stream(stream)));
+}
+
+moe_status moe_ep_recv_layout(const moe_config* cfg, const moe_ep_peers* peers, int32_t rank0,
+                              int32_t nlocal, int32_t* local_offsets, uint32_t epoch, int32_t* status,
+                              void* stream) {
+  moe_status st = ep_check(cfg, peers, rank0, nlocal);
+  if (st != MOE_OK) return st;
+  MOE_CHECK_PTR(local_offsets);
+  MOE_CHECK_PTR(status);
+  return cuda_status(launch_ep_recv_layout(*cfg, *peers, rank0, nlocal, local_offsets, status, epoch,
+                                           as_stream(stream)));
+}
+
+moe_status moe_ep_return_rows(const moe_config* cfg, const moe_ep_peers* peers, int32_t rank0,
+                              int32_t nlocal, const void* y_recv, const int32_t* local_offsets,
+                              uint32_t epoch, int32_t* done, int32_t* status, void* stream) {
+  moe_status st = ep_check(cfg, peers, rank0, nlocal);
+  if (st != MOE_OK) return st;
+  MOE_CHECK_PTR(local_offsets);
+  MOE_CHECK_PTR(done);
+  MOE_CHECK_PTR(status);
+  if (peers->cap > 0) MOE_CHECK_PTR(y_recv);
+  return cuda_status(launch_ep_return_rows(*cfg, *peers, rank0, nlocal, y_recv, local_offsets, done,
+                                           epoch, as_stream(stream)));
+}
+
+moe_status moe_ep_wait_returned(const moe_config* cfg, const moe_ep_peers* peers, int32_t rank0,
+                                int32_t nlocal, uint32_t epoch, int32_t* status, void* stream) {
+  moe_status st = ep_check(cfg, peers, rank0, nlocal);
+  if (st != MOE_OK) return st;
+  MOE_CHECK_PTR(status);
+  return cuda_status(launch_ep_wait_returned(*peers, rank0, nlocal, status, epoch, as_stream(stream)));
+}
+
 moe_status moe_check_wait_timeout(uint32_t* barrier, int32_t* status, void* stream) {
   MOE_CHECK_PTR(barrier);
   MOE_CHECK_PTR(status);
   return cuda_status(launch_barrier_timeout_check(barrier, status, as_stream(stream)));
+}
+
+moe_status moe_router_filter_view(const moe_config* cfg, size_t* approx_offset, int32_t* approx_ld,
+                                  size_t* wmax_offset, float* coef) {
+  moe_status st = moe_validate_config(cfg);
+  if (st != MOE_OK) return st;
+  MOE_CHECK_PTR(approx_offset);
+  MOE_CHECK_PTR(approx_ld);
+  MOE_CHECK_PTR(wmax_offset);
+  MOE_CHECK_PTR(coef);
+  const moe_config& c = *cfg;
+  const WsLayout L = ws_layout(c);
+  if (!route_takes_filter(c, L.r_wmax - L.r_split, false)) return MOE_ERR_UNSUPPORTED;
+  *approx_offset = L.r_approx;
+  *approx_ld = (c.E + 127) / 128 * 128;
+  *wmax_offset = L.r_wmax;
+  *coef = route_filter_coef(c.D);
+  return MOE_OK;
 }
 
 const char* moe_status_string(moe_status s) {

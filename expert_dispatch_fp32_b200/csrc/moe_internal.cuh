@@ -29,7 +29,6 @@ struct WsLayout {
   size_t logits;        // fp32 [T, E]
   size_t block_counts;  // int32 [nblk, E]: preprocess per-block histograms
   size_t barrier;       // uint32 [2]: preprocess grid barrier (zeroed per call)
-  size_t mt_start;      // int32 [2][E + 1]: prefixes of ceil(count/128), ceil(count/256)
   size_t act_shared;    // bf16 [T, S*Fs]
   size_t r_split;       // bf16 [2*Epad, D]: tensor-core router weights
   size_t r_wmax;        // fp32 [D]
@@ -72,6 +71,10 @@ struct RouterScratch {
   double* part;     // fp64 slice totals of a split logits launch (aliases bsplit), or null
   size_t part_bytes;
 };
+// Whether moe_route (bf16 x) takes the tensor-core filter + exact refine for this
+// configuration, and the filter's per-unit error coefficient (eps_t = coef * S_t).
+bool route_takes_filter(const moe_config& c, size_t part_bytes, bool keep_logits);
+float route_filter_coef(int D);
 // logits: where the tiled path stores fp32 logits (caller's buffer or workspace);
 // keep_logits: the caller asked for them (the fused few-expert path then writes them).
 cudaError_t launch_route(const moe_config& c, const void* x, const float* w_router,
@@ -83,13 +86,28 @@ int preprocess_blocks(int64_t R);
 cudaError_t launch_preprocess(const moe_config& c, const int32_t* topk_idx, int32_t* counts,
                               int32_t* expert_offsets, int32_t* rank_splits,
                               int32_t* rank_offsets, int32_t* pos, int32_t* src,
-                              int32_t* block_counts, int max_blocks, int32_t* mt_start,
+                              int32_t* block_counts, int max_blocks,
                               unsigned* barrier, int32_t* status, cudaStream_t s);
 // Self-check of the bounded grid-barrier wait (preprocess.cu): one block, barrier for two.
 cudaError_t launch_barrier_timeout_check(unsigned* barrier, int32_t* status, cudaStream_t s);
 // Multi-rank helpers (ep.cu).
 cudaError_t launch_local_ids(const int32_t* topk_idx, const int32_t* src, int32_t* ids, int R, int El,
                              cudaStream_t s);
+// Peer-memory exchange (ep_peer.cu).
+cudaError_t launch_ep_send_counts(const moe_ep_peers& p, int rank0, int nlocal, const int32_t* counts,
+                                  int E, uint32_t epoch, cudaStream_t s);
+cudaError_t launch_ep_send_rows(const moe_config& c, const moe_ep_peers& p, int rank0, int nlocal,
+                                const void* x, const int32_t* topk_idx, const int32_t* pos,
+                                const int32_t* expert_offsets, int32_t* done, int32_t* status,
+                                uint32_t epoch, cudaStream_t s);
+cudaError_t launch_ep_recv_layout(const moe_config& c, const moe_ep_peers& p, int rank0, int nlocal,
+                                  int32_t* local_offsets, int32_t* status, uint32_t epoch,
+                                  cudaStream_t s);
+cudaError_t launch_ep_return_rows(const moe_config& c, const moe_ep_peers& p, int rank0, int nlocal,
+                                  const void* y_recv, const int32_t* local_offsets, int32_t* done,
+                                  uint32_t epoch, cudaStream_t s);
+cudaError_t launch_ep_wait_returned(const moe_ep_peers& p, int rank0, int nlocal, int32_t* status,
+                                    uint32_t epoch, cudaStream_t s);
 cudaError_t launch_gather_rows(const bf16* src, const int32_t* index, bf16* dst, int n, int n_src,
                                int D, cudaStream_t s);
 // Router + preprocess + dispatch in one cooperative launch (few experts; see
@@ -100,7 +118,7 @@ cudaError_t launch_route_pre_dispatch(const moe_config& c, const void* x, const 
                                       float* topk_w, int32_t* counts, int32_t* expert_offsets,
                                       int32_t* rank_splits, int32_t* rank_offsets, int32_t* pos,
                                       int32_t* src, int32_t* block_counts, int max_blocks,
-                                      int32_t* mt_start, unsigned* barrier, bool barrier_zeroed,
+                                      unsigned* barrier, bool barrier_zeroed,
                                       bf16* x_perm, int32_t* status, cudaStream_t s);
 cudaError_t launch_dispatch(const moe_config& c, const void* x, const int32_t* pos,
                             bf16* x_perm, cudaStream_t s);
@@ -119,13 +137,12 @@ struct GemmProblem {
   const bf16* B; int G;                   // B [G, N, K]
   int N, K;
   const int32_t* group_offsets;           // [G+1] device, or nullptr: one dense group
-  const int32_t* mt_start;                // [G+1] device, or nullptr
   int dense_rows;                         // rows of the dense group
   int64_t max_tiles;                      // host upper bound on tiles (grid size)
   bf16* out; int ldo;                     // output row stride in elements
   float* outf;                            // fp32 output (EPI_PAIRSUM_F32)
   int epi; int tile_n;
-  int pair;                               // 1: 256-row tiles on CTA pairs (mt_start per 256 rows)
+  int pair;                               // 1: 256-row tiles on CTA pairs
   int32_t* status;
   int32_t* counter;                       // device tile counter, zero when the launch starts
   int dep;                                // launch_grouped_pair: index of the phase whose output

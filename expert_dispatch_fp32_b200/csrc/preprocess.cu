@@ -14,7 +14,7 @@
 //  2. a grid barrier (bounded wait; a stuck barrier reports MOE_ERR_TIMEOUT);
 //  3. every block reads the histogram, forms its per-expert base (pairs of e in
 //     earlier blocks) and the global exclusive scan; block 0 writes counts,
-//     expert offsets, rank splits/offsets and the GEMM M-tile prefixes;
+//     expert offsets and rank splits/offsets;
 //  4. each block walks its chunk in order; a pair's row is offset[e] + base[e] +
 //     (earlier pairs of e in this block), the last term from __match_any_sync
 //     ranks within a warp plus per-warp counts of earlier warps.  Rows follow
@@ -32,7 +32,7 @@ struct PreArgs {
   int R, E, ep, chunk;
   int32_t* block_counts;   // [gridDim.x][E]
   unsigned* barrier;       // [2], zero at launch
-  int32_t *counts, *expert_offsets, *rank_splits, *rank_offsets, *mt_start, *pos, *src, *status;
+  int32_t *counts, *expert_offsets, *rank_splits, *rank_offsets, *pos, *src, *status;
 };
 
 __global__ void __launch_bounds__(kPreThreads)
@@ -66,8 +66,8 @@ pre_fused_kernel(const PreArgs a) {
   if (!grid_barrier(a.barrier, gridDim.x, a.status)) return;
 
   // 3. per-expert base of this block, global totals and the block-0 outputs
-  pre_totals<kPreThreads>(a.block_counts, E, a.ep, cnt, tmp, warp_cnt, warp_sums, &total, a.counts,
-                          a.expert_offsets, a.rank_splits, a.rank_offsets, a.mt_start);
+  pre_totals<kPreThreads>(a.block_counts, E, a.ep, cnt, tmp, warp_sums, &total, a.counts,
+                          a.expert_offsets, a.rank_splits, a.rank_offsets);
 
   // 4. in-order scatter of this block's chunk, kPreThreads pairs per round
   pre_positions<kPreThreads>(
@@ -103,7 +103,7 @@ int preprocess_blocks(int64_t R) {
 cudaError_t launch_preprocess(const moe_config& c, const int32_t* topk_idx, int32_t* counts,
                               int32_t* expert_offsets, int32_t* rank_splits,
                               int32_t* rank_offsets, int32_t* pos, int32_t* src,
-                              int32_t* block_counts, int max_blocks, int32_t* mt_start,
+                              int32_t* block_counts, int max_blocks,
                               unsigned* barrier, int32_t* status, cudaStream_t s) {
   const int R = c.T * c.top_k;
   const int sms = sm_count();
@@ -117,7 +117,7 @@ cudaError_t launch_preprocess(const moe_config& c, const int32_t* topk_idx, int3
   a.idx = topk_idx; a.R = R; a.E = c.E; a.ep = c.ep_size; a.chunk = chunk;
   a.block_counts = block_counts; a.barrier = barrier;
   a.counts = counts; a.expert_offsets = expert_offsets; a.rank_splits = rank_splits;
-  a.rank_offsets = rank_offsets; a.mt_start = mt_start; a.pos = pos; a.src = src; a.status = status;
+  a.rank_offsets = rank_offsets; a.pos = pos; a.src = src; a.status = status;
   const size_t smem = (size_t)c.E * sizeof(int) * (2 + kPreWarps);
   if (smem > (48u << 10)) {
     err = cudaFuncSetAttribute(pre_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -22,7 +22,7 @@
 namespace moe {
 namespace {
 
-// Scratch: grid-barrier words, the two GEMM tile prefixes, then block histograms.
+// Scratch: two grid-barrier words, then the block histograms.
 constexpr size_t kNoAllocScratchInts = MOE_NOALLOC_SCRATCH_BYTES / sizeof(int32_t);
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchInts];
 
@@ -106,19 +106,18 @@ extern "C" moe_status moe_preprocess_noalloc(const moe_config* cfg, const int32_
   }
   const size_t R = (size_t)c.T * c.top_k;
   const size_t nblk = (size_t)preprocess_blocks((int64_t)R);
-  // barrier words [2], tile prefixes [2 * (E + 1)], block histograms [nblk * E]
-  const size_t need = 2 + 2 * ((size_t)c.E + 1) + nblk * (size_t)c.E;
+  // barrier words [2], block histograms [nblk * E]
+  const size_t need = 2 + nblk * (size_t)c.E;
   if (need > kNoAllocScratchInts) return MOE_ERR_SCRATCH_LIMIT;
   int32_t* scratch = nullptr;
   if (scratch_for_current_device(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
   unsigned* barrier = reinterpret_cast<unsigned*>(scratch);
-  int32_t* mt_start = scratch + 2;
-  int32_t* block_counts = mt_start + 2 * ((size_t)c.E + 1);
+  int32_t* block_counts = scratch + 2;
   // The barrier words are zeroed on the stream before each launch; every histogram
   // entry is written before it is read, so nothing else needs clearing.
   const cudaError_t err = launch_preprocess(c, topk_idx, counts, expert_offsets, rank_splits,
                                             rank_offsets, pos, src, block_counts, (int)nblk,
-                                            mt_start, barrier, status,
+                                            barrier, status,
                                             reinterpret_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -85,8 +85,9 @@ MOE_API moe_status moe_validate_config(const moe_config* cfg);
 /* Bytes of scratch a caller must pass as `workspace` to moe_route,
  * moe_preprocess, moe_expert_ffn and moe_forward (one buffer serves all of them,
  * 256-byte aligned).  Holds the fp32 logits when the caller keeps none, the
- * preprocess block histograms, the per-expert GEMM tile prefix and the shared
- * experts' activations.  0 for an invalid config. */
+ * preprocess block histograms, the tensor-core router's intermediates, the shared
+ * experts' activations and the expert-FFN launch's tile and band counters.  0 for an
+ * invalid config. */
 MOE_API size_t moe_workspace_size(const moe_config* cfg);
 
 /* Bytes of the prepacked weight buffer written by moe_prepare_weights. */
@@ -137,7 +138,7 @@ MOE_API moe_status moe_route(const moe_config* cfg, const void* x, const float* 
  * Rows are ordered rank-major, then local expert, then token ascending (the
  * same as global expert order).  Bit-exact and deterministic.  An index outside
  * [0, E) sets *status = MOE_ERR_INDEX_OOB and that pair is skipped.
- * Also writes the GEMM tile prefix into `workspace` for moe_expert_ffn. */
+ * `workspace` holds the per-block histograms (scratch). */
 MOE_API moe_status moe_preprocess(const moe_config* cfg, const int32_t* topk_idx, int32_t* counts,
                           int32_t* expert_offsets, int32_t* rank_splits, int32_t* rank_offsets,
                           int32_t* pos, int32_t* src, void* workspace, int32_t* status,
@@ -168,10 +169,8 @@ MOE_API moe_status moe_dispatch_permute(const moe_config* cfg, const void* x, co
  *   y_perm         device bf16 [R, D], written
  *   shared_out     device bf16 [T, D], written when S > 0; NULL skips the shared
  *                  experts (moe_shared_ffn runs them alone)
- *   workspace      the buffer moe_preprocess (or moe_route_dispatch) wrote its tile
- *                  prefix into, for this same routing: moe_preprocess_noalloc writes no
- *                  prefix, so its outputs need a moe_preprocess of the same topk_idx
- *                  before this call, or the tiles follow an earlier routing
+ *   workspace      moe_workspace_size(cfg) bytes of scratch; the tile schedule comes
+ *                  from expert_offsets alone (each CTA derives the per-expert M tiles)
  *   status         device int32, MOE_ERR_TIMEOUT if a bounded wait expired */
 MOE_API moe_status moe_expert_ffn(const moe_config* cfg, const void* x_perm, const void* x,
                           const int32_t* expert_offsets, const void* packed, void* act,
@@ -245,11 +244,10 @@ MOE_API moe_status moe_forward(const moe_config* cfg, const void* x, const float
  * the process exits.
  *
  * Outputs, layouts, ordering and the device status word are exactly those of
- * moe_preprocess (bit-identical results); it does not write the GEMM tile prefix
- * that moe_expert_ffn reads from a workspace, so it is a drop-in for the
- * bookkeeping outputs only.
- *   Limit: max(1, min(160, ceil(T*k / 256))) * E + 2*(E + 1) + 2 int32 values must
- *   fit in the scratch (the check uses this count; the launch may then use fewer
+ * moe_preprocess (bit-identical results), and they are all moe_dispatch_permute,
+ * moe_expert_ffn and moe_combine_unpermute read.
+ *   Limit: max(1, min(160, ceil(T*k / 256))) * E + 2 int32 values must fit in the
+ *   scratch (the check uses this count; the launch may then use fewer
  *   blocks on a GPU with fewer SMs); larger configurations return
  *   MOE_ERR_SCRATCH_LIMIT before anything is enqueued.
  *   First call on each device: finds the scratch array's device address with
@@ -291,6 +289,80 @@ MOE_API moe_status moe_ep_local_ids(const moe_config* cfg, const int32_t* topk_i
 MOE_API moe_status moe_gather_rows(const void* src, const int32_t* index, void* dst, int32_t n,
                                    int32_t n_src, int32_t D, void* stream);
 
+/* Expert-parallel exchange over peer memory ("Expert Parallel (EP)", Communication
+ * Pattern steps 2-4; "Worked Example ...", Steps 2 and 4): the token pre- and
+ * post-all-to-all as stores into the other ranks' buffers, with no host round trip.
+ * P = cfg->ep_size ranks; rank r owns experts [r*El, (r+1)*El), El = E / P, and holds
+ * cfg->T tokens.  Every rank's exchange buffers are reachable from every rank through
+ * the tables below: device arrays of P device pointers, entry p = rank p's buffer
+ * (peer mappings of other GPUs' memory on a multi-GPU node; with several ranks on one
+ * GPU, buffers of that GPU).  Each call covers ranks [rank0, rank0 + nlocal), the
+ * ranks whose own data is on the calling device; their per-rank inputs are stacked
+ * (rank rank0 + i at slice i of each argument; an int32 argument of n values per rank
+ * has rows of (n + 3) / 4 * 4 values, so each rank's row is 16-byte aligned).  `epoch` numbers the exchange: every
+ * call of one forward passes the same value, the next forward a different one (flags
+ * are compared for equality, never reset).  Waits are bounded (~1 s of SM cycles) and
+ * report MOE_ERR_TIMEOUT in *status; after an error the caller zeroes `done` and the
+ * flag arrays before the next exchange.  Received rows of local expert l are ordered
+ * by sending rank, then token, which the grouped FFN takes as is.
+ * Order of one forward, on every rank: moe_route + moe_preprocess of its tokens,
+ * moe_ep_send_counts, moe_ep_send_rows, moe_ep_recv_layout, moe_expert_ffn on the
+ * received rows (a config with E = El, top_k = 1, T = cap, shared_out = NULL),
+ * moe_ep_return_rows, moe_ep_wait_returned, then moe_shared_ffn and
+ * moe_combine_unpermute with y_back in place of y_perm (same rows, same order). */
+typedef struct {
+  int32_t P;                   /* ranks in the exchange (== cfg->ep_size) */
+  int32_t cap;                 /* rows each rank's receive buffers hold */
+  int32_t* const* cnt;         /* int32 [P, E]: row s = counts sent by rank s */
+  uint32_t* const* flags;      /* uint32 [3, P], zero before the first exchange: epochs
+                                  of counts / rows / returned rows from each rank */
+  void* const* recv_x;         /* bf16 [cap, D]: rows received for the local experts */
+  int32_t* const* recv_src;    /* int32 [cap]: the sender's dispatch row of each */
+  int32_t* const* recv_rank;   /* int32 [cap]: the sender's rank of each */
+  void* const* y_back;         /* bf16 [T*k, D]: output rows returned to this rank, at
+                                  its own dispatch rows (pos) */
+} moe_ep_peers;
+
+/* Each covered rank's counts [E] (from moe_preprocess) into row `rank` of every rank's
+ * count matrix, then its count flag there.  counts: device int32 [nlocal, E]. */
+MOE_API moe_status moe_ep_send_counts(const moe_config* cfg, const moe_ep_peers* peers,
+                                      int32_t rank0, int32_t nlocal, const int32_t* counts,
+                                      uint32_t epoch, void* stream);
+
+/* The token pre-all-to-all: waits for every rank's counts, then stores each covered
+ * rank's k rows per token (bf16; an fp32 x is rounded to nearest even, as the dispatch
+ * does) into the owning ranks' recv_x, with recv_src / recv_rank beside them, and
+ * raises its row flag on every rank.  x [nlocal, T, D] (x_dtype), topk_idx and pos
+ * [nlocal, T*k], expert_offsets [nlocal, E+1] (moe_route / moe_preprocess outputs);
+ * done: device int32 [nlocal], zero (left zero).  A row beyond cap sets
+ * MOE_ERR_INVALID_ARG in *status and is dropped. */
+MOE_API moe_status moe_ep_send_rows(const moe_config* cfg, const moe_ep_peers* peers,
+                                    int32_t rank0, int32_t nlocal, const void* x,
+                                    const int32_t* topk_idx, const int32_t* pos,
+                                    const int32_t* expert_offsets, uint32_t epoch, int32_t* done,
+                                    int32_t* status, void* stream);
+
+/* Waits until every rank's rows have arrived, then writes each covered rank's local
+ * expert offsets [nlocal, El+1] over its received rows (the expert_offsets argument of
+ * the local moe_expert_ffn). */
+MOE_API moe_status moe_ep_recv_layout(const moe_config* cfg, const moe_ep_peers* peers,
+                                      int32_t rank0, int32_t nlocal, int32_t* local_offsets,
+                                      uint32_t epoch, int32_t* status, void* stream);
+
+/* The token post-all-to-all: each covered rank's output rows y_recv [nlocal, cap, D]
+ * (bf16, the local experts' y over the received rows, local_offsets as written by
+ * moe_ep_recv_layout) go back to their senders' y_back at the senders' rows; then the
+ * rank raises its return flag on every rank.  done: device int32 [nlocal], zero. */
+MOE_API moe_status moe_ep_return_rows(const moe_config* cfg, const moe_ep_peers* peers,
+                                      int32_t rank0, int32_t nlocal, const void* y_recv,
+                                      const int32_t* local_offsets, uint32_t epoch,
+                                      int32_t* done, int32_t* status, void* stream);
+
+/* Waits until every rank has returned the covered ranks' rows (y_back complete). */
+MOE_API moe_status moe_ep_wait_returned(const moe_config* cfg, const moe_ep_peers* peers,
+                                        int32_t rank0, int32_t nlocal, uint32_t epoch,
+                                        int32_t* status, void* stream);
+
 /* Self-check of device-side failure detection.  The cooperative kernels (moe_preprocess,
  * moe_route_dispatch) synchronise their blocks at a grid barrier whose wait is bounded
  * (~1 s of SM cycles); a block that gives up writes MOE_ERR_TIMEOUT to the status word
@@ -302,6 +374,25 @@ MOE_API moe_status moe_gather_rows(const void* src, const int32_t* index, void* 
  *   barrier: two device uint32 words of scratch (zeroed by the call);
  *   status: device int32, not reset by the call. */
 MOE_API moe_status moe_check_wait_timeout(uint32_t* barrier, int32_t* status, void* stream);
+
+/* Where moe_route's tensor-core router leaves its intermediate values, so that a
+ * caller (the parity tests) can measure how close the filter runs to its error bound.
+ * "Expert Parallel (EP)", Configuration: the router is computed in fp32
+ * (router_dtype='fp32'); for bf16 x with more experts than the shared-memory router
+ * holds, moe_route without returned logits finds each token's top-k in two steps:
+ * approx[t,e] = x_t . (hi_e + mid_e) on the tensor cores (W_r = hi + mid + lo, hi and
+ * mid bf16), and an exact fp32 logit for every expert whose approx + bias is at least
+ * the k-th largest minus 2 eps_t, eps_t = coef * sum_d |x_t,d| wmax_d.  That is sound
+ * when |approx - exact| <= eps_t, which this view lets a test check.
+ * After moe_route with this cfg and workspace (no logits returned), the workspace
+ * holds, until the next call that uses it:
+ *   approx [T, approx_ld] fp32 at byte *approx_offset (bias not added; columns >= E
+ *          are padding), wmax [D] fp32 at byte *wmax_offset; *coef is the coefficient.
+ * Returns MOE_ERR_UNSUPPORTED when moe_route takes another path for cfg (fp32 x, few
+ * experts, few tokens, no renormalisation, or MOE_ROUTER_TC=0 in the environment).
+ * Host-only: enqueues nothing. */
+MOE_API moe_status moe_router_filter_view(const moe_config* cfg, size_t* approx_offset,
+                                          int32_t* approx_ld, size_t* wmax_offset, float* coef);
 
 /* Static description of a status code. */
 MOE_API const char* moe_status_string(moe_status s);

@@ -122,3 +122,39 @@ def test_empty_batch_is_a_no_op(B):
     assert lib.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, None) == 0
     assert lib.moe_dispatch_permute(ctypes.byref(c), None, None, None, None) == 0
     assert lib.moe_combine_unpermute(ctypes.byref(c), None, None, None, None, None, None, None) == 0
+
+
+def test_router_filter_view_says_which_router_runs(B):
+    # the tensor-core filter: bf16 x, 256 experts, enough tokens, renormalised
+    ds = good_cfg(B, T=8192, D=7168, E=256, ep_size=8, top_k=8, F=2048, act=B.MOE_ACT_SWIGLU,
+                  x_dtype=B.MOE_DT_BF16)
+    ao, ld, wo, coef = B.moe_router_filter_view(ds)
+    assert ld == 256 and ao % 256 == 0 and wo % 256 == 0
+    assert ao + 8192 * ld * 4 <= B.moe_workspace_size(ds) and wo + 7168 * 4 <= ao
+    assert abs(coef - (4 * (7168 // 16 + 2) * 2.0 ** -23 + 2.0 ** -17)) < 1e-9
+    # other paths: fp32 x, few experts, few tokens, no renormalisation
+    assert B.moe_router_filter_view(good_cfg(B)) is None
+    for kw in ({"E": 16, "ep_size": 4, "D": 2048}, {"T": 32}, {"renormalize": 0}):
+        c = dict(T=8192, D=7168, E=256, ep_size=8, top_k=8, F=2048, act=B.MOE_ACT_SWIGLU,
+                 x_dtype=B.MOE_DT_BF16)
+        c.update(kw)
+        assert B.moe_router_filter_view(good_cfg(B, **c)) is None, kw
+
+
+def test_peer_exchange_calls_reject_bad_tables_on_host(B):
+    c = good_cfg(B)                       # ep_size 4
+    lib = B.lib()
+    import numpy as np
+    buf = np.zeros(1 << 12, dtype=np.uint8)
+    h = (buf.ctypes.data + 255) // 256 * 256       # real host memory, never enqueued on
+    peers = B.MoeEpPeers(4, 16, h, h, h, h, h, h)
+    by, pa = ctypes.byref(c), ctypes.addressof(peers)
+    assert lib.moe_ep_send_counts(by, None, 0, 4, h, 1, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_send_counts(by, pa, 3, 2, h, 1, None) == B.MOE_ERR_INVALID_ARG   # ranks 3..4 of 4
+    assert lib.moe_ep_send_counts(by, pa, 0, 0, h, 1, None) == B.MOE_ERR_INVALID_ARG
+    bad = B.MoeEpPeers(2, 16, h, h, h, h, h, h)   # P differs from ep_size
+    assert lib.moe_ep_wait_returned(by, ctypes.addressof(bad), 0, 1, 1, h, None) == B.MOE_ERR_INVALID_ARG
+    nul = B.MoeEpPeers(4, 16, h, None, h, h, h, h)
+    assert lib.moe_ep_recv_layout(by, ctypes.addressof(nul), 0, 1, h, 1, h, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_send_rows(by, pa, 0, 1, h, h, h, None, 1, h, h, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_return_rows(by, pa, 0, 1, h, h, 1, None, h, None) == B.MOE_ERR_INVALID_ARG

@@ -113,7 +113,7 @@ def test_few_expert_router_four_tokens_per_warp(T):
 def test_fused_route_dispatch_matches_stage_calls(T, D, E, k, xdt, renorm, logits, shared):
     """moe_route_dispatch as one cooperative launch gives the bits of moe_route +
     moe_preprocess + moe_dispatch_permute (routing, weights, logits, counts, offsets,
-    splits, rows, x_perm) and the same layer output (so the same GEMM tile prefix)."""
+    splits, rows, x_perm) and the same layer output."""
     wl = BASE.with_(T=T, D=D, E=E, ep_size=2 if E % 2 == 0 else 1, top_k=k, F=128, x_dtype=xdt,
                     renormalize=renorm, n_shared=1 if shared else 0, F_shared=128 if shared else 0,
                     seed=7)
@@ -421,11 +421,12 @@ def test_uneven_expert_tiles(act, extra):
     g.manual_seed(5)
     x_perm = torch.randn((T, wl.D), generator=g, device="cuda").to(torch.bfloat16)
     x_bf = inp["x"].to(torch.bfloat16) if shared else None
-    # CTA-pair kernel with skinny remainder tiles, with M = 128 remainders only, then
-    # the one-CTA kernel
-    for pair, skinny in (("1", "1"), ("1", "0"), ("0", "1")):
+    # CTA-pair kernel with skinny tiles and folded remainders (257..320-row last bands as
+    # one tile), without folding, without skinny tiles, then the one-CTA kernel
+    for pair, skinny, fold in (("1", "1", "1"), ("1", "1", "0"), ("1", "0", "1"), ("0", "1", "1")):
         os.environ["MOE_GEMM_CTA_PAIR"] = pair
         os.environ["MOE_GEMM_SKINNY"] = skinny
+        os.environ["MOE_GEMM_FOLD"] = fold
         try:
             b["y_perm"].zero_()
             M.moe_expert_ffn(cfg, x_perm, x_bf, b["expert_offsets"], layer.packed, b["act"],
@@ -434,6 +435,7 @@ def test_uneven_expert_tiles(act, extra):
         finally:
             del os.environ["MOE_GEMM_CTA_PAIR"]
             del os.environ["MOE_GEMM_SKINNY"]
+            del os.environ["MOE_GEMM_FOLD"]
         assert int(b["status"].item()) == 0
         off = b["expert_offsets"].cpu().numpy()
         assert np.array_equal(np.diff(off), counts)
@@ -450,11 +452,14 @@ def test_uneven_expert_tiles(act, extra):
             assert_layer_close(f64(b["shared_out"]), s_ref, np.zeros_like(s_ref), "shared_out")
 
 
-def test_fused_and_separate_ffn_launches_agree(monkeypatch):
+@pytest.mark.parametrize("T", [700, 1400])
+def test_fused_and_separate_ffn_launches_agree(monkeypatch, T):
     """The single persistent launch (gate_up, shared gate_up, down, shared down with
     band dependencies) gives the same bits as one launch per GEMM, and both match
-    the oracle (ragged expert ends and a partial last band of the shared expert)."""
-    wl = BASE.with_(T=700, D=512, E=16, ep_size=4, top_k=3, F=512, n_shared=2, F_shared=256, seed=9)
+    the oracle (ragged expert ends and a partial last band of the shared expert; with
+    1400 tokens most experts hold 257..320 rows, so their down tiles wait on folded
+    gate_up tiles)."""
+    wl = BASE.with_(T=T, D=512, E=16, ep_size=4, top_k=3, F=512, n_shared=2, F_shared=256, seed=9)
     inp = W.make_inputs(wl, device="cuda")
     outs = []
     for flag in ("1", "0"):

@@ -63,9 +63,9 @@ def test_noalloc_preprocess_matches_workspace_preprocess_twice():
 
 @pytest.mark.gpu
 def test_noalloc_rejects_configs_beyond_its_scratch():
-    # 2048 tokens x top-8 over 1024 experts: 64 histogram blocks x 1024 experts plus the
-    # prefixes need 67 588 int32, more than the 65 536 the scratch holds.  Real buffers of
-    # the right sizes, so nothing would fault even if a launch were enqueued.
+    # 2048 tokens x top-8 over 1024 experts: 64 histogram blocks x 1024 experts plus two
+    # barrier words need 65 538 int32, two more than the 65 536 the scratch holds.  Real
+    # buffers of the right sizes, so nothing would fault even if a launch were enqueued.
     wl = W.Workload(name="wide", T=2048, D=64, E=1024, ep_size=8, top_k=8, F=128)
     cfg = M.make_config(wl.T, wl.D, wl.E, wl.ep_size, wl.top_k, wl.F)
     idx = torch.zeros((wl.T, wl.top_k), dtype=torch.int32, device="cuda")
@@ -77,9 +77,8 @@ def test_noalloc_rejects_configs_beyond_its_scratch():
     assert st == M.MOE_ERR_SCRATCH_LIMIT
     torch.cuda.synchronize()
     assert int(got["counts"][0].item()) == -7          # nothing was written
-    # just under the limit: 1920 tokens -> 60 histogram blocks -> 63 492 int32 (1984 tokens
-    # would need 62 blocks, 65 540 int32, four too many)
-    wl2 = wl.with_(T=1920)
+    # just under the limit: 2016 tokens -> 63 histogram blocks -> 64 514 int32
+    wl2 = wl.with_(T=2016)
     cfg2 = M.make_config(wl2.T, wl2.D, wl2.E, wl2.ep_size, wl2.top_k, wl2.F)
     g = torch.Generator(device="cpu").manual_seed(5)
     idx2 = torch.rand((wl2.T, wl2.E), generator=g).argsort(dim=1)[:, :wl2.top_k]
