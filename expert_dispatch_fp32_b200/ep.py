@@ -162,3 +162,115 @@ class EPMoELayer:
         return o.shared_and_combine(x, st, y_back)
 
     __call__ = forward
+
+
+class PeerEPGroup:
+    """The expert-parallel forward of P ranks whose data is all on one device, the two
+    exchanges done by libmoe.so's peer-memory calls (moe_ep_*): stores straight into
+    the owning rank's receive buffer, flags with the forward's epoch, no host round
+    trip and no collective library.
+
+    Rank r owns experts [r*El, (r+1)*El) and its own T tokens; the shared experts and
+    the router are replicated.  The same calls take peer-mapped buffers of other GPUs
+    in their pointer tables; here every table entry is a slice of one device's tensors,
+    and each call covers all P ranks in one launch (kernels of different ranks never
+    wait on one another across launches).  forward(x) takes x [P, T, D] and returns
+    out [P, T, D]: rank r's rows equal moe_forward of its tokens with all E experts.
+    """
+
+    def __init__(self, *, D, E, P, top_k, F, T, w_router, w_gate_up, w_down, expert_bias=None,
+                 ws_gate_up=None, ws_down=None, act="swiglu", renormalize=True, x_dtype="bf16"):
+        if E % P:
+            raise ValueError("num_experts must be divisible by the number of ranks")
+        dev = w_router.device
+        self.D, self.E, self.P, self.k, self.F, self.T = D, E, P, top_k, F, T
+        self.El = El = E // P
+        self.S = 0 if ws_gate_up is None else ws_gate_up.shape[0]
+        self.Fs = 0 if ws_gate_up is None else ws_down.shape[1]
+        self.cap = cap = P * T * min(top_k, El)
+        self.w_router = w_router.contiguous()
+        self.bias = None if expert_bias is None else expert_bias.contiguous()
+        self.tok_cfg = make_config(T, D, E, P, top_k, F, act, renormalize, x_dtype, self.S, self.Fs)
+        self.loc_cfg = make_config(cap, D, El, 1, 1, F, act, True, "bf16", self.S, self.Fs)
+        self.sh_cfg = make_config(T, D, El, 1, 1, F, act, True, "bf16", self.S, self.Fs)
+        i32 = lambda *s: torch.zeros(s, dtype=torch.int32, device=dev)
+        bf = lambda *s: torch.zeros(s, dtype=torch.bfloat16, device=dev)
+        # stacked per-rank int32 rows padded to 16 bytes (the calls' row stride); [:, :n]
+        # views keep every rank's row aligned for the single-rank calls
+        pad = lambda n: (n + 3) // 4 * 4
+        rows = lambda n: torch.zeros((P, pad(n)), dtype=torch.int32, device=dev)[:, :n]
+        R = T * top_k
+        psize = B.moe_packed_weights_size(self.loc_cfg)
+        self.packed = torch.empty((P, psize), dtype=torch.uint8, device=dev)
+        for r in range(P):
+            B.moe_prepare_weights(self.loc_cfg, w_gate_up[r * El:(r + 1) * El].contiguous(),
+                                  w_down[r * El:(r + 1) * El].contiguous(),
+                                  None if ws_gate_up is None else ws_gate_up.contiguous(),
+                                  None if ws_down is None else ws_down.contiguous(), self.packed[r])
+        # each rank's own stage outputs (stacked: rank r at index r)
+        self.topk_idx, self.topk_w = rows(R), torch.zeros((P, T, top_k), device=dev)
+        self.counts, self.offsets = rows(E), rows(E + 1)
+        self.splits, self.rank_offsets = rows(P), rows(P + 1)
+        self.pos, self.src = rows(R), rows(R)
+        self.ws_tok = torch.empty((P, max(B.moe_workspace_size(self.tok_cfg), 256)), dtype=torch.uint8,
+                                  device=dev)
+        # exchange buffers, reached through the pointer tables
+        self.cnt = i32(P, P, E)
+        self.flags = i32(P, 3, P)
+        self.recv_x, self.recv_src, self.recv_rank = bf(P, cap, D), i32(P, cap), i32(P, cap)
+        self.y_back = bf(P, R, D)
+        # the local experts' inputs and outputs
+        self.local_off = rows(El + 1)
+        self.act, self.y_recv = bf(P, cap, F), bf(P, cap, D)
+        self.ws_loc = torch.empty((P, max(B.moe_workspace_size(self.loc_cfg), 256)), dtype=torch.uint8,
+                                  device=dev)
+        self.ws_sh = torch.empty((P, max(B.moe_workspace_size(self.sh_cfg), 256)), dtype=torch.uint8,
+                                 device=dev)
+        xdt = torch.float32 if x_dtype in ("f32", torch.float32) else torch.bfloat16
+        self.shared_out = bf(P, T, D) if self.S else None
+        self.out = torch.empty((P, T, D), dtype=xdt, device=dev)
+        self.done, self.status = i32(P), i32(1)
+        table = lambda t: torch.tensor([t[r].data_ptr() for r in range(P)], dtype=torch.int64, device=dev)
+        self._tables = [table(t) for t in (self.cnt, self.flags, self.recv_x, self.recv_src,
+                                          self.recv_rank, self.y_back)]
+        self.peers = B.MoeEpPeers(P, cap, *[t.data_ptr() for t in self._tables])
+        self.epoch = 0
+
+    def forward(self, x, stream=None):
+        P, c = self.P, self.tok_cfg
+        self.epoch = self.epoch % 0xFFFFFFFF + 1          # never 0, the flags' initial value
+        e = self.epoch
+        for r in range(P):                                 # 1. each rank routes its tokens
+            B.moe_route(c, x[r], self.w_router, self.bias, None, self.topk_idx[r], self.topk_w[r],
+                        self.ws_tok[r], stream)
+        for r in range(P):
+            B.moe_preprocess(c, self.topk_idx[r], self.counts[r], self.offsets[r], self.splits[r],
+                             self.rank_offsets[r], self.pos[r], self.src[r], self.ws_tok[r],
+                             self.status, stream)
+        # 2. counts, then the token pre-all-to-all into the owners' buffers
+        B.moe_ep_send_counts(c, self.peers, 0, P, self.counts, e, stream)
+        B.moe_ep_send_rows(c, self.peers, 0, P, x, self.topk_idx, self.pos, self.offsets, e, self.done,
+                           self.status, stream)
+        B.moe_ep_recv_layout(c, self.peers, 0, P, self.local_off, e, self.status, stream)
+        for d in range(P):                                 # 3. each rank's local experts
+            B.moe_expert_ffn(self.loc_cfg, self.recv_x[d], None, self.local_off[d], self.packed[d],
+                             self.act[d], self.y_recv[d], None, self.ws_loc[d], self.status, stream)
+        # 4. the token post-all-to-all back to the senders' dispatch rows
+        B.moe_ep_return_rows(c, self.peers, 0, P, self.y_recv, self.local_off, e, self.done,
+                             self.status, stream)
+        B.moe_ep_wait_returned(c, self.peers, 0, P, e, self.status, stream)
+        for r in range(P):                                 # 5. shared experts and combine
+            sh = None
+            if self.S:
+                sh = self.shared_out[r]
+                B.moe_shared_ffn(self.sh_cfg, x[r], self.packed[r], sh, self.ws_sh[r], self.status, stream)
+            B.moe_combine_unpermute(c, self.y_back[r], self.pos[r], self.topk_w[r], x[r], sh, self.out[r],
+                                    stream)
+        return self.out
+
+    __call__ = forward
+
+    def check_status(self):
+        v = int(self.status.item())
+        if v != B.MOE_OK:
+            raise B.MoeError("device status", v)
