@@ -56,6 +56,9 @@ def parse_args():
     ap.add_argument("--tokens", type=int, default=0,
                     help="run the workload's shapes with this many tokens instead of its T "
                          "(serving-sized batches; the line's workload name gets a _t<N> suffix)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="run the workload with this many routed experts (a multiple of its "
+                         "ep_size; reduced cases for profiling; the name gets an _e<N> suffix)")
     return ap.parse_args()
 
 
@@ -63,6 +66,8 @@ def pick_workload(args):
     wl = W.get(args.workload)
     if args.tokens > 0:
         wl = wl.with_(T=args.tokens, name=f"{wl.name}_t{args.tokens}")
+    if args.experts > 0:
+        wl = wl.with_(E=args.experts, name=f"{wl.name}_e{args.experts}")
     return wl
 
 

@@ -80,3 +80,38 @@ def test_reference_arm_tokens_override():
     line = json.loads(p.stdout.strip().splitlines()[-1])
     assert line["config"]["workload"] == "worked_example_t64_t9" and line["config"]["T"] == 9
     assert line["value"] > 0
+
+
+def test_streamed_oracle_inputs_match_the_full_arrays():
+    """bench.py's CPU baseline fetches one expert's weights at a time (so a 256-expert
+    layer never needs its float64 weights at once); the oracle's output must be the
+    same as with the full weight arrays."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import torch
+    import bench
+    import moe_workloads as W
+    import oracle
+    wl = W.get("zipf_skew_e64").with_(T=48, D=128, F=128, F_shared=128)
+    inp = W.make_inputs(wl)
+    host = bench.HostOracleInputs(wl, inp)
+    f = lambda t: t.to(torch.float64).numpy()
+    kw = dict(E=wl.E, ep_size=wl.ep_size, top_k=wl.top_k, act=wl.act, renormalize=True)
+    full = oracle.moe_layer(host.x, host.w_router, host.bias, f(inp["w_gate_up"]), f(inp["w_down"]),
+                            host.ws_up, host.ws_down, **kw)
+    streamed = oracle.moe_layer(host.x, host.w_router, host.bias, None, None, host.ws_up, host.ws_down,
+                                expert_weights=host.expert, **kw)
+    assert np.array_equal(full["out"], streamed["out"])
+    assert bench.cpu_oracle_time(wl, host, 20, seed=3) > 0
+
+
+def test_reference_arm_experts_override():
+    """--experts runs a reduced expert count (profiling cases) and names it so."""
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "worked_example_t64", "--experts", "8", "--tokens", "16",
+                        "--steps", "1", "--warmup", "0"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert p.returncode == 0, p.stderr
+    line = json.loads(p.stdout.strip().splitlines()[-1])
+    assert line["config"]["workload"] == "worked_example_t64_t16_e8" and line["config"]["E"] == 8
