@@ -72,6 +72,7 @@ _SIGS = {
     "moe_gather_rows": (ctypes.c_int, [_vp, _i32p, _vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                        _vp]),
     "moe_check_wait_timeout": (ctypes.c_int, [_vp, _i32p, _vp]),
+    "moe_mxfp8_quantize": (ctypes.c_int, [_vp, ctypes.c_int64, ctypes.c_int32, _vp, _vp, _vp]),
     "moe_ep_send_counts": (ctypes.c_int, [_cfgp, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, _i32p,
                                           ctypes.c_uint32, _vp]),
     "moe_ep_send_rows": (ctypes.c_int, [_cfgp, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, _vp,
@@ -156,6 +157,10 @@ def moe_ep_return_rows(cfg, peers, rank0, nlocal, y_recv, local_offsets, epoch, 
 def moe_ep_wait_returned(cfg, peers, rank0, nlocal, epoch, status, stream=None):
     _call("moe_ep_wait_returned", ctypes.byref(cfg), ctypes.addressof(peers), rank0, nlocal, epoch,
           _p(status), _s(stream))
+
+
+def moe_mxfp8_quantize(x, rows, K, q, scales, stream=None):
+    _call("moe_mxfp8_quantize", _p(x), rows, K, _p(q), _p(scales), _s(stream))
 
 
 def moe_router_filter_view(cfg):

@@ -605,6 +605,17 @@ moe_status moe_router_filter_view(const moe_config* cfg, size_t* approx_offset, 
   return MOE_OK;
 }
 
+moe_status moe_mxfp8_quantize(const void* x, int64_t rows, int32_t K, void* q, void* scales,
+                              void* stream) {
+  if (rows < 0 || K <= 0 || K % 32 != 0) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  MOE_CHECK_PTR(x);
+  MOE_CHECK_PTR(q);
+  if (scales == nullptr) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_mx_quant_rows((const bf16*)x, rows, K, (uint8_t*)q, (uint8_t*)scales,
+                                          as_stream(stream)));
+}
+
 const char* moe_status_string(moe_status s) {
   switch (s) {
     case MOE_OK: return "ok";

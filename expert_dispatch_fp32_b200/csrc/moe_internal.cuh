@@ -93,6 +93,9 @@ cudaError_t launch_barrier_timeout_check(unsigned* barrier, int32_t* status, cud
 // Multi-rank helpers (ep.cu).
 cudaError_t launch_local_ids(const int32_t* topk_idx, const int32_t* src, int32_t* ids, int R, int El,
                              cudaStream_t s);
+// MXFP8 quantisation of bf16 rows (mxfp8.cu).
+cudaError_t launch_mx_quant_rows(const bf16* x, int64_t rows, int K, uint8_t* q, uint8_t* scales,
+                                 cudaStream_t s);
 // Peer-memory exchange (ep_peer.cu).
 cudaError_t launch_ep_send_counts(const moe_ep_peers& p, int rank0, int nlocal, const int32_t* counts,
                                   int E, uint32_t epoch, cudaStream_t s);

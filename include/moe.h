@@ -394,6 +394,18 @@ MOE_API moe_status moe_check_wait_timeout(uint32_t* barrier, int32_t* status, vo
 MOE_API moe_status moe_router_filter_view(const moe_config* cfg, size_t* approx_offset,
                                           int32_t* approx_ld, size_t* wmax_offset, float* coef);
 
+/* MXFP8 quantisation of bf16 rows (OCP Microscaling v1.0 "MXFP8 (E4M3)"; the MXFP8
+ * routed-expert option of torchtitan issue 5554): every 32 consecutive elements of a row
+ * share one power-of-two scale 2^s, s = floor(log2 max|v|) - 8 clamped to [-127, 127]
+ * (-127 for an all-zero block), and each element becomes v / 2^s rounded to the nearest
+ * E4M3 value, ties to even, magnitudes above 448 clamped to 448.
+ *   x      device bf16 [rows, K], K % 32 == 0, 16-byte aligned
+ *   q      device uint8 [rows, K], written: E4M3 bit patterns
+ *   scales device uint8 [rows, K/32], written: s + 127 (E8M0)
+ * Errors: MOE_ERR_INVALID_ARG for a bad pointer, a negative size or K % 32 != 0. */
+MOE_API moe_status moe_mxfp8_quantize(const void* x, int64_t rows, int32_t K, void* q, void* scales,
+                                      void* stream);
+
 /* Static description of a status code. */
 MOE_API const char* moe_status_string(moe_status s);
 
