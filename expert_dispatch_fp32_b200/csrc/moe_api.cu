@@ -51,6 +51,33 @@ PackLayout pack_layout(const moe_config& c) {
   return L;
 }
 
+MxPackLayout mx_pack_layout(const moe_config& c) {
+  MxPackLayout L;
+  const size_t E = c.E, D = c.D, F = c.F;
+  const size_t nup = c.act == MOE_ACT_SWIGLU ? 2 * F : F;
+  size_t o = 0;
+  L.w_up = o;       o = align256(o + E * nup * D);
+  L.w_down = o;     o = align256(o + E * D * F);
+  L.sf_up = o;      o = align256(o + E * nup * (D / 32));
+  L.sf_down = o;    o = align256(o + E * D * (F / 32));
+  L.sf_scratch = o; o = align256(o + (E * nup * (D / 32) > E * D * (F / 32) ? E * nup * (D / 32) : E * D * (F / 32)));
+  L.total = o;
+  return L;
+}
+
+MxWsLayout mx_ws_layout(const moe_config& c) {
+  MxWsLayout L;
+  const size_t R = (size_t)c.T * c.top_k, D = c.D, F = c.F;
+  size_t o = ws_layout(c).total;
+  L.xq = o;       o = align256(o + R * D);
+  L.xs = o;       o = align256(o + R * (D / 32));
+  L.aq = o;       o = align256(o + R * F);
+  L.as = o;       o = align256(o + R * (F / 32));
+  L.counters = o; o = align256(o + 2 * sizeof(int32_t));
+  L.total = o;
+  return L;
+}
+
 int up_tile_n(const moe_config& c) {
   if (c.act == MOE_ACT_SWIGLU) return 256;
   return c.F % 256 == 0 ? 256 : c.F % 128 == 0 ? 128 : 64;
@@ -602,6 +629,100 @@ moe_status moe_router_filter_view(const moe_config* cfg, size_t* approx_offset, 
   *approx_ld = (c.E + 127) / 128 * 128;
   *wmax_offset = L.r_wmax;
   *coef = route_filter_coef(c.D);
+  return MOE_OK;
+}
+
+// MXFP8 routed experts need 128-deep K steps and 128-wide N tiles on both GEMMs.
+static moe_status mx_check(const moe_config* cfg) {
+  moe_status st = moe_validate_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->D % 128 != 0 || cfg->F % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+size_t moe_packed_weights_mxfp8_size(const moe_config* cfg) {
+  if (mx_check(cfg) != MOE_OK) return 0;
+  return mx_pack_layout(*cfg).total;
+}
+
+size_t moe_workspace_mxfp8_size(const moe_config* cfg) {
+  if (mx_check(cfg) != MOE_OK) return 0;
+  return mx_ws_layout(*cfg).total;
+}
+
+moe_status moe_prepare_weights_mxfp8(const moe_config* cfg, const void* packed, void* packed_mx,
+                                     void* stream) {
+  moe_status st = mx_check(cfg);
+  if (st != MOE_OK) return st;
+  MOE_CHECK_PTR(packed);
+  MOE_CHECK_PTR(packed_mx);
+  const moe_config& c = *cfg;
+  const PackLayout P = pack_layout(c);
+  const MxPackLayout Q = mx_pack_layout(c);
+  const uint8_t* pk = (const uint8_t*)packed;
+  uint8_t* mx = (uint8_t*)packed_mx;
+  cudaStream_t s = as_stream(stream);
+  const int64_t nup = c.act == MOE_ACT_SWIGLU ? 2 * (int64_t)c.F : c.F;
+  cudaError_t err = launch_mx_quant_rows((const bf16*)(pk + P.w_up), (int64_t)c.E * nup, c.D, mx + Q.w_up,
+                                         mx + Q.sf_scratch, s);
+  if (err == cudaSuccess) err = launch_mx_block_scales(mx + Q.sf_scratch, mx + Q.sf_up, (int64_t)c.E * nup, c.D, s);
+  if (err == cudaSuccess)
+    err = launch_mx_quant_rows((const bf16*)(pk + P.w_down), (int64_t)c.E * c.D, c.F, mx + Q.w_down,
+                               mx + Q.sf_scratch, s);
+  if (err == cudaSuccess) err = launch_mx_block_scales(mx + Q.sf_scratch, mx + Q.sf_down, (int64_t)c.E * c.D, c.F, s);
+  return cuda_status(err);
+}
+
+moe_status moe_expert_ffn_mxfp8(const moe_config* cfg, const void* x_perm, const void* x,
+                                const int32_t* expert_offsets, const void* packed, const void* packed_mx,
+                                void* act, void* y_perm, void* shared_out, void* workspace,
+                                int32_t* status, void* stream) {
+  moe_status st = mx_check(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  MOE_CHECK_PTR(expert_offsets);
+  MOE_CHECK_PTR(packed_mx);
+  MOE_CHECK_PTR(workspace);
+  MOE_CHECK_PTR(status);
+  const int64_t R = (int64_t)c.T * c.top_k;
+  if (R > 0) {
+    MOE_CHECK_PTR(x_perm);
+    MOE_CHECK_PTR(act);
+    MOE_CHECK_PTR(y_perm);
+  }
+  cudaStream_t s = as_stream(stream);
+  const MxPackLayout Q = mx_pack_layout(c);
+  const MxWsLayout L = mx_ws_layout(c);
+  const uint8_t* mx = (const uint8_t*)packed_mx;
+  uint8_t* ws = (uint8_t*)workspace;
+  const int nup = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
+  int32_t* ctr = (int32_t*)(ws + L.counters);
+  if (R > 0) {
+    cudaError_t err = cudaMemsetAsync(ctr, 0, 2 * sizeof(int32_t), s);
+    if (err == cudaSuccess) err = launch_mx_quant_rows((const bf16*)x_perm, R, c.D, ws + L.xq, ws + L.xs, s);
+    MxProblem up;
+    memset(&up, 0, sizeof(up));
+    up.A = ws + L.xq; up.a_rows = R; up.sa = ws + L.xs;
+    up.B = mx + Q.w_up; up.G = c.E; up.sb = mx + Q.sf_up;
+    up.N = nup; up.K = c.D;
+    up.group_offsets = expert_offsets;
+    up.out = (bf16*)act; up.ldo = c.F;
+    up.epi = c.act == MOE_ACT_SWIGLU ? EPI_SWIGLU : EPI_GELU;
+    up.status = status; up.counter = ctr;
+    if (err == cudaSuccess) err = launch_grouped_mx(up, s);
+    if (err == cudaSuccess) err = launch_mx_quant_rows((const bf16*)act, R, c.F, ws + L.aq, ws + L.as, s);
+    MxProblem dn = up;
+    dn.A = ws + L.aq; dn.sa = ws + L.as;
+    dn.B = mx + Q.w_down; dn.sb = mx + Q.sf_down;
+    dn.N = c.D; dn.K = c.F;
+    dn.out = (bf16*)y_perm; dn.ldo = c.D;
+    dn.epi = EPI_STORE; dn.counter = ctr + 1;
+    if (err == cudaSuccess) err = launch_grouped_mx(dn, s);
+    if (err != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  // the shared experts stay bf16 (the MXFP8 option covers the routed experts)
+  if (c.n_shared > 0 && shared_out != nullptr)
+    return moe_shared_ffn(cfg, x, packed, shared_out, workspace, status, stream);
   return MOE_OK;
 }
 

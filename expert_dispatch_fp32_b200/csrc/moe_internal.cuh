@@ -51,6 +51,19 @@ struct PackLayout {
 };
 PackLayout pack_layout(const moe_config& c);
 
+// MXFP8 routed-expert weights: E4M3 gate_up [E, Nup, D] and down [E, D, F] (the bf16
+// packing's row order), their scales in block order, and a row-major scale scratch.
+struct MxPackLayout {
+  size_t w_up, w_down, sf_up, sf_down, sf_scratch, total;
+};
+MxPackLayout mx_pack_layout(const moe_config& c);
+// Workspace of the MXFP8 FFN: the bf16 workspace, then the quantised x_perm and act with
+// their scales and two tile counters.
+struct MxWsLayout {
+  size_t xq, xs, aq, as, counters, total;
+};
+MxWsLayout mx_ws_layout(const moe_config& c);
+
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // GEMM tile widths chosen from the shapes
@@ -96,6 +109,26 @@ cudaError_t launch_local_ids(const int32_t* topk_idx, const int32_t* src, int32_
 // MXFP8 quantisation of bf16 rows (mxfp8.cu).
 cudaError_t launch_mx_quant_rows(const bf16* x, int64_t rows, int K, uint8_t* q, uint8_t* scales,
                                  cudaStream_t s);
+// MXFP8 grouped GEMM (grouped_gemm_mx.cu): E4M3 A [a_rows, K] with row-major scales
+// sa [a_rows, K/32]; E4M3 B [G, N, K] with scales in the tensor cores' block order sb
+// (launch_mx_block_scales); 128 x 128 tiles; `counter` zero at launch.
+struct MxProblem {
+  const uint8_t* A; int64_t a_rows;
+  const uint8_t* sa;
+  const uint8_t* B; int G;
+  const uint8_t* sb;
+  int N, K;
+  const int32_t* group_offsets;
+  bf16* out; int ldo;
+  int epi;
+  int32_t* status;
+  int32_t* counter;
+};
+cudaError_t launch_grouped_mx(const MxProblem& p, cudaStream_t s);
+// Row-major scales [rows, K/32] -> the block order of launch_grouped_mx's B operand
+// (rows % 128 == 0, K % 128 == 0).
+cudaError_t launch_mx_block_scales(const uint8_t* rowmajor, uint8_t* blocked, int64_t rows, int K,
+                                   cudaStream_t s);
 // Peer-memory exchange (ep_peer.cu).
 cudaError_t launch_ep_send_counts(const moe_ep_peers& p, int rank0, int nlocal, const int32_t* counts,
                                   int E, uint32_t epoch, cudaStream_t s);

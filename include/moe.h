@@ -406,6 +406,33 @@ MOE_API moe_status moe_router_filter_view(const moe_config* cfg, size_t* approx_
 MOE_API moe_status moe_mxfp8_quantize(const void* x, int64_t rows, int32_t K, void* q, void* scales,
                                       void* stream);
 
+/* MXFP8 routed experts (opt-in; the layer's default path is bf16).  torchtitan issue 5554
+ * names MXFP8 routed experts as an option; the expert FFN is the same two-layer network
+ * ("Expert Parallel (EP)", Communication Pattern step 3), with every operand of both
+ * GEMMs quantised to MXFP8 as moe_mxfp8_quantize does along its K axis: x_perm and the
+ * weights of gate_up along D, act and the down weights along F.  The tensor cores form
+ * the scaled products exactly and accumulate in fp32 (tcgen05 kind::mxf8f6f4 with block
+ * scales); the activation and its bf16 rounding are those of moe_expert_ffn.  Needs
+ * D % 128 == 0 and F % 128 == 0 (else MOE_ERR_UNSUPPORTED).
+ *
+ * Bytes of the MXFP8 weight buffer: */
+MOE_API size_t moe_packed_weights_mxfp8_size(const moe_config* cfg);
+/* Bytes of workspace for moe_expert_ffn_mxfp8 (includes moe_workspace_size's). */
+MOE_API size_t moe_workspace_mxfp8_size(const moe_config* cfg);
+/* Quantises the routed experts of `packed` (moe_prepare_weights' output for cfg) into
+ * packed_mx (caller-allocated, moe_packed_weights_mxfp8_size bytes); one time. */
+MOE_API moe_status moe_prepare_weights_mxfp8(const moe_config* cfg, const void* packed, void* packed_mx,
+                                             void* stream);
+/* moe_expert_ffn with MXFP8 routed experts: quantises x_perm, runs gate_up (activation
+ * fused, act written in bf16), quantises act, runs down into y_perm; the shared experts
+ * (if shared_out is not NULL) run in bf16 from `packed` as in moe_expert_ffn.  Arguments
+ * as moe_expert_ffn plus packed_mx; workspace: moe_workspace_mxfp8_size bytes. */
+MOE_API moe_status moe_expert_ffn_mxfp8(const moe_config* cfg, const void* x_perm, const void* x,
+                                        const int32_t* expert_offsets, const void* packed,
+                                        const void* packed_mx, void* act, void* y_perm,
+                                        void* shared_out, void* workspace, int32_t* status,
+                                        void* stream);
+
 /* Static description of a status code. */
 MOE_API const char* moe_status_string(moe_status s);
 

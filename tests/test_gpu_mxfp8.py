@@ -37,3 +37,71 @@ def test_quantize_matches_the_oracle_bit_for_bit(rows, K):
     assert np.array_equal(s.cpu().numpy().astype(np.int64) - 127, s_ref)
     qv = q.cpu().view(torch.float8_e4m3fn).to(torch.float64).numpy()
     assert np.array_equal(qv, qv_ref)
+
+
+def _mx_oracle_expert(x_rows, w_up, w_down, act):
+    """The expert FFN on MXFP8 operands: x and both weight matrices quantised along their
+    K axis (oracle/mxfp8.py), the activation rounded to bf16 (as the GPU stores it) and
+    quantised along F before the down projection."""
+    import oracle
+    dq = lambda a: mxfp8.dequantize_mxfp8(*mxfp8.quantize_mxfp8(a, axis=-1), axis=-1)
+    xq = dq(x_rows)
+    wu = dq(np.asarray(w_up).T).T            # [D, Nup], blocks of 32 along D
+    wd = dq(np.asarray(w_down).T).T          # [F, D], blocks of 32 along F
+    h = xq @ wu
+    if act == "swiglu":
+        F = wu.shape[1] // 2
+        a = oracle.silu(h[:, :F]) * h[:, F:]
+    else:
+        a = oracle.gelu(h)
+    a = oracle.bf16_round(a)
+    return dq(a) @ wd
+
+
+@pytest.mark.parametrize("case", ["swiglu_shared", "gelu", "deepseek_like"])
+def test_mxfp8_expert_ffn_matches_the_oracle(case):
+    import moe_workloads as W
+    from parity_helpers import assert_layer_close, f64, make_layer, up_weights
+    wl = {"swiglu_shared": W.Workload(name="mx1", T=300, D=512, E=8, ep_size=2, top_k=2, F=256,
+                                      n_shared=1, F_shared=256, seed=31),
+          "gelu": W.Workload(name="mx2", T=200, D=256, E=4, ep_size=2, top_k=2, F=256, act="gelu",
+                             seed=32),
+          "deepseek_like": W.Workload(name="mx3", T=512, D=1024, E=16, ep_size=4, top_k=8, F=512,
+                                      n_shared=1, F_shared=512, seed=33)}[case]
+    inp = W.make_inputs(wl, device="cuda")
+    layer = make_layer(wl, inp)
+    T = wl.T
+    b = layer.allocate(T)
+    cfg = layer.config(T)
+    layer.forward(inp["x"])                 # route, preprocess, dispatch (x_perm) and the bf16 FFN
+    torch.cuda.synchronize()
+    layer.check_status()
+    y_bf16 = b["y_perm"].clone()
+    packed_mx = torch.empty(M.moe_packed_weights_mxfp8_size(cfg), dtype=torch.uint8, device="cuda")
+    M.moe_prepare_weights_mxfp8(cfg, layer.packed, packed_mx)
+    ws = torch.zeros(M.moe_workspace_mxfp8_size(cfg), dtype=torch.uint8, device="cuda")
+    y = torch.full_like(b["y_perm"], float("nan"))
+    sh = None if b["shared_out"] is None else torch.empty_like(b["shared_out"])
+    for it in range(2):                     # twice: the scratch and counters are reused
+        M.moe_expert_ffn_mxfp8(cfg, b["x_perm"], inp["x"] if wl.x_dtype == "bf16" else None,
+                               b["expert_offsets"], layer.packed, packed_mx, b["act"], y, sh, ws,
+                               b["status"])
+        torch.cuda.synchronize()
+        layer.check_status()
+    off = b["expert_offsets"].cpu().numpy()
+    xp = f64(b["x_perm"])
+    wup = up_weights(wl, inp)
+    got, ref = [], []
+    for e in range(wl.E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi == lo:
+            continue
+        r = _mx_oracle_expert(xp[lo:hi], f64(wup[e]), f64(inp["w_down"][e]), wl.act)
+        g = f64(y[lo:hi])
+        assert_layer_close(g, r, np.zeros_like(r), f"mxfp8 y_perm expert {e}")
+        got.append(g); ref.append(r)
+    err = np.linalg.norm(np.concatenate(got) - np.concatenate(ref)) / np.linalg.norm(np.concatenate(ref))
+    vs_bf16 = (torch.linalg.norm(y.float() - y_bf16.float()) / torch.linalg.norm(y_bf16.float())).item()
+    print(f"\n{case}: MXFP8 y_perm vs oracle rel-L2 {err:.2e}; vs the bf16 path {vs_bf16:.2e}")
+    if sh is not None:
+        assert torch.equal(sh, b["shared_out"])     # the shared experts stay bf16
