@@ -76,8 +76,7 @@ _SIGS = {
     "moe_packed_weights_mxfp8_size": (ctypes.c_size_t, [_cfgp]),
     "moe_workspace_mxfp8_size": (ctypes.c_size_t, [_cfgp]),
     "moe_prepare_weights_mxfp8": (ctypes.c_int, [_cfgp, _vp, _vp, _vp]),
-    "moe_expert_ffn_mxfp8": (ctypes.c_int, [_cfgp, _vp, _vp, _i32p, _vp, _vp, _vp, _vp, _vp, _vp, _i32p,
-                                            _vp]),
+    "moe_expert_ffn_mxfp8": (ctypes.c_int, [_cfgp, _vp, _vp, _i32p, _vp, _vp, _vp, _vp, _vp, _i32p, _vp]),
     "moe_ep_send_counts": (ctypes.c_int, [_cfgp, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, _i32p,
                                           ctypes.c_uint32, _vp]),
     "moe_ep_send_rows": (ctypes.c_int, [_cfgp, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, _vp,
@@ -180,10 +179,10 @@ def moe_prepare_weights_mxfp8(cfg, packed, packed_mx, stream=None):
     _call("moe_prepare_weights_mxfp8", ctypes.byref(cfg), _p(packed), _p(packed_mx), _s(stream))
 
 
-def moe_expert_ffn_mxfp8(cfg, x_perm, x, expert_offsets, packed, packed_mx, act, y_perm, shared_out,
+def moe_expert_ffn_mxfp8(cfg, x_perm, x, expert_offsets, packed, packed_mx, y_perm, shared_out,
                          workspace, status, stream=None):
     _call("moe_expert_ffn_mxfp8", ctypes.byref(cfg), _p(x_perm), _p(x), _p(expert_offsets), _p(packed),
-          _p(packed_mx), _p(act), _p(y_perm), _p(shared_out), _p(workspace), _p(status), _s(stream))
+          _p(packed_mx), _p(y_perm), _p(shared_out), _p(workspace), _p(status), _s(stream))
 
 
 def moe_router_filter_view(cfg):

@@ -1,5 +1,6 @@
 // Grouped expert GEMM with MXFP8 operands on the 5th-generation tensor cores:
-// tcgen05.mma.kind::mxf8f6f4.block_scale, E4M3 A and B, one E8M0 scale per 32 K.
+// tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale, E4M3 A and B, one E8M0 scale
+// per 32 K, 256 x 256 output tiles on a cluster of two CTAs.
 //
 // torchtitan issue 5554 (shared-expert overlap) lists MXFP8 routed experts as an
 // option; "Expert Parallel (EP)", Communication Pattern step 3 and "Worked Example:
@@ -8,100 +9,145 @@
 // MXFP8 (E4M3): out[row, :] = epilogue( sum_k qa[row,k] 2^sa[row,k/32] qb[n,k] 2^sb[n,k/32] ),
 // accumulated in fp32 by the tensor cores (the scaled products are exact).
 //
-//   A   E4M3 [rows, K] (K-major) with its scales sa [rows, K/32] (row-major bytes,
-//       s + 127), from moe_mxfp8_quantize; rows of group g at [off[g], off[g+1]);
-//   B   E4M3 [G, N, K] (K-major) with its scales pre-arranged in the tensor cores'
-//       block order: for group g, 128-row block n and 128-deep K step s, 512 bytes at
-//       ((g * N/128 + n) * K/128 + s) * 512, row r's four scales (K blocks 4s..4s+3)
-//       at byte 16 (r % 32) + 4 (r / 32).
+// Operands (K-major E4M3 bytes):
+//   A   [rows, K]; rows of group g at [off[g], off[g+1]); M tiles of 256 rows per group,
+//       numbered across groups (tile t = tiles of the groups before g + m).
+//   B   [G, N, K]; N tiles of 256 rows.
+// Scales are stored "blocked": for tile t, K step s (128 K), half h (128 rows) a
+// 512-byte block holding row m's four scales (K blocks 4s..4s+3) at byte
+// 16 (m % 32) + 4 (m / 32) + j, the order tcgen05.cp .32x128b.warpx4 spreads over TMEM
+// (row m in lane m % 32 of every lane quarter, column m / 32, byte j).  Block (t, s, h)
+// sits at ((t * ksteps + s) * 2 + h) * 512 (mx_sf_offset), so CTA h of a pair loads its
+// A block and both B blocks of a K step with one TMA copy each.  A's blocks come from
+// the x_perm quantiser, which knows each row's tile, and from this kernel's own
+// epilogue for the down projection's A (the activation): the up projection and the down
+// projection tile the same groups the same way, so the epilogue of up tile t writes the
+// scales of down tile t.
 //
-// One CTA per SM, 128 x 128 output tiles, 6 warps as in the bf16 one-CTA kernel:
-//   warp 0      producer: every lane gathers four rows' scale words of the A tile
-//               into the 512-byte block order (one 16-byte store per lane), then lane 0
-//               posts the stage's expected bytes and issues the A and B tile loads (TMA,
-//               128 rows x 128 bytes, 128-byte swizzle) and B's 512-byte scale block
-//               (bulk copy) into a 6-stage ring;
-//   warp 1      allocates 512 TMEM columns (two 128-column accumulators, A and B scale
-//               columns at 256 and 260); one lane copies the stage's scale blocks into
-//               TMEM (tcgen05.cp 32x128b, broadcast to the four lane quarters) and issues
-//               four M=128 N=128 K=32 block-scaled MMAs, scale block j selected by the
-//               scale-id fields; commits free the stage and hand over the accumulator;
-//   warps 2-5   epilogue (tcgen05.ld, activation, bf16 rows masked at the group end).
-// The scale columns are rewritten every stage: tcgen05 operations of one thread run in
-// issue order, so a stage's copy lands after the previous stage's MMAs have read theirs.
-// Every wait is bounded and reports MOE_ERR_TIMEOUT.  The accumulators and scale columns
-// need 264 TMEM columns, so the tile is 128 wide: two 256-wide accumulators would fill TMEM.
+// A CTA pair, 10 warps per CTA:
+//   warp 0      TMA producer (lane 0, both CTAs): this CTA's 128 A rows, its 128 B rows,
+//               its A scale block and both B scale blocks of each K step into a 6-stage
+//               ring; the bytes complete on the leader's `full` barrier.
+//   warp 1      TMEM (512 columns, both CTAs); in the leader, lane 0 copies the stage's
+//               scale blocks into TMEM (tcgen05.cp) and issues four M=256 N=256 K=32
+//               block-scaled MMAs, scale byte j selected per MMA; commits free the stage
+//               in both CTAs and hand the accumulator to the epilogue.
+//   warps 2-9   epilogue: warp w reads lanes 32 (w % 4) .. of TMEM, columns
+//               128 ((w - 2) / 4) .. + 127, all into registers, then releases the
+//               accumulator (16 arrivals on the leader) before its math and stores.
+// The accumulator needs 256 TMEM columns and the scales 12, so there is one
+// accumulator: the early release keeps the tensor cores' wait per tile to the TMEM
+// read.  The scale columns are rewritten every K step: tcgen05 operations issued by one
+// thread run in order, so a step's copy lands after the previous step's MMAs read theirs.
+// Every wait is bounded and reports MOE_ERR_TIMEOUT.
+#include <cuda_fp8.h>
+
 #include "tc_common.cuh"
 
 namespace moe {
 
 namespace {
 
+constexpr int kMxThreads = 320;
+constexpr int kMxTileM = 256;
+
 struct MxArgs {
-  CUtensorMap tmap_a;        // E4M3 [rows, K], box 128 x 128 bytes
+  CUtensorMap tmap_a;        // E4M3 [rows, K], box 128 x 128 rows
   CUtensorMap tmap_b;        // E4M3 [G, N, K], box 128 x 128 x 1
-  const uint32_t* sa;        // A scales as 32-bit words: [rows, K/128] (four K blocks each)
-  const uint8_t* sb;         // B scales, block order (see above)
+  CUtensorMap tmap_sfa;      // A scale blocks as [bytes / 256, 256], box 256 x 2 (one block)
+  CUtensorMap tmap_sfb;      // B scale blocks, box 256 x 4 (both halves of a K step)
   const int32_t* group_offsets;
-  int32_t G, N, K, a_rows;
-  bf16* out;
+  int32_t G, N, K;
+  bf16* out;                 // EPI_STORE: bf16 [rows, ldo]
   int32_t ldo;
+  uint8_t* q_out;            // EPI_SWIGLU / EPI_GELU: E4M3 activation [rows, ldo]
+  uint8_t* q_sf;             //   and its scale blocks (ldo / 128 K steps)
   int32_t* status;
   int32_t* counter;          // tile counter, zero at launch
 };
 
 struct MxCfg {
-  static constexpr int BN = 128;
+  static constexpr int BN = 256;
   static constexpr int KS = 128;                     // K elements (bytes) per stage
   static constexpr int kStages = 6;
-  static constexpr int kABytes = kTileM * KS;        // 16 KB
-  static constexpr int kBBytes = BN * KS;            // 16 KB
-  static constexpr int kSfBytes = 512;
-  static constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;
+  static constexpr int kABytes = 128 * KS;           // this CTA's 128 A rows
+  static constexpr int kBBytes = 128 * KS;           // this CTA's 128 B rows
+  static constexpr int kSfaBytes = 512;
+  static constexpr int kSfbBytes = 1024;
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static constexpr int kTmemCols = 512;
-  static constexpr int kSfaCol = 256, kSfbCol = 260;
+  static constexpr int kSfaCol = 256, kSfbCol = 260;  // 4 + 8 scale columns after the accumulator
+  static constexpr int kCtrl = 512;
   static size_t smem_bytes(int G) {
-    return 1024 + (size_t)kStages * kStageBytes + kCtrlBytes + 2 * (size_t)(G + 1) * sizeof(int);
+    return 1024 + (size_t)kStages * kStageBytes + kCtrl + 2 * (size_t)(G + 1) * sizeof(int);
   }
 };
 
-// Block-scaled instruction descriptor, kind::mxf8f6f4: E4M3 A and B, K-major, E8M0 scales,
-// scale block `j` of A and of B (bits 29-30 and 4-5).
+// Block-scaled instruction descriptor, kind::mxf8f6f4: E4M3 A and B, K-major, E8M0 scales
+// (bit 23), scale byte `j` of A and of B (bits 29-30 and 4-5).
 __host__ __device__ constexpr uint32_t mx_idesc(int M, int N, int j) {
   return ((uint32_t)j << 4) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24) |
          ((uint32_t)j << 29);
 }
 
 // Shared-memory descriptor of a 512-byte scale block for tcgen05.cp: no swizzle,
-// K-major, 8-row core matrices of 16 bytes placed 128 bytes apart.
+// 8-row core matrices of 16-byte rows placed 128 bytes apart.
 __device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
   return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
 }
 
-__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+__device__ __forceinline__ void tc_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
-__device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate, uint32_t sfa, uint32_t sfb) {
+__device__ __forceinline__ void tc_mma_mx_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate, uint32_t sfa,
+                                               uint32_t sfb) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
           d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
       : "memory");
 }
 
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-      : "memory");
+// Byte offset of scale (row m of half h, K block j) of tile t's K step s.
+__host__ __device__ __forceinline__ size_t mx_sf_offset(int64_t t, int ksteps, int s, int h, int m, int j) {
+  return (size_t)((t * ksteps + s) * 2 + h) * 512 + 16 * (m & 31) + 4 * (m >> 5) + j;
+}
+
+__device__ __forceinline__ int mx_mtiles(int rows) { return (rows + kMxTileM - 1) / kMxTileM; }
+
+// E8M0 exponent of a block from its largest magnitude: floor(log2 amax) - 8, clamped to
+// [-127, 127] (-127 for a zero block; a subnormal amax also lands on -127).
+__device__ __forceinline__ int mx_exponent(float amax) {
+  const int e = (int)((__float_as_uint(amax) >> 23) & 0xFFu) - 127 - 8;
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// Quantise 32 values: E4M3 bytes of v * 2^-s (round to nearest even, saturated) into
+// dst (32 bytes, 16-byte aligned); returns the scale byte s + 127.
+__device__ __forceinline__ uint8_t mx_quant32(const float (&v)[32], uint8_t* dst) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const int s = mx_exponent(amax);
+  const float inv = __uint_as_float((uint32_t)(127 - s) << 23);
+  uint4 out[2];
+  uint16_t* o = reinterpret_cast<uint16_t*>(out);
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    o[i] = (uint16_t)__nv_cvt_float2_to_fp8x2(make_float2(v[2 * i] * inv, v[2 * i + 1] * inv), __NV_SATFINITE,
+                                              __NV_E4M3);
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  d[0] = out[0];
+  d[1] = out[1];
+  return (uint8_t)(s + 127);
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_mx_kernel(const __grid_constant__ MxArgs p) {
+__global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __grid_constant__ MxArgs p) {
   using C = MxCfg;
   constexpr int S = C::kStages, BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
@@ -110,173 +156,224 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_mx_kernel(const 
   uint8_t* a_smem = smem;
   uint8_t* b_smem = smem + S * C::kABytes;
   uint8_t* sfa_smem = smem + S * (C::kABytes + C::kBBytes);
-  uint8_t* sfb_smem = sfa_smem + S * C::kSfBytes;
+  uint8_t* sfb_smem = sfa_smem + S * C::kSfaBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
-  // bars: full[S], empty[S], tmem_full[2], tmem_empty[2], qfull[Q], qempty[Q]
-  volatile int* tq = reinterpret_cast<volatile int*>(bars + 2 * S + 4 + 2 * kTileQ);
+  // bars: full[S], empty[S], tmem_full, tmem_empty, qfull[Q], qempty[Q]
+  volatile int* tq = reinterpret_cast<volatile int*>(bars + 2 * S + 2 + 2 * kTileQ);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(tq) + kTileQ);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* wsum = const_cast<int*>(abort_flag) + 1;
-  int* mt = reinterpret_cast<int*>(smem + S * C::kStageBytes + kCtrlBytes);
+  int* wsum = const_cast<int*>(abort_flag) + 1;                 // [kMxThreads / 32]
+  int* mt = reinterpret_cast<int*>(smem + S * C::kStageBytes + C::kCtrl);
   const int G = p.G;
   int* off = mt + (G + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
-  const uint32_t tfull0 = smem_u32(bars + 2 * S), tempty0 = smem_u32(bars + 2 * S + 2);
-  const uint32_t qfull0 = smem_u32(bars + 2 * S + 4), qempty0 = smem_u32(bars + 2 * S + 4 + kTileQ);
+  const uint32_t tfull = smem_u32(bars + 2 * S), tempty = smem_u32(bars + 2 * S + 1);
+  const uint32_t qfull0 = smem_u32(bars + 2 * S + 2), qempty0 = smem_u32(bars + 2 * S + 2 + kTileQ);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(full0 + 8 * i, 1);
       mbar_init(empty0 + 8 * i, 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(tfull0 + 8 * i, 1);
-      mbar_init(tempty0 + 8 * i, 4);
-    }
+    mbar_init(tfull, 1);
+    mbar_init(tempty, 16);                   // 8 epilogue warps x 2 CTAs
     for (int i = 0; i < kTileQ; ++i) {
       mbar_init(qfull0 + 8 * i, 1);
-      mbar_init(qempty0 + 8 * i, 5);         // MMA issuer + 4 epilogue warps
+      // leader: MMA issuer + 8 epilogue warps; peer: producer + 8 epilogue warps
+      mbar_init(qempty0 + 8 * i, 18);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&p.tmap_a);
     prefetch_tmap(&p.tmap_b);
+    prefetch_tmap(&p.tmap_sfa);
+    prefetch_tmap(&p.tmap_sfb);
   }
   for (int i = threadIdx.x; i <= G; i += blockDim.x) off[i] = p.group_offsets[i];
-  __syncthreads();
-  group_tile_prefix(off, G, mt, wsum, [](int rows) { return (rows + kTileM - 1) / kTileM; });
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
                  "r"(C::kTmemCols)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
-  tc_fence_before();
   __syncthreads();
+  group_tile_prefix(off, G, mt, wsum, [](int rows) { return mx_mtiles(rows); });
+  tc_fence_before();
+  cluster_sync();               // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   const int nb = p.N / BN;
   const int total = mt[G] * nb;
   const int ksteps = p.K / C::KS;
-  const uint32_t qempty_sched = qempty0;
+  const uint32_t qempty_sched = map_to_cta(qempty0, 0);
 
   if (warp == 0) {
-    // ---------------- producer: scale gather (all lanes), TMA and bulk copies (lane 0) ----------------
-    int stage = 0;
-    uint32_t phase = 0;
-    int next = 0;
-    if (lane == 0) next = atomicAdd(p.counter, 1);
-    for (int qi = 0;; ++qi) {
-      int tile = 0;
-      if (lane == 0) tile = tq_post<false>(p.counter, next, total, qi, qfull0, qempty0, tq, abort_flag, p.status);
-      tile = __shfl_sync(0xffffffffu, tile, 0);
-      if (tile < 0) break;
-      int g, m, n;
-      decode_tile(tile, mt, G, nb, g, m, n);
-      const int row0 = off[g] + m * kTileM;
-      const uint8_t* sb_tile = p.sb + ((size_t)g * nb + n) * ksteps * C::kSfBytes;
-      bool ok = true;
-      for (int kb = 0; kb < ksteps; ++kb) {
-        int w = 1;
-        if (lane == 0) w = mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status) ? 1 : 0;
-        if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-        // this lane's rows lane, lane + 32, lane + 64, lane + 96: one word each (the four
-        // scales of the stage's K blocks); rows past the tensor take scale 0 (2^-127)
-        uint4 v;
-        uint32_t* vw = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int r = row0 + lane + 32 * j;
-          vw[j] = r < p.a_rows ? __ldg(p.sa + (size_t)r * ksteps + kb) : 0u;
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs; the leader's also schedules) ----------------
+      const uint32_t full0_leader = map_to_cta(full0, 0);
+      constexpr uint32_t stage_tx = 2u * (uint32_t)C::kStageBytes;
+      int stage = 0;
+      uint32_t phase = 0;
+      int next = leader ? atomicAdd(p.counter, 1) : 0;
+      for (int qi = 0;; ++qi) {
+        const int tile = leader
+            ? tq_post<true>(p.counter, next, total, qi, qfull0, qempty0, tq, abort_flag, p.status)
+            : tq_take<false>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
+        if (tile < 0) break;
+        int g, m, n;
+        decode_tile(tile, mt, G, nb, g, m, n);
+        const int arow = off[g] + m * kMxTileM + (int)rank * 128;
+        const int brow = n * BN + (int)rank * 128;
+        const int64_t ta = (int64_t)mt[g] + m;              // A's tile (scale blocks)
+        const int64_t tb = (int64_t)g * nb + n;              // B's tile
+        bool ok = true;
+        for (int kb = 0; kb < ksteps; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, stage_tx);
+          const uint32_t fb = full0_leader + 8 * stage;
+          tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * C::KS, arow);
+          tma_load_3d_pair(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * C::KS, brow, g);
+          tma_load_2d_pair(smem_u32(sfa_smem + stage * C::kSfaBytes), &p.tmap_sfa, fb, 0,
+                           (int)(((ta * ksteps + kb) * 2 + rank) * 2));
+          tma_load_2d_pair(smem_u32(sfb_smem + stage * C::kSfbBytes), &p.tmap_sfb, fb, 0,
+                           (int)((tb * ksteps + kb) * 4));
+          if (++stage == S) { stage = 0; phase ^= 1u; }
         }
-        *reinterpret_cast<uint4*>(sfa_smem + stage * C::kSfBytes + 16 * lane) = v;
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) {
-          const uint32_t fb = full0 + 8 * stage;
-          mbar_arrive_expect_tx(fb, C::kABytes + C::kBBytes + C::kSfBytes);
-          tma_load_2d(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * C::KS, row0);
-          tma_load_3d(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * C::KS, n * BN, g);
-          bulk_load(smem_u32(sfb_smem + stage * C::kSfBytes), sb_tile + (size_t)kb * C::kSfBytes,
-                    C::kSfBytes, fb);
-        }
-        if (++stage == S) { stage = 0; phase ^= 1u; }
+        if (!ok) break;
       }
-      if (!ok) break;
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- scale copies and block-scaled MMAs ----------------
+    if (lane == 0 && leader) {
+      // ---------------- scale copies and block-scaled pair MMAs (leader CTA) ----------------
       const uint32_t t_sfa = tmem_base + C::kSfaCol, t_sfb = tmem_base + C::kSfbCol;
       int stage = 0;
       uint32_t phase = 0;
-      int acc = 0;
       uint32_t acc_phase = 0;
       for (int qi = 0;; ++qi) {
         const int tile = tq_take<false>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
         if (tile < 0) break;
-        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, p.status)) break;
+        if (!mbar_wait(tempty, acc_phase ^ 1u, abort_flag, p.status)) break;
+        acc_phase ^= 1u;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         bool ok = true;
         for (int kb = 0; kb < ksteps; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
-          tc_cp_sf(t_sfa, sf_desc(smem_u32(sfa_smem + stage * C::kSfBytes)));
-          tc_cp_sf(t_sfb, sf_desc(smem_u32(sfb_smem + stage * C::kSfBytes)));
+          const uint32_t sa = smem_u32(sfa_smem + stage * C::kSfaBytes);
+          const uint32_t sb = smem_u32(sfb_smem + stage * C::kSfbBytes);
+          tc_cp_sf_pair(t_sfa, sf_desc(sa));
+          tc_cp_sf_pair(t_sfb, sf_desc(sb));              // B rows 0..127 of the tile
+          tc_cp_sf_pair(t_sfb + 4, sf_desc(sb + 512));    // B rows 128..255
           const uint64_t ad = sw128_desc(smem_u32(a_smem + stage * C::kABytes));
           const uint64_t bd = sw128_desc(smem_u32(b_smem + stage * C::kBBytes));
 #pragma unroll
           for (int j = 0; j < 4; ++j)          // K = 32 per MMA: +32 bytes
-            tc_mma_mx(d_tmem, ad + 2 * j, bd + 2 * j, mx_idesc(kTileM, BN, j), (kb | j) != 0,
-                      t_sfa | ((uint32_t)j << 30), t_sfb | ((uint32_t)j << 30));
-          tc_commit(empty0 + 8 * stage);
+            tc_mma_mx_pair(tmem_base, ad + 2 * j, bd + 2 * j, mx_idesc(kMxTileM, BN, j), (kb | j) != 0,
+                           t_sfa | ((uint32_t)j << 30), t_sfb | ((uint32_t)j << 30));
+          tc_commit_pair_both(empty0 + 8 * stage);
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        tc_commit(tfull0 + 8 * acc);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        tc_commit_pair_both(tfull);
       }
     }
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
-    const int q = warp & 3;
-    int acc = 0;
+    // ---------------- epilogue (warps 2..9 of both CTAs) ----------------
+    const int q = warp & 3;                 // TMEM lane quarter this warp may read
+    const int h = (warp - 2) >> 2;          // column half: TMEM columns 128 h .. 128 h + 127
+    const uint32_t tempty_leader = map_to_cta(tempty, 0);
     uint32_t acc_phase = 0;
     for (int qi = 0;; ++qi) {
       const int tile = tq_take<true>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
       if (__any_sync(0xffffffffu, tile < 0)) break;
       int g, m, n;
       decode_tile(tile, mt, G, nb, g, m, n);
-      const int row0 = off[g] + m * kTileM;
-      const int rows_valid = min(kTileM, off[g + 1] - row0);
       bool ok = true;
-      if (lane == 0) ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status);
+      if (lane == 0) ok = mbar_wait(tfull, acc_phase, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;
+      acc_phase ^= 1u;
       tc_fence_after();
-      const int r = q * 32 + lane;
-      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      const bool paired = EPI == EPI_SWIGLU;
-      epilogue_row<EPI>(p.out, nullptr, p.ldo, tb, 0, paired ? BN / 2 : BN, (int64_t)row0 + r,
-                        paired ? n * (BN / 2) : n * BN, r < rows_valid);
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * 128);
+      uint32_t v0[32], v1[32], v2[32], v3[32];
+      tmem_ld32(tbase, v0);
+      tmem_ld32(tbase + 32, v1);
+      tmem_ld32(tbase + 64, v2);
+      tmem_ld32(tbase + 96, v3);
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (lane == 0) mbar_arrive_cluster(tempty_leader);      // the accumulator may be reused
+      const int r = q * 32 + lane;
+      const int64_t row = (int64_t)off[g] + m * kMxTileM + (int)rank * 128 + r;
+      if (row >= off[g + 1]) {
+        // a row past the group's end: nothing to store
+      } else if (EPI == EPI_STORE) {
+        bf16* dst = p.out + row * p.ldo + n * BN + h * 128;
+        float f[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v0[i]);
+        store_row32(dst, f);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v1[i]);
+        store_row32(dst + 32, f);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v2[i]);
+        store_row32(dst + 64, f);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v3[i]);
+        store_row32(dst + 96, f);
+      } else {
+        // the activation, quantised for the down projection: this row's scales go to the
+        // down projection's tile mt[g] + m (the same tiling), half `rank`, row r
+        const int qk = p.ldo / C::KS;
+        const int64_t t = (int64_t)mt[g] + m;
+        float f[32];
+        if (EPI == EPI_SWIGLU) {
+          // [gate 64 | up 64] -> outputs n*128 + 64h + [0, 64): K step n, blocks 2h, 2h + 1
+          const int oc = n * 128 + h * 64;
+          uint8_t* dst = p.q_out + row * p.ldo + oc;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = silu_f(__uint_as_float(v0[i])) * __uint_as_float(v2[i]);
+          p.q_sf[mx_sf_offset(t, qk, n, (int)rank, r, 2 * h)] = mx_quant32(f, dst);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = silu_f(__uint_as_float(v1[i])) * __uint_as_float(v3[i]);
+          p.q_sf[mx_sf_offset(t, qk, n, (int)rank, r, 2 * h + 1)] = mx_quant32(f, dst + 32);
+        } else {
+          // GELU: outputs n*256 + 128h + [0, 128): K step 2n + h, blocks 0..3
+          const int oc = n * BN + h * 128;
+          const int s = 2 * n + h;
+          uint8_t* dst = p.q_out + row * p.ldo + oc;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = gelu_f(__uint_as_float(v0[i]));
+          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 0)] = mx_quant32(f, dst);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = gelu_f(__uint_as_float(v1[i]));
+          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 1)] = mx_quant32(f, dst + 32);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = gelu_f(__uint_as_float(v2[i]));
+          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 2)] = mx_quant32(f, dst + 64);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = gelu_f(__uint_as_float(v3[i]));
+          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 3)] = mx_quant32(f, dst + 96);
+        }
+      }
+      __syncwarp();
     }
   }
 
+  // Neither CTA leaves (or frees TMEM) while the pair's MMAs may still touch it.
   __syncwarp();
-  __syncthreads();
+  tc_fence_before();
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(C::kTmemCols)
                  : "memory");
   }
@@ -294,71 +391,162 @@ bool make_map_u8(CUtensorMap* m, const void* base, int rank, const uint64_t* dim
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Scale blocks viewed as rows of 256 bytes; a box of `box_rows` rows (2: one block, 4: two).
+bool make_map_sf(CUtensorMap* m, const void* base, size_t bytes, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || bytes % 256 != 0 || bytes == 0) return false;
+  cuuint64_t d[2] = {256, bytes / 256};
+  cuuint64_t strides[1] = {256};
+  cuuint32_t box[2] = {256, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), d, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int EPI>
-cudaError_t launch_mx(const MxArgs& a, int grid, cudaStream_t s) {
+cudaError_t launch_mx(const MxArgs& a, int clusters, cudaStream_t s) {
   const size_t smem = MxCfg::smem_bytes(a.G);
   auto kern = grouped_gemm_mx_kernel<EPI>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  kern<<<grid, kGemmThreads, smem, s>>>(a);
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kMxThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, kern, a);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
-// Scale blocks of a B operand in the order above, from row-major scales [G * N, K/32]:
-// one thread per (row, K step) writes the row's four scales as one word.
+// B's scale blocks from row-major scales [G * N, K/32] (N % 256 == 0): one thread per
+// (row, K step) moves the row's four scales as one word.  Tile t of B is rows
+// [256 t, 256 t + 256) of the stacked [G * N] rows.
 __global__ void __launch_bounds__(256)
-mx_block_scales_kernel(const uint32_t* __restrict__ rowmajor, uint32_t* __restrict__ blocked, int64_t rows,
+mx_block_scales_kernel(const uint32_t* __restrict__ rowmajor, uint8_t* __restrict__ blocked, int64_t rows,
                        int ksteps) {
   const int64_t n = rows * ksteps;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t row = i / ksteps;
-    const int kb = (int)(i % ksteps);
-    const int64_t blk = row / 128;
-    const int r = (int)(row % 128);
-    // block (blk, kb) holds 128 words; row r's word at (16 (r % 32) + 4 (r / 32)) / 4
-    blocked[(blk * ksteps + kb) * 128 + 4 * (r % 32) + r / 32] = __ldg(rowmajor + i);
+    const int s = (int)(i % ksteps);
+    const int64_t t = row / kMxTileM;
+    const int h = (int)((row / 128) & 1), m = (int)(row % 128);
+    *reinterpret_cast<uint32_t*>(blocked + mx_sf_offset(t, ksteps, s, h, m, 0)) = __ldg(rowmajor + i);
+  }
+}
+
+// x_perm -> E4M3 rows with A's scale blocks.  One warp per row: the row's group (binary
+// search of the offsets), its M tile and place in it, then 32-element blocks lane-strided.
+__global__ void __launch_bounds__(256)
+mx_quant_a_kernel(const bf16* __restrict__ x, const int32_t* __restrict__ group_offsets, int G, int K,
+                  uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+  extern __shared__ int sh[];
+  int* mt = sh;                 // [G + 1]
+  int* off = sh + (G + 1);      // [G + 1]
+  int* wsum = off + (G + 1);    // [8]
+  for (int i = threadIdx.x; i <= G; i += blockDim.x) off[i] = group_offsets[i];
+  __syncthreads();
+  group_tile_prefix(off, G, mt, wsum, [](int rows) { return mx_mtiles(rows); });
+  const int lane = threadIdx.x & 31;
+  const int warps = (int)(gridDim.x * blockDim.x) >> 5;
+  const int nblk = K / 32, ksteps = K / MxCfg::KS;
+  const int rows = off[G];
+  for (int r = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); r < rows; r += warps) {
+    int lo = 0, hi = G;           // off[lo] <= r < off[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (off[mid] <= r) lo = mid; else hi = mid;
+    }
+    const int rr = r - off[lo];
+    const int64_t t = (int64_t)mt[lo] + rr / kMxTileM;
+    const int within = rr % kMxTileM, h = within >> 7, m = within & 127;
+    for (int b = lane; b < nblk; b += 32) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)r * K + b * 32);
+      float v[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint4 u = __ldg(src + c);
+        const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(hh[i]);
+          v[8 * c + 2 * i] = f.x;
+          v[8 * c + 2 * i + 1] = f.y;
+        }
+      }
+      sf[mx_sf_offset(t, ksteps, b >> 2, h, m, b & 3)] = mx_quant32(v, q + (int64_t)r * K + b * 32);
+    }
   }
 }
 
 }  // namespace
 
+size_t mx_sf_bytes(int64_t tiles, int K) { return (size_t)tiles * (K / MxCfg::KS) * 1024; }
+
 cudaError_t launch_mx_block_scales(const uint8_t* rowmajor, uint8_t* blocked, int64_t rows, int K,
                                    cudaStream_t s) {
-  if (rows % 128 != 0 || K % 128 != 0) return cudaErrorInvalidValue;
-  const int64_t n = rows * (K / 128);
+  if (rows % kMxTileM != 0 || K % MxCfg::KS != 0) return cudaErrorInvalidValue;
+  const int64_t n = rows * (K / MxCfg::KS);
   if (n == 0) return cudaSuccess;
   int64_t grid = (n + 255) / 256;
   if (grid > 8 * (int64_t)sm_count()) grid = 8 * (int64_t)sm_count();
-  mx_block_scales_kernel<<<(int)grid, 256, 0, s>>>(reinterpret_cast<const uint32_t*>(rowmajor),
-                                                   reinterpret_cast<uint32_t*>(blocked), rows, K / 128);
+  mx_block_scales_kernel<<<(int)grid, 256, 0, s>>>(reinterpret_cast<const uint32_t*>(rowmajor), blocked, rows,
+                                                   K / MxCfg::KS);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mx_quant_a(const bf16* x, int64_t rows, const int32_t* group_offsets, int G, int K,
+                              uint8_t* q, uint8_t* sf, cudaStream_t s) {
+  if (K % MxCfg::KS != 0 || G <= 0) return cudaErrorInvalidValue;
+  if (rows == 0) return cudaSuccess;
+  const size_t smem = (2 * (size_t)(G + 1) + 8) * sizeof(int);
+  if (smem > 48 * 1024) return cudaErrorInvalidValue;
+  int64_t grid = (rows + 7) / 8;                 // 8 rows (warps) per block
+  if (grid > 4 * (int64_t)sm_count()) grid = 4 * (int64_t)sm_count();
+  mx_quant_a_kernel<<<(int)grid, 256, smem, s>>>(x, group_offsets, G, K, q, sf);
   return cudaGetLastError();
 }
 
 cudaError_t launch_grouped_mx(const MxProblem& p, cudaStream_t s) {
-  if (p.N % MxCfg::BN != 0 || p.K % MxCfg::KS != 0 || p.counter == nullptr || p.group_offsets == nullptr)
+  if (p.N % MxCfg::BN != 0 || p.K % MxCfg::KS != 0 || p.counter == nullptr || p.group_offsets == nullptr ||
+      p.G <= 0)
     return cudaErrorInvalidValue;
+  if (p.epi != EPI_STORE && (p.ldo % MxCfg::KS != 0 || p.q_out == nullptr || p.q_sf == nullptr))
+    return cudaErrorInvalidValue;
+  const int64_t tiles_m = p.a_rows / kMxTileM + p.G;      // at least the sum of ceil(rows_g / 256)
   MxArgs a;
   memset(&a, 0, sizeof(a));
   const uint64_t da[2] = {(uint64_t)p.K, (uint64_t)p.a_rows};
   const uint64_t db[3] = {(uint64_t)p.K, (uint64_t)p.N, (uint64_t)p.G};
-  if (!make_map_u8(&a.tmap_a, p.A, 2, da, kTileM) || !make_map_u8(&a.tmap_b, p.B, 3, db, MxCfg::BN))
+  if (!make_map_u8(&a.tmap_a, p.A, 2, da, 128) || !make_map_u8(&a.tmap_b, p.B, 3, db, 128) ||
+      !make_map_sf(&a.tmap_sfa, p.sa, mx_sf_bytes(tiles_m, p.K), 2) ||
+      !make_map_sf(&a.tmap_sfb, p.sb, mx_sf_bytes((int64_t)p.G * (p.N / MxCfg::BN), p.K), 4))
     return cudaErrorInvalidValue;
-  a.sa = reinterpret_cast<const uint32_t*>(p.sa);
-  a.sb = p.sb;
   a.group_offsets = p.group_offsets;
   a.G = p.G;
   a.N = p.N;
   a.K = p.K;
-  a.a_rows = (int32_t)p.a_rows;
   a.out = p.out;
   a.ldo = p.ldo;
+  a.q_out = p.q_out;
+  a.q_sf = p.q_sf;
   a.status = p.status;
   a.counter = p.counter;
-  const int64_t tiles = (p.a_rows / kTileM + p.G) * (int64_t)(p.N / MxCfg::BN);
-  const int grid = (int)(tiles < sm_count() ? (tiles > 0 ? tiles : 1) : sm_count());
-  if (p.epi == EPI_SWIGLU) return launch_mx<EPI_SWIGLU>(a, grid, s);
-  if (p.epi == EPI_GELU) return launch_mx<EPI_GELU>(a, grid, s);
-  return launch_mx<EPI_STORE>(a, grid, s);
+  const int64_t tiles = tiles_m * (int64_t)(p.N / MxCfg::BN);
+  const int pairs = sm_count() / 2;
+  const int clusters = (int)(tiles < pairs ? (tiles > 0 ? tiles : 1) : pairs);
+  if (p.epi == EPI_SWIGLU) return launch_mx<EPI_SWIGLU>(a, clusters, s);
+  if (p.epi == EPI_GELU) return launch_mx<EPI_GELU>(a, clusters, s);
+  return launch_mx<EPI_STORE>(a, clusters, s);
 }
 
 }  // namespace moe

@@ -68,11 +68,12 @@ MxPackLayout mx_pack_layout(const moe_config& c) {
 MxWsLayout mx_ws_layout(const moe_config& c) {
   MxWsLayout L;
   const size_t R = (size_t)c.T * c.top_k, D = c.D, F = c.F;
+  const int64_t tiles = (int64_t)(R / 256) + c.E;     // bounds the 256-row tiles of all experts
   size_t o = ws_layout(c).total;
   L.xq = o;       o = align256(o + R * D);
-  L.xs = o;       o = align256(o + R * (D / 32));
+  L.xsf = o;      o = align256(o + mx_sf_bytes(tiles, c.D));
   L.aq = o;       o = align256(o + R * F);
-  L.as = o;       o = align256(o + R * (F / 32));
+  L.asf = o;      o = align256(o + mx_sf_bytes(tiles, c.F));
   L.counters = o; o = align256(o + 2 * sizeof(int32_t));
   L.total = o;
   return L;
@@ -632,11 +633,13 @@ moe_status moe_router_filter_view(const moe_config* cfg, size_t* approx_offset, 
   return MOE_OK;
 }
 
-// MXFP8 routed experts need 128-deep K steps and 128-wide N tiles on both GEMMs.
+// MXFP8 routed experts: 256-wide N tiles on both GEMMs (gate_up width and D multiples of
+// 256) and 128-deep K steps (D and F multiples of 128).
 static moe_status mx_check(const moe_config* cfg) {
   moe_status st = moe_validate_config(cfg);
   if (st != MOE_OK) return st;
-  if (cfg->D % 128 != 0 || cfg->F % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  const int nup = cfg->act == MOE_ACT_SWIGLU ? 2 * cfg->F : cfg->F;
+  if (cfg->D % 256 != 0 || cfg->F % 128 != 0 || nup % 256 != 0) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 
@@ -675,8 +678,8 @@ moe_status moe_prepare_weights_mxfp8(const moe_config* cfg, const void* packed, 
 
 moe_status moe_expert_ffn_mxfp8(const moe_config* cfg, const void* x_perm, const void* x,
                                 const int32_t* expert_offsets, const void* packed, const void* packed_mx,
-                                void* act, void* y_perm, void* shared_out, void* workspace,
-                                int32_t* status, void* stream) {
+                                void* y_perm, void* shared_out, void* workspace, int32_t* status,
+                                void* stream) {
   moe_status st = mx_check(cfg);
   if (st != MOE_OK) return st;
   const moe_config& c = *cfg;
@@ -687,7 +690,6 @@ moe_status moe_expert_ffn_mxfp8(const moe_config* cfg, const void* x_perm, const
   const int64_t R = (int64_t)c.T * c.top_k;
   if (R > 0) {
     MOE_CHECK_PTR(x_perm);
-    MOE_CHECK_PTR(act);
     MOE_CHECK_PTR(y_perm);
   }
   cudaStream_t s = as_stream(stream);
@@ -699,22 +701,24 @@ moe_status moe_expert_ffn_mxfp8(const moe_config* cfg, const void* x_perm, const
   int32_t* ctr = (int32_t*)(ws + L.counters);
   if (R > 0) {
     cudaError_t err = cudaMemsetAsync(ctr, 0, 2 * sizeof(int32_t), s);
-    if (err == cudaSuccess) err = launch_mx_quant_rows((const bf16*)x_perm, R, c.D, ws + L.xq, ws + L.xs, s);
+    if (err == cudaSuccess)
+      err = launch_mx_quant_a((const bf16*)x_perm, R, expert_offsets, c.E, c.D, ws + L.xq, ws + L.xsf, s);
+    // gate_up (or W1): the activation comes out quantised, with the down projection's scales
     MxProblem up;
     memset(&up, 0, sizeof(up));
-    up.A = ws + L.xq; up.a_rows = R; up.sa = ws + L.xs;
+    up.A = ws + L.xq; up.a_rows = R; up.sa = ws + L.xsf;
     up.B = mx + Q.w_up; up.G = c.E; up.sb = mx + Q.sf_up;
     up.N = nup; up.K = c.D;
     up.group_offsets = expert_offsets;
-    up.out = (bf16*)act; up.ldo = c.F;
+    up.q_out = ws + L.aq; up.q_sf = ws + L.asf; up.ldo = c.F;
     up.epi = c.act == MOE_ACT_SWIGLU ? EPI_SWIGLU : EPI_GELU;
     up.status = status; up.counter = ctr;
     if (err == cudaSuccess) err = launch_grouped_mx(up, s);
-    if (err == cudaSuccess) err = launch_mx_quant_rows((const bf16*)act, R, c.F, ws + L.aq, ws + L.as, s);
     MxProblem dn = up;
-    dn.A = ws + L.aq; dn.sa = ws + L.as;
+    dn.A = ws + L.aq; dn.sa = ws + L.asf;
     dn.B = mx + Q.w_down; dn.sb = mx + Q.sf_down;
     dn.N = c.D; dn.K = c.F;
+    dn.q_out = nullptr; dn.q_sf = nullptr;
     dn.out = (bf16*)y_perm; dn.ldo = c.D;
     dn.epi = EPI_STORE; dn.counter = ctr + 1;
     if (err == cudaSuccess) err = launch_grouped_mx(dn, s);

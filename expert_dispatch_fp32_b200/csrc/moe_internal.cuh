@@ -57,10 +57,10 @@ struct MxPackLayout {
   size_t w_up, w_down, sf_up, sf_down, sf_scratch, total;
 };
 MxPackLayout mx_pack_layout(const moe_config& c);
-// Workspace of the MXFP8 FFN: the bf16 workspace, then the quantised x_perm and act with
-// their scales and two tile counters.
+// Workspace of the MXFP8 FFN: the bf16 workspace, then the quantised x_perm and
+// activation with their scale blocks, and two tile counters.
 struct MxWsLayout {
-  size_t xq, xs, aq, as, counters, total;
+  size_t xq, xsf, aq, asf, counters, total;
 };
 MxWsLayout mx_ws_layout(const moe_config& c);
 
@@ -113,22 +113,28 @@ cudaError_t launch_mx_quant_rows(const bf16* x, int64_t rows, int K, uint8_t* q,
 // sa [a_rows, K/32]; E4M3 B [G, N, K] with scales in the tensor cores' block order sb
 // (launch_mx_block_scales); 128 x 128 tiles; `counter` zero at launch.
 struct MxProblem {
-  const uint8_t* A; int64_t a_rows;
-  const uint8_t* sa;
-  const uint8_t* B; int G;
-  const uint8_t* sb;
-  int N, K;
+  const uint8_t* A; int64_t a_rows;       // E4M3 [a_rows, K]
+  const uint8_t* sa;                      // A's scale blocks (launch_mx_quant_a or an EPI_SWIGLU/GELU run)
+  const uint8_t* B; int G;                // E4M3 [G, N, K]
+  const uint8_t* sb;                      // B's scale blocks (launch_mx_block_scales)
+  int N, K;                               // N % 256 == 0, K % 128 == 0
   const int32_t* group_offsets;
-  bf16* out; int ldo;
+  bf16* out; int ldo;                     // EPI_STORE: bf16 [a_rows, ldo]
+  uint8_t* q_out; uint8_t* q_sf;          // EPI_SWIGLU / EPI_GELU: E4M3 [a_rows, ldo] + scale blocks
   int epi;
   int32_t* status;
   int32_t* counter;
 };
 cudaError_t launch_grouped_mx(const MxProblem& p, cudaStream_t s);
-// Row-major scales [rows, K/32] -> the block order of launch_grouped_mx's B operand
-// (rows % 128 == 0, K % 128 == 0).
+// Bytes of the scale blocks of `tiles` 256-row tiles over K.
+size_t mx_sf_bytes(int64_t tiles, int K);
+// Row-major scales [rows, K/32] -> the scale blocks of a B operand (rows % 256 == 0,
+// K % 128 == 0).
 cudaError_t launch_mx_block_scales(const uint8_t* rowmajor, uint8_t* blocked, int64_t rows, int K,
                                    cudaStream_t s);
+// bf16 rows grouped by group_offsets -> E4M3 rows and the scale blocks of an A operand.
+cudaError_t launch_mx_quant_a(const bf16* x, int64_t rows, const int32_t* group_offsets, int G, int K,
+                              uint8_t* q, uint8_t* sf, cudaStream_t s);
 // Peer-memory exchange (ep_peer.cu).
 cudaError_t launch_ep_send_counts(const moe_ep_peers& p, int rank0, int nlocal, const int32_t* counts,
                                   int E, uint32_t epoch, cudaStream_t s);

@@ -410,10 +410,12 @@ MOE_API moe_status moe_mxfp8_quantize(const void* x, int64_t rows, int32_t K, vo
  * names MXFP8 routed experts as an option; the expert FFN is the same two-layer network
  * ("Expert Parallel (EP)", Communication Pattern step 3), with every operand of both
  * GEMMs quantised to MXFP8 as moe_mxfp8_quantize does along its K axis: x_perm and the
- * weights of gate_up along D, act and the down weights along F.  The tensor cores form
- * the scaled products exactly and accumulate in fp32 (tcgen05 kind::mxf8f6f4 with block
- * scales); the activation and its bf16 rounding are those of moe_expert_ffn.  Needs
- * D % 128 == 0 and F % 128 == 0 (else MOE_ERR_UNSUPPORTED).
+ * weights of gate_up along D, the activation and the down weights along F.  The tensor
+ * cores form the scaled products exactly and accumulate in fp32 (tcgen05 kind::mxf8f6f4
+ * with block scales); the activation (SiLU(gate) * up, or GELU) is formed in fp32 and
+ * quantised from fp32, never rounded to bf16.  Needs D % 256 == 0, F % 128 == 0 and a
+ * gate_up width (2F for SwiGLU, F for GELU) that is a multiple of 256, else
+ * MOE_ERR_UNSUPPORTED.
  *
  * Bytes of the MXFP8 weight buffer: */
 MOE_API size_t moe_packed_weights_mxfp8_size(const moe_config* cfg);
@@ -423,15 +425,17 @@ MOE_API size_t moe_workspace_mxfp8_size(const moe_config* cfg);
  * packed_mx (caller-allocated, moe_packed_weights_mxfp8_size bytes); one time. */
 MOE_API moe_status moe_prepare_weights_mxfp8(const moe_config* cfg, const void* packed, void* packed_mx,
                                              void* stream);
-/* moe_expert_ffn with MXFP8 routed experts: quantises x_perm, runs gate_up (activation
- * fused, act written in bf16), quantises act, runs down into y_perm; the shared experts
- * (if shared_out is not NULL) run in bf16 from `packed` as in moe_expert_ffn.  Arguments
- * as moe_expert_ffn plus packed_mx; workspace: moe_workspace_mxfp8_size bytes. */
+/* moe_expert_ffn with MXFP8 routed experts: quantises x_perm (E4M3 rows and their
+ * scales, ordered for the GEMM's tiles), runs gate_up with the activation and its
+ * quantisation in the epilogue (the quantised activation stays in the workspace; no
+ * bf16 act is written), then down into y_perm (bf16 [T*k, D]).  The shared experts (if
+ * shared_out is not NULL) run in bf16 from `packed` as in moe_expert_ffn.  Other
+ * arguments as moe_expert_ffn; workspace: moe_workspace_mxfp8_size bytes, nothing in it
+ * needs clearing.  Errors as moe_expert_ffn. */
 MOE_API moe_status moe_expert_ffn_mxfp8(const moe_config* cfg, const void* x_perm, const void* x,
                                         const int32_t* expert_offsets, const void* packed,
-                                        const void* packed_mx, void* act, void* y_perm,
-                                        void* shared_out, void* workspace, int32_t* status,
-                                        void* stream);
+                                        const void* packed_mx, void* y_perm, void* shared_out,
+                                        void* workspace, int32_t* status, void* stream);
 
 /* Static description of a status code. */
 MOE_API const char* moe_status_string(moe_status s);
