@@ -2,6 +2,7 @@
 """Benchmark of the expert-parallel MoE-layer forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--mxfp8]
 
 One step = one forward of the whole layer (route -> preprocess -> dispatch ->
 grouped expert FFN -> combine) over one batch of T synthetic tokens, inputs
@@ -12,6 +13,9 @@ each step is timed with CUDA events on the launching stream; the max over ranks
 is taken.  With N > 1 (torchrun) every rank runs an independent replica on its
 own batch (replicas only: the layer needs no collective on one node here), so
 scaling is weak and value = tokens of all ranks / max time.
+
+`--mxfp8` runs the routed experts in MXFP8 (E4M3 with one E8M0 scale per 32; the
+opt-in path, MoELayer(mxfp8=True)); routing, shared experts and combine are unchanged.
 
 `--impl reference` times the CPU oracle (float64 numpy, the definition the CUDA
 path is checked against) on host cores over a bounded token sample per step.
@@ -56,6 +60,8 @@ def parse_args():
     ap.add_argument("--tokens", type=int, default=0,
                     help="run the workload's shapes with this many tokens instead of its T "
                          "(serving-sized batches; the line's workload name gets a _t<N> suffix)")
+    ap.add_argument("--mxfp8", action="store_true",
+                    help="routed experts in MXFP8 (the opt-in path); the workload name gets _mxfp8")
     ap.add_argument("--experts", type=int, default=0,
                     help="run the workload with this many routed experts (a multiple of its "
                          "ep_size; reduced cases for profiling; the name gets an _e<N> suffix)")
@@ -310,7 +316,8 @@ def run_ours(args):
     if rank > 0:
         inp["x"] = W.make_x(wl, device="cuda", seed=wl.seed + 1000 * rank)
     cpu_host = None
-    want_cpu = (rank == 0 and ws == 1 and not args.no_cpu_baseline)
+    # (the oracle is the bf16 layer's definition: no CPU baseline for the MXFP8 variant)
+    want_cpu = (rank == 0 and ws == 1 and not args.no_cpu_baseline and not args.mxfp8)
     if want_cpu:
         # keeps the drawn weights (bf16, on the device) for the oracle to fetch per expert
         cpu_host = HostOracleInputs(wl, inp)
@@ -318,7 +325,8 @@ def run_ours(args):
     layer = M.MoELayer(D=wl.D, E=wl.E, ep_size=wl.ep_size, top_k=wl.top_k, F=wl.F,
                        w_router=inp["w_router"], w_gate_up=up, w_down=inp["w_down"],
                        expert_bias=inp["bias"], ws_gate_up=inp["ws_gate_up"], ws_down=inp["ws_down"],
-                       act=wl.act, renormalize=wl.renormalize, x_dtype=wl.x_dtype)
+                       act=wl.act, renormalize=wl.renormalize, x_dtype=wl.x_dtype, mxfp8=args.mxfp8)
+    mx = args.mxfp8
     torch.cuda.synchronize()
     for key in ("w_gate_up", "w1", "w_down", "ws_gate_up", "ws_down"):
         inp.pop(key, None)
@@ -339,6 +347,14 @@ def run_ours(args):
 
     x_bf = x if wl.x_dtype == "bf16" else None
 
+    def expert_ffn():
+        if mx:
+            M.moe_expert_ffn_mxfp8(cfg, b["x_perm"], x_bf, b["expert_offsets"], layer.packed,
+                                   layer.packed_mx, b["y_perm"], b["shared_out"], b["workspace"],
+                                   b["status"], stream)
+        else:
+            M.moe_expert_ffn(cfg, b["x_perm"], x_bf, b["expert_offsets"], layer.packed, b["act"],
+                             b["y_perm"], b["shared_out"], b["workspace"], b["status"], stream)
 
     def stages(ev):
         ev[0].record(stream)
@@ -350,8 +366,7 @@ def run_ours(args):
         ev[2].record(stream)
         M.moe_dispatch_permute(cfg, x, b["pos"], b["x_perm"], stream)
         ev[3].record(stream)
-        M.moe_expert_ffn(cfg, b["x_perm"], x_bf, b["expert_offsets"], layer.packed, b["act"],
-                         b["y_perm"], b["shared_out"], b["workspace"], b["status"], stream)
+        expert_ffn()
         ev[4].record(stream)
         M.moe_combine_unpermute(cfg, b["y_perm"], b["pos"], b["topk_w"], x, b["shared_out"],
                                 b["out"], stream)
@@ -365,8 +380,7 @@ def run_ours(args):
                              b["rank_offsets"], b["pos"], b["src"], b["x_perm"], b["workspace"],
                              b["status"], stream)
         ev[1].record(stream)
-        M.moe_expert_ffn(cfg, b["x_perm"], x_bf, b["expert_offsets"], layer.packed, b["act"],
-                         b["y_perm"], b["shared_out"], b["workspace"], b["status"], stream)
+        expert_ffn()
         ev[2].record(stream)
         M.moe_combine_unpermute(cfg, b["y_perm"], b["pos"], b["topk_w"], x, b["shared_out"],
                                 b["out"], stream)
@@ -380,12 +394,12 @@ def run_ours(args):
     fused = M.moe_route_dispatch_is_fused(cfg)
 
     mk = lambda n=6: [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-    # the stage-by-stage step is moe_forward: check once that both give the same bits
+    # the stage-by-stage step is the layer's forward: check once that both give the same bits
     stages(mk())
     ref_out = b["out"].clone()
     layer.forward(x, stream)
     torch.cuda.synchronize()
-    assert torch.equal(ref_out, b["out"]), "stage-by-stage step differs from moe_forward"
+    assert torch.equal(ref_out, b["out"]), "stage-by-stage step differs from the layer's forward"
     layer.check_status()
 
     for _ in range(args.warmup):
@@ -457,11 +471,7 @@ def run_ours(args):
             stream.wait_event(up_done[i])
             if i >= NBUF:
                 stream.wait_event(dn_done[i - NBUF])           # out_dev[j] already read back
-            M.moe_forward(cfg, x_dev[j], layer.w_router, layer.expert_bias, layer.packed, None,
-                          b["topk_idx"], b["topk_w"], b["counts"], b["expert_offsets"],
-                          b["rank_splits"], b["rank_offsets"], b["pos"], b["src"], b["x_perm"],
-                          b["act"], b["y_perm"], b["shared_out"], out_dev[j], b["workspace"],
-                          b["status"], stream)
+            layer.forward_into(x_dev[j], out_dev[j], stream)      # moe_forward (bf16 path)
             fw_done[i].record(stream)
             with torch.cuda.stream(d2h):
                 d2h.wait_event(fw_done[i])
@@ -490,11 +500,13 @@ def run_ours(args):
     ffn_ms = stage_ms[3] / args.steps
     ffn_tflops = wl.ffn_flop() / (ffn_ms / 1e3) / 1e12
     peak_key = "bf16_tflops"
-    peak_tf = peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
-    sust_tf = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    # MXFP8: dense fp8 runs at twice the bf16 rate (nominal ratio) on the measured figure
+    pmul = 2.0 if mx else 1.0
+    peak_tf = pmul * peaks.get(peak_key, FALLBACK_PEAKS[peak_key])
+    sust_tf = pmul * peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "ffn_traffic.json")
-    if os.path.exists(tpath):
+    if os.path.exists(tpath) and not mx:
         try:
             import hashlib
             with open(tpath) as f:
@@ -509,7 +521,9 @@ def run_ours(args):
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     disp_gbs = disp_b / (stage_ms[2] / args.steps / 1e3) / 1e9
     comb_gbs = comb_b / (stage_ms[4] / args.steps / 1e3) / 1e9
-    launches_per_step = (1 if fused else route_launches(wl) + 1 + 1) + ffn_launches(wl) + 1
+    # MXFP8 FFN: x_perm quantiser, gate_up, down, and the shared experts' launch
+    n_ffn = (3 + (1 if wl.n_shared else 0)) if mx else ffn_launches(wl)
+    launches_per_step = (1 if fused else route_launches(wl) + 1 + 1) + n_ffn + 1
 
     # layer roofline: the sum of every stage's ideal time over the measured step.  Ideal
     # times: route = max(bytes / HBM, flop / fp32 peak), the fp32 peak from the unit counts
@@ -520,7 +534,7 @@ def run_ours(args):
     fp32_tf = sms * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
     hit = int((b["counts"][:wl.E] > 0).sum().item())
     mats = 3 if wl.act == "swiglu" else 2
-    w_bytes = hit * mats * wl.D * wl.F * 2 + wl.n_shared * 3 * wl.D * wl.F_shared * 2
+    w_bytes = hit * mats * wl.D * wl.F * (1 if mx else 2) + wl.n_shared * 3 * wl.D * wl.F_shared * 2
     hbm_bs = hbm * 1e9
     ideal_us = {
         "route": 1e6 * max((wl.T * wl.D * sx + wl.E * wl.D * 4 + wl.R * 8) / hbm_bs,
@@ -538,20 +552,26 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "T": wl.T, "D": wl.D, "E": wl.E, "ep_size": wl.ep_size,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "mxfp8 routed experts (e4m3, e8m0 per 32), bf16 elsewhere" if mx else "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name + ("_mxfp8" if mx else ""), "T": wl.T, "D": wl.D, "E": wl.E, "ep_size": wl.ep_size,
                    "top_k": wl.top_k, "F": wl.F, "act": wl.act, "n_shared": wl.n_shared,
                    "F_shared": wl.F_shared, "router": "fp32", "parallelism": f"replicas{ws}",
                    "l2": "flushed before every timed step: 256 MiB write, then a read of it (no dirty lines left)"},
         "roofline": {"bound": "tensor", "achieved": ffn_tflops, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": ffn_tflops / peak_tf, "traffic": traffic,
-                     "kernel": ("grouped_gemm_pair_kernel, one launch" if ffn_launches(wl) == 1
-                                else "grouped_gemm_kernel launches")
-                               + " (expert FFN stage: routed gate_up+down"
-                               + (", shared gate_up+down" if wl.n_shared else "") + ")",
+                     "kernel": (("mx_quant_a_kernel + grouped_gemm_mx_kernel x2 (routed gate_up, "
+                                 "down; MXFP8)" + (" + shared experts' bf16 launch" if wl.n_shared else ""))
+                                if mx else
+                                ("grouped_gemm_pair_kernel, one launch" if ffn_launches(wl) == 1
+                                 else "grouped_gemm_kernel launches")
+                                + " (expert FFN stage: routed gate_up+down"
+                                + (", shared gate_up+down" if wl.n_shared else "") + ")"),
                      "timed": "CUDA events around the FFN stage call in a stage-by-stage pass "
                               "of the same kernels, after an L2 flush per step",
-                     "peak_source": f"{peak_src} bf16 burst (cuBLAS 8192^3, best of 10)",
+                     "peak_source": (f"2 x {peak_src} bf16 burst (fp8 dense = 2 x bf16, nominal ratio)"
+                                     if mx else f"{peak_src} bf16 burst (cuBLAS 8192^3, best of 10)"),
                      "frac_of_sustained": ffn_tflops / sust_tf},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * wl.D * sx,
                 "d2h_bytes_per_step": T * wl.D * sx},

@@ -24,6 +24,11 @@
 // projection tile the same groups the same way, so the epilogue of up tile t writes the
 // scales of down tile t.
 //
+// The last tile of a group with at most 128 rows left runs as M = 128 (64 rows per CTA):
+// its A scales use the same blocks (rows 0..63 of each), B's scales go to lane quarters
+// 0-1 (rows 0..127) and 2-3 (rows 128..255), and the accumulator holds the CTA's row i in
+// lane i for tile columns [0, 128) and in lane 64 + i for [128, 256).
+//
 // A CTA pair, 10 warps per CTA:
 //   warp 0      TMA producer (lane 0, both CTAs): this CTA's 128 A rows, its 128 B rows,
 //               its A scale block and both B scale blocks of each K step into a 6-stage
@@ -53,6 +58,7 @@ constexpr int kMxTileM = 256;
 
 struct MxArgs {
   CUtensorMap tmap_a;        // E4M3 [rows, K], box 128 x 128 rows
+  CUtensorMap tmap_a64;      // the same, box 128 x 64 rows (half tiles)
   CUtensorMap tmap_b;        // E4M3 [G, N, K], box 128 x 128 x 1
   CUtensorMap tmap_sfa;      // A scale blocks as [bytes / 256, 256], box 256 x 2 (one block)
   CUtensorMap tmap_sfb;      // B scale blocks, box 256 x 4 (both halves of a K step)
@@ -62,6 +68,7 @@ struct MxArgs {
   int32_t ldo;
   uint8_t* q_out;            // EPI_SWIGLU / EPI_GELU: E4M3 activation [rows, ldo]
   uint8_t* q_sf;             //   and its scale blocks (ldo / 128 K steps)
+  int32_t half;              // run a group's last <= 128 rows as an M = 128 tile
   int32_t* status;
   int32_t* counter;          // tile counter, zero at launch
 };
@@ -119,6 +126,26 @@ __host__ __device__ __forceinline__ size_t mx_sf_offset(int64_t t, int ksteps, i
 
 __device__ __forceinline__ int mx_mtiles(int rows) { return (rows + kMxTileM - 1) / kMxTileM; }
 
+// M tile m of a group of `rows` rows is a half tile (M = 128: 64 rows per CTA) when at
+// most 128 rows are left for it and half tiles are enabled; otherwise M = 256.
+__device__ __forceinline__ bool mx_is_half(int rows, int m, int half) {
+  return half && rows - m * kMxTileM <= 128;
+}
+
+// Place of tile row `within` (0..255) in the scale blocks: CTA half h and row m in it
+// (M = 256: 128 rows per CTA; M = 128: 64).
+__device__ __forceinline__ void mx_row_place(int within, bool half_tile, int& h, int& m) {
+  if (half_tile) { h = within >> 6; m = within & 63; }
+  else { h = within >> 7; m = within & 127; }
+}
+
+// 64 rows of 16 bytes: rows 0..31 into lane quarters 0 and 1, rows 32..63 into quarters 2
+// and 3 (the scale layout of B for an M = 128 pair MMA; measured: the ::02_13 form gives
+// wrong products there).
+__device__ __forceinline__ void tc_cp_sf_pair_64(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.64x128b.warpx2::01_23 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // E8M0 exponent of a block from its largest magnitude: floor(log2 amax) - 8, clamped to
 // [-127, 127] (-127 for a zero block; a subnormal amax also lands on -127).
 __device__ __forceinline__ int mx_exponent(float amax) {
@@ -144,6 +171,26 @@ __device__ __forceinline__ uint8_t mx_quant32(const float (&v)[32], uint8_t* dst
   d[0] = out[0];
   d[1] = out[1];
   return (uint8_t)(s + 127);
+}
+
+__device__ __forceinline__ void store32(bf16* dst, const uint32_t (&v)[32]) {
+  float f[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+  store_row32(dst, f);
+}
+__device__ __forceinline__ uint8_t quant_swiglu32(const uint32_t (&gate)[32], const uint32_t (&up)[32],
+                                                  uint8_t* dst) {
+  float f[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) f[i] = silu_f(__uint_as_float(gate[i])) * __uint_as_float(up[i]);
+  return mx_quant32(f, dst);
+}
+__device__ __forceinline__ uint8_t quant_gelu32(const uint32_t (&v)[32], uint8_t* dst) {
+  float f[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) f[i] = gelu_f(__uint_as_float(v[i]));
+  return mx_quant32(f, dst);
 }
 
 template <int EPI>
@@ -189,6 +236,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&p.tmap_a);
+    prefetch_tmap(&p.tmap_a64);
     prefetch_tmap(&p.tmap_b);
     prefetch_tmap(&p.tmap_sfa);
     prefetch_tmap(&p.tmap_sfb);
@@ -217,7 +265,6 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
     if (lane == 0) {
       // ---------------- TMA producer (both CTAs; the leader's also schedules) ----------------
       const uint32_t full0_leader = map_to_cta(full0, 0);
-      constexpr uint32_t stage_tx = 2u * (uint32_t)C::kStageBytes;
       int stage = 0;
       uint32_t phase = 0;
       int next = leader ? atomicAdd(p.counter, 1) : 0;
@@ -228,7 +275,10 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
         if (tile < 0) break;
         int g, m, n;
         decode_tile(tile, mt, G, nb, g, m, n);
-        const int arow = off[g] + m * kMxTileM + (int)rank * 128;
+        const bool hf = mx_is_half(off[g + 1] - off[g], m, p.half);
+        const int arow = off[g] + m * kMxTileM + (int)rank * (hf ? 64 : 128);
+        const CUtensorMap* amap = hf ? &p.tmap_a64 : &p.tmap_a;
+        const uint32_t stage_tx = 2u * (uint32_t)(C::kStageBytes - (hf ? C::kABytes / 2 : 0));
         const int brow = n * BN + (int)rank * 128;
         const int64_t ta = (int64_t)mt[g] + m;              // A's tile (scale blocks)
         const int64_t tb = (int64_t)g * nb + n;              // B's tile
@@ -237,7 +287,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
           if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, stage_tx);
           const uint32_t fb = full0_leader + 8 * stage;
-          tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), &p.tmap_a, fb, kb * C::KS, arow);
+          tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), amap, fb, kb * C::KS, arow);
           tma_load_3d_pair(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * C::KS, brow, g);
           tma_load_2d_pair(smem_u32(sfa_smem + stage * C::kSfaBytes), &p.tmap_sfa, fb, 0,
                            (int)(((ta * ksteps + kb) * 2 + rank) * 2));
@@ -258,6 +308,9 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
       for (int qi = 0;; ++qi) {
         const int tile = tq_take<false>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
         if (tile < 0) break;
+        int g, m, n;
+        decode_tile(tile, mt, G, nb, g, m, n);
+        const bool hf = mx_is_half(off[g + 1] - off[g], m, p.half);
         if (!mbar_wait(tempty, acc_phase ^ 1u, abort_flag, p.status)) break;
         acc_phase ^= 1u;
         tc_fence_after();
@@ -268,13 +321,20 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
           const uint32_t sa = smem_u32(sfa_smem + stage * C::kSfaBytes);
           const uint32_t sb = smem_u32(sfb_smem + stage * C::kSfbBytes);
           tc_cp_sf_pair(t_sfa, sf_desc(sa));
-          tc_cp_sf_pair(t_sfb, sf_desc(sb));              // B rows 0..127 of the tile
-          tc_cp_sf_pair(t_sfb + 4, sf_desc(sb + 512));    // B rows 128..255
+          if (!hf) {
+            // M = 256: B's scales for rows n (0..255) in lane n % 32 of every quarter, column n / 32
+            tc_cp_sf_pair(t_sfb, sf_desc(sb));              // B rows 0..127 of the tile
+            tc_cp_sf_pair(t_sfb + 4, sf_desc(sb + 512));    // B rows 128..255
+          } else {
+            // M = 128: rows 0..127 in lane quarters 0 and 1, rows 128..255 in quarters 2 and 3
+            tc_cp_sf_pair_64(t_sfb, sf_desc(sb));
+          }
           const uint64_t ad = sw128_desc(smem_u32(a_smem + stage * C::kABytes));
           const uint64_t bd = sw128_desc(smem_u32(b_smem + stage * C::kBBytes));
+          const int mm = hf ? kMxTileM / 2 : kMxTileM;
 #pragma unroll
           for (int j = 0; j < 4; ++j)          // K = 32 per MMA: +32 bytes
-            tc_mma_mx_pair(tmem_base, ad + 2 * j, bd + 2 * j, mx_idesc(kMxTileM, BN, j), (kb | j) != 0,
+            tc_mma_mx_pair(tmem_base, ad + 2 * j, bd + 2 * j, mx_idesc(mm, BN, j), (kb | j) != 0,
                            t_sfa | ((uint32_t)j << 30), t_sfb | ((uint32_t)j << 30));
           tc_commit_pair_both(empty0 + 8 * stage);
           if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -299,68 +359,75 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
       if (!__all_sync(0xffffffffu, ok)) break;
       acc_phase ^= 1u;
       tc_fence_after();
-      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * 128);
+      const bool hf = mx_is_half(off[g + 1] - off[g], m, p.half);
+      // M = 256: this CTA's rows 0..127 in lanes 0..127, tile columns 0..255; this warp takes
+      //   columns 128 h .. + 127 of lanes 32 q ...
+      // M = 128: this CTA's rows 0..63 in lanes 0..63 for tile columns [0, 128) and in lanes
+      //   64..127 for [128, 256), at TMEM columns 0..127; this warp takes 64 of them (SwiGLU:
+      //   32 gate and the matching 32 up columns).
+      const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16);
       uint32_t v0[32], v1[32], v2[32], v3[32];
-      tmem_ld32(tbase, v0);
-      tmem_ld32(tbase + 32, v1);
-      tmem_ld32(tbase + 64, v2);
-      tmem_ld32(tbase + 96, v3);
+      if (!hf) {
+        tmem_ld32(tl + h * 128, v0);
+        tmem_ld32(tl + h * 128 + 32, v1);
+        tmem_ld32(tl + h * 128 + 64, v2);
+        tmem_ld32(tl + h * 128 + 96, v3);
+      } else if (EPI == EPI_SWIGLU) {
+        tmem_ld32(tl + h * 32, v0);
+        tmem_ld32(tl + 64 + h * 32, v2);
+      } else {
+        tmem_ld32(tl + h * 64, v0);
+        tmem_ld32(tl + h * 64 + 32, v1);
+      }
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader);      // the accumulator may be reused
-      const int r = q * 32 + lane;
-      const int64_t row = (int64_t)off[g] + m * kMxTileM + (int)rank * 128 + r;
+      const int r = hf ? (q & 1) * 32 + lane : q * 32 + lane;
+      const int64_t row = (int64_t)off[g] + m * kMxTileM + (int)rank * (hf ? 64 : 128) + r;
+      // the activation's scales go to the down projection's tile mt[g] + m (the same
+      // tiling), CTA half `rank`, row r
+      const int qk = p.ldo / C::KS;
+      const int64_t t = (int64_t)mt[g] + m;
       if (row >= off[g + 1]) {
         // a row past the group's end: nothing to store
-      } else if (EPI == EPI_STORE) {
-        bf16* dst = p.out + row * p.ldo + n * BN + h * 128;
-        float f[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v0[i]);
-        store_row32(dst, f);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v1[i]);
-        store_row32(dst + 32, f);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v2[i]);
-        store_row32(dst + 64, f);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v3[i]);
-        store_row32(dst + 96, f);
-      } else {
-        // the activation, quantised for the down projection: this row's scales go to the
-        // down projection's tile mt[g] + m (the same tiling), half `rank`, row r
-        const int qk = p.ldo / C::KS;
-        const int64_t t = (int64_t)mt[g] + m;
-        float f[32];
-        if (EPI == EPI_SWIGLU) {
+      } else if (!hf) {
+        if (EPI == EPI_STORE) {
+          bf16* dst = p.out + row * p.ldo + n * BN + h * 128;
+          store32(dst, v0);
+          store32(dst + 32, v1);
+          store32(dst + 64, v2);
+          store32(dst + 96, v3);
+        } else if (EPI == EPI_SWIGLU) {
           // [gate 64 | up 64] -> outputs n*128 + 64h + [0, 64): K step n, blocks 2h, 2h + 1
-          const int oc = n * 128 + h * 64;
-          uint8_t* dst = p.q_out + row * p.ldo + oc;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) f[i] = silu_f(__uint_as_float(v0[i])) * __uint_as_float(v2[i]);
-          p.q_sf[mx_sf_offset(t, qk, n, (int)rank, r, 2 * h)] = mx_quant32(f, dst);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) f[i] = silu_f(__uint_as_float(v1[i])) * __uint_as_float(v3[i]);
-          p.q_sf[mx_sf_offset(t, qk, n, (int)rank, r, 2 * h + 1)] = mx_quant32(f, dst + 32);
+          uint8_t* dst = p.q_out + row * p.ldo + n * 128 + h * 64;
+          p.q_sf[mx_sf_offset(t, qk, n, (int)rank, r, 2 * h)] = quant_swiglu32(v0, v2, dst);
+          p.q_sf[mx_sf_offset(t, qk, n, (int)rank, r, 2 * h + 1)] = quant_swiglu32(v1, v3, dst + 32);
         } else {
           // GELU: outputs n*256 + 128h + [0, 128): K step 2n + h, blocks 0..3
-          const int oc = n * BN + h * 128;
+          uint8_t* dst = p.q_out + row * p.ldo + n * BN + h * 128;
           const int s = 2 * n + h;
-          uint8_t* dst = p.q_out + row * p.ldo + oc;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) f[i] = gelu_f(__uint_as_float(v0[i]));
-          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 0)] = mx_quant32(f, dst);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) f[i] = gelu_f(__uint_as_float(v1[i]));
-          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 1)] = mx_quant32(f, dst + 32);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) f[i] = gelu_f(__uint_as_float(v2[i]));
-          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 2)] = mx_quant32(f, dst + 64);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) f[i] = gelu_f(__uint_as_float(v3[i]));
-          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 3)] = mx_quant32(f, dst + 96);
+          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 0)] = quant_gelu32(v0, dst);
+          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 1)] = quant_gelu32(v1, dst + 32);
+          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 2)] = quant_gelu32(v2, dst + 64);
+          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 3)] = quant_gelu32(v3, dst + 96);
+        }
+      } else {
+        const int cq = q >> 1;               // tile columns 128 cq .. 128 cq + 127
+        if (EPI == EPI_STORE) {
+          bf16* dst = p.out + row * p.ldo + n * BN + cq * 128 + h * 64;
+          store32(dst, v0);
+          store32(dst + 32, v1);
+        } else if (EPI == EPI_SWIGLU) {
+          // outputs n*128 + 64 cq + 32 h + [0, 32): K step n, block 2 cq + h
+          uint8_t* dst = p.q_out + row * p.ldo + n * 128 + cq * 64 + h * 32;
+          p.q_sf[mx_sf_offset(t, qk, n, (int)rank, r, 2 * cq + h)] = quant_swiglu32(v0, v2, dst);
+        } else {
+          // outputs n*256 + 128 cq + 64 h + [0, 64): K step 2n + cq, blocks 2h, 2h + 1
+          uint8_t* dst = p.q_out + row * p.ldo + n * BN + cq * 128 + h * 64;
+          const int s = 2 * n + cq;
+          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 2 * h)] = quant_gelu32(v0, dst);
+          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 2 * h + 1)] = quant_gelu32(v1, dst + 32);
         }
       }
       __syncwarp();
@@ -448,7 +515,7 @@ mx_block_scales_kernel(const uint32_t* __restrict__ rowmajor, uint8_t* __restric
 // search of the offsets), its M tile and place in it, then 32-element blocks lane-strided.
 __global__ void __launch_bounds__(256)
 mx_quant_a_kernel(const bf16* __restrict__ x, const int32_t* __restrict__ group_offsets, int G, int K,
-                  uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+                  int half, uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
   extern __shared__ int sh[];
   int* mt = sh;                 // [G + 1]
   int* off = sh + (G + 1);      // [G + 1]
@@ -468,7 +535,8 @@ mx_quant_a_kernel(const bf16* __restrict__ x, const int32_t* __restrict__ group_
     }
     const int rr = r - off[lo];
     const int64_t t = (int64_t)mt[lo] + rr / kMxTileM;
-    const int within = rr % kMxTileM, h = within >> 7, m = within & 127;
+    int h, m;
+    mx_row_place(rr % kMxTileM, mx_is_half(off[lo + 1] - off[lo], rr / kMxTileM, half), h, m);
     for (int b = lane; b < nblk; b += 32) {
       const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)r * K + b * 32);
       float v[32];
@@ -505,14 +573,14 @@ cudaError_t launch_mx_block_scales(const uint8_t* rowmajor, uint8_t* blocked, in
 }
 
 cudaError_t launch_mx_quant_a(const bf16* x, int64_t rows, const int32_t* group_offsets, int G, int K,
-                              uint8_t* q, uint8_t* sf, cudaStream_t s) {
+                              int half_tiles, uint8_t* q, uint8_t* sf, cudaStream_t s) {
   if (K % MxCfg::KS != 0 || G <= 0) return cudaErrorInvalidValue;
   if (rows == 0) return cudaSuccess;
   const size_t smem = (2 * (size_t)(G + 1) + 8) * sizeof(int);
   if (smem > 48 * 1024) return cudaErrorInvalidValue;
   int64_t grid = (rows + 7) / 8;                 // 8 rows (warps) per block
   if (grid > 4 * (int64_t)sm_count()) grid = 4 * (int64_t)sm_count();
-  mx_quant_a_kernel<<<(int)grid, 256, smem, s>>>(x, group_offsets, G, K, q, sf);
+  mx_quant_a_kernel<<<(int)grid, 256, smem, s>>>(x, group_offsets, G, K, half_tiles, q, sf);
   return cudaGetLastError();
 }
 
@@ -527,7 +595,8 @@ cudaError_t launch_grouped_mx(const MxProblem& p, cudaStream_t s) {
   memset(&a, 0, sizeof(a));
   const uint64_t da[2] = {(uint64_t)p.K, (uint64_t)p.a_rows};
   const uint64_t db[3] = {(uint64_t)p.K, (uint64_t)p.N, (uint64_t)p.G};
-  if (!make_map_u8(&a.tmap_a, p.A, 2, da, 128) || !make_map_u8(&a.tmap_b, p.B, 3, db, 128) ||
+  if (!make_map_u8(&a.tmap_a, p.A, 2, da, 128) || !make_map_u8(&a.tmap_a64, p.A, 2, da, 64) ||
+      !make_map_u8(&a.tmap_b, p.B, 3, db, 128) ||
       !make_map_sf(&a.tmap_sfa, p.sa, mx_sf_bytes(tiles_m, p.K), 2) ||
       !make_map_sf(&a.tmap_sfb, p.sb, mx_sf_bytes((int64_t)p.G * (p.N / MxCfg::BN), p.K), 4))
     return cudaErrorInvalidValue;
@@ -539,6 +608,7 @@ cudaError_t launch_grouped_mx(const MxProblem& p, cudaStream_t s) {
   a.ldo = p.ldo;
   a.q_out = p.q_out;
   a.q_sf = p.q_sf;
+  a.half = p.half_tiles;
   a.status = p.status;
   a.counter = p.counter;
   const int64_t tiles = tiles_m * (int64_t)(p.N / MxCfg::BN);

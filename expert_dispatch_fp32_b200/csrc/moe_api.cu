@@ -700,9 +700,12 @@ moe_status moe_expert_ffn_mxfp8(const moe_config* cfg, const void* x_perm, const
   const int nup = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
   int32_t* ctr = (int32_t*)(ws + L.counters);
   if (R > 0) {
+    // a group's last <= 128 rows run as an M = 128 tile (MOE_MX_HALF=0: as M = 256, for comparison)
+    const char* half_env = getenv("MOE_MX_HALF");
+    const int half = (half_env && half_env[0] == '0') ? 0 : 1;
     cudaError_t err = cudaMemsetAsync(ctr, 0, 2 * sizeof(int32_t), s);
     if (err == cudaSuccess)
-      err = launch_mx_quant_a((const bf16*)x_perm, R, expert_offsets, c.E, c.D, ws + L.xq, ws + L.xsf, s);
+      err = launch_mx_quant_a((const bf16*)x_perm, R, expert_offsets, c.E, c.D, half, ws + L.xq, ws + L.xsf, s);
     // gate_up (or W1): the activation comes out quantised, with the down projection's scales
     MxProblem up;
     memset(&up, 0, sizeof(up));
@@ -712,6 +715,7 @@ moe_status moe_expert_ffn_mxfp8(const moe_config* cfg, const void* x_perm, const
     up.group_offsets = expert_offsets;
     up.q_out = ws + L.aq; up.q_sf = ws + L.asf; up.ldo = c.F;
     up.epi = c.act == MOE_ACT_SWIGLU ? EPI_SWIGLU : EPI_GELU;
+    up.half_tiles = half;
     up.status = status; up.counter = ctr;
     if (err == cudaSuccess) err = launch_grouped_mx(up, s);
     MxProblem dn = up;

@@ -37,11 +37,15 @@ class MoELayer:
     [E, F, D]; ws_gate_up bf16 [S, D, 2Fs] and ws_down bf16 [S, Fs, D] or None.
     The expert weights are repacked once at construction (moe_prepare_weights);
     the caller may drop its copies afterwards.
+
+    mxfp8=True runs the routed experts in MXFP8 (moe_expert_ffn_mxfp8: E4M3 operands with
+    one E8M0 scale per 32, quantised once for the weights at construction and per batch
+    for the rows); routing, the shared experts and the combine stay as in the bf16 path.
     """
 
     def __init__(self, *, D, E, ep_size, top_k, F, w_router, w_gate_up, w_down, expert_bias=None,
                  ws_gate_up=None, ws_down=None, act="swiglu", renormalize=True, x_dtype="bf16",
-                 keep_router_logits=False, stream=None):
+                 keep_router_logits=False, mxfp8=False, stream=None):
         self.D, self.E, self.ep_size, self.top_k, self.F = D, E, ep_size, top_k, F
         self.act, self.renormalize, self.x_dtype = act, renormalize, x_dtype
         self.n_shared = 0 if ws_gate_up is None else ws_gate_up.shape[0]
@@ -55,6 +59,14 @@ class MoELayer:
         B.moe_prepare_weights(cfg, w_gate_up.contiguous(), w_down.contiguous(),
                               None if ws_gate_up is None else ws_gate_up.contiguous(),
                               None if ws_down is None else ws_down.contiguous(), self.packed, stream)
+        self.mxfp8 = bool(mxfp8)
+        self.packed_mx = None
+        if self.mxfp8:
+            n = B.moe_packed_weights_mxfp8_size(cfg)
+            if n == 0:
+                raise B.MoeError("moe_packed_weights_mxfp8_size", B.MOE_ERR_UNSUPPORTED)
+            self.packed_mx = _empty(n, torch.uint8, self.device)
+            B.moe_prepare_weights_mxfp8(cfg, self.packed, self.packed_mx, stream)
         self._bufT = None
         self.buf = {}
 
@@ -81,7 +93,8 @@ class MoELayer:
             y_perm=_empty((R, D), torch.bfloat16, dev),
             shared_out=_empty((T, D), torch.bfloat16, dev) if self.n_shared else None,
             out=_empty((T, D), xdt, dev),
-            workspace=_empty(max(B.moe_workspace_size(cfg), 256), torch.uint8, dev),
+            workspace=_empty(max(B.moe_workspace_mxfp8_size(cfg) if self.mxfp8 else
+                                 B.moe_workspace_size(cfg), 256), torch.uint8, dev),
             status=torch.zeros(1, dtype=torch.int32, device=dev),
         )
         self._bufT = T
@@ -90,13 +103,30 @@ class MoELayer:
 
     def forward(self, x, stream=None):
         """Enqueue the whole layer on ``stream``; returns the output buffer."""
+        b = self.allocate(x.shape[0])
+        self.forward_into(x, b["out"], stream)
+        return b["out"]
+
+    def forward_into(self, x, out, stream=None):
+        """Enqueue the whole layer on ``stream`` with its output written to ``out``
+        (a device tensor shaped like x)."""
         T = x.shape[0]
         b = self.allocate(T)
-        B.moe_forward(self._cfg, x, self.w_router, self.expert_bias, self.packed, b["logits"],
-                      b["topk_idx"], b["topk_w"], b["counts"], b["expert_offsets"], b["rank_splits"],
-                      b["rank_offsets"], b["pos"], b["src"], b["x_perm"], b["act"], b["y_perm"],
-                      b["shared_out"], b["out"], b["workspace"], b["status"], stream)
-        return b["out"]
+        if not self.mxfp8:
+            B.moe_forward(self._cfg, x, self.w_router, self.expert_bias, self.packed, b["logits"],
+                          b["topk_idx"], b["topk_w"], b["counts"], b["expert_offsets"], b["rank_splits"],
+                          b["rank_offsets"], b["pos"], b["src"], b["x_perm"], b["act"], b["y_perm"],
+                          b["shared_out"], out, b["workspace"], b["status"], stream)
+            return
+        B.moe_route_dispatch(self._cfg, x, self.w_router, self.expert_bias, b["logits"], b["topk_idx"],
+                             b["topk_w"], b["counts"], b["expert_offsets"], b["rank_splits"],
+                             b["rank_offsets"], b["pos"], b["src"], b["x_perm"], b["workspace"],
+                             b["status"], stream)
+        B.moe_expert_ffn_mxfp8(self._cfg, b["x_perm"], x if self.x_dtype == "bf16" else None,
+                               b["expert_offsets"], self.packed, self.packed_mx, b["y_perm"],
+                               b["shared_out"], b["workspace"], b["status"], stream)
+        B.moe_combine_unpermute(self._cfg, b["y_perm"], b["pos"], b["topk_w"], x, b["shared_out"], out,
+                                stream)
 
     __call__ = forward
 

@@ -57,8 +57,11 @@ def _mx_oracle_expert(x_rows, w_up, w_down, act):
     return dq(a) @ wd
 
 
-@pytest.mark.parametrize("case", ["swiglu_shared", "gelu", "deepseek_like"])
-def test_mxfp8_expert_ffn_matches_the_oracle(case):
+@pytest.mark.parametrize("case,half", [("swiglu_shared", "1"), ("gelu", "1"), ("deepseek_like", "1"),
+                                       ("swiglu_shared", "0"), ("deepseek_like", "0")])
+def test_mxfp8_expert_ffn_matches_the_oracle(case, half, monkeypatch):
+    # half "1": a group's last <= 128 rows run as an M = 128 tile (the default); "0": M = 256
+    monkeypatch.setenv("MOE_MX_HALF", half)
     import moe_workloads as W
     from parity_helpers import assert_layer_close, f64, make_layer, up_weights
     wl = {"swiglu_shared": W.Workload(name="mx1", T=300, D=512, E=8, ep_size=2, top_k=2, F=256,
@@ -103,3 +106,41 @@ def test_mxfp8_expert_ffn_matches_the_oracle(case):
     print(f"\n{case}: MXFP8 y_perm vs oracle rel-L2 {err:.2e}; vs the bf16 path {vs_bf16:.2e}")
     if sh is not None:
         assert torch.equal(sh, b["shared_out"])     # the shared experts stay bf16
+
+
+def test_mxfp8_layer_forward_is_its_stages():
+    """MoELayer(mxfp8=True): the forward is route+dispatch, the MXFP8 FFN and the combine
+    (same bits as the calls one by one), and its MoE part stays within the format's error
+    of the bf16 layer's."""
+    import moe_workloads as W
+    from parity_helpers import f64
+    wl = W.Workload(name="mxl", T=640, D=512, E=16, ep_size=4, top_k=4, F=256, n_shared=1,
+                    F_shared=256, seed=41)
+    inp = W.make_inputs(wl, device="cuda")
+    kw = dict(D=wl.D, E=wl.E, ep_size=wl.ep_size, top_k=wl.top_k, F=wl.F, w_router=inp["w_router"],
+              w_gate_up=inp["w_gate_up"], w_down=inp["w_down"], expert_bias=inp["bias"],
+              ws_gate_up=inp["ws_gate_up"], ws_down=inp["ws_down"])
+    ref = M.MoELayer(**kw)
+    mx = M.MoELayer(**kw, mxfp8=True)
+    x = inp["x"]
+    out_ref = ref.forward(x).clone()
+    out = mx.forward(x).clone()
+    torch.cuda.synchronize()
+    mx.check_status()
+    b, cfg = mx.buf, mx.config(wl.T)
+    y = torch.empty_like(b["y_perm"])
+    sh = torch.empty_like(b["shared_out"])
+    o = torch.empty_like(out)
+    M.moe_route_dispatch(cfg, x, mx.w_router, mx.expert_bias, None, b["topk_idx"], b["topk_w"],
+                         b["counts"], b["expert_offsets"], b["rank_splits"], b["rank_offsets"], b["pos"],
+                         b["src"], b["x_perm"], b["workspace"], b["status"])
+    M.moe_expert_ffn_mxfp8(cfg, b["x_perm"], x, b["expert_offsets"], mx.packed, mx.packed_mx, y, sh,
+                           b["workspace"], b["status"])
+    M.moe_combine_unpermute(cfg, y, b["pos"], b["topk_w"], x, sh, o)
+    torch.cuda.synchronize()
+    mx.check_status()
+    assert torch.equal(o, out)
+    moe_mx, moe_ref = f64(out) - f64(x), f64(out_ref) - f64(x)
+    rel = np.linalg.norm(moe_mx - moe_ref) / np.linalg.norm(moe_ref)
+    print(f"\nMoE part, MXFP8 layer vs bf16 layer: rel-L2 {rel:.3e}")
+    assert rel < 0.15
