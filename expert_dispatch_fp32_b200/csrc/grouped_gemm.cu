@@ -83,6 +83,8 @@ struct PairArgs {
   int32_t G, nph;
   int32_t skinny;            // 1: groups of <= 64 rows run as skinny (weights-as-M) tiles
   int32_t fold;              // 1: a last band of 257..320 rows runs as one folded tile
+  int32_t fold_m256;         // 1: a folded remainder is one M = 256 product per K slice (needs
+                             //    the gate/up exchange buffer in shared memory)
   int32_t* status;
   int32_t* counter;          // tile counter, zero at launch
   int32_t* done;             // band completion counts, zero at launch
@@ -306,8 +308,12 @@ struct PairCfg {
   static constexpr int kTmemCols = 2 * BN;
   static constexpr uint32_t kIdesc = make_idesc(2 * kTileM, BN);
   static constexpr uint32_t kIdescHalf = make_idesc(kTileM, BN);
-  static size_t smem_bytes(int G) {
-    return 1024 + (size_t)kStages * kStageBytes + kCtrlBytes + 2 * (size_t)(G + 1) * sizeof(int);
+  // gate/up exchange of a folded remainder's SwiGLU epilogue: 64 slab rows x 16 columns,
+  // then its two mbarriers
+  static constexpr int kFoldXBytes = 64 * 16 * 4 + 16;
+  static size_t smem_bytes(int G, bool fold_x) {
+    const size_t base = 1024 + (size_t)kStages * kStageBytes + kCtrlBytes + 2 * (size_t)(G + 1) * sizeof(int);
+    return fold_x ? ((base + 15) & ~(size_t)15) + kFoldXBytes : base;
   }
 };
 // Largest remainder folded into a single-band group's tile (rows beyond 256).
@@ -418,6 +424,80 @@ __device__ __forceinline__ void epilogue_skinny(int epi, bf16* out, float* outf,
   }
 }
 
+// Epilogue of a folded remainder computed as ONE M = 256 product per K slice (weights as
+// M, the remainder rows as N = ns): in CTA r, TMEM lane m (0..127) holds slab row m of
+// the CTA and columns 0..ns-1 the remainder rows 0..ns-1, which start at row `rbase`.
+// Slab row m is, per 256-wide N block n: paired (SwiGLU / router pairs) the first
+// factor of output n*128 + 64r + m (m < 64) or the second factor of output
+// n*128 + 64r + m - 64; plain: output n*256 + 128r + m.  Paired, the warps holding the
+// second factors (lane quarters 2, 3) pass them through shared memory (xbuf: 64 rows x
+// 16 columns of fp32) to the warps holding the first (quarters 0, 1), 16 columns at a
+// time, handing the buffer over on two mbarriers (xfull: 2 arrivals by the second-factor
+// warps; xempty: 2 by the first-factor warps) with bounded waits.  `xk` counts the
+// hand-overs so far (the same in every epilogue warp).  One element per store (a warp
+// writes 32 consecutive output columns of a row).  Returns false if a wait gave up.
+__device__ __forceinline__ bool epilogue_fold256(int epi, bf16* out, float* outf, int ldo, uint32_t tb,
+                                                 const PairTile& t, int rbase, int rank, int q, int lane,
+                                                 int ns, float* xbuf, uint32_t xfull, uint32_t xempty,
+                                                 uint32_t& xk, volatile int* abort_flag, int32_t* status) {
+  const bool paired = epi == EPI_SWIGLU || epi == EPI_PAIRSUM_F32;
+  for (int c0 = 0; c0 < ns; c0 += 16) {
+    uint32_t v[16];
+    __syncwarp();          // tcgen05.ld is warp-collective: reconverge after the masked stores
+    tmem_ld16(tb + c0, v);
+    tmem_ld_wait();
+    if (!paired) {
+      const int col = t.n * 256 + rank * 128 + q * 32 + lane;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const int64_t row = (int64_t)rbase + c0 + c;
+        if (c0 + c < ns && row < t.end) {
+          const float x = __uint_as_float(v[c]);
+          out[row * ldo + col] = __float2bfloat16_rn(epi == EPI_GELU ? gelu_f(x) : x);
+        }
+      }
+      continue;
+    }
+    const int i = (q & 1) * 32 + lane;              // output among the CTA's 64
+    float4* xr = reinterpret_cast<float4*>(xbuf + i * 16);
+    const uint32_t par = xk & 1u;
+    ++xk;
+    bool ok = true;
+    if (q >= 2) {
+      if (lane == 0) ok = mbar_wait(xempty, par ^ 1u, abort_flag, status);
+      if (!__all_sync(0xffffffffu, ok)) return false;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        xr[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                            __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xfull);
+    } else {
+      if (lane == 0) ok = mbar_wait(xfull, par, abort_flag, status);
+      if (!__all_sync(0xffffffffu, ok)) return false;
+      float u[16];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 f = xr[j];
+        u[4 * j] = f.x; u[4 * j + 1] = f.y; u[4 * j + 2] = f.z; u[4 * j + 3] = f.w;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xempty);           // xbuf may be rewritten
+      const int col = t.n * 128 + rank * 64 + i;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const int64_t row = (int64_t)rbase + c0 + c;
+        if (c0 + c < ns && row < t.end) {
+          const float g = __uint_as_float(v[c]);
+          if (epi == EPI_SWIGLU) out[row * ldo + col] = __float2bfloat16_rn(silu_f(g) * u[c]);
+          else outf[row * ldo + col] = g + u[c];
+        }
+      }
+    }
+  }
+  return true;
+}
+
 // Bounded wait (cycle count) until *cnt >= need, read with acquire semantics.
 __device__ __noinline__ bool wait_count(const int32_t* cnt, int need, volatile int* abort_flag,
                                         int32_t* status) {
@@ -469,6 +549,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
   int* mt = reinterpret_cast<int*>(smem + S * C::kStageBytes + kCtrlBytes);
   const int G = p.G > 0 ? p.G : 1;
   int* off = mt + (G + 1);
+  // gate/up exchange of folded remainders and its two mbarriers (present when p.fold_m256)
+  float* xbuf = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(off + (G + 1)) + 15) & ~(uintptr_t)15);
+  const uint32_t xfull = smem_u32(xbuf + 64 * 16), xempty = xfull + 8;
   const int nph = p.nph;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -485,6 +568,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
     }
     for (int i = 0; i < 2; ++i) mbar_init(tfull0 + 8 * i, 1);
     for (int i = 0; i < 4; ++i) mbar_init(tfree0 + 8 * i, 8);     // 4 epilogue warps x 2 CTAs
+    if (p.fold_m256) {
+      mbar_init(xfull, 2);                 // the two second-factor warps of this CTA
+      mbar_init(xempty, 2);                // the two first-factor warps
+    }
     for (int i = 0; i < kTileQ; ++i) {
       mbar_init(qfull0 + 8 * i, 1);
       // leader: MMA issuer + 4 epilogue warps; peer: producer + 4 epilogue warps
@@ -606,6 +693,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         const uint32_t idesc = kind == TK_FULL || kind == TK_FOLD ? C::kIdesc
                                : kind == TK_HALF ? C::kIdescHalf : make_idesc(kTileM, ns);
         const uint32_t idesc_s = make_idesc(kTileM, ns);        // skinny / folded remainder
+        const uint32_t idesc_f = make_idesc(2 * kTileM, ns);    // folded remainder, M = 256 form
         const int ksteps = p.ph[t.ph].K / kTileK;
         // the TMEM regions this tile writes: this buffer's head, its tail unless skinny,
         // the other buffer's head if folded
@@ -638,11 +726,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
             }
           } else if (kind == TK_FOLD) {
             const uint64_t rd = sw128_desc(smem_u32(r_smem + stage * C::kRemBytes));
+            if (p.fold_m256) {
+              // the remainder as one M = 256 product: both CTAs' whole weight slabs as M
 #pragma unroll
-            for (int kk = 0; kk < kTileK / 16; ++kk) {
-              tc_mma_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
-              tc_mma_pair(s_tmem, bd + 2 * kk, rd + 2 * kk, idesc_s, (kb | kk) != 0);
-              tc_mma_pair(s_tmem + kSkinnyHi, bd_hi + 2 * kk, rd + 2 * kk, idesc_s, (kb | kk) != 0);
+              for (int kk = 0; kk < kTileK / 16; ++kk) {
+                tc_mma_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                tc_mma_pair(s_tmem, bd + 2 * kk, rd + 2 * kk, idesc_f, (kb | kk) != 0);
+              }
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < kTileK / 16; ++kk) {
+                tc_mma_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                tc_mma_pair(s_tmem, bd + 2 * kk, rd + 2 * kk, idesc_s, (kb | kk) != 0);
+                tc_mma_pair(s_tmem + kSkinnyHi, bd_hi + 2 * kk, rd + 2 * kk, idesc_s, (kb | kk) != 0);
+              }
             }
           } else {
 #pragma unroll
@@ -663,6 +760,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
     const uint32_t tfree_leader = map_to_cta(tfree0, 0);
     int acc = 0;
     uint32_t acc_phase = 0;
+    uint32_t xk = 0;             // gate/up hand-overs of folded remainders so far
     // release TMEM region i: this warp has read all of its columns
     auto release = [&](int i) {
       tc_fence_before();
@@ -686,8 +784,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
       const uint32_t tb = tmem_base + lanes + (uint32_t)(acc * BN);
       if (kind == TK_FOLD) {
         // the remainder rows (after the first 256), from the other buffer's head
-        epilogue_skinny(P.epi, P.out, P.outf, P.ldo, tmem_base + lanes + (uint32_t)((acc ^ 1) * BN), t,
-                        t.base + 2 * kTileM, (int)rank, q, lane, ns);
+        const uint32_t tr = tmem_base + lanes + (uint32_t)((acc ^ 1) * BN);
+        if (p.fold_m256) {
+          if (!epilogue_fold256(P.epi, P.out, P.outf, P.ldo, tr, t, t.base + 2 * kTileM, (int)rank, q, lane, ns,
+                                xbuf, xfull, xempty, xk, abort_flag, p.status))
+            break;
+        } else
+          epilogue_skinny(P.epi, P.out, P.outf, P.ldo, tr, t, t.base + 2 * kTileM, (int)rank, q, lane, ns);
         release(acc ^ 1);
       }
       if (kind == TK_SKINNY) {
@@ -700,8 +803,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         const int r = q * 32 + lane;
         const int col0 = paired ? t.n * (BN / 2) : t.n * BN;
         const bool valid = r < min(t.end - row0, kTileM);
-        epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, 0, 64, (int64_t)row0 + r, col0, valid);
-        release(acc);
+        // the head (TMEM columns 0..63) is released as soon as it is in registers: a folded
+        // tile that follows puts its remainder there
+        epilogue_head_rt(P.epi, P.out, P.outf, P.ldo, tb, (int64_t)row0 + r, col0, valid,
+                         [&] { release(acc); });
         epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, 64, paired ? BN / 2 : BN, (int64_t)row0 + r,
                         col0, valid);
         release(2 + acc);
@@ -773,7 +878,7 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t K, uint64_t N, uint6
 }
 
 cudaError_t launch_tc_pair(const PairArgs& a, int clusters, cudaStream_t s) {
-  const size_t smem = PairCfg::smem_bytes(a.group_offsets ? a.G : 1);
+  const size_t smem = PairCfg::smem_bytes(a.group_offsets ? a.G : 1, a.fold_m256 != 0);
   auto kern = grouped_gemm_pair_kernel;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
@@ -825,6 +930,18 @@ int sm_count() {
   return n;
 }
 
+// Largest dynamic shared memory a block may opt in to on this device.
+int smem_optin() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 232448;
+  static int cache[64] = {0};
+  if (dev < 64 && cache[dev]) return cache[dev];
+  int n = 232448;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (dev < 64) cache[dev] = n;
+  return n;
+}
+
 int64_t pair_band_bound(const GemmProblem& p) {
   // 256-row bands of a phase: ceil(rows / 256) for a dense group; for the expert
   // groups at most rows / 256 + G (each group adds at most one partial band)
@@ -853,6 +970,9 @@ cudaError_t launch_grouped_pair(const GemmProblem* probs, int n, int32_t* counte
     a.skinny = (env && env[0] == '0') ? 0 : 1;
     env = getenv("MOE_GEMM_FOLD");
     a.fold = (env && env[0] == '0') ? 0 : 1;
+    // MOE_GEMM_FOLD256=0 runs a folded remainder as two M = 128 products per K slice
+    env = getenv("MOE_GEMM_FOLD256");
+    a.fold_m256 = (a.fold && !(env && env[0] == '0')) ? 1 : 0;
   }
   a.status = probs[0].status;
   a.counter = counter;
@@ -904,6 +1024,9 @@ cudaError_t launch_grouped_pair(const GemmProblem* probs, int n, int32_t* counte
     }
     tiles += (p.max_tiles > 0 ? p.max_tiles : 1);
   }
+  // the M = 256 fold needs its exchange buffer next to the ring (room for about 700 groups)
+  if (a.fold_m256 && PairCfg::smem_bytes(a.group_offsets ? a.G : 1, true) > (size_t)smem_optin())
+    a.fold_m256 = 0;
   const int64_t pairs = sm_count() / 2;
   const int clusters = (int)(tiles < pairs ? tiles : pairs);
   return launch_tc_pair(a, clusters, s);

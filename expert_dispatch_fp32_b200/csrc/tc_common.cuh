@@ -136,6 +136,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -333,6 +342,7 @@ __device__ __forceinline__ void epilogue_row(bf16* out, float* outf, int ldo, ui
     for (int c = cb; c < ce; c += 32) {
       const int tc = (c >> 6) * 128 + (c & 63);
       uint32_t a[32], b[32];
+      __syncwarp();        // tcgen05.ld is warp-collective: reconverge after the masked stores
       tmem_ld32(tb + tc, a);
       tmem_ld32(tb + tc + 64, b);
       tmem_ld_wait();
@@ -351,6 +361,7 @@ __device__ __forceinline__ void epilogue_row(bf16* out, float* outf, int ldo, ui
 #pragma unroll 1
     for (int c = cb; c < ce; c += 32) {
       uint32_t h[32];
+      __syncwarp();        // tcgen05.ld is warp-collective: reconverge after the masked stores
       tmem_ld32(tb + c, h);
       tmem_ld_wait();
       float v[32];
@@ -372,6 +383,56 @@ __device__ __forceinline__ void epilogue_row_rt(int epi, bf16* out, float* outf,
     case EPI_GELU: epilogue_row<EPI_GELU>(out, outf, ldo, tb, cb, ce, row, col0, valid); break;
     case EPI_PAIRSUM_F32: epilogue_row<EPI_PAIRSUM_F32>(out, outf, ldo, tb, cb, ce, row, col0, valid); break;
     default: epilogue_row<EPI_STORE>(out, outf, ldo, tb, cb, ce, row, col0, valid); break;
+  }
+}
+
+// 32 output columns at dst from accumulator values a (and b, paired).
+template <int EPI>
+__device__ __forceinline__ void epilogue_cols32(bf16* out, float* outf, int64_t off, const uint32_t (&a)[32],
+                                                const uint32_t (&b)[32]) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float x = __uint_as_float(a[i]);
+    if (EPI == EPI_SWIGLU) v[i] = silu_f(x) * __uint_as_float(b[i]);
+    else if (EPI == EPI_PAIRSUM_F32) v[i] = x + __uint_as_float(b[i]);
+    else if (EPI == EPI_GELU) v[i] = gelu_f(x);
+    else v[i] = x;
+  }
+  if (EPI == EPI_PAIRSUM_F32) store_row32_f32(outf + off, v);
+  else store_row32(out + off, v);
+}
+
+// The first 64 output columns of a row (TMEM columns 0..63, and 64..127 for a paired
+// epilogue) with the TMEM reads done before `release` runs: the columns' region may be
+// reused as soon as they are in registers, before the math and the stores.
+template <int EPI, class Release>
+__device__ __forceinline__ void epilogue_head(bf16* out, float* outf, int ldo, uint32_t tb, int64_t row,
+                                              int col0, bool valid, Release release) {
+  constexpr bool kPaired = EPI == EPI_SWIGLU || EPI == EPI_PAIRSUM_F32;
+  uint32_t a0[32], a1[32], b0[32], b1[32];
+  tmem_ld32(tb, a0);
+  tmem_ld32(tb + 32, a1);
+  if (kPaired) {
+    tmem_ld32(tb + 64, b0);
+    tmem_ld32(tb + 96, b1);
+  }
+  tmem_ld_wait();
+  release();
+  if (valid) {
+    epilogue_cols32<EPI>(out, outf, row * ldo + col0, a0, b0);
+    epilogue_cols32<EPI>(out, outf, row * ldo + col0 + 32, a1, b1);
+  }
+  __syncwarp();          // the caller's next tcgen05.ld needs the whole warp converged
+}
+template <class Release>
+__device__ __forceinline__ void epilogue_head_rt(int epi, bf16* out, float* outf, int ldo, uint32_t tb,
+                                                 int64_t row, int col0, bool valid, Release release) {
+  switch (epi) {
+    case EPI_SWIGLU: epilogue_head<EPI_SWIGLU>(out, outf, ldo, tb, row, col0, valid, release); break;
+    case EPI_GELU: epilogue_head<EPI_GELU>(out, outf, ldo, tb, row, col0, valid, release); break;
+    case EPI_PAIRSUM_F32: epilogue_head<EPI_PAIRSUM_F32>(out, outf, ldo, tb, row, col0, valid, release); break;
+    default: epilogue_head<EPI_STORE>(out, outf, ldo, tb, row, col0, valid, release); break;
   }
 }
 

@@ -421,12 +421,15 @@ def test_uneven_expert_tiles(act, extra):
     g.manual_seed(5)
     x_perm = torch.randn((T, wl.D), generator=g, device="cuda").to(torch.bfloat16)
     x_bf = inp["x"].to(torch.bfloat16) if shared else None
-    # CTA-pair kernel with skinny tiles and folded remainders (257..320-row last bands as
-    # one tile), without folding, without skinny tiles, then the one-CTA kernel
-    for pair, skinny, fold in (("1", "1", "1"), ("1", "1", "0"), ("1", "0", "1"), ("0", "1", "1")):
+    # CTA-pair kernel with skinny tiles and folded remainders (257..288-row last bands as
+    # one tile; the remainder as one M = 256 product, then as two M = 128 products),
+    # without folding, without skinny tiles, then the one-CTA kernel
+    for pair, skinny, fold, f256 in (("1", "1", "1", "1"), ("1", "1", "1", "0"), ("1", "1", "0", "1"),
+                                     ("1", "0", "1", "1"), ("0", "1", "1", "1")):
         os.environ["MOE_GEMM_CTA_PAIR"] = pair
         os.environ["MOE_GEMM_SKINNY"] = skinny
         os.environ["MOE_GEMM_FOLD"] = fold
+        os.environ["MOE_GEMM_FOLD256"] = f256
         try:
             b["y_perm"].zero_()
             M.moe_expert_ffn(cfg, x_perm, x_bf, b["expert_offsets"], layer.packed, b["act"],
@@ -436,6 +439,7 @@ def test_uneven_expert_tiles(act, extra):
             del os.environ["MOE_GEMM_CTA_PAIR"]
             del os.environ["MOE_GEMM_SKINNY"]
             del os.environ["MOE_GEMM_FOLD"]
+            del os.environ["MOE_GEMM_FOLD256"]
         assert int(b["status"].item()) == 0
         off = b["expert_offsets"].cpu().numpy()
         assert np.array_equal(np.diff(off), counts)
