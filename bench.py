@@ -511,7 +511,9 @@ def run_ours(args):
             import hashlib
             with open(tpath) as f:
                 tj = json.load(f)
-            src = open(os.path.join(ROOT, "expert_dispatch_fp32_b200", "csrc", "grouped_gemm.cu"), "rb").read()
+            # the FFN kernel's source: grouped_gemm.cu and the tcgen05 helpers it includes
+            csrc = os.path.join(ROOT, "expert_dispatch_fp32_b200", "csrc")
+            src = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ("grouped_gemm.cu", "tc_common.cuh"))
             ent = tj.get(wl.name)
             if ent and ent.get("kernel_sha256") == hashlib.sha256(src).hexdigest():
                 traffic = ent["dram_bytes_per_step"]
