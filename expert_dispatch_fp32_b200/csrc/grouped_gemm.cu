@@ -392,7 +392,7 @@ __device__ __forceinline__ void decode_pair_tile(int tile, const int* pstart, in
 // second factor of outputs n*128 + 64r + i; plain outputs: columns n*256 + 128r + i
 // and + 64.  One output element per store (a warp writes 32 consecutive columns).
 constexpr int kSkinnyHi = 32;     // TMEM column offset of the second 64 slab rows' product
-__device__ __forceinline__ void epilogue_skinny(int epi, bf16* out, float* outf, int ldo, uint32_t tb,
+__device__ __noinline__ void epilogue_skinny(int epi, bf16* out, float* outf, int ldo, uint32_t tb,
                                                 const PairTile& t, int rbase, int rank, int q,
                                                 int lane, int ns) {
   uint32_t r0[32], r1[32];
@@ -436,7 +436,9 @@ __device__ __forceinline__ void epilogue_skinny(int epi, bf16* out, float* outf,
 // warps; xempty: 2 by the first-factor warps) with bounded waits.  `xk` counts the
 // hand-overs so far (the same in every epilogue warp).  One element per store (a warp
 // writes 32 consecutive output columns of a row).  Returns false if a wait gave up.
-__device__ __forceinline__ bool epilogue_fold256(int epi, bf16* out, float* outf, int ldo, uint32_t tb,
+// Out of line, like epilogue_skinny: both run on few tiles, and inlined they made the main
+// epilogue's code slower.
+__device__ __noinline__ bool epilogue_fold256(int epi, bf16* out, float* outf, int ldo, uint32_t tb,
                                                  const PairTile& t, int rbase, int rank, int q, int lane,
                                                  int ns, float* xbuf, uint32_t xfull, uint32_t xempty,
                                                  uint32_t& xk, volatile int* abort_flag, int32_t* status) {
@@ -546,6 +548,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
   int* dmt = pstart + kMaxPhases + 1;                           // [kMaxPhases][2]
   int* doff = dmt + 2 * kMaxPhases;                             // [kMaxPhases][2]
   int* wsum = doff + 2 * kMaxPhases;                            // [kGemmThreads / 32]
+  int* any_fold = wsum + kGemmThreads / 32;                     // 1: some group folds
   int* mt = reinterpret_cast<int*>(smem + S * C::kStageBytes + kCtrlBytes);
   const int G = p.G > 0 ? p.G : 1;
   int* off = mt + (G + 1);
@@ -600,9 +603,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   __syncthreads();
+  if (threadIdx.x == 0) *any_fold = 0;
   if (p.group_offsets != nullptr) {
     const int fold = p.fold;
     group_tile_prefix(off, G, mt, wsum, [fold](int rows) { return pair_mtiles(rows, fold); });
+    if (fold) {
+      for (int g = threadIdx.x; g < G; g += blockDim.x) {
+        const int rows = off[g + 1] - off[g];
+        if (rows > 2 * kTileM && rows <= 2 * kTileM + kFoldMax) atomicOr(any_fold, 1);
+      }
+    }
   }
   if (threadIdx.x == 0) {          // tile numbering: phase after phase
     int acc_t = 0;
@@ -803,10 +813,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         const int r = q * 32 + lane;
         const int col0 = paired ? t.n * (BN / 2) : t.n * BN;
         const bool valid = r < min(t.end - row0, kTileM);
-        // the head (TMEM columns 0..63) is released as soon as it is in registers: a folded
-        // tile that follows puts its remainder there
-        epilogue_head_rt(P.epi, P.out, P.outf, P.ldo, tb, (int64_t)row0 + r, col0, valid,
-                         [&] { release(acc); });
+        if (*any_fold) {
+          // the head (TMEM columns 0..63) is released as soon as it is in registers: a
+          // folded tile that follows puts its remainder there
+          epilogue_head_rt(P.epi, P.out, P.outf, P.ldo, tb, (int64_t)row0 + r, col0, valid,
+                           [&] { release(acc); });
+        } else {
+          // no folded tile waits for a head: loads and stores interleaved, 32 columns at a time
+          epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, 0, 64, (int64_t)row0 + r, col0, valid);
+          release(acc);
+        }
         epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, 64, paired ? BN / 2 : BN, (int64_t)row0 + r,
                         col0, valid);
         release(2 + acc);

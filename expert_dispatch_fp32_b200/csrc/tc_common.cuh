@@ -301,7 +301,10 @@ __device__ __forceinline__ void decode_tile(int tile, const int* mt, int G, int 
   m = band * kBandM + (rem - n * bw);
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+// SiLU with the fast exp and divide intrinsics (a few ulp of fp32): its result is rounded to
+// bf16 (or quantised) next, and the exact form kept the epilogue on the critical path of
+// short-K launches.  g -> -inf gives g / inf = -0, the limit.
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 __device__ __forceinline__ float gelu_f(float h) {
   return 0.5f * h * (1.0f + erff(h * 0.70710678118654752f));
 }
