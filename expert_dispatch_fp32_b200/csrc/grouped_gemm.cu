@@ -82,7 +82,8 @@ struct PairArgs {
   const int32_t* group_offsets;   // [G + 1] (grouped phases); the kernel derives the M tiles
   int32_t G, nph;
   int32_t skinny;            // 1: groups of <= 64 rows run as skinny (weights-as-M) tiles
-  int32_t fold;              // 1: a last band of 257..320 rows runs as one folded tile
+  int32_t fold;              // > 0: a single-band group of 257..256 + fold rows runs as one
+                             //    folded tile (fold = 32 or 64, the largest remainder)
   int32_t fold_m256;         // 1: a folded remainder is one M = 256 product per K slice (needs
                              //    the gate/up exchange buffer in shared memory)
   int32_t* status;
@@ -316,8 +317,9 @@ struct PairCfg {
     return fold_x ? ((base + 15) & ~(size_t)15) + kFoldXBytes : base;
   }
 };
-// Largest remainder folded into a single-band group's tile (rows beyond 256).
-constexpr int kFoldMax = PairCfg::kRemRows;
+// Largest remainder folded into a single-band group's tile (rows beyond 256): the
+// remainder box holds kRemRows rows per CTA.
+constexpr int kFoldMax = 2 * PairCfg::kRemRows;
 
 // Where a pair tile sits: phase, group, M tile (256 rows), N block, its first row,
 // the group's end row, and its band slot (the M tile's index across the phase).
@@ -332,24 +334,24 @@ struct PairTile {
 //     the weights on the M side (M = 128: 64 weight rows per CTA, twice) and the rows
 //     on the N side, N = rows rounded up to 32 (N/2 rows per CTA; a multiple of 32 is
 //     a valid N for every 2-CTA MMA shape), for 2N/256 of an M = 128 tile's MMA work;
-//   with folding enabled, a group of 257..320 rows in all: TK_FOLD, the M = 256 tile
-//     of the first 256 rows plus, on every K step and from the same weight slab in
-//     shared memory, the skinny product of the remainder rows.  The remainder then
-//     costs two small MMAs per K step instead of a second tile that streams the whole
-//     weight panel again for a few rows (on deepseek_v3's routing, 256 +- 18 rows per
-//     expert, half the experts have one).  Measured on 256 experts of 272 rows each
-//     (deepseek_v3 shapes): the folded tile costs 1.46 full tiles, a full tile plus an
-//     M = 128 tile 1.51; with 320 rows (N = 64) folding was slower (1.61 vs 1.51), as it
-//     was for the last band of larger groups (small_e8_d2048, 1035..1096 rows: 0.503 vs
-//     0.475 ms), where the folded tile falls behind the group's other tiles that share
-//     its weight tiles through L2.  So only single-band groups with a remainder of at
-//     most 32 rows fold.
+//   with folding enabled, a single-band group of 257..256 + fold rows in all: TK_FOLD,
+//     the M = 256 tile of the first 256 rows plus, on every K step and from the same
+//     weight slab in shared memory, the product of the remainder rows (weights as M,
+//     rows as N).  The remainder then costs one small MMA per K16 slice instead of a
+//     second tile that streams the whole weight panel again for a few rows (on
+//     deepseek_v3's routing, 256 +- 18 rows per expert, half the experts have one).
+//     Measured per tile on deepseek_v3: a folded K step 879-905 cycles against 613-630
+//     for a full tile (1.44 full tiles), an M = 128 tile 614-623 (1.0).  The folded tile
+//     falls behind when other tiles of its group share its weight tiles through L2
+//     (the last band of larger groups, small_e8_d2048: 0.503 vs 0.475 ms), so only
+//     single-band groups fold; with the one-product remainder a limit of 64 rows was
+//     1.9 % faster than 32 on deepseek_v3's launch (6.94-7.03 vs 7.05-7.25 ms, one box).
 // ns: the skinny (or folded) product's N, the row count rounded up to 32.
 enum TileKind { TK_FULL = 0, TK_HALF = 1, TK_SKINNY = 2, TK_FOLD = 3 };
 __device__ __forceinline__ int tile_kind(const PairTile& t, int skinny, int fold, int& ns) {
   const int left = t.end - t.base;
   ns = 0;
-  if (fold && t.m == 0 && left > 2 * kTileM && left <= 2 * kTileM + kFoldMax) {
+  if (fold > 0 && t.m == 0 && left > 2 * kTileM && left <= 2 * kTileM + fold) {
     ns = (left - 2 * kTileM + 31) & ~31;
     return TK_FOLD;
   }
@@ -360,10 +362,10 @@ __device__ __forceinline__ int tile_kind(const PairTile& t, int skinny, int fold
 }
 
 // M tiles of a group of `rows` rows: 256 rows each; with folding, a group of 257..
-// 256 + kFoldMax rows is one tile.
+// 256 + fold rows is one tile.
 __device__ __forceinline__ int pair_mtiles(int rows, int fold) {
   if (rows <= 0) return 0;
-  if (fold && rows > 2 * kTileM && rows <= 2 * kTileM + kFoldMax) return 1;
+  if (fold > 0 && rows > 2 * kTileM && rows <= 2 * kTileM + fold) return 1;
   return (rows + 2 * kTileM - 1) / (2 * kTileM);
 }
 
@@ -610,7 +612,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
     if (fold) {
       for (int g = threadIdx.x; g < G; g += blockDim.x) {
         const int rows = off[g + 1] - off[g];
-        if (rows > 2 * kTileM && rows <= 2 * kTileM + kFoldMax) atomicOr(any_fold, 1);
+        if (rows > 2 * kTileM && rows <= 2 * kTileM + fold) atomicOr(any_fold, 1);
       }
     }
   }
@@ -985,10 +987,15 @@ cudaError_t launch_grouped_pair(const GemmProblem* probs, int n, int32_t* counte
     const char* env = getenv("MOE_GEMM_SKINNY");
     a.skinny = (env && env[0] == '0') ? 0 : 1;
     env = getenv("MOE_GEMM_FOLD");
-    a.fold = (env && env[0] == '0') ? 0 : 1;
+    const bool fold_on = !(env && env[0] == '0');
     // MOE_GEMM_FOLD256=0 runs a folded remainder as two M = 128 products per K slice
     env = getenv("MOE_GEMM_FOLD256");
-    a.fold_m256 = (a.fold && !(env && env[0] == '0')) ? 1 : 0;
+    a.fold_m256 = (fold_on && !(env && env[0] == '0')) ? 1 : 0;
+    // the largest folded remainder: kFoldMax rows with the one-product form
+    // (MOE_GEMM_FOLD_MAX=32 for 32), 32 with the two-product form
+    env = getenv("MOE_GEMM_FOLD_MAX");
+    const int fmax = (env && atoi(env) == 32) ? 32 : kFoldMax;
+    a.fold = fold_on ? (a.fold_m256 ? fmax : 32) : 0;
   }
   a.status = probs[0].status;
   a.counter = counter;
@@ -1041,8 +1048,10 @@ cudaError_t launch_grouped_pair(const GemmProblem* probs, int n, int32_t* counte
     tiles += (p.max_tiles > 0 ? p.max_tiles : 1);
   }
   // the M = 256 fold needs its exchange buffer next to the ring (room for about 700 groups)
-  if (a.fold_m256 && PairCfg::smem_bytes(a.group_offsets ? a.G : 1, true) > (size_t)smem_optin())
+  if (a.fold_m256 && PairCfg::smem_bytes(a.group_offsets ? a.G : 1, true) > (size_t)smem_optin()) {
     a.fold_m256 = 0;
+    if (a.fold > 32) a.fold = 32;
+  }
   const int64_t pairs = sm_count() / 2;
   const int clusters = (int)(tiles < pairs ? tiles : pairs);
   return launch_tc_pair(a, clusters, s);
