@@ -347,9 +347,13 @@ def run_ours(args):
 
     x_bf = x if wl.x_dtype == "bf16" else None
 
+    fused = M.moe_route_dispatch_is_fused(cfg)
+    mx_fused_dispatch = mx and not fused and wl.x_dtype == "bf16"
+
     def expert_ffn():
         if mx:
-            M.moe_expert_ffn_mxfp8(cfg, b["x_perm"], x_bf, b["expert_offsets"], layer.packed,
+            M.moe_expert_ffn_mxfp8(cfg, None if mx_fused_dispatch else b["x_perm"], x_bf,
+                                   b["expert_offsets"], layer.packed,
                                    layer.packed_mx, b["y_perm"], b["shared_out"], b["workspace"],
                                    b["status"], stream)
         else:
@@ -364,7 +368,11 @@ def run_ours(args):
         M.moe_preprocess(cfg, b["topk_idx"], b["counts"], b["expert_offsets"], b["rank_splits"],
                          b["rank_offsets"], b["pos"], b["src"], b["workspace"], b["status"], stream)
         ev[2].record(stream)
-        M.moe_dispatch_permute(cfg, x, b["pos"], b["x_perm"], stream)
+        if mx_fused_dispatch:
+            # MXFP8: the dispatch writes the quantised rows (the layer's forward does the same)
+            M.moe_dispatch_mxfp8(cfg, x, b["src"], b["expert_offsets"], b["workspace"], stream)
+        else:
+            M.moe_dispatch_permute(cfg, x, b["pos"], b["x_perm"], stream)
         ev[3].record(stream)
         expert_ffn()
         ev[4].record(stream)
@@ -390,8 +398,6 @@ def run_ours(args):
         ev[0].record(stream)
         layer.forward(x, stream)
         ev[1].record(stream)
-
-    fused = M.moe_route_dispatch_is_fused(cfg)
 
     mk = lambda n=6: [torch.cuda.Event(enable_timing=True) for _ in range(n)]
     # the stage-by-stage step is the layer's forward: check once that both give the same bits
@@ -523,7 +529,8 @@ def run_ours(args):
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     disp_gbs = disp_b / (stage_ms[2] / args.steps / 1e3) / 1e9
     comb_gbs = comb_b / (stage_ms[4] / args.steps / 1e3) / 1e9
-    # MXFP8 FFN: x_perm quantiser, gate_up, down, and the shared experts' launch
+    # MXFP8 FFN: x_perm quantiser (inside the dispatch when that is a separate stage),
+    # gate_up, down, and the shared experts' launch
     n_ffn = (3 + (1 if wl.n_shared else 0)) if mx else ffn_launches(wl)
     launches_per_step = (1 if fused else route_launches(wl) + 1 + 1) + n_ffn + 1
 

@@ -12,7 +12,7 @@ from ._binding import (  # noqa: F401
     MOE_ERR_INDEX_OOB, MOE_ERR_INVALID_ARG, MOE_ERR_SCRATCH_LIMIT, MOE_ERR_TIMEOUT,
     MOE_ERR_UNSUPPORTED, MOE_OK,
     MoeConfig, MoeEpPeers, MoeError, lib, moe_abi_version, moe_check_wait_timeout,
-    moe_combine_unpermute, moe_dispatch_permute,
+    moe_combine_unpermute, moe_dispatch_mxfp8, moe_dispatch_permute,
     moe_ep_local_ids, moe_ep_recv_layout, moe_ep_return_rows, moe_ep_send_counts, moe_ep_send_rows,
     moe_ep_wait_returned, moe_expert_ffn_mxfp8, moe_mxfp8_quantize, moe_packed_weights_mxfp8_size,
     moe_prepare_weights_mxfp8, moe_workspace_mxfp8_size, moe_expert_ffn, moe_forward, moe_gather_rows, moe_packed_weights_size,

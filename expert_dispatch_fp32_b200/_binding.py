@@ -77,6 +77,7 @@ _SIGS = {
     "moe_workspace_mxfp8_size": (ctypes.c_size_t, [_cfgp]),
     "moe_prepare_weights_mxfp8": (ctypes.c_int, [_cfgp, _vp, _vp, _vp]),
     "moe_expert_ffn_mxfp8": (ctypes.c_int, [_cfgp, _vp, _vp, _i32p, _vp, _vp, _vp, _vp, _vp, _i32p, _vp]),
+    "moe_dispatch_mxfp8": (ctypes.c_int, [_cfgp, _vp, _i32p, _i32p, _vp, _vp]),
     "moe_ep_send_counts": (ctypes.c_int, [_cfgp, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, _i32p,
                                           ctypes.c_uint32, _vp]),
     "moe_ep_send_rows": (ctypes.c_int, [_cfgp, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, _vp,
@@ -96,6 +97,9 @@ _SIGS = {
 }
 
 
+ABI_VERSION = 2          # MOE_ABI_VERSION of include/moe.h
+
+
 def lib() -> ctypes.CDLL:
     """Load libmoe.so (built in-tree by ``expert_dispatch_fp32_b200.build``)."""
     global _lib
@@ -107,6 +111,9 @@ def lib() -> ctypes.CDLL:
         for name, (res, args) in _SIGS.items():
             fn = getattr(L, name)
             fn.restype, fn.argtypes = res, args
+        if L.moe_abi_version() != ABI_VERSION:
+            raise ImportError(f"{LIB_PATH} has ABI version {L.moe_abi_version()}, this binding expects "
+                              f"{ABI_VERSION} (rebuild with `python -m expert_dispatch_fp32_b200.build`)")
         _lib = L
     return _lib
 
@@ -183,6 +190,11 @@ def moe_expert_ffn_mxfp8(cfg, x_perm, x, expert_offsets, packed, packed_mx, y_pe
                          workspace, status, stream=None):
     _call("moe_expert_ffn_mxfp8", ctypes.byref(cfg), _p(x_perm), _p(x), _p(expert_offsets), _p(packed),
           _p(packed_mx), _p(y_perm), _p(shared_out), _p(workspace), _p(status), _s(stream))
+
+
+def moe_dispatch_mxfp8(cfg, x, src, expert_offsets, workspace, stream=None):
+    _call("moe_dispatch_mxfp8", ctypes.byref(cfg), _p(x), _p(src), _p(expert_offsets), _p(workspace),
+          _s(stream))
 
 
 def moe_router_filter_view(cfg):

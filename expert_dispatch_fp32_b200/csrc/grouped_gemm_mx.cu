@@ -401,16 +401,17 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
         } else if (EPI == EPI_SWIGLU) {
           // [gate 64 | up 64] -> outputs n*128 + 64h + [0, 64): K step n, blocks 2h, 2h + 1
           uint8_t* dst = p.q_out + row * p.ldo + n * 128 + h * 64;
-          p.q_sf[mx_sf_offset(t, qk, n, (int)rank, r, 2 * h)] = quant_swiglu32(v0, v2, dst);
-          p.q_sf[mx_sf_offset(t, qk, n, (int)rank, r, 2 * h + 1)] = quant_swiglu32(v1, v3, dst + 32);
+          const uint32_t s0 = quant_swiglu32(v0, v2, dst), s1 = quant_swiglu32(v1, v3, dst + 32);
+          *reinterpret_cast<uint16_t*>(p.q_sf + mx_sf_offset(t, qk, n, (int)rank, r, 2 * h)) =
+              (uint16_t)(s0 | (s1 << 8));
         } else {
           // GELU: outputs n*256 + 128h + [0, 128): K step 2n + h, blocks 0..3
           uint8_t* dst = p.q_out + row * p.ldo + n * BN + h * 128;
           const int s = 2 * n + h;
-          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 0)] = quant_gelu32(v0, dst);
-          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 1)] = quant_gelu32(v1, dst + 32);
-          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 2)] = quant_gelu32(v2, dst + 64);
-          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 3)] = quant_gelu32(v3, dst + 96);
+          const uint32_t s0 = quant_gelu32(v0, dst), s1 = quant_gelu32(v1, dst + 32);
+          const uint32_t s2 = quant_gelu32(v2, dst + 64), s3 = quant_gelu32(v3, dst + 96);
+          *reinterpret_cast<uint32_t*>(p.q_sf + mx_sf_offset(t, qk, s, (int)rank, r, 0)) =
+              s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
         }
       } else {
         const int cq = q >> 1;               // tile columns 128 cq .. 128 cq + 127
@@ -426,8 +427,9 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
           // outputs n*256 + 128 cq + 64 h + [0, 64): K step 2n + cq, blocks 2h, 2h + 1
           uint8_t* dst = p.q_out + row * p.ldo + n * BN + cq * 128 + h * 64;
           const int s = 2 * n + cq;
-          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 2 * h)] = quant_gelu32(v0, dst);
-          p.q_sf[mx_sf_offset(t, qk, s, (int)rank, r, 2 * h + 1)] = quant_gelu32(v1, dst + 32);
+          const uint32_t s0 = quant_gelu32(v0, dst), s1 = quant_gelu32(v1, dst + 32);
+          *reinterpret_cast<uint16_t*>(p.q_sf + mx_sf_offset(t, qk, s, (int)rank, r, 2 * h)) =
+              (uint16_t)(s0 | (s1 << 8));
         }
       }
       __syncwarp();
@@ -511,11 +513,15 @@ mx_block_scales_kernel(const uint32_t* __restrict__ rowmajor, uint8_t* __restric
   }
 }
 
-// x_perm -> E4M3 rows with A's scale blocks.  One warp per row: the row's group (binary
+// Rows of A -> E4M3 rows with A's scale blocks.  One warp per row: the row's group (binary
 // search of the offsets), its M tile and place in it, then 32-element blocks lane-strided.
+// Row r's bf16 source is x[r] (x_perm), or, with src, x[src[r] / k]: the dispatch itself
+// ("Expert Parallel (EP)", Communication Pattern step 2: each chosen expert gets a copy
+// of the token), so the bf16 x_perm is never written.
 __global__ void __launch_bounds__(256)
-mx_quant_a_kernel(const bf16* __restrict__ x, const int32_t* __restrict__ group_offsets, int G, int K,
-                  int half, uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+mx_quant_a_kernel(const bf16* __restrict__ x, const int32_t* __restrict__ src, int k,
+                  const int32_t* __restrict__ group_offsets, int G, int K, int half, uint8_t* __restrict__ q,
+                  uint8_t* __restrict__ sf) {
   extern __shared__ int sh[];
   int* mt = sh;                 // [G + 1]
   int* off = sh + (G + 1);      // [G + 1]
@@ -537,21 +543,35 @@ mx_quant_a_kernel(const bf16* __restrict__ x, const int32_t* __restrict__ group_
     const int64_t t = (int64_t)mt[lo] + rr / kMxTileM;
     int h, m;
     mx_row_place(rr % kMxTileM, mx_is_half(off[lo + 1] - off[lo], rr / kMxTileM, half), h, m);
-    for (int b = lane; b < nblk; b += 32) {
-      const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)r * K + b * 32);
-      float v[32];
+    const bf16* xr = x + (src != nullptr ? (int64_t)(__ldg(src + r) / k) : (int64_t)r) * K;
+    // lane b takes block b (coalesced); the four blocks of a K step sit in four
+    // consecutive lanes (nblk % 4 == 0), whose scales go out as one word
+    for (int b0 = 0; b0 < nblk; b0 += 32) {
+      const int b = b0 + lane;
+      const bool ok = b < nblk;
+      uint32_t sc = 0;
+      if (ok) {
+        const uint4* xs = reinterpret_cast<const uint4*>(xr + b * 32);
+        float v[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint4 u = __ldg(src + c);
-        const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&u);
+        for (int c = 0; c < 4; ++c) {
+          const uint4 u = __ldg(xs + c);
+          const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = __bfloat1622float2(hh[i]);
-          v[8 * c + 2 * i] = f.x;
-          v[8 * c + 2 * i + 1] = f.y;
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(hh[i]);
+            v[8 * c + 2 * i] = f.x;
+            v[8 * c + 2 * i + 1] = f.y;
+          }
         }
+        sc = mx_quant32(v, q + (int64_t)r * K + b * 32);
       }
-      sf[mx_sf_offset(t, ksteps, b >> 2, h, m, b & 3)] = mx_quant32(v, q + (int64_t)r * K + b * 32);
+      const uint32_t s1 = __shfl_down_sync(0xffffffffu, sc, 1);
+      const uint32_t s2 = __shfl_down_sync(0xffffffffu, sc, 2);
+      const uint32_t s3 = __shfl_down_sync(0xffffffffu, sc, 3);
+      if (ok && (lane & 3) == 0)
+        *reinterpret_cast<uint32_t*>(sf + mx_sf_offset(t, ksteps, b >> 2, h, m, 0)) =
+            sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
     }
   }
 }
@@ -572,15 +592,16 @@ cudaError_t launch_mx_block_scales(const uint8_t* rowmajor, uint8_t* blocked, in
   return cudaGetLastError();
 }
 
-cudaError_t launch_mx_quant_a(const bf16* x, int64_t rows, const int32_t* group_offsets, int G, int K,
-                              int half_tiles, uint8_t* q, uint8_t* sf, cudaStream_t s) {
+cudaError_t launch_mx_quant_a(const bf16* x, const int32_t* src, int k, int64_t rows,
+                              const int32_t* group_offsets, int G, int K, int half_tiles, uint8_t* q, uint8_t* sf,
+                              cudaStream_t s) {
   if (K % MxCfg::KS != 0 || G <= 0) return cudaErrorInvalidValue;
   if (rows == 0) return cudaSuccess;
   const size_t smem = (2 * (size_t)(G + 1) + 8) * sizeof(int);
   if (smem > 48 * 1024) return cudaErrorInvalidValue;
   int64_t grid = (rows + 7) / 8;                 // 8 rows (warps) per block
   if (grid > 4 * (int64_t)sm_count()) grid = 4 * (int64_t)sm_count();
-  mx_quant_a_kernel<<<(int)grid, 256, smem, s>>>(x, group_offsets, G, K, half_tiles, q, sf);
+  mx_quant_a_kernel<<<(int)grid, 256, smem, s>>>(x, src, k, group_offsets, G, K, half_tiles, q, sf);
   return cudaGetLastError();
 }
 

@@ -633,6 +633,13 @@ moe_status moe_router_filter_view(const moe_config* cfg, size_t* approx_offset, 
   return MOE_OK;
 }
 
+// A group's last <= 128 rows run as an M = 128 tile in the MXFP8 GEMMs (MOE_MX_HALF=0: as
+// M = 256, for comparison); the quantiser of their A rows must lay the scales out the same way.
+static int mx_half_tiles() {
+  const char* env = getenv("MOE_MX_HALF");
+  return (env && env[0] == '0') ? 0 : 1;
+}
+
 // MXFP8 routed experts: 256-wide N tiles on both GEMMs (gate_up width and D multiples of
 // 256) and 128-deep K steps (D and F multiples of 128).
 static moe_status mx_check(const moe_config* cfg) {
@@ -689,7 +696,7 @@ moe_status moe_expert_ffn_mxfp8(const moe_config* cfg, const void* x_perm, const
   MOE_CHECK_PTR(status);
   const int64_t R = (int64_t)c.T * c.top_k;
   if (R > 0) {
-    MOE_CHECK_PTR(x_perm);
+    if (x_perm != nullptr) MOE_CHECK_PTR(x_perm);
     MOE_CHECK_PTR(y_perm);
   }
   cudaStream_t s = as_stream(stream);
@@ -700,12 +707,12 @@ moe_status moe_expert_ffn_mxfp8(const moe_config* cfg, const void* x_perm, const
   const int nup = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
   int32_t* ctr = (int32_t*)(ws + L.counters);
   if (R > 0) {
-    // a group's last <= 128 rows run as an M = 128 tile (MOE_MX_HALF=0: as M = 256, for comparison)
-    const char* half_env = getenv("MOE_MX_HALF");
-    const int half = (half_env && half_env[0] == '0') ? 0 : 1;
+    const int half = mx_half_tiles();
     cudaError_t err = cudaMemsetAsync(ctr, 0, 2 * sizeof(int32_t), s);
-    if (err == cudaSuccess)
-      err = launch_mx_quant_a((const bf16*)x_perm, R, expert_offsets, c.E, c.D, half, ws + L.xq, ws + L.xsf, s);
+    // x_perm NULL: moe_dispatch_mxfp8 has already put the quantised rows in the workspace
+    if (err == cudaSuccess && x_perm != nullptr)
+      err = launch_mx_quant_a((const bf16*)x_perm, nullptr, 1, R, expert_offsets, c.E, c.D, half, ws + L.xq,
+                              ws + L.xsf, s);
     // gate_up (or W1): the activation comes out quantised, with the down projection's scales
     MxProblem up;
     memset(&up, 0, sizeof(up));
@@ -732,6 +739,24 @@ moe_status moe_expert_ffn_mxfp8(const moe_config* cfg, const void* x_perm, const
   if (c.n_shared > 0 && shared_out != nullptr)
     return moe_shared_ffn(cfg, x, packed, shared_out, workspace, status, stream);
   return MOE_OK;
+}
+
+moe_status moe_dispatch_mxfp8(const moe_config* cfg, const void* x, const int32_t* src,
+                              const int32_t* expert_offsets, void* workspace, void* stream) {
+  moe_status st = mx_check(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  if (c.x_dtype != MOE_DT_BF16) return MOE_ERR_UNSUPPORTED;
+  MOE_CHECK_PTR(expert_offsets);
+  MOE_CHECK_PTR(workspace);
+  const int64_t R = (int64_t)c.T * c.top_k;
+  if (R == 0) return MOE_OK;
+  MOE_CHECK_PTR(x);
+  MOE_CHECK_PTR(src);
+  const MxWsLayout L = mx_ws_layout(c);
+  uint8_t* ws = (uint8_t*)workspace;
+  return cuda_status(launch_mx_quant_a((const bf16*)x, src, c.top_k, R, expert_offsets, c.E, c.D,
+                                       mx_half_tiles(), ws + L.xq, ws + L.xsf, as_stream(stream)));
 }
 
 moe_status moe_mxfp8_quantize(const void* x, int64_t rows, int32_t K, void* q, void* scales,

@@ -134,9 +134,11 @@ size_t mx_sf_bytes(int64_t tiles, int K);
 cudaError_t launch_mx_block_scales(const uint8_t* rowmajor, uint8_t* blocked, int64_t rows, int K,
                                    cudaStream_t s);
 // bf16 rows grouped by group_offsets -> E4M3 rows and the scale blocks of an A operand.
-// half_tiles: the tiling of the GEMM that reads the blocks (MxProblem::half_tiles).
-cudaError_t launch_mx_quant_a(const bf16* x, int64_t rows, const int32_t* group_offsets, int G, int K,
-                              int half_tiles, uint8_t* q, uint8_t* sf, cudaStream_t s);
+// half_tiles: the tiling of the GEMM that reads the blocks (MxProblem::half_tiles).  Row r
+// comes from x[r], or with src from x[src[r] / k] (dispatch and quantisation in one pass).
+cudaError_t launch_mx_quant_a(const bf16* x, const int32_t* src, int k, int64_t rows,
+                              const int32_t* group_offsets, int G, int K, int half_tiles, uint8_t* q, uint8_t* sf,
+                              cudaStream_t s);
 // Peer-memory exchange (ep_peer.cu).
 cudaError_t launch_ep_send_counts(const moe_ep_peers& p, int rank0, int nlocal, const int32_t* counts,
                                   int E, uint32_t epoch, cudaStream_t s);

@@ -118,11 +118,23 @@ class MoELayer:
                           b["rank_offsets"], b["pos"], b["src"], b["x_perm"], b["act"], b["y_perm"],
                           b["shared_out"], out, b["workspace"], b["status"], stream)
             return
-        B.moe_route_dispatch(self._cfg, x, self.w_router, self.expert_bias, b["logits"], b["topk_idx"],
-                             b["topk_w"], b["counts"], b["expert_offsets"], b["rank_splits"],
-                             b["rank_offsets"], b["pos"], b["src"], b["x_perm"], b["workspace"],
-                             b["status"], stream)
-        B.moe_expert_ffn_mxfp8(self._cfg, b["x_perm"], x if self.x_dtype == "bf16" else None,
+        if self.x_dtype != "bf16" or B.moe_route_dispatch_is_fused(self._cfg):
+            # the one-launch router + preprocess + dispatch writes the bf16 x_perm; the
+            # FFN call quantises it
+            B.moe_route_dispatch(self._cfg, x, self.w_router, self.expert_bias, b["logits"],
+                                 b["topk_idx"], b["topk_w"], b["counts"], b["expert_offsets"],
+                                 b["rank_splits"], b["rank_offsets"], b["pos"], b["src"], b["x_perm"],
+                                 b["workspace"], b["status"], stream)
+            x_perm = b["x_perm"]
+        else:
+            # route and preprocess, then the dispatch quantises the rows as it copies them
+            B.moe_route(self._cfg, x, self.w_router, self.expert_bias, b["logits"], b["topk_idx"],
+                        b["topk_w"], b["workspace"], stream)
+            B.moe_preprocess(self._cfg, b["topk_idx"], b["counts"], b["expert_offsets"], b["rank_splits"],
+                             b["rank_offsets"], b["pos"], b["src"], b["workspace"], b["status"], stream)
+            B.moe_dispatch_mxfp8(self._cfg, x, b["src"], b["expert_offsets"], b["workspace"], stream)
+            x_perm = None
+        B.moe_expert_ffn_mxfp8(self._cfg, x_perm, x if self.x_dtype == "bf16" else None,
                                b["expert_offsets"], self.packed, self.packed_mx, b["y_perm"],
                                b["shared_out"], b["workspace"], b["status"], stream)
         B.moe_combine_unpermute(self._cfg, b["y_perm"], b["pos"], b["topk_w"], x, b["shared_out"], out,

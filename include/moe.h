@@ -40,7 +40,9 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+/* 2: the MXFP8 routed-expert calls, moe_dispatch_mxfp8, the router filter view and the
+ * peer-memory exchange calls. */
+#define MOE_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -425,8 +427,21 @@ MOE_API size_t moe_workspace_mxfp8_size(const moe_config* cfg);
  * packed_mx (caller-allocated, moe_packed_weights_mxfp8_size bytes); one time. */
 MOE_API moe_status moe_prepare_weights_mxfp8(const moe_config* cfg, const void* packed, void* packed_mx,
                                              void* stream);
+/* Dispatch straight into MXFP8 (bf16 x only): each routed row r, in the expert-grouped
+ * order of moe_preprocess, is quantised from x[src[r] / k] ("Expert Parallel (EP)",
+ * Communication Pattern step 2) into the MXFP8 workspace, E4M3 elements with their
+ * scales ordered for the expert GEMM's tiles; moe_expert_ffn_mxfp8 with x_perm = NULL
+ * then uses them.  Equal, bit for bit, to moe_dispatch_permute followed by the
+ * quantisation inside moe_expert_ffn_mxfp8, without writing the bf16 x_perm.
+ *   x              device bf16 [T, D];  src, expert_offsets from moe_preprocess
+ *   workspace      the MXFP8 workspace later passed to moe_expert_ffn_mxfp8
+ * Errors: MOE_ERR_UNSUPPORTED for fp32 x or a shape moe_expert_ffn_mxfp8 refuses;
+ * MOE_ERR_INVALID_ARG for a bad pointer. */
+MOE_API moe_status moe_dispatch_mxfp8(const moe_config* cfg, const void* x, const int32_t* src,
+                                      const int32_t* expert_offsets, void* workspace, void* stream);
 /* moe_expert_ffn with MXFP8 routed experts: quantises x_perm (E4M3 rows and their
- * scales, ordered for the GEMM's tiles), runs gate_up with the activation and its
+ * scales, ordered for the GEMM's tiles; x_perm NULL: the rows moe_dispatch_mxfp8 left in
+ * the workspace), runs gate_up with the activation and its
  * quantisation in the epilogue (the quantised activation stays in the workspace; no
  * bf16 act is written), then down into y_perm (bf16 [T*k, D]).  The shared experts (if
  * shared_out is not NULL) run in bf16 from `packed` as in moe_expert_ffn.  Other

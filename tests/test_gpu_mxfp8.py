@@ -108,13 +108,15 @@ def test_mxfp8_expert_ffn_matches_the_oracle(case, half, monkeypatch):
         assert torch.equal(sh, b["shared_out"])     # the shared experts stay bf16
 
 
-def test_mxfp8_layer_forward_is_its_stages():
+@pytest.mark.parametrize("E", [16, 64])
+def test_mxfp8_layer_forward_is_its_stages(E):
     """MoELayer(mxfp8=True): the forward is route+dispatch, the MXFP8 FFN and the combine
-    (same bits as the calls one by one), and its MoE part stays within the format's error
-    of the bf16 layer's."""
+    (same bits as the calls one by one; with more than 32 experts the dispatch writes the
+    quantised rows itself), and its MoE part stays within the format's error of the bf16
+    layer's."""
     import moe_workloads as W
     from parity_helpers import f64
-    wl = W.Workload(name="mxl", T=640, D=512, E=16, ep_size=4, top_k=4, F=256, n_shared=1,
+    wl = W.Workload(name="mxl", T=640, D=512, E=E, ep_size=4, top_k=4, F=256, n_shared=1,
                     F_shared=256, seed=41)
     inp = W.make_inputs(wl, device="cuda")
     kw = dict(D=wl.D, E=wl.E, ep_size=wl.ep_size, top_k=wl.top_k, F=wl.F, w_router=inp["w_router"],
@@ -134,7 +136,11 @@ def test_mxfp8_layer_forward_is_its_stages():
     M.moe_route_dispatch(cfg, x, mx.w_router, mx.expert_bias, None, b["topk_idx"], b["topk_w"],
                          b["counts"], b["expert_offsets"], b["rank_splits"], b["rank_offsets"], b["pos"],
                          b["src"], b["x_perm"], b["workspace"], b["status"])
-    M.moe_expert_ffn_mxfp8(cfg, b["x_perm"], x, b["expert_offsets"], mx.packed, mx.packed_mx, y, sh,
+    x_perm = b["x_perm"]
+    if not M.moe_route_dispatch_is_fused(cfg):
+        M.moe_dispatch_mxfp8(cfg, x, b["src"], b["expert_offsets"], b["workspace"])
+        x_perm = None
+    M.moe_expert_ffn_mxfp8(cfg, x_perm, x, b["expert_offsets"], mx.packed, mx.packed_mx, y, sh,
                            b["workspace"], b["status"])
     M.moe_combine_unpermute(cfg, y, b["pos"], b["topk_w"], x, sh, o)
     torch.cuda.synchronize()
@@ -144,3 +150,36 @@ def test_mxfp8_layer_forward_is_its_stages():
     rel = np.linalg.norm(moe_mx - moe_ref) / np.linalg.norm(moe_ref)
     print(f"\nMoE part, MXFP8 layer vs bf16 layer: rel-L2 {rel:.3e}")
     assert rel < 0.15
+
+
+@pytest.mark.parametrize("half", ["1", "0"])
+def test_mxfp8_dispatch_equals_quantised_x_perm(half, monkeypatch):
+    """moe_dispatch_mxfp8 (each row quantised straight from x[src / k]) followed by the
+    MXFP8 FFN with x_perm = NULL gives the bits of the bf16 dispatch followed by the FFN's
+    own quantisation of x_perm, with M = 128 remainder tiles on and off."""
+    import moe_workloads as W
+    from parity_helpers import make_layer
+    monkeypatch.setenv("MOE_MX_HALF", half)
+    wl = W.Workload(name="mxd", T=700, D=512, E=64, ep_size=8, top_k=4, F=256, seed=43)
+    inp = W.make_inputs(wl, device="cuda")
+    layer = make_layer(wl, inp)
+    x = inp["x"]
+    layer.forward(x)
+    torch.cuda.synchronize()
+    layer.check_status()
+    b, cfg = layer.buf, layer.config(wl.T)
+    pmx = torch.empty(M.moe_packed_weights_mxfp8_size(cfg), dtype=torch.uint8, device="cuda")
+    M.moe_prepare_weights_mxfp8(cfg, layer.packed, pmx)
+    n = M.moe_workspace_mxfp8_size(cfg)
+    ws_a = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    ws_b = torch.full((n,), 0x7F, dtype=torch.uint8, device="cuda")   # stale bytes everywhere
+    y_a = torch.empty_like(b["y_perm"])
+    y_b = torch.full_like(b["y_perm"], float("nan"))
+    M.moe_expert_ffn_mxfp8(cfg, b["x_perm"], None, b["expert_offsets"], layer.packed, pmx, y_a, None,
+                           ws_a, b["status"])
+    M.moe_dispatch_mxfp8(cfg, x, b["src"], b["expert_offsets"], ws_b)
+    M.moe_expert_ffn_mxfp8(cfg, None, None, b["expert_offsets"], layer.packed, pmx, y_b, None, ws_b,
+                           b["status"])
+    torch.cuda.synchronize()
+    layer.check_status()
+    assert torch.equal(y_a, y_b)
