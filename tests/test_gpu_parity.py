@@ -197,3 +197,54 @@ def test_forward_end_to_end(ctx):
     e = assert_layer_close(got, res["out"], f64(inp["x"][torch.from_numpy(toks).cuda()]))
     print(f"\n{wl.name}: tokens checked {toks.size}, rel-L2 {e[0]:.2e}, max-abs {e[1]:.2e}, "
           f"MoE-part rel-L2 {e[2]:.2e}; near-tie {n_exempt}, differ {n_differ}")
+
+
+def _mx_dq(a):
+    """MXFP8 quantise-and-dequantise along the last axis (oracle/mxfp8.py)."""
+    from oracle import mxfp8
+    return mxfp8.dequantize_mxfp8(*mxfp8.quantize_mxfp8(a, axis=-1), axis=-1)
+
+
+def test_mxfp8_expert_ffn_stage(ctx):
+    """The MXFP8 routed experts at full size (the FFN stage of `bench.py --mxfp8`): y_perm
+    of three experts (sampled rows, tile edges included) against the oracle's expert FFN
+    on MXFP8-quantised rows, weights and activation.  Quantising a whole expert's weights
+    takes the oracle seconds, hence three experts; the quantiser and the GEMM tiling are
+    checked on every row of smaller cases in test_gpu_mxfp8.py."""
+    wl, inp, layer, pre = ctx["wl"], ctx["inp"], ctx["layer"], ctx["pre"]
+    if wl.name not in ("deepseek_v3", "zipf_skew_e64"):
+        pytest.skip("MXFP8 full-size check runs on deepseek_v3 and zipf_skew_e64")
+    cfg = layer.config(wl.T)
+    b = _preprocess_on_gpu(ctx, ctx["ref"]["idx"])
+    src = torch.from_numpy(pre["src"]).cuda()
+    x_perm = inp["x"].to(torch.bfloat16)[src.long() // wl.top_k].contiguous()
+    pmx = torch.empty(M.moe_packed_weights_mxfp8_size(cfg), dtype=torch.uint8, device="cuda")
+    M.moe_prepare_weights_mxfp8(cfg, layer.packed, pmx)
+    ws = torch.empty(M.moe_workspace_mxfp8_size(cfg), dtype=torch.uint8, device="cuda")
+    y = torch.full_like(b["y_perm"], float("nan"))
+    M.moe_expert_ffn_mxfp8(cfg, x_perm, None, b["expert_offsets"], layer.packed, pmx, y, None, ws,
+                           b["status"])
+    torch.cuda.synchronize()
+    assert int(b["status"].item()) == 0
+    counts = pre["counts"]
+    # the busiest expert, the last non-empty one, and one with a remainder past 256 rows
+    nz = np.nonzero(counts)[0]
+    picks = [int(nz[np.argmax(counts[nz])]), int(nz[-1])]
+    over = [int(e) for e in nz if counts[e] % 256 != 0 and counts[e] > 256 and int(e) not in picks]
+    if over:
+        picks.append(over[0])
+    rows_of = _sample_rows(pre, np.random.default_rng(2))
+    wup = up_weights(wl, inp)
+    for e in picks:
+        rows = rows_of[e]
+        xr = f64(x_perm[torch.from_numpy(rows).cuda()])
+        wu = _mx_dq(f64(wup[e]).T).T              # [D, Nup], blocks along D
+        wd = _mx_dq(f64(inp["w_down"][e]).T).T    # [F, D], blocks along F
+        h = _mx_dq(xr) @ wu
+        F = wu.shape[1] // 2
+        a = oracle.silu(h[:, :F]) * h[:, F:] if wl.act == "swiglu" else oracle.gelu(h)
+        ref = _mx_dq(a) @ wd
+        got = f64(y[torch.from_numpy(rows).cuda()])
+        e_ = assert_layer_close(got, ref, np.zeros_like(ref), f"mxfp8 y_perm expert {e}")
+        print(f"\n{wl.name}: MXFP8 expert {e} ({counts[e]} rows, {rows.size} checked): "
+              f"rel-L2 {e_[0]:.2e}, max-abs {e_[1]:.2e}")
