@@ -59,9 +59,11 @@ constexpr int kMxTileM = 256;
 struct MxArgs {
   CUtensorMap tmap_a;        // E4M3 [rows, K], box 128 x 128 rows
   CUtensorMap tmap_a64;      // the same, box 128 x 64 rows (half tiles)
+  CUtensorMap tmap_a32;      // the same, box 128 x 32 rows (a folded tile's remainder rows)
   CUtensorMap tmap_b;        // E4M3 [G, N, K], box 128 x 128 x 1
   CUtensorMap tmap_sfa;      // A scale blocks as [bytes / 256, 256], box 256 x 2 (one block)
   CUtensorMap tmap_sfb;      // B scale blocks, box 256 x 4 (both halves of a K step)
+  CUtensorMap tmap_sfb1;     // B scale blocks, box 256 x 2 (one half)
   const int32_t* group_offsets;
   int32_t G, N, K;
   bf16* out;                 // EPI_STORE: bf16 [rows, ldo]
@@ -69,26 +71,41 @@ struct MxArgs {
   uint8_t* q_out;            // EPI_SWIGLU / EPI_GELU: E4M3 activation [rows, ldo]
   uint8_t* q_sf;             //   and its scale blocks (ldo / 128 K steps)
   int32_t half;              // run a group's last <= 128 rows as an M = 128 tile
+  int32_t fold;              // > 0: a group of 257..256 + fold rows runs as one folded tile
   int32_t* status;
   int32_t* counter;          // tile counter, zero at launch
 };
 
-struct MxCfg {
+// Shared memory per stage: this CTA's A and B halves and the scale blocks; with folding
+// (kFold) also a folded tile's remainder rows (a 32-row box), their scale block and this
+// CTA's own B scale block (the remainder product's A scales), in 5 stages instead of 6.
+template <bool kFold>
+struct MxCfgT {
   static constexpr int BN = 256;
   static constexpr int KS = 128;                     // K elements (bytes) per stage
-  static constexpr int kStages = 6;
+  static constexpr int kStages = kFold ? 5 : 6;
   static constexpr int kABytes = 128 * KS;           // this CTA's 128 A rows
   static constexpr int kBBytes = 128 * KS;           // this CTA's 128 B rows
+  static constexpr int kRemBytes = kFold ? 32 * KS : 0;
   static constexpr int kSfaBytes = 512;
   static constexpr int kSfbBytes = 1024;
-  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kSfoBytes = kFold ? 512 : 0;  // own B block (remainder product's A scales)
+  static constexpr int kSfrBytes = kFold ? 512 : 0;  // remainder rows' scales
+  static constexpr int kStageBytes =
+      kABytes + kBBytes + kRemBytes + kSfaBytes + kSfbBytes + kSfoBytes + kSfrBytes;
   static constexpr int kTmemCols = 512;
-  static constexpr int kSfaCol = 256, kSfbCol = 260;  // 4 + 8 scale columns after the accumulator
+  // scale columns after the accumulator, then the remainder product's accumulator
+  static constexpr int kSfaCol = 256, kSfbCol = 260, kSsfaCol = 268, kSsfbCol = 272, kRemCol = 320;
   static constexpr int kCtrl = 512;
+  // gate/up exchange of a folded remainder: per column half, 64 outputs x 32 columns fp32,
+  // then 4 mbarriers
+  static constexpr int kXBytes = kFold ? 2 * 64 * 32 * 4 + 32 : 0;
   static size_t smem_bytes(int G) {
-    return 1024 + (size_t)kStages * kStageBytes + kCtrl + 2 * (size_t)(G + 1) * sizeof(int);
+    const size_t base = 1024 + (size_t)kStages * kStageBytes + kCtrl + 2 * (size_t)(G + 1) * sizeof(int);
+    return ((base + 15) & ~(size_t)15) + kXBytes;
   }
 };
+using MxCfg = MxCfgT<false>;
 
 // Block-scaled instruction descriptor, kind::mxf8f6f4: E4M3 A and B, K-major, E8M0 scales
 // (bit 23), scale byte `j` of A and of B (bits 29-30 and 4-5).
@@ -119,12 +136,32 @@ __device__ __forceinline__ void tc_mma_mx_pair(uint32_t d_tmem, uint64_t adesc, 
       : "memory");
 }
 
-// Byte offset of scale (row m of half h, K block j) of tile t's K step s.
+// Byte offset of B's scale (row m of half h, K block j) of tile t's K step s: two blocks
+// (halves of 128 rows) per tile and K step.
 __host__ __device__ __forceinline__ size_t mx_sf_offset(int64_t t, int ksteps, int s, int h, int m, int j) {
   return (size_t)((t * ksteps + s) * 2 + h) * 512 + 16 * (m & 31) + 4 * (m >> 5) + j;
 }
+// The same for A: three blocks per tile and K step, the third for a folded tile's
+// remainder rows (rows 256.. of the group, m = row - 256).
+__host__ __device__ __forceinline__ size_t mx_sfa_offset(int64_t t, int ksteps, int s, int h, int m, int j) {
+  return (size_t)((t * ksteps + s) * 3 + h) * 512 + 16 * (m & 31) + 4 * (m >> 5) + j;
+}
 
-__device__ __forceinline__ int mx_mtiles(int rows) { return (rows + kMxTileM - 1) / kMxTileM; }
+// M tiles of a group of `rows` rows: 256 rows each, a group of 257..256 + fold rows one.
+__device__ __forceinline__ int mx_mtiles(int rows, int fold) {
+  if (fold > 0 && rows > kMxTileM && rows <= kMxTileM + fold) return 1;
+  return (rows + kMxTileM - 1) / kMxTileM;
+}
+// Whether tile m of a group of `rows` rows is folded; ns: the remainder's N (rows past
+// 256 rounded up to 32).
+__device__ __forceinline__ bool mx_is_fold(int rows, int m, int fold, int& ns) {
+  ns = 0;
+  if (fold > 0 && m == 0 && rows > kMxTileM && rows <= kMxTileM + fold) {
+    ns = (rows - kMxTileM + 31) & ~31;
+    return true;
+  }
+  return false;
+}
 
 // M tile m of a group of `rows` rows is a half tile (M = 128: 64 rows per CTA) when at
 // most 128 rows are left for it and half tiles are enabled; otherwise M = 256.
@@ -132,10 +169,19 @@ __device__ __forceinline__ bool mx_is_half(int rows, int m, int half) {
   return half && rows - m * kMxTileM <= 128;
 }
 
-// Place of tile row `within` (0..255) in the scale blocks: CTA half h and row m in it
-// (M = 256: 128 rows per CTA; M = 128: 64).
-__device__ __forceinline__ void mx_row_place(int within, bool half_tile, int& h, int& m) {
-  if (half_tile) { h = within >> 6; m = within & 63; }
+// Scale-block place of row `rr` of a group of `rows` rows: tile offset dt (from the
+// group's first tile), block h and row m in it.
+__device__ __forceinline__ void mx_a_place(int rows, int rr, int half, int fold, int& dt, int& h, int& m) {
+  int ns;
+  if (mx_is_fold(rows, 0, fold, ns)) {
+    dt = 0;
+    if (rr < kMxTileM) { h = rr >> 7; m = rr & 127; }
+    else { h = 2; m = rr - kMxTileM; }
+    return;
+  }
+  dt = rr / kMxTileM;
+  const int within = rr % kMxTileM;
+  if (mx_is_half(rows, dt, half)) { h = within >> 6; m = within & 63; }
   else { h = within >> 7; m = within & 127; }
 }
 
@@ -193,17 +239,32 @@ __device__ __forceinline__ uint8_t quant_gelu32(const uint32_t (&v)[32], uint8_t
   return mx_quant32(f, dst);
 }
 
-template <int EPI>
+// Quantises, along the 32 lanes of a warp (32 consecutive outputs of one row), the value
+// v of this lane: returns the E4M3 byte, and the block's scale byte through `sc`.
+__device__ __forceinline__ uint8_t mx_quant_lanes(float v, uint8_t& sc) {
+  float amax = fabsf(v);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const int s = mx_exponent(amax);
+  const float inv = __uint_as_float((uint32_t)(127 - s) << 23);
+  sc = (uint8_t)(s + 127);
+  return (uint8_t)__nv_cvt_float_to_fp8(v * inv, __NV_SATFINITE, __NV_E4M3);
+}
+
+template <int EPI, bool FOLD>
 __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __grid_constant__ MxArgs p) {
-  using C = MxCfg;
+  using C = MxCfgT<FOLD>;
   constexpr int S = C::kStages, BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* a_smem = smem;
   uint8_t* b_smem = smem + S * C::kABytes;
-  uint8_t* sfa_smem = smem + S * (C::kABytes + C::kBBytes);
+  uint8_t* r_smem = smem + S * (C::kABytes + C::kBBytes);
+  uint8_t* sfa_smem = r_smem + S * C::kRemBytes;
   uint8_t* sfb_smem = sfa_smem + S * C::kSfaBytes;
+  uint8_t* sfo_smem = sfb_smem + S * C::kSfbBytes;
+  uint8_t* sfr_smem = sfo_smem + S * C::kSfoBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
   // bars: full[S], empty[S], tmem_full, tmem_empty, qfull[Q], qempty[Q]
   volatile int* tq = reinterpret_cast<volatile int*>(bars + 2 * S + 2 + 2 * kTileQ);
@@ -213,6 +274,10 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
   int* mt = reinterpret_cast<int*>(smem + S * C::kStageBytes + C::kCtrl);
   const int G = p.G;
   int* off = mt + (G + 1);
+  // gate/up exchange of folded remainders: xbuf[h] = 64 outputs x 32 columns, then
+  // xfull[h], xempty[h] (FOLD only)
+  float* xbuf = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(off + (G + 1)) + 15) & ~(uintptr_t)15);
+  const uint32_t xbar0 = smem_u32(xbuf + 2 * 64 * 32);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -220,6 +285,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
   const uint32_t tfull = smem_u32(bars + 2 * S), tempty = smem_u32(bars + 2 * S + 1);
   const uint32_t qfull0 = smem_u32(bars + 2 * S + 2), qempty0 = smem_u32(bars + 2 * S + 2 + kTileQ);
+  const int fold = FOLD ? p.fold : 0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -233,6 +299,9 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
       // leader: MMA issuer + 8 epilogue warps; peer: producer + 8 epilogue warps
       mbar_init(qempty0 + 8 * i, 18);
     }
+    if (FOLD) {
+      for (int i = 0; i < 4; ++i) mbar_init(xbar0 + 8 * i, 2);   // xfull[2]: up warps; xempty[2]: gate warps
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tmap(&p.tmap_a);
@@ -240,6 +309,10 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
     prefetch_tmap(&p.tmap_b);
     prefetch_tmap(&p.tmap_sfa);
     prefetch_tmap(&p.tmap_sfb);
+    if (FOLD) {
+      prefetch_tmap(&p.tmap_a32);
+      prefetch_tmap(&p.tmap_sfb1);
+    }
   }
   for (int i = threadIdx.x; i <= G; i += blockDim.x) off[i] = p.group_offsets[i];
   if (warp == 1) {
@@ -250,7 +323,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   __syncthreads();
-  group_tile_prefix(off, G, mt, wsum, [](int rows) { return mx_mtiles(rows); });
+  group_tile_prefix(off, G, mt, wsum, [fold](int rows) { return mx_mtiles(rows, fold); });
   tc_fence_before();
   cluster_sync();               // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
@@ -275,11 +348,17 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
         if (tile < 0) break;
         int g, m, n;
         decode_tile(tile, mt, G, nb, g, m, n);
-        const bool hf = mx_is_half(off[g + 1] - off[g], m, p.half);
+        const int rows = off[g + 1] - off[g];
+        int ns;
+        const bool fd = FOLD && mx_is_fold(rows, m, fold, ns);
+        const bool hf = !fd && mx_is_half(rows, m, p.half);
         const int arow = off[g] + m * kMxTileM + (int)rank * (hf ? 64 : 128);
         const CUtensorMap* amap = hf ? &p.tmap_a64 : &p.tmap_a;
-        const uint32_t stage_tx = 2u * (uint32_t)(C::kStageBytes - (hf ? C::kABytes / 2 : 0));
+        const uint32_t stage_tx =
+            fd ? 2u * (uint32_t)C::kStageBytes
+               : 2u * (uint32_t)(C::kABytes + C::kBBytes + C::kSfaBytes + C::kSfbBytes - (hf ? C::kABytes / 2 : 0));
         const int brow = n * BN + (int)rank * 128;
+        const int rrow = off[g] + kMxTileM + (int)rank * (ns / 2);
         const int64_t ta = (int64_t)mt[g] + m;              // A's tile (scale blocks)
         const int64_t tb = (int64_t)g * nb + n;              // B's tile
         bool ok = true;
@@ -290,9 +369,18 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
           tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), amap, fb, kb * C::KS, arow);
           tma_load_3d_pair(smem_u32(b_smem + stage * C::kBBytes), &p.tmap_b, fb, kb * C::KS, brow, g);
           tma_load_2d_pair(smem_u32(sfa_smem + stage * C::kSfaBytes), &p.tmap_sfa, fb, 0,
-                           (int)(((ta * ksteps + kb) * 2 + rank) * 2));
+                           (int)(((ta * ksteps + kb) * 3 + rank) * 2));
           tma_load_2d_pair(smem_u32(sfb_smem + stage * C::kSfbBytes), &p.tmap_sfb, fb, 0,
                            (int)((tb * ksteps + kb) * 4));
+          if (FOLD && fd) {
+            // the remainder rows (this CTA's ns/2 of a 32-row box), their scale block
+            // (the third block, the same in both CTAs) and this CTA's own B scale block
+            tma_load_2d_pair(smem_u32(r_smem + stage * C::kRemBytes), &p.tmap_a32, fb, kb * C::KS, rrow);
+            tma_load_2d_pair(smem_u32(sfr_smem + stage * C::kSfrBytes), &p.tmap_sfa, fb, 0,
+                             (int)(((ta * ksteps + kb) * 3 + 2) * 2));
+            tma_load_2d_pair(smem_u32(sfo_smem + stage * C::kSfoBytes), &p.tmap_sfb1, fb, 0,
+                             (int)(((tb * ksteps + kb) * 2 + rank) * 2));
+          }
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -302,6 +390,8 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
     if (lane == 0 && leader) {
       // ---------------- scale copies and block-scaled pair MMAs (leader CTA) ----------------
       const uint32_t t_sfa = tmem_base + C::kSfaCol, t_sfb = tmem_base + C::kSfbCol;
+      const uint32_t t_ssfa = tmem_base + C::kSsfaCol, t_ssfb = tmem_base + C::kSsfbCol;
+      const uint32_t t_rem = tmem_base + C::kRemCol;
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_phase = 0;
@@ -310,7 +400,10 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
         if (tile < 0) break;
         int g, m, n;
         decode_tile(tile, mt, G, nb, g, m, n);
-        const bool hf = mx_is_half(off[g + 1] - off[g], m, p.half);
+        const int rows = off[g + 1] - off[g];
+        int ns;
+        const bool fd = FOLD && mx_is_fold(rows, m, fold, ns);
+        const bool hf = !fd && mx_is_half(rows, m, p.half);
         if (!mbar_wait(tempty, acc_phase ^ 1u, abort_flag, p.status)) break;
         acc_phase ^= 1u;
         tc_fence_after();
@@ -329,6 +422,12 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
             // M = 128: rows 0..127 in lane quarters 0 and 1, rows 128..255 in quarters 2 and 3
             tc_cp_sf_pair_64(t_sfb, sf_desc(sb));
           }
+          if (FOLD && fd) {
+            // remainder product: this CTA's weight slab as M (its own B block as A scales),
+            // the remainder rows as N (their block, rows n in lane n % 32, column n / 32)
+            tc_cp_sf_pair(t_ssfa, sf_desc(smem_u32(sfo_smem + stage * C::kSfoBytes)));
+            tc_cp_sf_pair(t_ssfb, sf_desc(smem_u32(sfr_smem + stage * C::kSfrBytes)));
+          }
           const uint64_t ad = sw128_desc(smem_u32(a_smem + stage * C::kABytes));
           const uint64_t bd = sw128_desc(smem_u32(b_smem + stage * C::kBBytes));
           const int mm = hf ? kMxTileM / 2 : kMxTileM;
@@ -336,6 +435,13 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
           for (int j = 0; j < 4; ++j)          // K = 32 per MMA: +32 bytes
             tc_mma_mx_pair(tmem_base, ad + 2 * j, bd + 2 * j, mx_idesc(mm, BN, j), (kb | j) != 0,
                            t_sfa | ((uint32_t)j << 30), t_sfb | ((uint32_t)j << 30));
+          if (FOLD && fd) {
+            const uint64_t rd = sw128_desc(smem_u32(r_smem + stage * C::kRemBytes));
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tc_mma_mx_pair(t_rem, bd + 2 * j, rd + 2 * j, mx_idesc(kMxTileM, ns, j), (kb | j) != 0,
+                             t_ssfa | ((uint32_t)j << 30), t_ssfb | ((uint32_t)j << 30));
+          }
           tc_commit_pair_both(empty0 + 8 * stage);
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
@@ -349,6 +455,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
     const int h = (warp - 2) >> 2;          // column half: TMEM columns 128 h .. 128 h + 127
     const uint32_t tempty_leader = map_to_cta(tempty, 0);
     uint32_t acc_phase = 0;
+    uint32_t xk = 0;                        // gate/up hand-overs of folded remainders so far
     for (int qi = 0;; ++qi) {
       const int tile = tq_take<true>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
       if (__any_sync(0xffffffffu, tile < 0)) break;
@@ -359,14 +466,19 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
       if (!__all_sync(0xffffffffu, ok)) break;
       acc_phase ^= 1u;
       tc_fence_after();
-      const bool hf = mx_is_half(off[g + 1] - off[g], m, p.half);
+      const int grows = off[g + 1] - off[g];
+      int ns;
+      const bool fd = FOLD && mx_is_fold(grows, m, fold, ns);
+      const bool hf = !fd && mx_is_half(grows, m, p.half);
       // M = 256: this CTA's rows 0..127 in lanes 0..127, tile columns 0..255; this warp takes
       //   columns 128 h .. + 127 of lanes 32 q ...
       // M = 128: this CTA's rows 0..63 in lanes 0..63 for tile columns [0, 128) and in lanes
       //   64..127 for [128, 256), at TMEM columns 0..127; this warp takes 64 of them (SwiGLU:
       //   32 gate and the matching 32 up columns).
+      // Folded: also the remainder product, CTA's weight row 32 q + lane x remainder rows
+      //   [h ns / 2, (h + 1) ns / 2) at TMEM columns kRemCol + ...
       const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16);
-      uint32_t v0[32], v1[32], v2[32], v3[32];
+      uint32_t v0[32], v1[32], v2[32], v3[32], ra[16], rb[16];
       if (!hf) {
         tmem_ld32(tl + h * 128, v0);
         tmem_ld32(tl + h * 128 + 32, v1);
@@ -378,6 +490,10 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
       } else {
         tmem_ld32(tl + h * 64, v0);
         tmem_ld32(tl + h * 64 + 32, v1);
+      }
+      if (FOLD && fd) {
+        tmem_ld16(tl + C::kRemCol + h * (ns / 2), ra);
+        if (ns == 64) tmem_ld16(tl + C::kRemCol + h * 32 + 16, rb);
       }
       tmem_ld_wait();
       tc_fence_before();
@@ -402,7 +518,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
           // [gate 64 | up 64] -> outputs n*128 + 64h + [0, 64): K step n, blocks 2h, 2h + 1
           uint8_t* dst = p.q_out + row * p.ldo + n * 128 + h * 64;
           const uint32_t s0 = quant_swiglu32(v0, v2, dst), s1 = quant_swiglu32(v1, v3, dst + 32);
-          *reinterpret_cast<uint16_t*>(p.q_sf + mx_sf_offset(t, qk, n, (int)rank, r, 2 * h)) =
+          *reinterpret_cast<uint16_t*>(p.q_sf + mx_sfa_offset(t, qk, n, (int)rank, r, 2 * h)) =
               (uint16_t)(s0 | (s1 << 8));
         } else {
           // GELU: outputs n*256 + 128h + [0, 128): K step 2n + h, blocks 0..3
@@ -410,7 +526,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
           const int s = 2 * n + h;
           const uint32_t s0 = quant_gelu32(v0, dst), s1 = quant_gelu32(v1, dst + 32);
           const uint32_t s2 = quant_gelu32(v2, dst + 64), s3 = quant_gelu32(v3, dst + 96);
-          *reinterpret_cast<uint32_t*>(p.q_sf + mx_sf_offset(t, qk, s, (int)rank, r, 0)) =
+          *reinterpret_cast<uint32_t*>(p.q_sf + mx_sfa_offset(t, qk, s, (int)rank, r, 0)) =
               s0 | (s1 << 8) | (s2 << 16) | (s3 << 24);
         }
       } else {
@@ -422,17 +538,85 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
         } else if (EPI == EPI_SWIGLU) {
           // outputs n*128 + 64 cq + 32 h + [0, 32): K step n, block 2 cq + h
           uint8_t* dst = p.q_out + row * p.ldo + n * 128 + cq * 64 + h * 32;
-          p.q_sf[mx_sf_offset(t, qk, n, (int)rank, r, 2 * cq + h)] = quant_swiglu32(v0, v2, dst);
+          p.q_sf[mx_sfa_offset(t, qk, n, (int)rank, r, 2 * cq + h)] = quant_swiglu32(v0, v2, dst);
         } else {
           // outputs n*256 + 128 cq + 64 h + [0, 64): K step 2n + cq, blocks 2h, 2h + 1
           uint8_t* dst = p.q_out + row * p.ldo + n * BN + cq * 128 + h * 64;
           const int s = 2 * n + cq;
           const uint32_t s0 = quant_gelu32(v0, dst), s1 = quant_gelu32(v1, dst + 32);
-          *reinterpret_cast<uint16_t*>(p.q_sf + mx_sf_offset(t, qk, s, (int)rank, r, 2 * h)) =
+          *reinterpret_cast<uint16_t*>(p.q_sf + mx_sfa_offset(t, qk, s, (int)rank, r, 2 * h)) =
               (uint16_t)(s0 | (s1 << 8));
         }
       }
       __syncwarp();
+      if (FOLD && fd) {
+        // The remainder: rows rbase + c, c in [h ns / 2, (h + 1) ns / 2) (local cc), and the
+        // CTA's weight row wm = 32 q + lane, i.e. per 256-wide N block n: paired, the gate
+        // (wm < 64) or up (wm >= 64) factor of output n*128 + 64 rank + wm % 64; plain,
+        // output n*256 + 128 rank + wm.  Stores go one element per lane (a warp writes 32
+        // consecutive outputs of a row); the activation is quantised across the warp's
+        // 32 lanes, one block per remainder row.
+        const int64_t rbase = (int64_t)off[g] + kMxTileM;
+        const int nh = ns / 2;
+        const int c0 = h * nh;
+        if (EPI == EPI_STORE) {
+          const int col = n * BN + (int)rank * 128 + q * 32 + lane;
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) {
+            if (cc < nh && rbase + c0 + cc < off[g + 1])
+              p.out[(rbase + c0 + cc) * p.ldo + col] = __float2bfloat16_rn(__uint_as_float(cc < 16 ? ra[cc] : rb[cc - 16]));
+          }
+        } else if (EPI == EPI_GELU) {
+          const int col = n * BN + (int)rank * 128 + q * 32 + lane;
+          const int ks = col / C::KS, jb = (col / 32) & 3;
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) {
+            if (cc < nh && rbase + c0 + cc < off[g + 1]) {       // warp-uniform
+              uint8_t sc;
+              const uint8_t qv = mx_quant_lanes(gelu_f(__uint_as_float(cc < 16 ? ra[cc] : rb[cc - 16])), sc);
+              p.q_out[(rbase + c0 + cc) * p.ldo + col] = qv;
+              if (lane == 0) p.q_sf[mx_sfa_offset(t, qk, ks, 2, c0 + cc, jb)] = sc;
+            }
+          }
+        } else {
+          // SwiGLU: the up factors (quarters 2, 3) pass through xbuf[h] to the gate warps
+          float* xb = xbuf + h * (64 * 32);
+          const uint32_t xfull = xbar0 + 8 * h, xempty = xbar0 + 16 + 8 * h;
+          const int i = (q & 1) * 32 + lane;                // output among the CTA's 64
+          const uint32_t par = xk & 1u;
+          ++xk;
+          bool xok = true;
+          if (q >= 2) {
+            if (lane == 0) xok = mbar_wait(xempty, par ^ 1u, abort_flag, p.status);
+            if (!__all_sync(0xffffffffu, xok)) break;
+#pragma unroll
+            for (int cc = 0; cc < 32; ++cc)
+              if (cc < nh) xb[cc * 64 + i] = __uint_as_float(cc < 16 ? ra[cc] : rb[cc - 16]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xfull);
+          } else {
+            if (lane == 0) xok = mbar_wait(xfull, par, abort_flag, p.status);
+            if (!__all_sync(0xffffffffu, xok)) break;
+            float u[32];
+#pragma unroll
+            for (int cc = 0; cc < 32; ++cc) u[cc] = cc < nh ? xb[cc * 64 + i] : 0.f;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xempty);              // xbuf[h] may be rewritten
+            const int col = n * 128 + (int)rank * 64 + i;    // a 32-block: lanes 0..31 of this warp
+            const int ks = col / C::KS, jb = (col / 32) & 3;
+#pragma unroll
+            for (int cc = 0; cc < 32; ++cc) {
+              if (cc < nh && rbase + c0 + cc < off[g + 1]) {     // warp-uniform
+                uint8_t sc;
+                const uint8_t qv = mx_quant_lanes(silu_f(__uint_as_float(cc < 16 ? ra[cc] : rb[cc - 16])) * u[cc], sc);
+                p.q_out[(rbase + c0 + cc) * p.ldo + col] = qv;
+                if (lane == 0) p.q_sf[mx_sfa_offset(t, qk, ks, 2, c0 + cc, jb)] = sc;
+              }
+            }
+          }
+        }
+        __syncwarp();
+      }
     }
   }
 
@@ -473,10 +657,10 @@ bool make_map_sf(CUtensorMap* m, const void* base, size_t bytes, uint32_t box_ro
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI>
+template <int EPI, bool FOLD>
 cudaError_t launch_mx(const MxArgs& a, int clusters, cudaStream_t s) {
-  const size_t smem = MxCfg::smem_bytes(a.G);
-  auto kern = grouped_gemm_mx_kernel<EPI>;
+  const size_t smem = MxCfgT<FOLD>::smem_bytes(a.G);
+  auto kern = grouped_gemm_mx_kernel<EPI, FOLD>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg;
@@ -520,15 +704,15 @@ mx_block_scales_kernel(const uint32_t* __restrict__ rowmajor, uint8_t* __restric
 // of the token), so the bf16 x_perm is never written.
 __global__ void __launch_bounds__(256)
 mx_quant_a_kernel(const bf16* __restrict__ x, const int32_t* __restrict__ src, int k,
-                  const int32_t* __restrict__ group_offsets, int G, int K, int half, uint8_t* __restrict__ q,
-                  uint8_t* __restrict__ sf) {
+                  const int32_t* __restrict__ group_offsets, int G, int K, int half, int fold,
+                  uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
   extern __shared__ int sh[];
   int* mt = sh;                 // [G + 1]
   int* off = sh + (G + 1);      // [G + 1]
   int* wsum = off + (G + 1);    // [8]
   for (int i = threadIdx.x; i <= G; i += blockDim.x) off[i] = group_offsets[i];
   __syncthreads();
-  group_tile_prefix(off, G, mt, wsum, [](int rows) { return mx_mtiles(rows); });
+  group_tile_prefix(off, G, mt, wsum, [fold](int rows) { return mx_mtiles(rows, fold); });
   const int lane = threadIdx.x & 31;
   const int warps = (int)(gridDim.x * blockDim.x) >> 5;
   const int nblk = K / 32, ksteps = K / MxCfg::KS;
@@ -540,9 +724,9 @@ mx_quant_a_kernel(const bf16* __restrict__ x, const int32_t* __restrict__ src, i
       if (off[mid] <= r) lo = mid; else hi = mid;
     }
     const int rr = r - off[lo];
-    const int64_t t = (int64_t)mt[lo] + rr / kMxTileM;
-    int h, m;
-    mx_row_place(rr % kMxTileM, mx_is_half(off[lo + 1] - off[lo], rr / kMxTileM, half), h, m);
+    int dt, h, m;
+    mx_a_place(off[lo + 1] - off[lo], rr, half, fold, dt, h, m);
+    const int64_t t = (int64_t)mt[lo] + dt;
     const bf16* xr = x + (src != nullptr ? (int64_t)(__ldg(src + r) / k) : (int64_t)r) * K;
     // lane b takes block b (coalesced); the four blocks of a K step sit in four
     // consecutive lanes (nblk % 4 == 0), whose scales go out as one word
@@ -570,7 +754,7 @@ mx_quant_a_kernel(const bf16* __restrict__ x, const int32_t* __restrict__ src, i
       const uint32_t s2 = __shfl_down_sync(0xffffffffu, sc, 2);
       const uint32_t s3 = __shfl_down_sync(0xffffffffu, sc, 3);
       if (ok && (lane & 3) == 0)
-        *reinterpret_cast<uint32_t*>(sf + mx_sf_offset(t, ksteps, b >> 2, h, m, 0)) =
+        *reinterpret_cast<uint32_t*>(sf + mx_sfa_offset(t, ksteps, b >> 2, h, m, 0)) =
             sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
     }
   }
@@ -579,6 +763,7 @@ mx_quant_a_kernel(const bf16* __restrict__ x, const int32_t* __restrict__ src, i
 }  // namespace
 
 size_t mx_sf_bytes(int64_t tiles, int K) { return (size_t)tiles * (K / MxCfg::KS) * 1024; }
+size_t mx_sfa_bytes(int64_t tiles, int K) { return (size_t)tiles * (K / MxCfg::KS) * 1536; }
 
 cudaError_t launch_mx_block_scales(const uint8_t* rowmajor, uint8_t* blocked, int64_t rows, int K,
                                    cudaStream_t s) {
@@ -593,15 +778,15 @@ cudaError_t launch_mx_block_scales(const uint8_t* rowmajor, uint8_t* blocked, in
 }
 
 cudaError_t launch_mx_quant_a(const bf16* x, const int32_t* src, int k, int64_t rows,
-                              const int32_t* group_offsets, int G, int K, int half_tiles, uint8_t* q, uint8_t* sf,
-                              cudaStream_t s) {
+                              const int32_t* group_offsets, int G, int K, int half_tiles, int fold, uint8_t* q,
+                              uint8_t* sf, cudaStream_t s) {
   if (K % MxCfg::KS != 0 || G <= 0) return cudaErrorInvalidValue;
   if (rows == 0) return cudaSuccess;
   const size_t smem = (2 * (size_t)(G + 1) + 8) * sizeof(int);
   if (smem > 48 * 1024) return cudaErrorInvalidValue;
   int64_t grid = (rows + 7) / 8;                 // 8 rows (warps) per block
   if (grid > 4 * (int64_t)sm_count()) grid = 4 * (int64_t)sm_count();
-  mx_quant_a_kernel<<<(int)grid, 256, smem, s>>>(x, src, k, group_offsets, G, K, half_tiles, q, sf);
+  mx_quant_a_kernel<<<(int)grid, 256, smem, s>>>(x, src, k, group_offsets, G, K, half_tiles, fold, q, sf);
   return cudaGetLastError();
 }
 
@@ -616,10 +801,11 @@ cudaError_t launch_grouped_mx(const MxProblem& p, cudaStream_t s) {
   memset(&a, 0, sizeof(a));
   const uint64_t da[2] = {(uint64_t)p.K, (uint64_t)p.a_rows};
   const uint64_t db[3] = {(uint64_t)p.K, (uint64_t)p.N, (uint64_t)p.G};
+  const size_t sfb_bytes = mx_sf_bytes((int64_t)p.G * (p.N / MxCfg::BN), p.K);
   if (!make_map_u8(&a.tmap_a, p.A, 2, da, 128) || !make_map_u8(&a.tmap_a64, p.A, 2, da, 64) ||
-      !make_map_u8(&a.tmap_b, p.B, 3, db, 128) ||
-      !make_map_sf(&a.tmap_sfa, p.sa, mx_sf_bytes(tiles_m, p.K), 2) ||
-      !make_map_sf(&a.tmap_sfb, p.sb, mx_sf_bytes((int64_t)p.G * (p.N / MxCfg::BN), p.K), 4))
+      !make_map_u8(&a.tmap_a32, p.A, 2, da, 32) || !make_map_u8(&a.tmap_b, p.B, 3, db, 128) ||
+      !make_map_sf(&a.tmap_sfa, p.sa, mx_sfa_bytes(tiles_m, p.K), 2) ||
+      !make_map_sf(&a.tmap_sfb, p.sb, sfb_bytes, 4) || !make_map_sf(&a.tmap_sfb1, p.sb, sfb_bytes, 2))
     return cudaErrorInvalidValue;
   a.group_offsets = p.group_offsets;
   a.G = p.G;
@@ -630,14 +816,20 @@ cudaError_t launch_grouped_mx(const MxProblem& p, cudaStream_t s) {
   a.q_out = p.q_out;
   a.q_sf = p.q_sf;
   a.half = p.half_tiles;
+  a.fold = p.fold;
   a.status = p.status;
   a.counter = p.counter;
   const int64_t tiles = tiles_m * (int64_t)(p.N / MxCfg::BN);
   const int pairs = sm_count() / 2;
   const int clusters = (int)(tiles < pairs ? (tiles > 0 ? tiles : 1) : pairs);
-  if (p.epi == EPI_SWIGLU) return launch_mx<EPI_SWIGLU>(a, clusters, s);
-  if (p.epi == EPI_GELU) return launch_mx<EPI_GELU>(a, clusters, s);
-  return launch_mx<EPI_STORE>(a, clusters, s);
+  if (p.fold > 0) {
+    if (p.epi == EPI_SWIGLU) return launch_mx<EPI_SWIGLU, true>(a, clusters, s);
+    if (p.epi == EPI_GELU) return launch_mx<EPI_GELU, true>(a, clusters, s);
+    return launch_mx<EPI_STORE, true>(a, clusters, s);
+  }
+  if (p.epi == EPI_SWIGLU) return launch_mx<EPI_SWIGLU, false>(a, clusters, s);
+  if (p.epi == EPI_GELU) return launch_mx<EPI_GELU, false>(a, clusters, s);
+  return launch_mx<EPI_STORE, false>(a, clusters, s);
 }
 
 }  // namespace moe

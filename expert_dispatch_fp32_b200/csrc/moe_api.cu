@@ -71,9 +71,9 @@ MxWsLayout mx_ws_layout(const moe_config& c) {
   const int64_t tiles = (int64_t)(R / 256) + c.E;     // bounds the 256-row tiles of all experts
   size_t o = ws_layout(c).total;
   L.xq = o;       o = align256(o + R * D);
-  L.xsf = o;      o = align256(o + mx_sf_bytes(tiles, c.D));
+  L.xsf = o;      o = align256(o + mx_sfa_bytes(tiles, c.D));
   L.aq = o;       o = align256(o + R * F);
-  L.asf = o;      o = align256(o + mx_sf_bytes(tiles, c.F));
+  L.asf = o;      o = align256(o + mx_sfa_bytes(tiles, c.F));
   L.counters = o; o = align256(o + 2 * sizeof(int32_t));
   L.total = o;
   return L;
@@ -639,6 +639,12 @@ static int mx_half_tiles() {
   const char* env = getenv("MOE_MX_HALF");
   return (env && env[0] == '0') ? 0 : 1;
 }
+// A single-band group of 257..320 rows runs as one folded tile (the remainder as a product
+// with the weights as M); MOE_MX_FOLD=0: as a full tile and a second one, for comparison.
+static int mx_fold() {
+  const char* env = getenv("MOE_MX_FOLD");
+  return (env && env[0] == '0') ? 0 : 64;
+}
 
 // MXFP8 routed experts: 256-wide N tiles on both GEMMs (gate_up width and D multiples of
 // 256) and 128-deep K steps (D and F multiples of 128).
@@ -707,12 +713,12 @@ moe_status moe_expert_ffn_mxfp8(const moe_config* cfg, const void* x_perm, const
   const int nup = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
   int32_t* ctr = (int32_t*)(ws + L.counters);
   if (R > 0) {
-    const int half = mx_half_tiles();
+    const int half = mx_half_tiles(), fold = mx_fold();
     cudaError_t err = cudaMemsetAsync(ctr, 0, 2 * sizeof(int32_t), s);
     // x_perm NULL: moe_dispatch_mxfp8 has already put the quantised rows in the workspace
     if (err == cudaSuccess && x_perm != nullptr)
-      err = launch_mx_quant_a((const bf16*)x_perm, nullptr, 1, R, expert_offsets, c.E, c.D, half, ws + L.xq,
-                              ws + L.xsf, s);
+      err = launch_mx_quant_a((const bf16*)x_perm, nullptr, 1, R, expert_offsets, c.E, c.D, half, fold,
+                              ws + L.xq, ws + L.xsf, s);
     // gate_up (or W1): the activation comes out quantised, with the down projection's scales
     MxProblem up;
     memset(&up, 0, sizeof(up));
@@ -723,6 +729,7 @@ moe_status moe_expert_ffn_mxfp8(const moe_config* cfg, const void* x_perm, const
     up.q_out = ws + L.aq; up.q_sf = ws + L.asf; up.ldo = c.F;
     up.epi = c.act == MOE_ACT_SWIGLU ? EPI_SWIGLU : EPI_GELU;
     up.half_tiles = half;
+    up.fold = fold;
     up.status = status; up.counter = ctr;
     if (err == cudaSuccess) err = launch_grouped_mx(up, s);
     MxProblem dn = up;
@@ -756,7 +763,7 @@ moe_status moe_dispatch_mxfp8(const moe_config* cfg, const void* x, const int32_
   const MxWsLayout L = mx_ws_layout(c);
   uint8_t* ws = (uint8_t*)workspace;
   return cuda_status(launch_mx_quant_a((const bf16*)x, src, c.top_k, R, expert_offsets, c.E, c.D,
-                                       mx_half_tiles(), ws + L.xq, ws + L.xsf, as_stream(stream)));
+                                       mx_half_tiles(), mx_fold(), ws + L.xq, ws + L.xsf, as_stream(stream)));
 }
 
 moe_status moe_mxfp8_quantize(const void* x, int64_t rows, int32_t K, void* q, void* scales,

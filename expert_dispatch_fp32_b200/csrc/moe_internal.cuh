@@ -123,22 +123,25 @@ struct MxProblem {
   uint8_t* q_out; uint8_t* q_sf;          // EPI_SWIGLU / EPI_GELU: E4M3 [a_rows, ldo] + scale blocks
   int epi;
   int half_tiles;                         // a group's last <= 128 rows as an M = 128 tile
+  int fold;                               // > 0: a group of 257..256 + fold rows as one folded tile
   int32_t* status;
   int32_t* counter;
 };
 cudaError_t launch_grouped_mx(const MxProblem& p, cudaStream_t s);
-// Bytes of the scale blocks of `tiles` 256-row tiles over K.
+// Bytes of the scale blocks of `tiles` 256-row tiles over K: a B operand (two 128-row
+// blocks per tile and K step) and an A operand (a third block for a folded remainder).
 size_t mx_sf_bytes(int64_t tiles, int K);
+size_t mx_sfa_bytes(int64_t tiles, int K);
 // Row-major scales [rows, K/32] -> the scale blocks of a B operand (rows % 256 == 0,
 // K % 128 == 0).
 cudaError_t launch_mx_block_scales(const uint8_t* rowmajor, uint8_t* blocked, int64_t rows, int K,
                                    cudaStream_t s);
 // bf16 rows grouped by group_offsets -> E4M3 rows and the scale blocks of an A operand.
-// half_tiles: the tiling of the GEMM that reads the blocks (MxProblem::half_tiles).  Row r
+// half_tiles, fold: the tiling of the GEMM that reads the blocks (MxProblem).  Row r
 // comes from x[r], or with src from x[src[r] / k] (dispatch and quantisation in one pass).
 cudaError_t launch_mx_quant_a(const bf16* x, const int32_t* src, int k, int64_t rows,
-                              const int32_t* group_offsets, int G, int K, int half_tiles, uint8_t* q, uint8_t* sf,
-                              cudaStream_t s);
+                              const int32_t* group_offsets, int G, int K, int half_tiles, int fold, uint8_t* q,
+                              uint8_t* sf, cudaStream_t s);
 // Peer-memory exchange (ep_peer.cu).
 cudaError_t launch_ep_send_counts(const moe_ep_peers& p, int rank0, int nlocal, const int32_t* counts,
                                   int E, uint32_t epoch, cudaStream_t s);

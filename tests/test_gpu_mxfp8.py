@@ -183,3 +183,54 @@ def test_mxfp8_dispatch_equals_quantised_x_perm(half, monkeypatch):
     torch.cuda.synchronize()
     layer.check_status()
     assert torch.equal(y_a, y_b)
+
+
+MX_UNEVEN = [0, 1, 64, 65, 128, 129, 200, 256, 257, 270, 288, 289, 300, 320, 321, 384, 385, 513, 3, 0,
+             700, 260]
+
+
+@pytest.mark.parametrize("act", ["swiglu", "gelu"])
+@pytest.mark.parametrize("fold", ["1", "0"])
+def test_mxfp8_uneven_expert_tiles(act, fold, monkeypatch):
+    """Every routed row of the MXFP8 expert FFN against the oracle on quantised operands,
+    with hand-set expert sizes that put each expert's last tile in every case: folded
+    remainders of 1..32 and 33..64 rows (257..320-row experts), M = 128 tiles, full tiles,
+    several bands, a single row and empty experts; folding on and off."""
+    import moe_workloads as W
+    from parity_helpers import f64, make_layer, up_weights
+    monkeypatch.setenv("MOE_MX_FOLD", fold)
+    counts = np.array(MX_UNEVEN)
+    E, T = counts.size, int(counts.sum())                # top-1: one row per token
+    wl = W.Workload(name="mxu", T=T, D=256, E=E, ep_size=2, top_k=1, F=256, act=act, seed=44)
+    inp = W.make_inputs(wl, device="cuda")
+    layer = make_layer(wl, inp)
+    b = layer.allocate(T)
+    cfg = layer.config(T)
+    rng = np.random.default_rng(12)
+    assign = rng.permutation(np.repeat(np.arange(E), counts)).astype(np.int32)
+    idx = torch.from_numpy(assign.reshape(T, 1)).cuda()
+    b["status"].zero_()
+    M.moe_preprocess(cfg, idx, b["counts"], b["expert_offsets"], b["rank_splits"], b["rank_offsets"],
+                     b["pos"], b["src"], b["workspace"], b["status"])
+    g = torch.Generator(device="cuda")
+    g.manual_seed(6)
+    x_perm = torch.randn((T, wl.D), generator=g, device="cuda").to(torch.bfloat16)
+    pmx = torch.empty(M.moe_packed_weights_mxfp8_size(cfg), dtype=torch.uint8, device="cuda")
+    M.moe_prepare_weights_mxfp8(cfg, layer.packed, pmx)
+    ws = torch.full((M.moe_workspace_mxfp8_size(cfg),), 0x7F, dtype=torch.uint8, device="cuda")
+    y = torch.full_like(b["y_perm"], float("nan"))
+    M.moe_expert_ffn_mxfp8(cfg, x_perm, None, b["expert_offsets"], layer.packed, pmx, y, None, ws, b["status"])
+    torch.cuda.synchronize()
+    assert int(b["status"].item()) == 0
+    off = b["expert_offsets"].cpu().numpy()
+    assert np.array_equal(np.diff(off), counts)
+    xp, yp = f64(x_perm), f64(y)
+    wup = up_weights(wl, inp)
+    for e in range(E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi == lo:
+            continue
+        ref = _mx_oracle_expert(xp[lo:hi], f64(wup[e]), f64(inp["w_down"][e]), act)
+        assert np.isfinite(yp[lo:hi]).all(), f"expert {e}: unwritten rows"
+        from parity_helpers import assert_layer_close
+        assert_layer_close(yp[lo:hi], ref, np.zeros_like(ref), f"mxfp8 y_perm expert {e} ({hi - lo} rows)")
