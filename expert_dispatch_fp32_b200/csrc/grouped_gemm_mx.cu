@@ -266,8 +266,8 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
   uint8_t* sfo_smem = sfb_smem + S * C::kSfbBytes;
   uint8_t* sfr_smem = sfo_smem + S * C::kSfoBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
-  // bars: full[S], empty[S], tmem_full, tmem_empty, qfull[Q], qempty[Q]
-  volatile int* tq = reinterpret_cast<volatile int*>(bars + 2 * S + 2 + 2 * kTileQ);
+  // bars: full[S], empty[S], tmem_full, tmem_empty, tmem_empty_rem, qfull[Q], qempty[Q]
+  volatile int* tq = reinterpret_cast<volatile int*>(bars + 2 * S + 3 + 2 * kTileQ);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(tq) + kTileQ);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* wsum = const_cast<int*>(abort_flag) + 1;                 // [kMxThreads / 32]
@@ -284,7 +284,9 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
   const bool leader = rank == 0;
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
   const uint32_t tfull = smem_u32(bars + 2 * S), tempty = smem_u32(bars + 2 * S + 1);
-  const uint32_t qfull0 = smem_u32(bars + 2 * S + 2), qempty0 = smem_u32(bars + 2 * S + 2 + kTileQ);
+  // the remainder accumulator is released on its own, after the main one
+  const uint32_t tempty_rem = smem_u32(bars + 2 * S + 2);
+  const uint32_t qfull0 = smem_u32(bars + 2 * S + 3), qempty0 = smem_u32(bars + 2 * S + 3 + kTileQ);
   const int fold = FOLD ? p.fold : 0;
 
   if (threadIdx.x == 0) {
@@ -294,6 +296,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
     }
     mbar_init(tfull, 1);
     mbar_init(tempty, 16);                   // 8 epilogue warps x 2 CTAs
+    mbar_init(tempty_rem, 16);
     for (int i = 0; i < kTileQ; ++i) {
       mbar_init(qfull0 + 8 * i, 1);
       // leader: MMA issuer + 8 epilogue warps; peer: producer + 8 epilogue warps
@@ -394,7 +397,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
       const uint32_t t_rem = tmem_base + C::kRemCol;
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t acc_phase = 0;
+      uint32_t acc_phase = 0, rem_phase = 0;
       for (int qi = 0;; ++qi) {
         const int tile = tq_take<false>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
         if (tile < 0) break;
@@ -406,6 +409,10 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
         const bool hf = !fd && mx_is_half(rows, m, p.half);
         if (!mbar_wait(tempty, acc_phase ^ 1u, abort_flag, p.status)) break;
         acc_phase ^= 1u;
+        if (fd) {                              // the previous folded tile's remainder is read out
+          if (!mbar_wait(tempty_rem, rem_phase ^ 1u, abort_flag, p.status)) break;
+          rem_phase ^= 1u;
+        }
         tc_fence_after();
         bool ok = true;
         for (int kb = 0; kb < ksteps; ++kb) {
@@ -454,6 +461,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
     const int q = warp & 3;                 // TMEM lane quarter this warp may read
     const int h = (warp - 2) >> 2;          // column half: TMEM columns 128 h .. 128 h + 127
     const uint32_t tempty_leader = map_to_cta(tempty, 0);
+    const uint32_t tempty_rem_leader = map_to_cta(tempty_rem, 0);
     uint32_t acc_phase = 0;
     uint32_t xk = 0;                        // gate/up hand-overs of folded remainders so far
     for (int qi = 0;; ++qi) {
@@ -478,7 +486,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
       // Folded: also the remainder product, CTA's weight row 32 q + lane x remainder rows
       //   [h ns / 2, (h + 1) ns / 2) at TMEM columns kRemCol + ...
       const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16);
-      uint32_t v0[32], v1[32], v2[32], v3[32], ra[16], rb[16];
+      uint32_t v0[32], v1[32], v2[32], v3[32];
       if (!hf) {
         tmem_ld32(tl + h * 128, v0);
         tmem_ld32(tl + h * 128 + 32, v1);
@@ -490,10 +498,6 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
       } else {
         tmem_ld32(tl + h * 64, v0);
         tmem_ld32(tl + h * 64 + 32, v1);
-      }
-      if (FOLD && fd) {
-        tmem_ld16(tl + C::kRemCol + h * (ns / 2), ra);
-        if (ns == 64) tmem_ld16(tl + C::kRemCol + h * 32 + 16, rb);
       }
       tmem_ld_wait();
       tc_fence_before();
@@ -550,6 +554,14 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
       }
       __syncwarp();
       if (FOLD && fd) {
+        uint32_t ra[16], rb[16];
+        tc_fence_after();
+        tmem_ld16(tl + C::kRemCol + h * (ns / 2), ra);
+        if (ns == 64) tmem_ld16(tl + C::kRemCol + h * 32 + 16, rb);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty_rem_leader);   // the remainder may be reused
         // The remainder: rows rbase + c, c in [h ns / 2, (h + 1) ns / 2) (local cc), and the
         // CTA's weight row wm = 32 q + lane, i.e. per 256-wide N block n: paired, the gate
         // (wm < 64) or up (wm >= 64) factor of output n*128 + 64 rank + wm % 64; plain,
