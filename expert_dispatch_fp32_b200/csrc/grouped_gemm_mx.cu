@@ -13,34 +13,45 @@
 //   A   [rows, K]; rows of group g at [off[g], off[g+1]); M tiles of 256 rows per group,
 //       numbered across groups (tile t = tiles of the groups before g + m).
 //   B   [G, N, K]; N tiles of 256 rows.
-// Scales are stored "blocked": for tile t, K step s (128 K), half h (128 rows) a
+// Scales are stored "blocked": for tile t, K step s (128 K), block h (128 rows) a
 // 512-byte block holding row m's four scales (K blocks 4s..4s+3) at byte
 // 16 (m % 32) + 4 (m / 32) + j, the order tcgen05.cp .32x128b.warpx4 spreads over TMEM
-// (row m in lane m % 32 of every lane quarter, column m / 32, byte j).  Block (t, s, h)
-// sits at ((t * ksteps + s) * 2 + h) * 512 (mx_sf_offset), so CTA h of a pair loads its
-// A block and both B blocks of a K step with one TMA copy each.  A's blocks come from
-// the x_perm quantiser, which knows each row's tile, and from this kernel's own
-// epilogue for the down projection's A (the activation): the up projection and the down
-// projection tile the same groups the same way, so the epilogue of up tile t writes the
-// scales of down tile t.
+// (row m in lane m % 32 of every lane quarter, column m / 32, byte j).  B has two blocks
+// per tile and K step, at ((t * ksteps + s) * 2 + h) * 512 (mx_sf_offset); A has three,
+// at ((t * ksteps + s) * 3 + h) * 512 (mx_sfa_offset), the third for a folded tile's
+// remainder rows; so CTA h of a pair loads its A block and both B blocks of a K step with
+// one TMA copy each.  A's blocks come from the row quantiser (the dispatch), which knows
+// each row's tile, and from this kernel's own epilogue for the down projection's A (the
+// activation): the up projection and the down projection tile the same groups the same
+// way, so the epilogue of up tile t writes the scales of down tile t.
 //
 // The last tile of a group with at most 128 rows left runs as M = 128 (64 rows per CTA):
 // its A scales use the same blocks (rows 0..63 of each), B's scales go to lane quarters
 // 0-1 (rows 0..127) and 2-3 (rows 128..255), and the accumulator holds the CTA's row i in
 // lane i for tile columns [0, 128) and in lane 64 + i for [128, 256).
 //
+// With folding (FOLD), a group of 257..256 + fold rows runs as ONE tile: per K step the
+// M = 256 product of its first 256 rows and an M = 256 product of the pair's weight slabs
+// (as M, their scales each CTA's own B block) with the remainder rows (as N = 32 or 64,
+// their scales the third A block, read by both CTAs) into TMEM columns 320.., released on
+// a barrier of its own.  The epilogue quantises a remainder row's activation across the
+// 32 lanes of a warp (one weight row, i.e. one output, per lane); SwiGLU's up factors
+// (lane quarters 2-3) reach the gate warps through shared memory on two mbarrier pairs.
+//
 // A CTA pair, 10 warps per CTA:
 //   warp 0      TMA producer (lane 0, both CTAs): this CTA's 128 A rows, its 128 B rows,
-//               its A scale block and both B scale blocks of each K step into a 6-stage
-//               ring; the bytes complete on the leader's `full` barrier.
+//               its A scale block and both B scale blocks of each K step (and a folded
+//               tile's remainder rows and scale blocks) into a 6-stage ring (5 with
+//               folding); the bytes complete on the leader's `full` barrier.
 //   warp 1      TMEM (512 columns, both CTAs); in the leader, lane 0 copies the stage's
 //               scale blocks into TMEM (tcgen05.cp) and issues four M=256 N=256 K=32
-//               block-scaled MMAs, scale byte j selected per MMA; commits free the stage
-//               in both CTAs and hand the accumulator to the epilogue.
+//               block-scaled MMAs (and four remainder MMAs), scale byte j selected per
+//               MMA; commits free the stage in both CTAs and hand the accumulator to the
+//               epilogue.
 //   warps 2-9   epilogue: warp w reads lanes 32 (w % 4) .. of TMEM, columns
 //               128 ((w - 2) / 4) .. + 127, all into registers, then releases the
 //               accumulator (16 arrivals on the leader) before its math and stores.
-// The accumulator needs 256 TMEM columns and the scales 12, so there is one
+// The accumulator needs 256 TMEM columns and the scales 20, so there is one
 // accumulator: the early release keeps the tensor cores' wait per tile to the TMEM
 // read.  The scale columns are rewritten every K step: tcgen05 operations issued by one
 // thread run in order, so a step's copy lands after the previous step's MMAs read theirs.
