@@ -599,13 +599,15 @@ def run_ours(args):
     if want_cpu:
         # sized for 10-20 s of oracle work: the calibration undersizes large samples
         # (their BLAS steps run more efficiently per token), so a sample that ran under
-        # 8 s is scaled up once and timed again (the line reports the second)
+        # 8 s is scaled up and timed again, at most twice (the line reports the last)
         n_tok = args.cpu_sample or pick_sample(wl, cpu_host, 15.0)
         t = cpu_oracle_time(wl, cpu_host, n_tok, seed=1)
         cap = 16 * wl.T
-        if not args.cpu_sample and t < 8.0 and n_tok < cap:
+        for rep in range(2):
+            if args.cpu_sample or t >= 8.0 or n_tok >= cap:
+                break
             n_tok = int(min(cap, n_tok * 15.0 / max(t, 1e-6)))
-            t = cpu_oracle_time(wl, cpu_host, n_tok, seed=2)
+            t = cpu_oracle_time(wl, cpu_host, n_tok, seed=2 + rep)
         line["cpu_baseline"] = {"value": n_tok / t, "unit": "tokens/s", "cores": cpu_threads(),
                                 "kind": "oracle",
                                 "sample": f"{n_tok} tokens drawn from the {wl.name} batch "
