@@ -641,9 +641,15 @@ static int mx_half_tiles() {
 }
 // A single-band group of 257..320 rows runs as one folded tile (the remainder as a product
 // with the weights as M); MOE_MX_FOLD=0: as a full tile and a second one, for comparison.
-static int mx_fold() {
+// The folding kernel's ring has 5 stages instead of 6 (the remainder rows take shared
+// memory), which costs 5-7 % where no group folds; so it runs only where groups of about
+// 256 rows are expected: at most 512 routed rows per expert on average.  The quantiser
+// of the A rows and both GEMMs take the same decision from the same config.
+static int mx_fold(const moe_config& c) {
   const char* env = getenv("MOE_MX_FOLD");
-  return (env && env[0] == '0') ? 0 : 64;
+  if (env && env[0] == '0') return 0;
+  if (env && env[0] == '1') return 64;
+  return (int64_t)c.T * c.top_k <= 512LL * c.E ? 64 : 0;
 }
 
 // MXFP8 routed experts: 256-wide N tiles on both GEMMs (gate_up width and D multiples of
@@ -713,7 +719,7 @@ moe_status moe_expert_ffn_mxfp8(const moe_config* cfg, const void* x_perm, const
   const int nup = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
   int32_t* ctr = (int32_t*)(ws + L.counters);
   if (R > 0) {
-    const int half = mx_half_tiles(), fold = mx_fold();
+    const int half = mx_half_tiles(), fold = mx_fold(c);
     cudaError_t err = cudaMemsetAsync(ctr, 0, 2 * sizeof(int32_t), s);
     // x_perm NULL: moe_dispatch_mxfp8 has already put the quantised rows in the workspace
     if (err == cudaSuccess && x_perm != nullptr)
@@ -763,7 +769,7 @@ moe_status moe_dispatch_mxfp8(const moe_config* cfg, const void* x, const int32_
   const MxWsLayout L = mx_ws_layout(c);
   uint8_t* ws = (uint8_t*)workspace;
   return cuda_status(launch_mx_quant_a((const bf16*)x, src, c.top_k, R, expert_offsets, c.E, c.D,
-                                       mx_half_tiles(), mx_fold(), ws + L.xq, ws + L.xsf, as_stream(stream)));
+                                       mx_half_tiles(), mx_fold(c), ws + L.xq, ws + L.xsf, as_stream(stream)));
 }
 
 moe_status moe_mxfp8_quantize(const void* x, int64_t rows, int32_t K, void* q, void* scales,
