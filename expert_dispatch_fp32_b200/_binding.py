@@ -92,12 +92,16 @@ _SIGS = {
                                               ctypes.POINTER(ctypes.c_int32),
                                               ctypes.POINTER(ctypes.c_size_t),
                                               ctypes.POINTER(ctypes.c_float)]),
+    "moe_ipc_handle_bytes": (ctypes.c_int32, []),
+    "moe_ipc_export": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint64)]),
+    "moe_ipc_import": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_uint64, ctypes.POINTER(ctypes.c_void_p)]),
+    "moe_ipc_close": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_uint64]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_abi_version": (ctypes.c_int32, []),
 }
 
 
-ABI_VERSION = 2          # MOE_ABI_VERSION of include/moe.h
+ABI_VERSION = 3          # MOE_ABI_VERSION of include/moe.h
 
 
 def lib() -> ctypes.CDLL:
@@ -168,6 +172,33 @@ def moe_ep_return_rows(cfg, peers, rank0, nlocal, y_recv, local_offsets, epoch, 
 def moe_ep_wait_returned(cfg, peers, rank0, nlocal, epoch, status, stream=None):
     _call("moe_ep_wait_returned", ctypes.byref(cfg), ctypes.addressof(peers), rank0, nlocal, epoch,
           _p(status), _s(stream))
+
+
+def moe_ipc_handle_bytes() -> int:
+    return lib().moe_ipc_handle_bytes()
+
+
+def moe_ipc_export(ptr) -> tuple[bytes, int]:
+    """(handle bytes, offset) of the device allocation holding ``ptr`` (a tensor or an
+    address)."""
+    n = lib().moe_ipc_handle_bytes()
+    h = ctypes.create_string_buffer(n)
+    off = ctypes.c_uint64(0)
+    _call("moe_ipc_export", _p(ptr), h, ctypes.byref(off))
+    return h.raw, off.value
+
+
+def moe_ipc_import(handle: bytes, offset: int) -> int:
+    """Device address of another process's buffer (handle and offset from its
+    moe_ipc_export)."""
+    h = ctypes.create_string_buffer(bytes(handle), len(handle))
+    out = ctypes.c_void_p(0)
+    _call("moe_ipc_import", h, offset, ctypes.byref(out))
+    return int(out.value or 0)
+
+
+def moe_ipc_close(ptr: int, offset: int) -> None:
+    _call("moe_ipc_close", ptr, offset)
 
 
 def moe_mxfp8_quantize(x, rows, K, q, scales, stream=None):

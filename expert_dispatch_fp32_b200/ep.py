@@ -274,3 +274,206 @@ class PeerEPGroup:
         v = int(self.status.item())
         if v != B.MOE_OK:
             raise B.MoeError("device status", v)
+
+
+# --------------------------------------------------------------------------------------
+# One process per GPU: the same peer-memory exchange, each rank's buffers mapped into
+# the other ranks' processes
+# --------------------------------------------------------------------------------------
+
+EXCHANGE_BUFFERS = ("cnt", "flags", "recv_x", "recv_src", "recv_rank", "y_back")
+
+
+def exchange_layout(P, E, D, T, top_k, cap):
+    """Byte offsets and sizes of one rank's exchange buffers inside its single exchange
+    allocation (the same on every rank, so a peer's buffer is its mapped base plus the
+    offset): count matrix int32 [P, E], flags uint32 [3, P], received rows bf16 [cap, D]
+    with their sender rows and ranks int32 [cap], returned rows bf16 [T*k, D]."""
+    sizes = {"cnt": 4 * P * E, "flags": 4 * 3 * P, "recv_x": 2 * cap * D, "recv_src": 4 * cap,
+             "recv_rank": 4 * cap, "y_back": 2 * T * top_k * D}
+    off, o = {}, 0
+    for name in EXCHANGE_BUFFERS:
+        off[name] = o
+        o += (sizes[name] + 255) // 256 * 256
+    return off, sizes, o
+
+
+class CudaIpc:
+    """Maps exchange allocations between the processes of one node (libmoe.so's
+    moe_ipc_* calls: a CUDA IPC handle of the allocation plus the buffer's offset)."""
+
+    def export(self, t):
+        return B.moe_ipc_export(t)
+
+    def import_(self, handle, offset):
+        return B.moe_ipc_import(handle, offset)
+
+    def close(self, ptr, offset):
+        B.moe_ipc_close(ptr, offset)
+
+
+def peer_tables(rank, own_base, offsets, infos, ipc):
+    """Pointer tables of one rank: for each exchange buffer, entry p is rank p's buffer,
+    i.e. rank p's exchange allocation (this rank's own, or rank p's export mapped into
+    this process) plus the buffer's offset.  infos[p] is what rank p shared: its
+    exported (handle, offset).  Returns the tables (name -> P addresses) and the
+    mappings opened, (address, offset) pairs for ipc.close."""
+    P = len(infos)
+    bases, opened = [0] * P, []
+    for p in range(P):
+        if p == rank:
+            bases[p] = own_base
+            continue
+        handle, off = infos[p]["export"]
+        ptr = ipc.import_(handle, off)
+        opened.append((ptr, off))
+        bases[p] = ptr
+    return {name: [bases[p] + offsets[name] for p in range(P)] for name in EXCHANGE_BUFFERS}, opened
+
+
+def gather_infos(info, group=None):
+    """Every rank's `info` (host-side: host name, device id, exported handle), in rank
+    order, over the process group (any backend; one rank without a group)."""
+    if not dist.is_initialized():
+        return [info]
+    infos = [None] * dist.get_world_size(group)
+    dist.all_gather_object(infos, info, group=group)
+    return infos
+
+
+def check_peer_devices(infos):
+    """Every rank on its own GPU of one node: kernels of two ranks on one device would
+    wait on each other across launches (PeerEPGroup runs such ranks in one launch), and
+    the handles map only within a node."""
+    hosts = {inf["host"] for inf in infos}
+    if len(hosts) > 1:
+        raise RuntimeError(f"peer-memory exchange needs one node; ranks are on {sorted(hosts)}")
+    seen = {}
+    for p, inf in enumerate(infos):
+        if inf["device"] in seen:
+            raise RuntimeError(f"ranks {seen[inf['device']]} and {p} share device {inf['device']}: "
+                               "run ranks that share a GPU as one PeerEPGroup")
+        seen[inf["device"]] = p
+
+
+class PeerEPRank:
+    """One rank of the expert-parallel forward over peer memory, one process per GPU.
+
+    "Expert Parallel (EP)", Communication Pattern: rank r (its rank in `group`, P = the
+    group's size = ep) owns experts [r*El, (r+1)*El) and its own T tokens; the router
+    and the shared experts are replicated.  The exchanges are the moe_ep_* calls of
+    PeerEPGroup, each covering this rank alone (rank0 = r, nlocal = 1), with pointer
+    tables whose other entries are the other ranks' exchange buffers mapped into this
+    process once, at construction (moe_ipc_*: each rank exports its exchange
+    allocation, the handles go round the group with all_gather_object, each rank maps
+    the others').  Rows are stored straight into the owners' memory over NVLink /
+    NVSwitch and every wait is a flag in peer memory: no collective library and no host
+    round trip per forward.  Every rank calls forward the same number of times, with T
+    tokens each; close() (after the last forward, on every rank) unmaps the peers.
+    """
+
+    def __init__(self, group=None, *, D, E, top_k, F, T, w_router, w_gate_up_local, w_down_local,
+                 expert_bias=None, ws_gate_up=None, ws_down=None, act="swiglu", renormalize=True,
+                 x_dtype="bf16", ipc=None):
+        import socket
+        self.group = group
+        on = dist.is_initialized()
+        P = dist.get_world_size(group) if on else 1
+        r = dist.get_rank(group) if on else 0
+        if E % P:
+            raise ValueError("num_experts must be divisible by the number of ranks")
+        dev = w_router.device
+        self.D, self.E, self.P, self.rank, self.k, self.F, self.T = D, E, P, r, top_k, F, T
+        self.El = El = E // P
+        self.S = 0 if ws_gate_up is None else ws_gate_up.shape[0]
+        self.Fs = 0 if ws_gate_up is None else ws_down.shape[1]
+        self.cap = cap = P * T * min(top_k, El)
+        self.w_router = w_router.contiguous()
+        self.bias = None if expert_bias is None else expert_bias.contiguous()
+        self.tok_cfg = make_config(T, D, E, P, top_k, F, act, renormalize, x_dtype, self.S, self.Fs)
+        self.loc_cfg = make_config(cap, D, El, 1, 1, F, act, True, "bf16", self.S, self.Fs)
+        self.sh_cfg = make_config(T, D, El, 1, 1, F, act, True, "bf16", self.S, self.Fs)
+        i32 = lambda n: torch.zeros(n, dtype=torch.int32, device=dev)
+        R = T * top_k
+        self.packed = torch.empty(B.moe_packed_weights_size(self.loc_cfg), dtype=torch.uint8, device=dev)
+        B.moe_prepare_weights(self.loc_cfg, w_gate_up_local.contiguous(), w_down_local.contiguous(),
+                              None if ws_gate_up is None else ws_gate_up.contiguous(),
+                              None if ws_down is None else ws_down.contiguous(), self.packed)
+        self.topk_idx = torch.zeros((T, top_k), dtype=torch.int32, device=dev)
+        self.topk_w = torch.zeros((T, top_k), dtype=torch.float32, device=dev)
+        self.counts, self.offsets = i32(E), i32(E + 1)
+        self.splits, self.rank_offsets = i32(P), i32(P + 1)
+        self.pos, self.src = i32(R), i32(R)
+        self.ws_tok = torch.empty(max(B.moe_workspace_size(self.tok_cfg), 256), dtype=torch.uint8, device=dev)
+        # the exchange buffers: one zeroed allocation (flags start at 0, the epoch never is)
+        self.offsets_x, sizes, total = exchange_layout(P, E, D, T, top_k, cap)
+        self.xbuf = torch.zeros(total, dtype=torch.uint8, device=dev)
+        view = lambda name, dt, shape: self.xbuf[self.offsets_x[name]:self.offsets_x[name] + sizes[name]] \
+            .view(dt).view(shape)
+        self.recv_x = view("recv_x", torch.bfloat16, (cap, D))
+        self.y_back = view("y_back", torch.bfloat16, (R, D))
+        self.local_off = i32(El + 1)
+        self.act = torch.zeros((cap, F), dtype=torch.bfloat16, device=dev)
+        self.y_recv = torch.zeros((cap, D), dtype=torch.bfloat16, device=dev)
+        self.ws_loc = torch.empty(max(B.moe_workspace_size(self.loc_cfg), 256), dtype=torch.uint8, device=dev)
+        self.ws_sh = torch.empty(max(B.moe_workspace_size(self.sh_cfg), 256), dtype=torch.uint8, device=dev)
+        xdt = torch.float32 if x_dtype in ("f32", torch.float32) else torch.bfloat16
+        self.shared_out = torch.zeros((T, D), dtype=torch.bfloat16, device=dev) if self.S else None
+        self.out = torch.empty((T, D), dtype=xdt, device=dev)
+        self.done, self.status = i32(1), i32(1)
+        # map the peers' exchange allocations; the handles travel as host bytes
+        self.ipc = ipc if ipc is not None else CudaIpc()
+        props = torch.cuda.get_device_properties(dev)
+        info = {"host": socket.gethostname(), "device": str(getattr(props, "uuid", dev)),
+                "export": self.ipc.export(self.xbuf) if P > 1 else None}
+        infos = gather_infos(info, group)
+        check_peer_devices(infos)
+        tables, self._opened = peer_tables(r, self.xbuf.data_ptr(), self.offsets_x, infos, self.ipc)
+        self._tables = [torch.tensor(tables[name], dtype=torch.int64, device=dev) for name in EXCHANGE_BUFFERS]
+        self.peers = B.MoeEpPeers(P, cap, *[t.data_ptr() for t in self._tables])
+        self.epoch = 0
+        torch.cuda.synchronize(dev)
+        if on:
+            dist.barrier(group)     # every rank's flags are zero before any rank's first store
+
+    def forward(self, x, stream=None):
+        c, r = self.tok_cfg, self.rank
+        self.epoch = self.epoch % 0xFFFFFFFF + 1          # never 0, the flags' initial value
+        e = self.epoch
+        B.moe_route(c, x, self.w_router, self.bias, None, self.topk_idx, self.topk_w, self.ws_tok, stream)
+        B.moe_preprocess(c, self.topk_idx, self.counts, self.offsets, self.splits, self.rank_offsets,
+                         self.pos, self.src, self.ws_tok, self.status, stream)
+        # counts, then the token pre-all-to-all into the owners' buffers
+        B.moe_ep_send_counts(c, self.peers, r, 1, self.counts, e, stream)
+        B.moe_ep_send_rows(c, self.peers, r, 1, x, self.topk_idx, self.pos, self.offsets, e, self.done,
+                           self.status, stream)
+        B.moe_ep_recv_layout(c, self.peers, r, 1, self.local_off, e, self.status, stream)
+        B.moe_expert_ffn(self.loc_cfg, self.recv_x, None, self.local_off, self.packed, self.act,
+                         self.y_recv, None, self.ws_loc, self.status, stream)
+        # the token post-all-to-all back to the senders' dispatch rows
+        B.moe_ep_return_rows(c, self.peers, r, 1, self.y_recv, self.local_off, e, self.done,
+                             self.status, stream)
+        B.moe_ep_wait_returned(c, self.peers, r, 1, e, self.status, stream)
+        sh = None
+        if self.S:
+            sh = self.shared_out
+            B.moe_shared_ffn(self.sh_cfg, x, self.packed, sh, self.ws_sh, self.status, stream)
+        B.moe_combine_unpermute(c, self.y_back, self.pos, self.topk_w, x, sh, self.out, stream)
+        return self.out
+
+    __call__ = forward
+
+    def check_status(self):
+        v = int(self.status.item())
+        if v != B.MOE_OK:
+            raise B.MoeError("device status", v)
+
+    def close(self):
+        """Unmap the peers' buffers once every rank is done with the exchange (all ranks
+        call it; the rank's own allocation stays valid until the object is dropped)."""
+        torch.cuda.synchronize(self.xbuf.device)
+        if dist.is_initialized():
+            dist.barrier(self.group)
+        for ptr, off in self._opened:
+            self.ipc.close(ptr, off)
+        self._opened = []

@@ -41,8 +41,9 @@ extern "C" {
 #endif
 
 /* 2: the MXFP8 routed-expert calls, moe_dispatch_mxfp8, the router filter view and the
- * peer-memory exchange calls. */
-#define MOE_ABI_VERSION 2
+ * peer-memory exchange calls.  3: the moe_ipc_* calls that map another process's
+ * exchange buffers. */
+#define MOE_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -364,6 +365,33 @@ MOE_API moe_status moe_ep_return_rows(const moe_config* cfg, const moe_ep_peers*
 MOE_API moe_status moe_ep_wait_returned(const moe_config* cfg, const moe_ep_peers* peers,
                                         int32_t rank0, int32_t nlocal, uint32_t epoch,
                                         int32_t* status, void* stream);
+
+/* One process per GPU: the moe_ep_peers tables of a rank hold pointers into the other
+ * ranks' processes, mapped once before the first exchange ("Expert Parallel (EP)",
+ * Communication Pattern, steps 2 and 4: rows are stored straight into the owning
+ * rank's buffers).  Each rank exports its exchange buffers, sends the handle bytes and
+ * offsets to the others over its process group (host memory), and imports theirs.
+ * Setup-time calls (synchronous, no stream); the buffers must come from cudaMalloc
+ * (a caching allocator's blocks are fine; memory from cuMemCreate is not exportable
+ * and gives MOE_ERR_CUDA).  A rank never imports its own handle: its own table entry
+ * is its own pointer.
+ *
+ * Size in bytes of an exported handle (the bytes the caller sends to the other ranks). */
+MOE_API int32_t moe_ipc_handle_bytes(void);
+/* ptr: a device pointer inside a cudaMalloc allocation of the calling process.
+ * handle: host buffer of moe_ipc_handle_bytes() bytes, written: the allocation's
+ * handle.  offset: host, written: ptr's byte offset from the allocation's start.
+ * MOE_ERR_INVALID_ARG for a null argument or a pointer the driver does not know. */
+MOE_API moe_status moe_ipc_export(const void* ptr, void* handle, uint64_t* offset);
+/* Maps another process's allocation (handle and offset from its moe_ipc_export, on
+ * another device of this node) into this process, with peer access enabled on first
+ * use; *ptr (host, written) = the mapped buffer's device address.  The mapping stays
+ * until moe_ipc_close; the exporting process must keep the buffer alive until every
+ * importer has closed it.  MOE_ERR_CUDA if the driver refuses the handle (for
+ * instance a handle of this same process). */
+MOE_API moe_status moe_ipc_import(const void* handle, uint64_t offset, void** ptr);
+/* Unmaps a buffer mapped by moe_ipc_import (the same ptr and offset). */
+MOE_API moe_status moe_ipc_close(void* ptr, uint64_t offset);
 
 /* Self-check of device-side failure detection.  The cooperative kernels (moe_preprocess,
  * moe_route_dispatch) synchronise their blocks at a grid barrier whose wait is bounded

@@ -55,7 +55,7 @@ def good_cfg(B, **kw):
 
 
 def test_version_and_strings(B):
-    assert B.moe_abi_version() == B.ABI_VERSION == 2
+    assert B.moe_abi_version() == B.ABI_VERSION == 3
     assert B.moe_status_string(B.MOE_OK) == "ok"
     assert "range" in B.moe_status_string(B.MOE_ERR_INDEX_OOB)
     assert B.moe_status_string(99) == "unknown status"

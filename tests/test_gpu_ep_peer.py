@@ -14,7 +14,7 @@ import torch
 
 import expert_dispatch_fp32_b200 as M
 import moe_workloads as W
-from expert_dispatch_fp32_b200.ep import PeerEPGroup
+from expert_dispatch_fp32_b200.ep import PeerEPGroup, PeerEPRank
 from parity_helpers import assert_layer_close, f64, make_layer, oracle_layer, up_weights
 
 pytestmark = pytest.mark.gpu
@@ -96,3 +96,39 @@ def test_peer_exchange_wait_reports_timeout():
     layer = make_layer(wl, inp)
     for r in range(P):
         assert torch.equal(out[r], layer.forward(xs[r]))
+
+
+def test_per_process_rank_alone_equals_single_gpu_forward():
+    """PeerEPRank, the one-process-per-GPU form, with no process group (one rank): its
+    exchange calls cover rank 0 alone (rank0 = 0, nlocal = 1) through tables built
+    from its own exchange allocation; two forwards (two epochs) equal moe_forward bit
+    for bit.  Ranks on other GPUs would fill the other table entries with mappings
+    of their allocations (tests/test_ep_ipc_gloo.py covers that setup on CPU ranks)."""
+    wl = W.Workload(name="ep_rank1", T=384, D=256, E=16, ep_size=1, top_k=4, F=256, n_shared=1,
+                    F_shared=256, seed=25)
+    inp = W.make_inputs(wl, device="cuda")
+    rank = PeerEPRank(D=wl.D, E=wl.E, top_k=wl.top_k, F=wl.F, T=wl.T, w_router=inp["w_router"],
+                      w_gate_up_local=up_weights(wl, inp), w_down_local=inp["w_down"],
+                      expert_bias=inp["bias"], ws_gate_up=inp["ws_gate_up"], ws_down=inp["ws_down"],
+                      act=wl.act, renormalize=wl.renormalize, x_dtype=wl.x_dtype)
+    layer = make_layer(wl, inp)
+    x = W.make_x(wl, device="cuda", seed=7)
+    for it in range(2):
+        out = rank.forward(x).clone()
+        torch.cuda.synchronize()
+        rank.check_status()
+        ref = layer.forward(x).clone()
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref), it
+    assert int(rank.local_off[-1].item()) == wl.T * wl.top_k
+    rank.close()
+
+
+def test_ipc_export_reports_the_offset_in_the_allocation():
+    """moe_ipc_export names the allocation that holds a buffer and the buffer's offset
+    in it, so a peer maps the allocation once and adds the offset."""
+    t = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    h0, o0 = M.moe_ipc_export(t)
+    h1, o1 = M.moe_ipc_export(t[4096:])
+    assert len(h0) == M.moe_ipc_handle_bytes() == 64
+    assert h0 == h1 and o1 - o0 == 4096
