@@ -88,6 +88,9 @@ _SIGS = {
                                           _i32p, ctypes.c_uint32, _i32p, _i32p, _vp]),
     "moe_ep_wait_returned": (ctypes.c_int, [_cfgp, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
                                             ctypes.c_uint32, _i32p, _vp]),
+    "moe_ep_expert_ffn_return": (ctypes.c_int, [_cfgp, _cfgp, ctypes.c_void_p, ctypes.c_int32, _vp, _i32p,
+                                                _i32p, _i32p, _vp, _vp, _vp, _vp, ctypes.c_uint32, _i32p,
+                                                _i32p, _vp]),
     "moe_router_filter_view": (ctypes.c_int, [_cfgp, ctypes.POINTER(ctypes.c_size_t),
                                               ctypes.POINTER(ctypes.c_int32),
                                               ctypes.POINTER(ctypes.c_size_t),
@@ -167,6 +170,13 @@ def moe_ep_recv_layout(cfg, peers, rank0, nlocal, local_offsets, epoch, status, 
 def moe_ep_return_rows(cfg, peers, rank0, nlocal, y_recv, local_offsets, epoch, done, status, stream=None):
     _call("moe_ep_return_rows", ctypes.byref(cfg), ctypes.addressof(peers), rank0, nlocal, _p(y_recv),
           _p(local_offsets), epoch, _p(done), _p(status), _s(stream))
+
+
+def moe_ep_expert_ffn_return(cfg, local_cfg, peers, rank, recv_x, recv_src, recv_rank, local_offsets,
+                             packed, act, y_recv, workspace, epoch, done, status, stream=None):
+    _call("moe_ep_expert_ffn_return", ctypes.byref(cfg), ctypes.byref(local_cfg), ctypes.addressof(peers),
+          rank, _p(recv_x), _p(recv_src), _p(recv_rank), _p(local_offsets), _p(packed), _p(act), _p(y_recv),
+          _p(workspace), epoch, _p(done), _p(status), _s(stream))
 
 
 def moe_ep_wait_returned(cfg, peers, rank0, nlocal, epoch, status, stream=None):

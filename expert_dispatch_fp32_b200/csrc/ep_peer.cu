@@ -240,6 +240,13 @@ ep_return_rows_kernel(uint32_t* const* flags, const int32_t* const* recv_src,
   last_block_signal(done + li, flags, P, 2, d, epoch);
 }
 
+__global__ void ep_signal_returned_kernel(uint32_t* const* flags, int r, int P, uint32_t epoch) {
+  if (threadIdx.x == 0) {
+    __threadfence_system();
+    for (int d = 0; d < P; ++d) st_release_sys(flags[d] + 2 * P + r, epoch);
+  }
+}
+
 __global__ void ep_wait_returned_kernel(uint32_t* const* flags, int32_t* status, int rank0, int P,
                                         uint32_t epoch) {
   if (threadIdx.x == 0) wait_epoch(flags[rank0 + (int)blockIdx.x] + 2 * P, P, epoch, status);
@@ -296,6 +303,11 @@ cudaError_t launch_ep_return_rows(const moe_config& c, const moe_ep_peers& p, in
   ep_return_rows_kernel<<<grid, row_threads(c.D), 0, s>>>(
       p.flags, p.recv_src, p.recv_rank, p.y_back, static_cast<const bf16*>(y_recv), local_offsets, done,
       rank0, p.P, c.E, c.D, p.cap, c.T * c.top_k, epoch);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ep_signal_returned(const moe_ep_peers& p, int r, uint32_t epoch, cudaStream_t s) {
+  ep_signal_returned_kernel<<<1, 32, 0, s>>>(p.flags, r, p.P, epoch);
   return cudaGetLastError();
 }
 

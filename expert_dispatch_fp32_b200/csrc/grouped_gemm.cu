@@ -76,6 +76,10 @@ struct PhaseArgs {
   int32_t dep;               // phase whose band must be complete before A is read, or -1
   int32_t signal;            // 1: the epilogue counts stored tiles per band in done[]
   int32_t done_base;         // first done[] slot of this phase's bands (signal or dep source)
+  bf16* const* sc_base;      // EPI_STORE: row i to sc_base[sc_rank[i]] + sc_row[i] * ldo, or null
+  const int32_t* sc_rank;
+  const int32_t* sc_row;
+  int32_t sc_P, sc_rows;
 };
 struct PairArgs {
   PhaseArgs ph[kMaxPhases];
@@ -89,7 +93,21 @@ struct PairArgs {
   int32_t* status;
   int32_t* counter;          // tile counter, zero at launch
   int32_t* done;             // band completion counts, zero at launch
+  int32_t scatter;           // 1: a phase stores rows into other ranks' buffers (sc_base)
 };
+
+// Where output row `orow` of a scattering phase goes: the owning rank's buffer and row
+// (rank and row checked against the table; a bad one stores nothing).
+__device__ __forceinline__ void scatter_dst(const PhaseArgs& P, bool& valid, bf16*& o, int64_t& orow) {
+  if (!valid) return;
+  const int s = __ldg(P.sc_rank + orow), row = __ldg(P.sc_row + orow);
+  if ((unsigned)s >= (unsigned)P.sc_P || (unsigned)row >= (unsigned)P.sc_rows) {
+    valid = false;
+    return;
+  }
+  o = P.sc_base[s];
+  orow = row;
+}
 
 template <int BN>
 struct GemmCfg {
@@ -814,19 +832,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         const int row0 = t.base + (int)rank * kTileM;
         const int r = q * 32 + lane;
         const int col0 = paired ? t.n * (BN / 2) : t.n * BN;
-        const bool valid = r < min(t.end - row0, kTileM);
+        bool valid = r < min(t.end - row0, kTileM);
+        bf16* o = P.out;
+        int64_t orow = (int64_t)row0 + r;
+        if (P.sc_base != nullptr) scatter_dst(P, valid, o, orow);
         if (*any_fold) {
           // the head (TMEM columns 0..63) is released as soon as it is in registers: a
           // folded tile that follows puts its remainder there
-          epilogue_head_rt(P.epi, P.out, P.outf, P.ldo, tb, (int64_t)row0 + r, col0, valid,
-                           [&] { release(acc); });
+          epilogue_head_rt(P.epi, o, P.outf, P.ldo, tb, orow, col0, valid, [&] { release(acc); });
         } else {
           // no folded tile waits for a head: loads and stores interleaved, 32 columns at a time
-          epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, 0, 64, (int64_t)row0 + r, col0, valid);
+          epilogue_row_rt(P.epi, o, P.outf, P.ldo, tb, 0, 64, orow, col0, valid);
           release(acc);
         }
-        epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, 64, paired ? BN / 2 : BN, (int64_t)row0 + r,
-                        col0, valid);
+        epilogue_row_rt(P.epi, o, P.outf, P.ldo, tb, 64, paired ? BN / 2 : BN, orow, col0, valid);
         release(2 + acc);
       } else {
         // M = 128: this CTA's 64 rows; lanes 0..63 hold tile columns [0, 128) and
@@ -834,12 +853,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         const int row0 = t.base + (int)rank * (kTileM / 2);
         const int r = (q & 1) * 32 + lane, ch = q >> 1;
         const int col0 = paired ? t.n * (BN / 2) + ch * (BN / 4) : t.n * BN + ch * (BN / 2);
-        const bool valid = r < t.end - row0;
-        epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, 0, paired ? BN / 4 : 64, (int64_t)row0 + r,
-                        col0, valid);
+        bool valid = r < t.end - row0;
+        bf16* o = P.out;
+        int64_t orow = (int64_t)row0 + r;
+        if (P.sc_base != nullptr) scatter_dst(P, valid, o, orow);
+        epilogue_row_rt(P.epi, o, P.outf, P.ldo, tb, 0, paired ? BN / 4 : 64, orow, col0, valid);
         release(acc);
-        if (!paired)
-          epilogue_row_rt(P.epi, P.out, P.outf, P.ldo, tb, 64, BN / 2, (int64_t)row0 + r, col0, valid);
+        if (!paired) epilogue_row_rt(P.epi, o, P.outf, P.ldo, tb, 64, BN / 2, orow, col0, valid);
         release(2 + acc);
       }
       if (P.signal) {
@@ -853,6 +873,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    // rows stored into other ranks' memory are visible system-wide before the kernel
+    // ends (the caller raises the ranks' flags after it)
+    if (p.scatter) __threadfence_system();
   }
 
   // Neither CTA leaves (or frees TMEM) while the pair's MMAs may still touch it.
@@ -1029,6 +1052,16 @@ cudaError_t launch_grouped_pair(const GemmProblem* probs, int n, int32_t* counte
     P.K = p.K;
     P.epi = p.epi;
     P.dep = p.dep;
+    if (p.sc_base != nullptr) {
+      if (p.epi != EPI_STORE || p.sc_rank == nullptr || p.sc_row == nullptr || p.sc_P < 1)
+        return cudaErrorInvalidValue;
+      P.sc_base = p.sc_base;
+      P.sc_rank = p.sc_rank;
+      P.sc_row = p.sc_row;
+      P.sc_P = p.sc_P;
+      P.sc_rows = p.sc_rows;
+      a.scatter = 1;
+    }
     P.signal = 0;
     P.done_base = 0;
     if (p.dep >= 0) {
@@ -1046,6 +1079,13 @@ cudaError_t launch_grouped_pair(const GemmProblem* probs, int n, int32_t* counte
       }
     }
     tiles += (p.max_tiles > 0 ? p.max_tiles : 1);
+  }
+  // a scattering launch runs only M = 256 and M = 128 tiles (the skinny and folded
+  // epilogues write rows of their own)
+  if (a.scatter) {
+    a.skinny = 0;
+    a.fold = 0;
+    a.fold_m256 = 0;
   }
   // the M = 256 fold needs its exchange buffer next to the ring (room for about 700 groups)
   if (a.fold_m256 && PairCfg::smem_bytes(a.group_offsets ? a.G : 1, true) > (size_t)smem_optin()) {

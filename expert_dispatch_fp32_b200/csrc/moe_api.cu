@@ -286,10 +286,19 @@ namespace {
 
 // The expert-FFN stage: the routed experts over x_perm (`routed`) and/or the shared
 // experts over x (`shared`), one persistent launch when all tiles are 256 wide.
+// Where the routed down projection's rows go when they are stored straight into other
+// ranks' buffers (moe_ep_expert_ffn_return): row i to base[rank[i]] at row[i].
+struct FfnScatter {
+  bf16* const* base;
+  const int32_t* rank;
+  const int32_t* row;
+  int P, rows;
+};
+
 moe_status ffn_run(const moe_config* cfg, const void* x_perm, const void* x,
                    const int32_t* expert_offsets, const void* packed, void* act, void* y_perm,
                    void* shared_out, void* workspace, int32_t* status, void* stream, bool routed,
-                   bool shared, bool counters_zeroed = false) {
+                   bool shared, bool counters_zeroed = false, const FfnScatter* scatter = nullptr) {
   moe_status st = moe_validate_config(cfg);
   if (st != MOE_OK) return st;
   const moe_config& c = *cfg;
@@ -299,8 +308,9 @@ moe_status ffn_run(const moe_config* cfg, const void* x_perm, const void* x,
     MOE_CHECK_PTR(x_perm);
     MOE_CHECK_PTR(expert_offsets);
     MOE_CHECK_PTR(act);
-    MOE_CHECK_PTR(y_perm);
+    if (scatter == nullptr) MOE_CHECK_PTR(y_perm);
   }
+  if (scatter != nullptr && (!routed || shared)) return MOE_ERR_INVALID_ARG;
   MOE_CHECK_PTR(packed);
   MOE_CHECK_PTR(workspace);
   MOE_CHECK_PTR(status);
@@ -347,6 +357,13 @@ moe_status ffn_run(const moe_config* cfg, const void* x_perm, const void* x,
   dn.out = (bf16*)y_perm; dn.ldo = c.D;
   dn.epi = EPI_STORE;
   dn.counter = ctr + 2;
+  if (scatter != nullptr) {
+    dn.sc_base = scatter->base;
+    dn.sc_rank = scatter->rank;
+    dn.sc_row = scatter->row;
+    dn.sc_P = scatter->P;
+    dn.sc_rows = scatter->rows;
+  }
 
   // Shared experts: one dense SwiGLU expert of intermediate S*Fs over all tokens.
   const int Fc = c.n_shared * c.F_shared;
@@ -406,6 +423,8 @@ moe_status ffn_run(const moe_config* cfg, const void* x_perm, const void* x,
     return cuda_status(launch_grouped_pair(ph, n, ctr + kFfnCounter, ctr + 8, s));
   }
 
+  // the scattering store exists in the persistent pair launch only
+  if (scatter != nullptr) return MOE_ERR_UNSUPPORTED;
   // Otherwise one launch per GEMM, each with its own tile counter.
   if (cudaMemsetAsync(ctr + 1, 0, 4 * sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
   dn.dep = -1;
@@ -599,6 +618,53 @@ moe_status moe_ep_return_rows(const moe_config* cfg, const moe_ep_peers* peers, 
   if (peers->cap > 0) MOE_CHECK_PTR(y_recv);
   return cuda_status(launch_ep_return_rows(*cfg, *peers, rank0, nlocal, y_recv, local_offsets, done,
                                            epoch, as_stream(stream)));
+}
+
+moe_status moe_ep_expert_ffn_return(const moe_config* cfg, const moe_config* local_cfg,
+                                    const moe_ep_peers* peers, int32_t rank, const void* recv_x,
+                                    const int32_t* recv_src, const int32_t* recv_rank,
+                                    const int32_t* local_offsets, const void* packed, void* act,
+                                    void* y_recv, void* workspace, uint32_t epoch, int32_t* done,
+                                    int32_t* status, void* stream) {
+  moe_status st = ep_check(cfg, peers, rank, 1);
+  if (st != MOE_OK) return st;
+  st = moe_validate_config(local_cfg);
+  if (st != MOE_OK) return st;
+  const moe_config& c = *cfg;
+  const moe_config& l = *local_cfg;
+  if (l.E * c.ep_size != c.E || l.D != c.D || l.F != c.F || l.act != c.act || l.top_k != 1 ||
+      l.T != peers->cap || l.n_shared != c.n_shared || l.F_shared != c.F_shared)
+    return MOE_ERR_INVALID_ARG;
+  // int32 words read one at a time: 4-byte alignment is enough for these
+  auto ptr4 = [](const void* q) { return q != nullptr && ((uintptr_t)q & 3u) == 0; };
+  MOE_CHECK_PTR(local_offsets);
+  if (!ptr4(done)) return MOE_ERR_INVALID_ARG;
+  MOE_CHECK_PTR(status);
+  if (peers->cap == 0) {
+    return cuda_status(launch_ep_signal_returned(*peers, rank, epoch, as_stream(stream)));
+  }
+  MOE_CHECK_PTR(recv_x);
+  if (!ptr4(recv_src) || !ptr4(recv_rank)) return MOE_ERR_INVALID_ARG;
+  MOE_CHECK_PTR(packed);
+  MOE_CHECK_PTR(act);
+  MOE_CHECK_PTR(workspace);
+  cudaStream_t s = as_stream(stream);
+  // MOE_EP_FUSED_RETURN=0: the FFN into y_recv, then the separate return copy (for
+  // comparison; also the form taken where the down GEMM does not run as a pair launch)
+  const char* env = getenv("MOE_EP_FUSED_RETURN");
+  if (!(env && env[0] == '0')) {
+    const FfnScatter sc{(bf16* const*)peers->y_back, recv_rank, recv_src, peers->P, c.T * c.top_k};
+    const int32_t* off = local_offsets;
+    st = ffn_run(local_cfg, recv_x, nullptr, off, packed, act, nullptr, nullptr, workspace, status, stream,
+                 true, false, false, &sc);
+    if (st == MOE_OK) return cuda_status(launch_ep_signal_returned(*peers, rank, epoch, s));
+    if (st != MOE_ERR_UNSUPPORTED) return st;
+  }
+  MOE_CHECK_PTR(y_recv);
+  st = ffn_run(local_cfg, recv_x, nullptr, local_offsets, packed, act, y_recv, nullptr, workspace, status,
+               stream, true, false);
+  if (st != MOE_OK) return st;
+  return cuda_status(launch_ep_return_rows(c, *peers, rank, 1, y_recv, local_offsets, done, epoch, s));
 }
 
 moe_status moe_ep_wait_returned(const moe_config* cfg, const moe_ep_peers* peers, int32_t rank0,

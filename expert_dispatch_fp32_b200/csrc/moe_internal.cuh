@@ -155,6 +155,9 @@ cudaError_t launch_ep_recv_layout(const moe_config& c, const moe_ep_peers& p, in
 cudaError_t launch_ep_return_rows(const moe_config& c, const moe_ep_peers& p, int rank0, int nlocal,
                                   const void* y_recv, const int32_t* local_offsets, int32_t* done,
                                   uint32_t epoch, cudaStream_t s);
+// Rank r's return flag on every rank (after a system-scope fence): its output rows
+// were stored into the senders' y_back by the expert FFN itself.
+cudaError_t launch_ep_signal_returned(const moe_ep_peers& p, int r, uint32_t epoch, cudaStream_t s);
 cudaError_t launch_ep_wait_returned(const moe_ep_peers& p, int rank0, int nlocal, int32_t* status,
                                     uint32_t epoch, cudaStream_t s);
 cudaError_t launch_gather_rows(const bf16* src, const int32_t* index, bf16* dst, int n, int n_src,
@@ -196,6 +199,13 @@ struct GemmProblem {
   int32_t* counter;                       // device tile counter, zero when the launch starts
   int dep;                                // launch_grouped_pair: index of the phase whose output
                                           // rows this phase reads as A, or -1
+  // launch_grouped_pair, EPI_STORE: output row i goes to sc_base[sc_rank[i]] at row
+  // sc_row[i] (another rank's buffer, through a table of sc_P device pointers, each
+  // buffer of sc_rows rows) instead of out; null: out.  No skinny or folded tiles then.
+  bf16* const* sc_base;
+  const int32_t* sc_rank;
+  const int32_t* sc_row;
+  int sc_P, sc_rows;
 };
 // Up to 4 GEMMs (all 256-wide tiles) in one persistent CTA-pair launch, tiles taken
 // phase after phase; probs[i].dep = j (j < i) makes phase i read phase j's output

@@ -173,9 +173,12 @@ class PeerEPGroup:
     Rank r owns experts [r*El, (r+1)*El) and its own T tokens; the shared experts and
     the router are replicated.  The same calls take peer-mapped buffers of other GPUs
     in their pointer tables; here every table entry is a slice of one device's tensors,
-    and each call covers all P ranks in one launch (kernels of different ranks never
-    wait on one another across launches).  forward(x) takes x [P, T, D] and returns
-    out [P, T, D]: rank r's rows equal moe_forward of its tokens with all E experts.
+    and each exchange call covers all P ranks in one launch (kernels of different ranks
+    never wait on one another across launches); each rank's local experts run as their
+    own launch whose down-projection epilogue stores the output rows straight into the
+    senders' y_back (moe_ep_expert_ffn_return).  forward(x) takes x [P, T, D] and
+    returns out [P, T, D]: rank r's rows equal moe_forward of its tokens with all E
+    experts.
     """
 
     def __init__(self, *, D, E, P, top_k, F, T, w_router, w_gate_up, w_down, expert_bias=None,
@@ -252,12 +255,13 @@ class PeerEPGroup:
         B.moe_ep_send_rows(c, self.peers, 0, P, x, self.topk_idx, self.pos, self.offsets, e, self.done,
                            self.status, stream)
         B.moe_ep_recv_layout(c, self.peers, 0, P, self.local_off, e, self.status, stream)
-        for d in range(P):                                 # 3. each rank's local experts
-            B.moe_expert_ffn(self.loc_cfg, self.recv_x[d], None, self.local_off[d], self.packed[d],
-                             self.act[d], self.y_recv[d], None, self.ws_loc[d], self.status, stream)
-        # 4. the token post-all-to-all back to the senders' dispatch rows
-        B.moe_ep_return_rows(c, self.peers, 0, P, self.y_recv, self.local_off, e, self.done,
-                             self.status, stream)
+        # 3.-4. each rank's local experts, their output rows stored by the down GEMM's
+        # epilogue straight back into the senders' y_back at their dispatch rows
+        for d in range(P):
+            B.moe_ep_expert_ffn_return(c, self.loc_cfg, self.peers, d, self.recv_x[d], self.recv_src[d],
+                                       self.recv_rank[d], self.local_off[d], self.packed[d], self.act[d],
+                                       self.y_recv[d], self.ws_loc[d], e, self.done[d:d + 1], self.status,
+                                       stream)
         B.moe_ep_wait_returned(c, self.peers, 0, P, e, self.status, stream)
         for r in range(P):                                 # 5. shared experts and combine
             sh = None
@@ -411,6 +415,8 @@ class PeerEPRank:
         view = lambda name, dt, shape: self.xbuf[self.offsets_x[name]:self.offsets_x[name] + sizes[name]] \
             .view(dt).view(shape)
         self.recv_x = view("recv_x", torch.bfloat16, (cap, D))
+        self.recv_src = view("recv_src", torch.int32, (cap,))
+        self.recv_rank = view("recv_rank", torch.int32, (cap,))
         self.y_back = view("y_back", torch.bfloat16, (R, D))
         self.local_off = i32(El + 1)
         self.act = torch.zeros((cap, F), dtype=torch.bfloat16, device=dev)
@@ -448,11 +454,11 @@ class PeerEPRank:
         B.moe_ep_send_rows(c, self.peers, r, 1, x, self.topk_idx, self.pos, self.offsets, e, self.done,
                            self.status, stream)
         B.moe_ep_recv_layout(c, self.peers, r, 1, self.local_off, e, self.status, stream)
-        B.moe_expert_ffn(self.loc_cfg, self.recv_x, None, self.local_off, self.packed, self.act,
-                         self.y_recv, None, self.ws_loc, self.status, stream)
-        # the token post-all-to-all back to the senders' dispatch rows
-        B.moe_ep_return_rows(c, self.peers, r, 1, self.y_recv, self.local_off, e, self.done,
-                             self.status, stream)
+        # the local experts; the down GEMM's epilogue stores each output row straight into
+        # its sender's y_back (the token post-all-to-all, tile by tile)
+        B.moe_ep_expert_ffn_return(c, self.loc_cfg, self.peers, r, self.recv_x, self.recv_src,
+                                   self.recv_rank, self.local_off, self.packed, self.act, self.y_recv,
+                                   self.ws_loc, e, self.done, self.status, stream)
         B.moe_ep_wait_returned(c, self.peers, r, 1, e, self.status, stream)
         sh = None
         if self.S:

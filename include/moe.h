@@ -42,7 +42,7 @@ extern "C" {
 
 /* 2: the MXFP8 routed-expert calls, moe_dispatch_mxfp8, the router filter view and the
  * peer-memory exchange calls.  3: the moe_ipc_* calls that map another process's
- * exchange buffers. */
+ * exchange buffers, and moe_ep_expert_ffn_return. */
 #define MOE_ABI_VERSION 3
 
 #if defined(__GNUC__)
@@ -311,8 +311,9 @@ MOE_API moe_status moe_gather_rows(const void* src, const int32_t* index, void* 
  * Order of one forward, on every rank: moe_route + moe_preprocess of its tokens,
  * moe_ep_send_counts, moe_ep_send_rows, moe_ep_recv_layout, moe_expert_ffn on the
  * received rows (a config with E = El, top_k = 1, T = cap, shared_out = NULL),
- * moe_ep_return_rows, moe_ep_wait_returned, then moe_shared_ffn and
- * moe_combine_unpermute with y_back in place of y_perm (same rows, same order). */
+ * moe_ep_return_rows (or the last two as one: moe_ep_expert_ffn_return),
+ * moe_ep_wait_returned, then moe_shared_ffn and moe_combine_unpermute with y_back in
+ * place of y_perm (same rows, same order). */
 typedef struct {
   int32_t P;                   /* ranks in the exchange (== cfg->ep_size) */
   int32_t cap;                 /* rows each rank's receive buffers hold */
@@ -360,6 +361,27 @@ MOE_API moe_status moe_ep_return_rows(const moe_config* cfg, const moe_ep_peers*
                                       int32_t rank0, int32_t nlocal, const void* y_recv,
                                       const int32_t* local_offsets, uint32_t epoch,
                                       int32_t* done, int32_t* status, void* stream);
+
+/* The local experts and the token post-all-to-all as one step, for rank `rank` (one
+ * rank per call): moe_expert_ffn on the received rows (local_cfg: E = El, top_k = 1,
+ * T = peers->cap, the tokens config's D, F, act and shared-expert sizes; the shared
+ * experts are not run) whose down-projection epilogue stores each output row straight
+ * into its sender's y_back at the sender's dispatch row (recv_rank / recv_src, this
+ * rank's own buffers), over NVLink / NVSwitch peer memory as each tile finishes, so the
+ * return overlaps the GEMM tile by tile and the rows never pass through a y_recv
+ * buffer; then the rank's return flag on every rank.  Equivalent to moe_expert_ffn into
+ * y_recv followed by moe_ep_return_rows, which is what runs where the down GEMM is not
+ * a CTA-pair launch (D not a multiple of 256) or MOE_EP_FUSED_RETURN=0 is set: y_recv
+ * (bf16 [cap, D]) is needed then and may be NULL otherwise.  recv_x: bf16 [cap, D];
+ * recv_src, recv_rank: int32 [cap] (4-byte aligned); local_offsets: [El+1] from
+ * moe_ep_recv_layout; act: bf16 [cap, F] scratch; workspace:
+ * moe_workspace_size(local_cfg) bytes; done: one device int32 (4-byte aligned), zero. */
+MOE_API moe_status moe_ep_expert_ffn_return(const moe_config* cfg, const moe_config* local_cfg,
+                                            const moe_ep_peers* peers, int32_t rank, const void* recv_x,
+                                            const int32_t* recv_src, const int32_t* recv_rank,
+                                            const int32_t* local_offsets, const void* packed, void* act,
+                                            void* y_recv, void* workspace, uint32_t epoch, int32_t* done,
+                                            int32_t* status, void* stream);
 
 /* Waits until every rank has returned the covered ranks' rows (y_back complete). */
 MOE_API moe_status moe_ep_wait_returned(const moe_config* cfg, const moe_ep_peers* peers,

@@ -74,6 +74,25 @@ def test_peer_exchange_equals_single_gpu_forward(P, wl):
                        f64(xs[1][torch.from_numpy(toks).cuda()]))
 
 
+@pytest.mark.parametrize("fused", ["1", "0"])
+def test_fused_and_separate_return_agree(fused, monkeypatch):
+    """The local experts' down GEMM storing its rows straight into the senders' y_back
+    (moe_ep_expert_ffn_return's default) and the FFN into y_recv followed by the return
+    copy (MOE_EP_FUSED_RETURN=0) give the same bits, equal to moe_forward."""
+    monkeypatch.setenv("MOE_EP_FUSED_RETURN", fused)
+    P, wl = CASES[1]
+    wl = wl.with_(ep_size=P)
+    inp = W.make_inputs(wl, device="cuda")
+    grp = _group(wl, P, inp)
+    xs = _rank_batches(wl, P)
+    layer = make_layer(wl, inp)
+    out = grp.forward(xs).clone()
+    torch.cuda.synchronize()
+    grp.check_status()
+    for r in range(P):
+        assert torch.equal(out[r], layer.forward(xs[r])), r
+
+
 def test_peer_exchange_wait_reports_timeout():
     """A wait for an exchange that never happened (a later epoch nobody signals) runs
     out after about a second and reports MOE_ERR_TIMEOUT; the context stays usable and
