@@ -14,7 +14,7 @@ from ._binding import (  # noqa: F401
     MoeConfig, MoeEpPeers, MoeError, lib, moe_abi_version, moe_check_wait_timeout,
     moe_combine_unpermute, moe_dispatch_mxfp8, moe_dispatch_permute,
     moe_ep_local_ids, moe_ep_recv_layout, moe_ep_return_rows, moe_ep_send_counts, moe_ep_send_rows,
-    moe_ipc_close, moe_ipc_export, moe_ipc_handle_bytes, moe_ipc_import,
+    moe_ipc_close, moe_ipc_export, moe_ipc_handle_bytes, moe_ipc_import, moe_instr_read,
     moe_ep_wait_returned, moe_ep_expert_ffn_return, moe_expert_ffn_mxfp8, moe_mxfp8_quantize, moe_packed_weights_mxfp8_size,
     moe_prepare_weights_mxfp8, moe_workspace_mxfp8_size, moe_expert_ffn, moe_forward, moe_gather_rows, moe_packed_weights_size,
     moe_prepare_weights, moe_preprocess, moe_preprocess_noalloc, moe_shared_ffn,

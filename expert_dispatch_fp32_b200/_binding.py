@@ -99,6 +99,7 @@ _SIGS = {
     "moe_ipc_export": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint64)]),
     "moe_ipc_import": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_uint64, ctypes.POINTER(ctypes.c_void_p)]),
     "moe_ipc_close": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_uint64]),
+    "moe_instr_read": (ctypes.c_int, [ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_abi_version": (ctypes.c_int32, []),
 }
@@ -209,6 +210,18 @@ def moe_ipc_import(handle: bytes, offset: int) -> int:
 
 def moe_ipc_close(ptr: int, offset: int) -> None:
     _call("moe_ipc_close", ptr, offset)
+
+
+INSTR_CTAS, INSTR_SLOTS = 160, 24
+
+
+def moe_instr_read(kernel: int):
+    """Cycle counters of an instrumented library (kernel 0: bf16 GEMMs, 1: MXFP8) as a
+    [160, 24] uint64 numpy array; zeroes them on the device."""
+    import numpy as np
+    buf = (ctypes.c_uint64 * (INSTR_CTAS * INSTR_SLOTS))()
+    _call("moe_instr_read", kernel, buf, INSTR_CTAS * INSTR_SLOTS)
+    return np.frombuffer(buf, dtype=np.uint64).reshape(INSTR_CTAS, INSTR_SLOTS).copy()
 
 
 def moe_mxfp8_quantize(x, rows, K, q, scales, stream=None):

@@ -19,9 +19,11 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-BUILD = os.path.join(ROOT, "_build")
+_BUILD = os.path.join(ROOT, "_build")
+_BUILD_INSTR = os.path.join(ROOT, "_build", "instr")
 LIBDIR = os.path.join(PKG, "lib")
-LIB = os.path.join(LIBDIR, "libmoe.so")
+LIB_PLAIN = os.path.join(LIBDIR, "libmoe.so")
+LIB_INSTR = os.path.join(LIBDIR, "libmoe_instr.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -39,7 +41,13 @@ def _headers():
     return glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(ROOT, "include", "*.h"))
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False,
+          instrument: bool = False) -> str:
+    """Build libmoe.so (or, instrument=True, libmoe_instr.so: the same sources with the
+    kernels' cycle counters compiled in, -DMOE_INSTRUMENT, in a build folder of its own)."""
+    BUILD = _BUILD_INSTR if instrument else _BUILD
+    LIB = LIB_INSTR if instrument else LIB_PLAIN
+    extra = ["-DMOE_INSTRUMENT"] if instrument else []
     os.makedirs(BUILD, exist_ok=True)
     os.makedirs(LIBDIR, exist_ok=True)
     hdr_mtime = max((os.path.getmtime(h) for h in _headers()), default=0)
@@ -51,7 +59,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
         if (not force and os.path.exists(obj)
                 and os.path.getmtime(obj) >= max(os.path.getmtime(src), hdr_mtime)):
             continue
-        cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-c", src, "-o", obj]
+        cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *extra, "-c", src, "-o", obj]
         if ptxas_verbose:
             cmd += ["-Xptxas", "-v"]
         if verbose:
@@ -73,6 +81,7 @@ if __name__ == "__main__":
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true")
+    ap.add_argument("--instrument", action="store_true", help="build libmoe_instr.so (cycle counters)")
     a = ap.parse_args()
-    print(build(a.force, a.verbose, a.ptxas_verbose))
+    print(build(a.force, a.verbose, a.ptxas_verbose, a.instrument))
     sys.exit(0)

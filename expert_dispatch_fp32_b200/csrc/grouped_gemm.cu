@@ -657,6 +657,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
       int stage = 0;
       uint32_t phase = 0;
       int next = leader ? atomicAdd(p.counter, 1) : 0;
+      const long long ti0 = instr_clock();
       for (int qi = 0;; ++qi) {
         const int tile = leader
             ? tq_post<true>(p.counter, next, total, qi, qfull0, qempty0, tq, abort_flag, p.status)
@@ -693,7 +694,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         const int ksteps = P.K / kTileK;
         bool ok = true;
         for (int kb = 0; kb < ksteps; ++kb) {
+          const long long tw = instr_clock();
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          instr_add(IS_PROD_WAIT, instr_clock() - tw);
           if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, stage_tx);
           const uint32_t fb = full0_leader + 8 * stage;
           tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), amap, fb, kb * kTileK, arow);
@@ -705,6 +708,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         }
         if (!ok) break;
       }
+      instr_add(IS_PROD_TOTAL, instr_clock() - ti0);
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
@@ -713,6 +717,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
       uint32_t phase = 0;
       int acc = 0;
       uint32_t freeph = 0;       // bit i: parity of the next wait on TMEM region i
+      const long long ti0 = instr_clock();
       for (int qi = 0;; ++qi) {
         const int tile = tq_take<false>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
         if (tile < 0) break;
@@ -730,19 +735,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
         const uint32_t need = (1u << acc) | (kind != TK_SKINNY ? 4u << acc : 0u) |
                               (kind == TK_FOLD ? 1u << (acc ^ 1) : 0u);
         bool ok = true;
+        const long long tw = instr_clock();
         for (int i = 0; i < 4 && ok; ++i) {
           if (!((need >> i) & 1u)) continue;
           ok = mbar_wait(tfree0 + 8 * i, ((freeph >> i) & 1u) ^ 1u, abort_flag, p.status);
           freeph ^= 1u << i;
         }
         if (!ok) break;
+        const long long tk0 = instr_clock();
+        instr_add(IS_MMA_WAIT_ACC, tk0 - tw);
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         // skinny products (and a folded remainder, in the other buffer's head): the
         // first 64 weight rows into columns [0, ns/2), the second 64 into [32, 32 + ns/2)
         const uint32_t s_tmem = kind == TK_FOLD ? tmem_base + (uint32_t)((acc ^ 1) * BN) : d_tmem;
         for (int kb = 0; kb < ksteps; ++kb) {
+          const long long tf = instr_clock();
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.status)) { ok = false; break; }
+          instr_add(IS_MMA_WAIT_FULL, instr_clock() - tf);
           tc_fence_after();
           const uint64_t ad = sw128_desc(smem_u32(a_smem + stage * C::kABytes));
           const uint64_t bd = sw128_desc(smem_u32(b_smem + stage * C::kBBytes));
@@ -780,9 +790,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
+        {
+          const int ki = kind == TK_FULL ? 0 : kind == TK_HALF ? 1 : kind == TK_FOLD ? 2 : 3;
+          instr_add(IS_FULL_N + 2 * ki, 1);
+          instr_add(IS_FULL_CYC + 2 * ki, instr_clock() - tk0);
+          instr_add(IS_FULL_K + ki, ksteps);
+          instr_add(IS_KSTEPS, ksteps);
+        }
         tc_commit_pair_both(tfull0 + 8 * acc);
         acc ^= 1;
       }
+      instr_add(IS_MMA_TOTAL, instr_clock() - ti0);
     }
   } else {
     // ---------------- epilogue (warps 2..5 of both CTAs) ----------------
@@ -791,6 +809,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t xk = 0;             // gate/up hand-overs of folded remainders so far
+    const bool instr_epi = warp == 2 && lane == 0;
+    const long long ti0 = instr_clock();
     // release TMEM region i: this warp has read all of its columns
     auto release = [&](int i) {
       tc_fence_before();
@@ -806,7 +826,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
       int ns;
       const int kind = tile_kind(t, p.skinny, p.fold, ns);
       bool ok = true;
+      const long long tw = instr_clock();
       if (lane == 0) ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, p.status);
+      if (instr_epi) instr_add(IS_EPI_WAIT, instr_clock() - tw);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const bool paired = P.epi == EPI_SWIGLU || P.epi == EPI_PAIRSUM_F32;
@@ -876,6 +898,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) grouped_gemm_pair_kernel(cons
     // rows stored into other ranks' memory are visible system-wide before the kernel
     // ends (the caller raises the ranks' flags after it)
     if (p.scatter) __threadfence_system();
+    if (instr_epi) instr_add(IS_EPI_TOTAL, instr_clock() - ti0);
   }
 
   // Neither CTA leaves (or frees TMEM) while the pair's MMAs may still touch it.
@@ -1141,5 +1164,8 @@ cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s) {
   }
   return cudaErrorInvalidValue;
 }
+
+// The pair and one-CTA kernels' cycle counters (instrumented builds; else not supported).
+cudaError_t instr_read_pair(unsigned long long* host, int n) { return instr_read_tu(host, n); }
 
 }  // namespace moe

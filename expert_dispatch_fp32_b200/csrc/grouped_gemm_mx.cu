@@ -355,6 +355,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
       int stage = 0;
       uint32_t phase = 0;
       int next = leader ? atomicAdd(p.counter, 1) : 0;
+      const long long ti0 = instr_clock();
       for (int qi = 0;; ++qi) {
         const int tile = leader
             ? tq_post<true>(p.counter, next, total, qi, qfull0, qempty0, tq, abort_flag, p.status)
@@ -377,7 +378,9 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
         const int64_t tb = (int64_t)g * nb + n;              // B's tile
         bool ok = true;
         for (int kb = 0; kb < ksteps; ++kb) {
+          const long long tw = instr_clock();
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
+          instr_add(IS_PROD_WAIT, instr_clock() - tw);
           if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, stage_tx);
           const uint32_t fb = full0_leader + 8 * stage;
           tma_load_2d_pair(smem_u32(a_smem + stage * C::kABytes), amap, fb, kb * C::KS, arow);
@@ -399,6 +402,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
         }
         if (!ok) break;
       }
+      instr_add(IS_PROD_TOTAL, instr_clock() - ti0);
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
@@ -409,6 +413,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_phase = 0, rem_phase = 0;
+      const long long ti0 = instr_clock();
       for (int qi = 0;; ++qi) {
         const int tile = tq_take<false>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
         if (tile < 0) break;
@@ -418,16 +423,21 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
         int ns;
         const bool fd = FOLD && mx_is_fold(rows, m, fold, ns);
         const bool hf = !fd && mx_is_half(rows, m, p.half);
+        const long long tw = instr_clock();
         if (!mbar_wait(tempty, acc_phase ^ 1u, abort_flag, p.status)) break;
         acc_phase ^= 1u;
         if (fd) {                              // the previous folded tile's remainder is read out
           if (!mbar_wait(tempty_rem, rem_phase ^ 1u, abort_flag, p.status)) break;
           rem_phase ^= 1u;
         }
+        const long long tk0 = instr_clock();
+        instr_add(IS_MMA_WAIT_ACC, tk0 - tw);
         tc_fence_after();
         bool ok = true;
         for (int kb = 0; kb < ksteps; ++kb) {
+          const long long tf = instr_clock();
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, p.status)) { ok = false; break; }
+          instr_add(IS_MMA_WAIT_FULL, instr_clock() - tf);
           tc_fence_after();
           const uint32_t sa = smem_u32(sfa_smem + stage * C::kSfaBytes);
           const uint32_t sb = smem_u32(sfb_smem + stage * C::kSfbBytes);
@@ -464,8 +474,16 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
+        {
+          const int ki = fd ? 2 : hf ? 1 : 0;
+          instr_add(IS_FULL_N + 2 * ki, 1);
+          instr_add(IS_FULL_CYC + 2 * ki, instr_clock() - tk0);
+          instr_add(IS_FULL_K + ki, ksteps);
+          instr_add(IS_KSTEPS, ksteps);
+        }
         tc_commit_pair_both(tfull);
       }
+      instr_add(IS_MMA_TOTAL, instr_clock() - ti0);
     }
   } else {
     // ---------------- epilogue (warps 2..9 of both CTAs) ----------------
@@ -475,13 +493,17 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
     const uint32_t tempty_rem_leader = map_to_cta(tempty_rem, 0);
     uint32_t acc_phase = 0;
     uint32_t xk = 0;                        // gate/up hand-overs of folded remainders so far
+    const bool instr_epi = warp == 2 && lane == 0;
+    const long long ti0 = instr_clock();
     for (int qi = 0;; ++qi) {
       const int tile = tq_take<true>(qi, qfull0, qempty_sched, tq, abort_flag, p.status);
       if (__any_sync(0xffffffffu, tile < 0)) break;
       int g, m, n;
       decode_tile(tile, mt, G, nb, g, m, n);
       bool ok = true;
+      const long long tw = instr_clock();
       if (lane == 0) ok = mbar_wait(tfull, acc_phase, abort_flag, p.status);
+      if (instr_epi) instr_add(IS_EPI_WAIT, instr_clock() - tw);
       if (!__all_sync(0xffffffffu, ok)) break;
       acc_phase ^= 1u;
       tc_fence_after();
@@ -641,6 +663,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) grouped_gemm_mx_kernel(const __
         __syncwarp();
       }
     }
+    if (instr_epi) instr_add(IS_EPI_TOTAL, instr_clock() - ti0);
   }
 
   // Neither CTA leaves (or frees TMEM) while the pair's MMAs may still touch it.
@@ -854,5 +877,8 @@ cudaError_t launch_grouped_mx(const MxProblem& p, cudaStream_t s) {
   if (p.epi == EPI_GELU) return launch_mx<EPI_GELU, false>(a, clusters, s);
   return launch_mx<EPI_STORE, false>(a, clusters, s);
 }
+
+// The MXFP8 kernel's cycle counters (instrumented builds; else not supported).
+cudaError_t instr_read_mx(unsigned long long* host, int n) { return instr_read_tu(host, n); }
 
 }  // namespace moe

@@ -864,4 +864,12 @@ const char* moe_status_string(moe_status s) {
 
 int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
 
+moe_status moe_instr_read(int32_t kernel, uint64_t* counters, int32_t n) {
+  if (counters == nullptr || n < 0 || (kernel != 0 && kernel != 1)) return MOE_ERR_INVALID_ARG;
+  unsigned long long* h = reinterpret_cast<unsigned long long*>(counters);
+  const cudaError_t e = kernel == 0 ? instr_read_pair(h, n) : instr_read_mx(h, n);
+  if (e == cudaErrorNotSupported) return MOE_ERR_UNSUPPORTED;
+  return cuda_status(e);
+}
+
 }  // extern "C"

@@ -217,5 +217,9 @@ int64_t pair_done_slots(const GemmProblem* probs, int n);
 cudaError_t launch_grouped_gemm(const GemmProblem& p, cudaStream_t s);
 
 int sm_count();
+// Cycle counters of an instrumented build (-DMOE_INSTRUMENT): copied to host and zeroed;
+// cudaErrorNotSupported in an ordinary build.
+cudaError_t instr_read_pair(unsigned long long* host, int n);
+cudaError_t instr_read_mx(unsigned long long* host, int n);
 
 }  // namespace moe

@@ -17,6 +17,58 @@ constexpr int kGemmThreads = 192;
 constexpr int kCtrlBytes = 512;     // barriers, tile queue, TMEM slot, abort flag
 
 // ---------------------------------------------------------------------------
+// Cycle counters of an instrumented build (-DMOE_INSTRUMENT; compiled out otherwise):
+// per CTA, kInstrSlots 64-bit sums of SM cycles (clock64), each slot written by one
+// thread of its CTA only, read back with moe_instr_read.  They show where a GEMM
+// launch's MMA issuer, producer and epilogue spend their cycles, per tile kind.
+// ---------------------------------------------------------------------------
+constexpr int kInstrSlots = 24;
+constexpr int kInstrCtas = 160;     // >= one CTA per SM
+enum InstrSlot {
+  IS_MMA_TOTAL = 0,   // MMA issuer: the whole tile loop
+  IS_MMA_WAIT_ACC,    //   waiting for its accumulator (TMEM) to be drained
+  IS_MMA_WAIT_FULL,   //   waiting for a filled stage
+  IS_FULL_N,          // tiles of each kind and the issuer's cycles from their first to
+  IS_FULL_CYC,        //   their last K step (stage waits included)
+  IS_HALF_N,
+  IS_HALF_CYC,
+  IS_FOLD_N,
+  IS_FOLD_CYC,
+  IS_SKINNY_N,
+  IS_SKINNY_CYC,
+  IS_KSTEPS,          // K steps issued
+  IS_PROD_WAIT,       // producer (lane 0 of warp 0, both CTAs): waiting for a free stage
+  IS_PROD_TOTAL,
+  IS_EPI_WAIT,        // first epilogue warp (lane 0): waiting for a full accumulator
+  IS_EPI_TOTAL,
+  IS_FULL_K,          // K steps of full, M = 128, folded and skinny tiles
+  IS_HALF_K,
+  IS_FOLD_K,
+  IS_SKINNY_K,
+};
+#ifdef MOE_INSTRUMENT
+__device__ unsigned long long g_instr[kInstrCtas * kInstrSlots];
+__device__ __forceinline__ long long instr_clock() { return clock64(); }
+__device__ __forceinline__ void instr_add(int slot, long long v) {
+  if (blockIdx.x < kInstrCtas) g_instr[blockIdx.x * kInstrSlots + slot] += (unsigned long long)v;
+}
+// Copies this translation unit's counters to host[] (n values at most) and zeroes them.
+inline cudaError_t instr_read_tu(unsigned long long* host, int n) {
+  const size_t bytes = sizeof(unsigned long long) * (size_t)(n < kInstrCtas * kInstrSlots ? n : kInstrCtas * kInstrSlots);
+  cudaError_t e = cudaMemcpyFromSymbol(host, g_instr, bytes);
+  if (e != cudaSuccess) return e;
+  void* d = nullptr;
+  e = cudaGetSymbolAddress(&d, g_instr);
+  if (e != cudaSuccess) return e;
+  return cudaMemset(d, 0, sizeof(unsigned long long) * kInstrCtas * kInstrSlots);
+}
+#else
+__device__ __forceinline__ long long instr_clock() { return 0; }
+__device__ __forceinline__ void instr_add(int, long long) {}
+inline cudaError_t instr_read_tu(unsigned long long*, int) { return cudaErrorNotSupported; }
+#endif
+
+// ---------------------------------------------------------------------------
 // PTX wrappers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

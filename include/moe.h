@@ -42,7 +42,7 @@ extern "C" {
 
 /* 2: the MXFP8 routed-expert calls, moe_dispatch_mxfp8, the router filter view and the
  * peer-memory exchange calls.  3: the moe_ipc_* calls that map another process's
- * exchange buffers, and moe_ep_expert_ffn_return. */
+ * exchange buffers, moe_ep_expert_ffn_return and moe_instr_read. */
 #define MOE_ABI_VERSION 3
 
 #if defined(__GNUC__)
@@ -507,6 +507,17 @@ MOE_API const char* moe_status_string(moe_status s);
 
 /* MOE_ABI_VERSION of the loaded library. */
 MOE_API int32_t moe_abi_version(void);
+
+/* Cycle counters of an instrumented build of the library (compiled with
+ * -DMOE_INSTRUMENT: `python -m expert_dispatch_fp32_b200.instrument`).  kernel 0: the bf16
+ * grouped-GEMM kernels, 1: the MXFP8 kernel.  counters: host uint64 [n], written with up
+ * to 160 CTAs x 24 slots of summed SM cycles and counts (slot order: MMA issuer total, its
+ * waits for the accumulator, its waits for a filled stage, then tiles and issuer cycles of
+ * full, M = 128, folded and skinny tiles, K steps, the producer's waits for a free stage
+ * and its total, the first epilogue warp's waits for a full accumulator and its total,
+ * then the K steps of full, M = 128, folded and skinny tiles); the device counters are
+ * zeroed.  Synchronous.  MOE_ERR_UNSUPPORTED in an ordinary build. */
+MOE_API moe_status moe_instr_read(int32_t kernel, uint64_t* counters, int32_t n);
 
 #ifdef __cplusplus
 }
