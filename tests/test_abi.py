@@ -158,3 +158,17 @@ def test_peer_exchange_calls_reject_bad_tables_on_host(B):
     assert lib.moe_ep_recv_layout(by, ctypes.addressof(nul), 0, 1, h, 1, h, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_ep_send_rows(by, pa, 0, 1, h, h, h, None, 1, h, h, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_ep_return_rows(by, pa, 0, 1, h, h, 1, None, h, None) == B.MOE_ERR_INVALID_ARG
+
+
+def test_cycle_counters_exist_only_in_an_instrumented_build(B):
+    """moe_instr_read answers MOE_ERR_UNSUPPORTED from the ordinary library (the counters
+    are compiled out) and checks its arguments on the host first."""
+    import numpy as np
+    lib = B.lib()
+    buf = np.zeros(B.INSTR_CTAS * B.INSTR_SLOTS, dtype=np.uint64)
+    p = buf.ctypes.data
+    assert lib.moe_instr_read(0, p, buf.size) == B.MOE_ERR_UNSUPPORTED
+    assert lib.moe_instr_read(1, p, buf.size) == B.MOE_ERR_UNSUPPORTED
+    assert lib.moe_instr_read(2, p, buf.size) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_instr_read(0, None, buf.size) == B.MOE_ERR_INVALID_ARG
+    assert not buf.any()
