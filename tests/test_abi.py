@@ -172,3 +172,32 @@ def test_cycle_counters_exist_only_in_an_instrumented_build(B):
     assert lib.moe_instr_read(2, p, buf.size) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_instr_read(0, None, buf.size) == B.MOE_ERR_INVALID_ARG
     assert not buf.any()
+
+
+def test_fused_return_call_checks_its_configs_on_host(B):
+    """moe_ep_expert_ffn_return rejects, before enqueuing anything, a local config that is
+    not the tokens config's local-expert view (E/P experts, top-1, T = cap, same D/F/act),
+    a rank outside the exchange, a null or misaligned `done`, and a null table."""
+    c = good_cfg(B, act=B.MOE_ACT_SWIGLU, F=128, x_dtype=B.MOE_DT_BF16)    # E 16, ep 4, D 64
+    lib = B.lib()
+    import numpy as np
+    buf = np.zeros(1 << 12, dtype=np.uint8)
+    h = (buf.ctypes.data + 255) // 256 * 256
+    peers = B.MoeEpPeers(4, 16, h, h, h, h, h, h)
+    pa = ctypes.addressof(peers)
+    mk = lambda **kw: B.MoeConfig(**{**dict(T=16, D=64, E=4, ep_size=1, top_k=1, F=128,
+                                            act=B.MOE_ACT_SWIGLU, renormalize=1, x_dtype=B.MOE_DT_BF16,
+                                            router_dtype=B.MOE_DT_F32, n_shared=0, F_shared=0), **kw})
+    call = lambda loc, rank=0, done=h, p=pa: lib.moe_ep_expert_ffn_return(
+        ctypes.byref(c), ctypes.byref(loc), p, rank, h, h, h, h, h, h, None, h, 1, done, h, None)
+    # both configs are valid on their own, so each rejection below is the one field changed
+    # (a fully valid call would enqueue, which this host-memory test never does)
+    assert lib.moe_validate_config(ctypes.byref(c)) == 0 and lib.moe_validate_config(ctypes.byref(mk())) == 0
+    assert call(mk(E=8)) == B.MOE_ERR_INVALID_ARG          # not E / P experts
+    assert call(mk(T=32)) == B.MOE_ERR_INVALID_ARG         # T is not the receive capacity
+    assert call(mk(top_k=2)) == B.MOE_ERR_INVALID_ARG
+    assert call(mk(F=256)) == B.MOE_ERR_INVALID_ARG
+    assert call(mk(), rank=4) == B.MOE_ERR_INVALID_ARG
+    assert call(mk(), done=None) == B.MOE_ERR_INVALID_ARG
+    assert call(mk(), done=h + 2) == B.MOE_ERR_INVALID_ARG
+    assert call(mk(), p=None) == B.MOE_ERR_INVALID_ARG
