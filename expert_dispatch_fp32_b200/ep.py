@@ -453,6 +453,12 @@ class PeerEPRank:
         B.moe_ep_send_counts(c, self.peers, r, 1, self.counts, e, stream)
         B.moe_ep_send_rows(c, self.peers, r, 1, x, self.topk_idx, self.pos, self.offsets, e, self.done,
                            self.status, stream)
+        # the shared experts need only this rank's tokens: they run while the other ranks'
+        # rows are still on their way (the wait below then finds them there)
+        sh = None
+        if self.S:
+            sh = self.shared_out
+            B.moe_shared_ffn(self.sh_cfg, x, self.packed, sh, self.ws_sh, self.status, stream)
         B.moe_ep_recv_layout(c, self.peers, r, 1, self.local_off, e, self.status, stream)
         # the local experts; the down GEMM's epilogue stores each output row straight into
         # its sender's y_back (the token post-all-to-all, tile by tile)
@@ -460,10 +466,6 @@ class PeerEPRank:
                                    self.recv_rank, self.local_off, self.packed, self.act, self.y_recv,
                                    self.ws_loc, e, self.done, self.status, stream)
         B.moe_ep_wait_returned(c, self.peers, r, 1, e, self.status, stream)
-        sh = None
-        if self.S:
-            sh = self.shared_out
-            B.moe_shared_ffn(self.sh_cfg, x, self.packed, sh, self.ws_sh, self.status, stream)
         B.moe_combine_unpermute(c, self.y_back, self.pos, self.topk_w, x, sh, self.out, stream)
         return self.out
 
