@@ -373,7 +373,9 @@ class PeerEPRank:
     the others').  Rows are stored straight into the owners' memory over NVLink /
     NVSwitch and every wait is a flag in peer memory: no collective library and no host
     round trip per forward.  Every rank calls forward the same number of times, with T
-    tokens each; close() (after the last forward, on every rank) unmaps the peers.
+    tokens each; close() (after the last forward, on every rank) unmaps the peers.  Each
+    process selects its own GPU (torch.cuda.set_device) before constructing the rank, and
+    its weights live there.
     """
 
     def __init__(self, group=None, *, D, E, top_k, F, T, w_router, w_gate_up_local, w_down_local,
